@@ -1,0 +1,201 @@
+"""fp64 CPU oracle for MiniMax Sparse Attention (MSA) over GQA -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+import this package. It shares nothing with the CUDA library (``block_sparse_gqa_branch_b200``)
+and the library never imports it. The arithmetic lives in ``msa_oracle.c``; this file only
+builds it with gcc, marshals numpy arrays through ctypes, and loops over sequences and groups.
+
+Parity status of each function (what pins it) is listed in the tests that exercise it:
+``oracle_pool``, ``block_scores``, ``select`` and ``attend`` are pinned (tests/test_oracle_pins.py);
+nothing here is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "msa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libmsa_oracle.so")
+_lib = None
+
+P = ctypes.c_void_p
+I64 = ctypes.c_int64
+INT = ctypes.c_int
+
+
+def build(force: bool = False) -> str:
+    """Compile msa_oracle.c with gcc (plain C, -O2, no fast-math) into libmsa_oracle.so."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        # MSA_ORACLE_LIB lets the mutation test load a deliberately broken copy of the oracle
+        _lib = ctypes.CDLL(os.environ.get("MSA_ORACLE_LIB") or build())
+        _lib.oracle_bf16_to_f64.restype = ctypes.c_double
+        _lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        _lib.oracle_pool.argtypes = [P, I64, I64, I64, I64, I64, P, P]
+        _lib.oracle_block_scores.argtypes = [P, P, I64, I64, P]
+        _lib.oracle_select_from_scores.restype = I64
+        _lib.oracle_select_from_scores.argtypes = [P, I64, I64, P, P]
+        _lib.oracle_select_fullsort.restype = I64
+        _lib.oracle_select_fullsort.argtypes = [P, I64, I64, P]
+        _lib.oracle_attend_row.restype = I64
+        _lib.oracle_attend_row.argtypes = [P, P, P, I64, I64, P, I64, I64, P, P]
+        _lib.oracle_select_rows.argtypes = [I64, P, P, P, I64, I64, I64, INT, P, P, P]
+        _lib.oracle_attend_rows.argtypes = [I64, P, P, I64, P, P, I64, P, I64, I64, INT, INT,
+                                            P, P, P]
+    return _lib
+
+
+def default_threads() -> int:
+    return os.cpu_count() or 1
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# --------------------------------------------------------------------------- thin wrappers
+def pool(k_idx_seq: np.ndarray, Bk: int = 128, nb_cap: Optional[int] = None):
+    """k_idx_seq: [N, G, dI] bf16 bits of one sequence -> (pooled [G, nb_cap, dI] f64,
+    tail_sum [G, dI] f64)."""
+    k = _c(k_idx_seq, np.uint16)
+    N, G, dI = k.shape
+    nb = N // Bk if nb_cap is None else nb_cap
+    pooled = np.zeros((G, max(nb, 1), dI), np.float64)
+    tail = np.zeros((G, dI), np.float64)
+    lib().oracle_pool(_p(k), N, G, dI, Bk, max(nb, 1), _p(pooled), _p(tail))
+    return pooled[:, :nb], tail
+
+
+def block_scores(q_idx_row: np.ndarray, pooled_g: np.ndarray, n_cand: int) -> np.ndarray:
+    q = _c(q_idx_row, np.uint16)
+    pg = _c(pooled_g, np.float64)
+    s = np.zeros(max(n_cand, 1), np.float64)
+    lib().oracle_block_scores(_p(q), _p(pg), q.shape[-1], n_cand, _p(s))
+    return s[:n_cand]
+
+
+def select_from_scores(s: np.ndarray, c: int, topk: int = 16):
+    s = _c(s, np.float64) if len(s) else np.zeros(1, np.float64)
+    sel = np.zeros(topk, np.int32)
+    kth = np.zeros(1, np.float64)
+    n = lib().oracle_select_from_scores(_p(s), c, topk, _p(sel), _p(kth))
+    return sel, int(n), float(kth[0])
+
+
+def select_fullsort(s: np.ndarray, c: int, topk: int = 16):
+    s = _c(s, np.float64) if len(s) else np.zeros(1, np.float64)
+    sel = np.zeros(topk, np.int32)
+    n = lib().oracle_select_fullsort(_p(s), c, topk, _p(sel))
+    return sel, int(n)
+
+
+def select_rows(t: np.ndarray, q_idx_rows: np.ndarray, pooled_g: np.ndarray, Bk: int = 128,
+                topk: int = 16, nthreads: Optional[int] = None):
+    """Selection for queries of one (sequence, group). Returns (sel [n,topk], kth [n], nsel [n])."""
+    t = _c(t, np.int64)
+    q = _c(q_idx_rows, np.uint16)
+    pg = _c(pooled_g, np.float64)
+    n = len(t)
+    sel = np.zeros((n, topk), np.int32)
+    kth = np.zeros(n, np.float64)
+    nsel = np.zeros(n, np.int64)
+    lib().oracle_select_rows(n, _p(t), _p(q), _p(pg), q.shape[-1], Bk, topk,
+                             nthreads or default_threads(), _p(sel), _p(kth), _p(nsel))
+    return sel, kth, nsel
+
+
+def attend_rows(t: np.ndarray, q_rows: np.ndarray, K: np.ndarray, V: np.ndarray,
+                sel: Optional[np.ndarray], Bk: int = 128, topk: int = 16, dense: bool = False,
+                nthreads: Optional[int] = None):
+    """Attention for queries of one (sequence, group).
+    q_rows [n, Hg, d]; K, V [L, d] of the group; sel [n, topk] (ignored when dense).
+    Returns (o [n, Hg, d] f64, lse [n, Hg] f64, nkeys [n])."""
+    t = _c(t, np.int64)
+    q = _c(q_rows, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    n, Hg, d = q.shape
+    s = _c(sel if sel is not None else np.full((n, topk), -1), np.int32)
+    o = np.zeros((n, Hg, d), np.float64)
+    lse = np.zeros((n, Hg), np.float64)
+    nk = np.zeros(n, np.int64)
+    lib().oracle_attend_rows(n, _p(t), _p(q), Hg, _p(K), _p(V), d, _p(s), topk, Bk,
+                             1 if dense else 0, nthreads or default_threads(), _p(o), _p(lse),
+                             _p(nk))
+    return o, lse, nk
+
+
+# --------------------------------------------------------------------------- whole passes
+def prefill(x: dict, Hq: int, G: int, Bk: int = 128, topk: int = 16, sel: Optional[np.ndarray] = None,
+            nthreads: Optional[int] = None, with_attention: bool = True):
+    """MSA prefill over whole host tensors (bf16 bits, library layouts):
+    q [B,N,Hq,d], k/v [B,G,N,d], q_idx/k_idx [B,N,G,dI].
+    If ``sel`` [B,N,G,topk] is given, attention runs on that selection instead of the
+    oracle's own. Returns dict(sel, kth, nsel, out [B,N,Hq,d], lse [B,N,Hq], nkeys [B,N,G],
+    pooled [B,G,nb,dI])."""
+    q, k, v, qi, ki = x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"]
+    B, N, _, d = q.shape
+    dI = qi.shape[-1]
+    Hg = Hq // G
+    nb = N // Bk
+    t = np.arange(N, dtype=np.int64)
+    res = {
+        "sel": np.zeros((B, N, G, topk), np.int32),
+        "kth": np.zeros((B, N, G), np.float64),
+        "nsel": np.zeros((B, N, G), np.int64),
+        "pooled": np.zeros((B, G, nb, dI), np.float64),
+    }
+    if with_attention:
+        res["out"] = np.zeros((B, N, Hq, d), np.float64)
+        res["lse"] = np.zeros((B, N, Hq), np.float64)
+        res["nkeys"] = np.zeros((B, N, G), np.int64)
+    for b in range(B):
+        pooled, _ = pool(ki[b], Bk)
+        res["pooled"][b] = pooled
+        for g in range(G):
+            s_, kth, ns = select_rows(t, qi[b, :, g, :], pooled[g], Bk, topk, nthreads)
+            res["sel"][b, :, g], res["kth"][b, :, g], res["nsel"][b, :, g] = s_, kth, ns
+            if with_attention:
+                use = s_ if sel is None else sel[b, :, g]
+                o, lse, nk = attend_rows(t, q[b, :, g * Hg:(g + 1) * Hg, :], k[b, g], v[b, g],
+                                         use, Bk, topk, False, nthreads)
+                res["out"][b, :, g * Hg:(g + 1) * Hg] = o
+                res["lse"][b, :, g * Hg:(g + 1) * Hg] = lse
+                res["nkeys"][b, :, g] = nk
+    return res
+
+
+def dense_gqa(x: dict, Hq: int, G: int, nthreads: Optional[int] = None):
+    """Dense causal GQA attention (every key u <= t) with the same layouts; the comparator
+    the pages measure MSA against. Returns (out [B,N,Hq,d], lse [B,N,Hq])."""
+    q, k, v = x["q"], x["k"], x["v"]
+    B, N, _, d = q.shape
+    Hg = Hq // G
+    t = np.arange(N, dtype=np.int64)
+    out = np.zeros((B, N, Hq, d), np.float64)
+    lse = np.zeros((B, N, Hq), np.float64)
+    for b in range(B):
+        for g in range(G):
+            o, l, _ = attend_rows(t, q[b, :, g * Hg:(g + 1) * Hg, :], k[b, g], v[b, g], None,
+                                  dense=True, nthreads=nthreads)
+            out[b, :, g * Hg:(g + 1) * Hg] = o
+            lse[b, :, g * Hg:(g + 1) * Hg] = l
+    return out, lse

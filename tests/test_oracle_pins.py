@@ -1,0 +1,248 @@
+"""Pins of the fp64 oracle against things other than itself (CPU only).
+
+Every check uses an independent route: a numpy / torch library routine (mean, matmul,
+lexsort, scaled_dot_product_attention, logsumexp), a closed form, an invariant of the
+definition, or a constructed case whose answer is known by design. Sources for the
+definition: the youmind article "MiniMax M3 sparse attention agents" (paragraph "The
+mechanism that changes this", figure 1 caption, bullet "Predictable cost at every length":
+Bk = 128, k = 16, 2,048 tokens) and the KuCoin flash "MiniMax launches MSA sparse attention
+method and MiniMax-M3 model" (summary: GQA-based, exact softmax over the 16 blocks, exp-free
+top-k).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import synth
+from tests.msa_check import compare_selection_row, sel_sorted_ok
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def f32(bits):
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def make(N, Hq, G, d=128, dI=64, seed=1):
+    w = synth.small_workload(N=N, Hq=Hq, G=G, d=d, dI=dI, seed=seed)
+    return w, synth.prefill_inputs_np(w)
+
+
+# ----------------------------------------------------------------------------- pooling
+def test_pool_is_block_mean_and_tail_sum():
+    rng = np.random.default_rng(0)
+    N, G, dI, Bk = 37, 3, 8, 5
+    bits = synth.f64_to_bf16_bits(rng.standard_normal((N, G, dI)))
+    pooled, tail = oracle.pool(bits, Bk)
+    ref = f32(bits)[: (N // Bk) * Bk].reshape(N // Bk, Bk, G, dI).mean(axis=1).transpose(1, 0, 2)
+    assert pooled.shape == (G, N // Bk, dI)
+    np.testing.assert_allclose(pooled, ref, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(tail, f32(bits)[(N // Bk) * Bk:].sum(axis=0), rtol=0, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- scores
+def test_block_scores_match_matmul():
+    rng = np.random.default_rng(1)
+    dI, nb = 64, 50
+    q = synth.f64_to_bf16_bits(rng.standard_normal(dI))
+    pooled = rng.standard_normal((nb, dI))
+    s = oracle.block_scores(q, pooled, 40)
+    ref = pooled[:40] @ f32(q) / np.sqrt(dI)
+    np.testing.assert_allclose(s, ref, rtol=1e-13, atol=1e-15)
+
+
+# ----------------------------------------------------------------------------- selection
+def _lexsort_select(s, c, topk):
+    if c + 1 <= topk:
+        return np.arange(c + 1)
+    order = np.lexsort((np.arange(c), -s[:c]))     # primary: -s (score desc), secondary: id
+    return np.sort(np.concatenate([order[: topk - 1], [c]]))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_select_matches_library_sort_with_ties(seed):
+    rng = np.random.default_rng(seed)
+    for c in [0, 1, 7, 14, 15, 16, 17, 40, 300]:
+        # quantised scores force many exact ties
+        s = np.round(rng.standard_normal(max(c, 1)) * 4) / 4
+        sel, n, kth = oracle.select_from_scores(s, c, 16)
+        ref = _lexsort_select(s, c, 16)
+        assert n == len(ref)
+        assert list(sel[:n]) == list(ref)
+        assert all(v == -1 for v in sel[n:])
+        assert sel_sorted_ok(sel)
+        sel2, n2 = oracle.select_fullsort(s, c, 16)
+        assert list(sel2) == list(sel)
+        if c + 1 > 16:
+            ranked = s[np.lexsort((np.arange(c), -s[:c]))]
+            assert kth == ranked[14]
+        else:
+            assert np.isnan(kth)
+
+
+def test_select_few_blocks_takes_all():
+    for c in range(16):
+        sel, n, _ = oracle.select_from_scores(np.zeros(max(c, 1)), c, 16)
+        assert n == c + 1 and list(sel[: c + 1]) == list(range(c + 1))
+
+
+def test_equal_scores_take_lowest_ids():
+    # constant k_I (all pooled keys equal) or q_I = 0: every score ties -> {0..14, c}
+    N, G, dI, Bk = 128 * 40, 1, 64, 128
+    k_idx = np.full((N, G, dI), synth.f64_to_bf16_bits(np.array([0.75]))[0], np.uint16)
+    pooled, _ = oracle.pool(k_idx, Bk)
+    rng = np.random.default_rng(3)
+    q = synth.f64_to_bf16_bits(rng.standard_normal((1, dI)))
+    t = np.array([N - 1])
+    sel, _, _ = oracle.select_rows(t, q, pooled[0], Bk, 16)
+    assert list(sel[0]) == list(range(15)) + [39]
+    zero_q = np.zeros((1, dI), np.uint16)
+    k_rand = synth.f64_to_bf16_bits(rng.standard_normal((N, G, dI)))
+    pooled2, _ = oracle.pool(k_rand, Bk)
+    sel, _, _ = oracle.select_rows(t, zero_q, pooled2[0], Bk, 16)
+    assert list(sel[0]) == list(range(15)) + [39]
+
+
+def test_planted_blocks_are_selected():
+    rng = np.random.default_rng(4)
+    N, dI, Bk = 128 * 64, 64, 128
+    k_idx = synth.f64_to_bf16_bits(rng.standard_normal((N, 1, dI)))
+    q = synth.f64_to_bf16_bits(rng.standard_normal((1, dI)))
+    planted = np.sort(rng.choice(63, 15, replace=False))
+    qv = f32(q[0])
+    for j in planted:                # add a large multiple of q_I to every key of the block
+        k_idx[j * Bk:(j + 1) * Bk, 0] = synth.f64_to_bf16_bits(f32(k_idx[j * Bk:(j + 1) * Bk, 0]) + 6 * qv)
+    pooled, _ = oracle.pool(k_idx, Bk)
+    sel, _, _ = oracle.select_rows(np.array([N - 1]), q, pooled[0], Bk, 16)
+    assert list(sel[0]) == list(planted) + [63]
+
+
+def test_near_tie_rule():
+    s = np.array([1.0, 0.5, 0.5 + 4e-6, 0.2])
+    kth = 0.5 + 4e-6
+    assert compare_selection_row([1, 3, -1], [2, 3, -1], s, kth) == (True, 2, 0)
+    assert compare_selection_row([0, 3, -1], [2, 3, -1], s, kth)[0] is False
+    assert compare_selection_row([2, 3, 3], [2, 3, -1], s, kth)[0] is False
+
+
+# ----------------------------------------------------------------------------- attention
+def _sdpa_masked(qf, kf, vf, mask):
+    """torch fp64 attention. qf [H, T, d], kf/vf [U, d], mask [T, U] bool (True = attend)."""
+    out = F.scaled_dot_product_attention(qf[None], kf[None, None].expand(1, qf.shape[0], -1, -1),
+                                         vf[None, None].expand(1, qf.shape[0], -1, -1),
+                                         attn_mask=mask[None, None])
+    return out[0]
+
+
+def test_dense_equivalence_when_all_blocks_fit():
+    # c + 1 <= 16 for every query (N <= 2048): MSA reduces to dense causal GQA attention.
+    w, x = make(N=300, Hq=4, G=2, seed=11)
+    r = oracle.prefill(x, w.Hq, w.G)
+    q = torch.from_numpy(f32(x["q"]))[0]            # [N, Hq, d]
+    k = torch.from_numpy(f32(x["k"]))[0]            # [G, N, d]
+    v = torch.from_numpy(f32(x["v"]))[0]
+    Hg = w.Hq // w.G
+    kk = k.repeat_interleave(Hg, dim=0)             # head h uses group h // Hg
+    vv = v.repeat_interleave(Hg, dim=0)
+    ref = F.scaled_dot_product_attention(q.permute(1, 0, 2)[None], kk[None], vv[None], is_causal=True)
+    ref = ref[0].permute(1, 0, 2).numpy()
+    np.testing.assert_allclose(r["out"][0], ref, rtol=0, atol=1e-12)
+    lse_ref = torch.logsumexp((q.permute(1, 0, 2) @ kk.transpose(1, 2)) / np.sqrt(128)
+                              + torch.triu(torch.full((300, 300), -np.inf, dtype=torch.float64), 1),
+                              dim=-1).permute(1, 0).numpy()
+    np.testing.assert_allclose(r["lse"][0], lse_ref, rtol=0, atol=1e-11)
+    od, _ = oracle.dense_gqa(x, w.Hq, w.G)
+    np.testing.assert_allclose(od, r["out"], rtol=0, atol=1e-13)
+
+
+def test_sparse_attention_matches_masked_sdpa():
+    # small blocks (Bk = 4, k = 4) so that selection really drops blocks
+    rng = np.random.default_rng(5)
+    N, d, Bk, topk = 70, 32, 4, 4
+    qb = synth.f64_to_bf16_bits(rng.standard_normal((N, 2, d)))
+    kb = synth.f64_to_bf16_bits(rng.standard_normal((N, d)))
+    vb = synth.f64_to_bf16_bits(rng.standard_normal((N, d)))
+    sel = np.full((N, topk), -1, np.int32)
+    for t in range(N):
+        c = t // Bk
+        cand = rng.permutation(c)[: topk - 1] if c + 1 > topk else np.arange(c)
+        ids = np.sort(np.concatenate([cand, [c]]))
+        sel[t, : len(ids)] = ids
+    o, lse, nk = oracle.attend_rows(np.arange(N), qb, kb, vb, sel, Bk, topk)
+    mask = np.zeros((N, N), bool)
+    for t in range(N):
+        for u in range(t + 1):
+            mask[t, u] = (u // Bk) in set(sel[t][sel[t] >= 0])
+    ref = _sdpa_masked(torch.from_numpy(f32(qb)).permute(1, 0, 2), torch.from_numpy(f32(kb)),
+                       torch.from_numpy(f32(vb)), torch.from_numpy(mask))
+    np.testing.assert_allclose(o, ref.permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+    assert list(nk) == list(mask.sum(1))
+
+
+def test_constant_v_gives_v():
+    w, x = make(N=2600, Hq=4, G=1, seed=12)
+    x["v"][:] = synth.f64_to_bf16_bits(np.array([-1.375]))[0]
+    t = np.array([0, 1, 127, 128, 2047, 2048, 2599])
+    pooled, _ = oracle.pool(x["k_idx"][0], 128)
+    sel, _, _ = oracle.select_rows(t, x["q_idx"][0, t, 0], pooled[0])
+    o, _, _ = oracle.attend_rows(t, x["q"][0, t], x["k"][0, 0], x["v"][0, 0], sel)
+    np.testing.assert_allclose(o, -1.375, rtol=0, atol=1e-13)
+
+
+def test_permutation_inside_selected_block_is_invariant():
+    w, x = make(N=128 * 24, Hq=4, G=1, seed=13)
+    t = np.arange(128 * 23, 128 * 24)
+    r0 = _rows(x, t)
+    # the non-diagonal block that the most queries of the last block selected
+    counts = np.bincount(r0["sel"][r0["sel"] >= 0].ravel(), minlength=24)[:23]
+    j = int(np.argmax(counts))
+    assert counts[j] > 0
+    perm = np.random.default_rng(0).permutation(128) + 128 * j
+    y = {k: v.copy() for k, v in x.items()}
+    y["k"][0, 0, 128 * j:128 * (j + 1)] = x["k"][0, 0, perm]
+    y["v"][0, 0, 128 * j:128 * (j + 1)] = x["v"][0, 0, perm]
+    y["k_idx"][0, 128 * j:128 * (j + 1)] = x["k_idx"][0, perm]
+    r1 = _rows(y, t)
+    assert (r0["sel"] == r1["sel"]).all()
+    np.testing.assert_allclose(r1["o"], r0["o"], rtol=0, atol=1e-13)
+
+
+def _rows(x, t):
+    pooled, _ = oracle.pool(x["k_idx"][0], 128)
+    sel, kth, _ = oracle.select_rows(t, x["q_idx"][0, t, 0], pooled[0])
+    o, lse, nk = oracle.attend_rows(t, x["q"][0, t], x["k"][0, 0], x["v"][0, 0], sel)
+    return {"sel": sel, "o": o, "lse": lse, "nk": nk}
+
+
+# ----------------------------------------------------------------------------- key counts
+def closed_form_total_keys(N, Bk=128, k=16):
+    """Sum over queries of attended keys: t < k*Bk attend t+1 keys; later queries at offset
+    i of their block attend (k-1)*Bk + i + 1 keys."""
+    assert N % Bk == 0 and N >= k * Bk
+    head = (k * Bk) * (k * Bk + 1) // 2
+    per_block = Bk * (k - 1) * Bk + Bk * (Bk + 1) // 2
+    return head + (N // Bk - k) * per_block
+
+
+def test_closed_form_key_counts_golden():
+    with open(os.path.join(GOLDEN, "key_counts.json")) as f:
+        gold = json.load(f)
+    for n, total in gold["totals"].items():
+        assert closed_form_total_keys(int(n)) == total
+
+
+def test_oracle_key_counts_match_closed_form():
+    w, x = make(N=4096, Hq=4, G=1, seed=14)
+    x["q"] = x["q"][:, :, :1]          # one head is enough to count keys
+    pooled, _ = oracle.pool(x["k_idx"][0], 128)
+    t = np.arange(4096)
+    sel, _, _ = oracle.select_rows(t, x["q_idx"][0, :, 0], pooled[0])
+    _, _, nk = oracle.attend_rows(t, x["q"][0], x["k"][0, 0], x["v"][0, 0], sel)
+    assert int(nk.sum()) == closed_form_total_keys(4096) == 6162432
+    for tt in [2048, 2049, 3000, 4095]:
+        assert nk[tt] == 1920 + tt % 128 + 1
