@@ -1,0 +1,261 @@
+// capi.cu -- the extern "C" boundary of libmsa: argument validation on the host, workspace
+// sizing, TMA descriptor encoding, and kernel launches on the caller's stream. Nothing here
+// allocates device memory or synchronises (except msa_get_device_status, which must).
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+
+#include "msa_common.cuh"
+
+namespace msa {
+// kernels (other translation units)
+void launch_pool(const void*, int, int, int64_t, float*, int64_t, float*, cudaStream_t);
+void launch_append(const void*, const void*, const void*, const int32_t*, int, int, void*, void*, int64_t,
+                   float*, float*, int64_t, void*, cudaStream_t);
+void launch_select_prefill_simt(const void*, int, int, int64_t, const float*, int64_t, int32_t*, cudaStream_t);
+void launch_select_decode(const void*, const int32_t*, int64_t, int, int, const float*, int64_t, int32_t*,
+                          void*, cudaStream_t);
+size_t decode_select_ws_bytes(int, int, int64_t);
+void launch_attn_decode(const CUtensorMap&, const CUtensorMap&, const void*, int64_t, const int32_t*, int64_t,
+                        const int32_t*, int, int, int, void*, float*, void*, cudaStream_t);
+size_t decode_attn_ws_bytes(int, int, int);
+void launch_attn_prefill_simt(const void*, const void*, const void*, int64_t, int, int, int, const int32_t*,
+                              void*, float*, cudaStream_t);
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace msa
+
+using namespace msa;
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+constexpr int64_t kMaxPos = (int64_t(1) << 24) - 1;   // decode select merge supports 1024 chunks
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+msa_status_t check_shape(const msa_shape_t* s) {
+    if (s == nullptr) return MSA_ERR_INVALID_ARGUMENT;
+    if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_groups < 1 || s->batch > 65535 || s->n_kv_groups > 65535)
+        return MSA_ERR_INVALID_ARGUMENT;
+    if (s->n_q_heads % s->n_kv_groups != 0) return MSA_ERR_INVALID_ARGUMENT;
+    if (s->head_dim != kHeadDim || s->index_dim != kIndexDim || s->block_size != kBlock || s->top_k != kTopK)
+        return MSA_ERR_UNSUPPORTED;
+    const int hg = s->n_q_heads / s->n_kv_groups;
+    if (!(hg == 1 || hg == 2 || hg == 4 || hg == 8 || hg == 16)) return MSA_ERR_UNSUPPORTED;
+    return MSA_OK;
+}
+
+msa_status_t cuda_status() {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        g_last_cuda_error = int(e);
+        return MSA_ERR_CUDA;
+    }
+    return MSA_OK;
+}
+
+#define MSA_TRY(x)                            \
+    do {                                      \
+        msa_status_t _s = (x);                \
+        if (_s != MSA_OK) return _s;          \
+    } while (0)
+
+#define MSA_REQ(cond, code)                   \
+    do {                                      \
+        if (!(cond)) return (code);           \
+    } while (0)
+
+size_t header_only() { return sizeof(WsHeader); }
+
+size_t ws_size(const msa_shape_t* s, int32_t op, int64_t n) {
+    if (check_shape(s) != MSA_OK || n < 0) return 0;
+    const int hg = s->n_q_heads / s->n_kv_groups;
+    switch (op) {
+        case MSA_OP_INDEX_SELECT_PREFILL: return header_only();
+        case MSA_OP_INDEX_SELECT_DECODE:
+            if (n > kMaxPos) return 0;
+            return decode_select_ws_bytes(s->batch, s->n_kv_groups, n);
+        case MSA_OP_ATTN_PREFILL: return header_only();
+        case MSA_OP_ATTN_DECODE: return decode_attn_ws_bytes(s->batch, s->n_kv_groups, hg);
+        default: return 0;
+    }
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// bf16 matrix of `rows` x `cols` (row stride = cols), box = box_cols x box_rows, 128B swizzle
+msa_status_t make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                            uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return MSA_ERR_CUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error = int(r);
+        return MSA_ERR_CUDA;
+    }
+    return MSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t msa_abi_version(void) { return 1; }
+
+const char* msa_status_string(msa_status_t s) {
+    switch (s) {
+        case MSA_OK: return "ok";
+        case MSA_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case MSA_ERR_UNSUPPORTED: return "unsupported shape or constant";
+        case MSA_ERR_WORKSPACE: return "workspace missing or too small";
+        case MSA_ERR_CUDA: return "CUDA error";
+        case MSA_ERR_TIMEOUT: return "device wait timed out";
+        case MSA_ERR_DEVICE_BOUNDS: return "device index out of bounds";
+        default: return "unknown status";
+    }
+}
+
+int32_t msa_last_cuda_error(void) { return g_last_cuda_error; }
+
+uint64_t msa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t msa_workspace_size(const msa_shape_t* shape, int32_t op, int64_t n) { return ws_size(shape, op, n); }
+
+msa_status_t msa_pool_index_keys(const msa_shape_t* shape, const void* k_idx, int64_t n_tokens, float* pooled,
+                                 int64_t nb_cap, float* tail_sum, msa_stream_t stream) {
+    MSA_TRY(check_shape(shape));
+    MSA_REQ(n_tokens >= 0 && n_tokens < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(n_tokens == 0 || (k_idx != nullptr && aligned16(k_idx)), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(nb_cap >= n_tokens / kBlock && nb_cap >= 0, MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(n_tokens < kBlock || (pooled != nullptr && aligned16(pooled)), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(tail_sum == nullptr || aligned16(tail_sum), MSA_ERR_INVALID_ARGUMENT);
+    launch_pool(k_idx, shape->batch, shape->n_kv_groups, n_tokens, pooled, nb_cap, tail_sum,
+                reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status();
+}
+
+msa_status_t msa_index_select(const msa_shape_t* shape, const void* q_idx, int64_t n_queries, const int32_t* q_pos,
+                              int64_t max_pos, const float* pooled, int64_t nb_cap, int32_t* sel, void* workspace,
+                              size_t workspace_bytes, msa_stream_t stream) {
+    MSA_TRY(check_shape(shape));
+    MSA_REQ(q_idx != nullptr && aligned16(q_idx) && sel != nullptr && aligned16(sel), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(pooled == nullptr ? max_pos < kBlock : aligned16(pooled), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(n_queries >= 1 && n_queries < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(max_pos >= 0 && nb_cap >= 0, MSA_ERR_INVALID_ARGUMENT);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int B = shape->batch, G = shape->n_kv_groups;
+    if (q_pos == nullptr) {                        // prefill: positions 0..n_queries-1
+        MSA_REQ(max_pos >= n_queries - 1, MSA_ERR_INVALID_ARGUMENT);
+        MSA_REQ(nb_cap >= (n_queries - 1) / kBlock, MSA_ERR_INVALID_ARGUMENT);
+        const size_t need = ws_size(shape, MSA_OP_INDEX_SELECT_PREFILL, n_queries);
+        MSA_REQ(workspace != nullptr && workspace_bytes >= need, MSA_ERR_WORKSPACE);
+        launch_select_prefill_simt(q_idx, B, G, n_queries, pooled, nb_cap, sel, st);
+    } else {                                       // decode: one query per sequence at q_pos[b]
+        MSA_REQ(n_queries == 1, MSA_ERR_INVALID_ARGUMENT);
+        MSA_REQ(max_pos <= kMaxPos, MSA_ERR_UNSUPPORTED);
+        MSA_REQ(nb_cap >= max_pos / kBlock, MSA_ERR_INVALID_ARGUMENT);
+        const size_t need = ws_size(shape, MSA_OP_INDEX_SELECT_DECODE, max_pos);
+        MSA_REQ(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need, MSA_ERR_WORKSPACE);
+        launch_select_decode(q_idx, q_pos, max_pos, B, G, pooled, nb_cap, sel, workspace, st);
+    }
+    return cuda_status();
+}
+
+msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const void* q, const void* k, const void* v,
+                                     int64_t n_tokens, const int32_t* sel, void* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, msa_stream_t stream) {
+    MSA_TRY(check_shape(shape));
+    MSA_REQ(n_tokens >= 1 && n_tokens < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(q && k && v && sel && out && aligned16(q) && aligned16(k) && aligned16(v) && aligned16(sel) &&
+                aligned16(out) && (lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u) == 0),
+            MSA_ERR_INVALID_ARGUMENT);
+    const size_t need = ws_size(shape, MSA_OP_ATTN_PREFILL, n_tokens);
+    MSA_REQ(workspace != nullptr && workspace_bytes >= need, MSA_ERR_WORKSPACE);
+    const int hg = shape->n_q_heads / shape->n_kv_groups;
+    launch_attn_prefill_simt(q, k, v, n_tokens, shape->batch, shape->n_kv_groups, hg, sel, out, lse,
+                             reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status();
+}
+
+msa_status_t msa_pooled_keys_append(const msa_shape_t* shape, const void* k_idx_new, const void* k_new,
+                                    const void* v_new, const int32_t* ctx_len, void* k_cache, void* v_cache,
+                                    int64_t l_cap, float* tail_sum, float* pooled, int64_t nb_cap, void* workspace,
+                                    size_t workspace_bytes, msa_stream_t stream) {
+    MSA_TRY(check_shape(shape));
+    MSA_REQ(k_idx_new && aligned16(k_idx_new) && ctx_len && tail_sum && aligned16(tail_sum) && pooled &&
+                aligned16(pooled),
+            MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ((k_new == nullptr) == (v_new == nullptr), MSA_ERR_INVALID_ARGUMENT);
+    if (k_new != nullptr)
+        MSA_REQ(aligned16(k_new) && aligned16(v_new) && k_cache && v_cache && aligned16(k_cache) &&
+                    aligned16(v_cache) && l_cap >= 1,
+                MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(nb_cap >= 1, MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(workspace != nullptr && workspace_bytes >= header_only(), MSA_ERR_WORKSPACE);
+    launch_append(k_idx_new, k_new, v_new, ctx_len, shape->batch, shape->n_kv_groups, k_cache, v_cache,
+                  k_new ? l_cap : int64_t(1) << 62, tail_sum, pooled, nb_cap, workspace,
+                  reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status();
+}
+
+msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const void* q, const void* k_cache,
+                                    const void* v_cache, int64_t l_cap, const int32_t* q_pos, int64_t max_pos,
+                                    const int32_t* sel, void* out, float* lse, void* workspace,
+                                    size_t workspace_bytes, msa_stream_t stream) {
+    MSA_TRY(check_shape(shape));
+    MSA_REQ(q && k_cache && v_cache && q_pos && sel && out && aligned16(q) && aligned16(k_cache) &&
+                aligned16(v_cache) && aligned16(sel) && aligned16(out) &&
+                (lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u) == 0),
+            MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(l_cap >= 1 && max_pos >= 0 && max_pos < l_cap, MSA_ERR_INVALID_ARGUMENT);
+    const int B = shape->batch, G = shape->n_kv_groups;
+    MSA_REQ(int64_t(B) * G * l_cap + kBlock < (int64_t(1) << 31), MSA_ERR_UNSUPPORTED);
+    const size_t need = ws_size(shape, MSA_OP_ATTN_DECODE, max_pos);
+    MSA_REQ(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need, MSA_ERR_WORKSPACE);
+    CUtensorMap tmK, tmV;
+    const uint64_t rows = uint64_t(B) * G * uint64_t(l_cap);
+    MSA_TRY(make_tmap_bf16(&tmK, k_cache, rows, kHeadDim, 64, 32));
+    MSA_TRY(make_tmap_bf16(&tmV, v_cache, rows, kHeadDim, 64, 32));
+    launch_attn_decode(tmK, tmV, q, l_cap, q_pos, max_pos, sel, B, G, shape->n_q_heads / G, out, lse, workspace,
+                       reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status();
+}
+
+msa_status_t msa_get_device_status(void* workspace, int32_t* info, msa_stream_t stream) {
+    MSA_REQ(workspace != nullptr, MSA_ERR_INVALID_ARGUMENT);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    WsHeader h;
+    if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return cuda_status();
+    if (info) std::memcpy(info, h.info, sizeof(h.info));
+    if (h.err != 0) {
+        if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+            return cuda_status();
+    }
+    return static_cast<msa_status_t>(h.err);
+}
+
+}  // extern "C"

@@ -1,0 +1,135 @@
+// pool_append.cu -- Index Branch block pooling (prefill) and the incremental pooled-key /
+// KV-cache update of a decode step.
+//
+// Pooling: a block's pooled index key is the mean of its Bk = 128 index keys (youmind
+// article "MiniMax M3 sparse attention agents", bullet "Predictable cost at every length"
+// fixes Bk; the mean is this library's reading of the unspecified block summary).
+// One CTA reads one 128-token block of all G groups: with G = 8 that is 128 contiguous
+// 1 KB rows (128 KB), loaded as 16-byte vectors, so the kernel streams k_I once at HBM speed.
+#include "msa_common.cuh"
+
+namespace msa {
+
+// grid (ceil(N / Bk), B), 256 threads.
+__global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ k_idx, int64_t n_tokens,
+                                                   int G, float* __restrict__ pooled, int64_t nb_cap,
+                                                   float* __restrict__ tail_sum) {
+    extern __shared__ float red[];                      // [nparts][G*dI]
+    const int b = blockIdx.y;
+    const int64_t blk = blockIdx.x;
+    const int ncol = G * kIndexDim;                     // bf16 values per token row
+    const int nchunk = ncol / 8;                        // 16-byte chunks per row
+    const int nparts = nchunk >= 256 ? 1 : 256 / nchunk;
+    const int64_t t0 = blk * kBlock;
+    const int ntok = int((n_tokens - t0 < kBlock ? n_tokens - t0 : int64_t(kBlock)));
+    const uint4* base = reinterpret_cast<const uint4*>(k_idx + (size_t(b) * n_tokens + t0) * ncol);
+
+    for (int c0 = 0; c0 < nchunk; c0 += 256 / nparts) {
+        const int chunk = c0 + (threadIdx.x % (256 / nparts));
+        const int part = threadIdx.x / (256 / nparts);
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (chunk < nchunk && part < nparts) {
+#pragma unroll 4
+            for (int t = part; t < ntok; t += nparts) {
+                uint4 v = __ldg(base + size_t(t) * nchunk + chunk);
+                acc[0] += bf16_lo(v.x); acc[1] += bf16_hi(v.x);
+                acc[2] += bf16_lo(v.y); acc[3] += bf16_hi(v.y);
+                acc[4] += bf16_lo(v.z); acc[5] += bf16_hi(v.z);
+                acc[6] += bf16_lo(v.w); acc[7] += bf16_hi(v.w);
+            }
+            float* r = red + (size_t(part) * nchunk + chunk) * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) r[e] = acc[e];
+        }
+    }
+    __syncthreads();
+    const bool full = ntok == kBlock;
+    for (int col = threadIdx.x; col < ncol; col += 256) {
+        float s = 0.f;
+        for (int p = 0; p < nparts; ++p) s += red[size_t(p) * ncol + col];
+        const int g = col / kIndexDim, i = col % kIndexDim;
+        if (full) {
+            pooled[((size_t(b) * G + g) * nb_cap + blk) * kIndexDim + i] = s * (1.0f / kBlock);
+        } else if (tail_sum) {
+            tail_sum[(size_t(b) * G + g) * kIndexDim + i] = s;
+        }
+    }
+}
+
+__global__ void zero_kernel(float* p, int64_t n) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
+        p[i] = 0.f;
+}
+
+void launch_pool(const void* k_idx, int B, int G, int64_t n_tokens, float* pooled, int64_t nb_cap,
+                 float* tail_sum, cudaStream_t st) {
+    if (tail_sum && n_tokens % kBlock == 0) {
+        int64_t n = int64_t(B) * G * kIndexDim;
+        count_launch();
+        zero_kernel<<<int((n + 255) / 256), 256, 0, st>>>(tail_sum, n);
+    }
+    if (n_tokens == 0) return;
+    const int nchunk = G * kIndexDim / 8;
+    const int nparts = nchunk >= 256 ? 1 : 256 / nchunk;
+    size_t smem = size_t(nparts) * G * kIndexDim * sizeof(float);
+    if (smem > 48 * 1024) cudaFuncSetAttribute(pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    dim3 grid(unsigned((n_tokens + kBlock - 1) / kBlock), unsigned(B));
+    count_launch();
+    pool_kernel<<<grid, 256, smem, st>>>(static_cast<const uint16_t*>(k_idx), n_tokens, G, pooled,
+                                          nb_cap, tail_sum);
+}
+
+// ---------------------------------------------------------------- decode append
+// grid B, block 256. Writes the new token's K/V rows into the caches at position L_b and
+// folds its index keys into the open block's running sum; closes the block into `pooled`
+// when it becomes full.
+__global__ void __launch_bounds__(256) append_kernel(const uint16_t* __restrict__ k_idx_new,
+                                                     const uint16_t* __restrict__ k_new,
+                                                     const uint16_t* __restrict__ v_new,
+                                                     const int32_t* __restrict__ ctx_len, int G,
+                                                     uint16_t* __restrict__ k_cache,
+                                                     uint16_t* __restrict__ v_cache, int64_t l_cap,
+                                                     float* __restrict__ tail_sum,
+                                                     float* __restrict__ pooled, int64_t nb_cap,
+                                                     WsHeader* hdr) {
+    const int b = blockIdx.x;
+    const int pos = ctx_len[b];
+    const int64_t j = pos / kBlock;
+    const bool close = ((pos + 1) % kBlock) == 0;
+    if (pos < 0 || pos >= l_cap || (close && j >= nb_cap)) {
+        if (threadIdx.x == 0) record_error(hdr, MSA_ERR_DEVICE_BOUNDS, KID_APPEND, b, 0, pos);
+        return;
+    }
+    if (k_new != nullptr) {
+        const int nvec = G * kHeadDim / 8;                 // 16-byte vectors per token
+        for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+            const int g = i / (kHeadDim / 8), c = i % (kHeadDim / 8);
+            const size_t src = (size_t(b) * G + g) * (kHeadDim / 8) + c;
+            const size_t dst = ((size_t(b) * G + g) * l_cap + pos) * (kHeadDim / 8) + c;
+            reinterpret_cast<uint4*>(k_cache)[dst] = reinterpret_cast<const uint4*>(k_new)[src];
+            reinterpret_cast<uint4*>(v_cache)[dst] = reinterpret_cast<const uint4*>(v_new)[src];
+        }
+    }
+    const bool fresh = (pos % kBlock) == 0;
+    for (int i = threadIdx.x; i < G * kIndexDim; i += blockDim.x) {
+        const int g = i / kIndexDim, e = i % kIndexDim;
+        const size_t o = (size_t(b) * G + g) * kIndexDim + e;
+        const float x = bf16_to_f32(k_idx_new[o]);
+        const float s = fresh ? x : tail_sum[o] + x;
+        tail_sum[o] = s;
+        if (close) pooled[((size_t(b) * G + g) * nb_cap + j) * kIndexDim + e] = s * (1.0f / kBlock);
+    }
+}
+
+void launch_append(const void* k_idx_new, const void* k_new, const void* v_new, const int32_t* ctx_len,
+                   int B, int G, void* k_cache, void* v_cache, int64_t l_cap, float* tail_sum,
+                   float* pooled, int64_t nb_cap, void* ws, cudaStream_t st) {
+    count_launch();
+    append_kernel<<<B, 256, 0, st>>>(static_cast<const uint16_t*>(k_idx_new),
+                                     static_cast<const uint16_t*>(k_new),
+                                     static_cast<const uint16_t*>(v_new), ctx_len, G,
+                                     static_cast<uint16_t*>(k_cache), static_cast<uint16_t*>(v_cache),
+                                     l_cap, tail_sum, pooled, nb_cap, static_cast<WsHeader*>(ws));
+}
+
+}  // namespace msa

@@ -1,0 +1,257 @@
+// select.cu -- Index Branch scoring and exp-free top-k block selection.
+//
+// Sources: youmind article "MiniMax M3 sparse attention agents", paragraph "The mechanism
+// that changes this" (score the context in blocks, keep the most relevant per query and
+// GQA group) and bullet "Predictable cost at every length" (k = 16); KuCoin flash "MiniMax
+// launches MSA sparse attention method and MiniMax-M3 model", summary (exp-free top-k).
+//
+// Every score is s_j = q_I . kbar_j in fp32 (the 1/sqrt(d_I) factor is an exact power of two
+// and cannot change the order, so it is not applied). Ranking uses only compares: the
+// running top-15 keeps the earlier (lower) block on equal scores, which is the order
+// (score desc, id asc). The query's own block is added and the ids are written ascending.
+#include "msa_common.cuh"
+
+namespace msa {
+
+constexpr int kKeep = kTopK - 1;   // best fully-past blocks kept besides the diagonal one
+
+// Sort 16 ids ascending in registers (odd-even transposition network).
+__device__ __forceinline__ void sort16(int (&x)[16]) {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+#pragma unroll
+        for (int i = (r & 1); i + 1 < 16; i += 2) {
+            const int a = min(x[i], x[i + 1]), bb = max(x[i], x[i + 1]);
+            x[i] = a; x[i + 1] = bb;
+        }
+    }
+}
+
+__device__ __forceinline__ void write_all_blocks(int32_t* out, int c) {
+    int4* o = reinterpret_cast<int4*>(out);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        int4 v;
+        v.x = (4 * q + 0 <= c) ? 4 * q + 0 : -1;
+        v.y = (4 * q + 1 <= c) ? 4 * q + 1 : -1;
+        v.z = (4 * q + 2 <= c) ? 4 * q + 2 : -1;
+        v.w = (4 * q + 3 <= c) ? 4 * q + 3 : -1;
+        o[q] = v;
+    }
+}
+
+// ------------------------------------------------------------------ prefill, CUDA cores
+// grid (ceil(N / 128), G, B), 128 threads: thread i owns query t = 128 * blockIdx.x + i.
+// All queries of one 128-token block share the candidate set [0, c), c = blockIdx.x, so the
+// CTA stages the pooled keys through shared memory 64 candidates at a time.
+__global__ void __launch_bounds__(128) select_prefill_simt_kernel(const uint16_t* __restrict__ q_idx,
+                                                                  int64_t N, int G,
+                                                                  const float* __restrict__ pooled,
+                                                                  int64_t nb_cap, int32_t* __restrict__ sel) {
+    __shared__ __align__(16) float kb[64][kIndexDim];
+    const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int64_t t = int64_t(c) * kBlock + threadIdx.x;
+    const bool live = t < N;
+    int32_t* out = sel + ((size_t(b) * N + t) * G + g) * kTopK;
+    if (c + 1 <= kTopK) {
+        if (live) write_all_blocks(out, c);
+        return;
+    }
+    float q[kIndexDim];
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(q_idx + ((size_t(b) * N + (live ? t : 0)) * G + g) * kIndexDim);
+#pragma unroll
+        for (int v = 0; v < kIndexDim / 8; ++v) {
+            uint4 w = __ldg(src + v);
+            q[8 * v + 0] = bf16_lo(w.x); q[8 * v + 1] = bf16_hi(w.x);
+            q[8 * v + 2] = bf16_lo(w.y); q[8 * v + 3] = bf16_hi(w.y);
+            q[8 * v + 4] = bf16_lo(w.z); q[8 * v + 5] = bf16_hi(w.z);
+            q[8 * v + 6] = bf16_lo(w.w); q[8 * v + 7] = bf16_hi(w.w);
+        }
+    }
+    float best[kKeep];
+    int bid[kKeep];
+#pragma unroll
+    for (int k = 0; k < kKeep; ++k) { best[k] = -INFINITY; bid[k] = 0x7fffffff; }
+
+    const float4* pk = reinterpret_cast<const float4*>(pooled + (size_t(b) * G + g) * nb_cap * kIndexDim);
+    for (int j0 = 0; j0 < c; j0 += 64) {
+        const int nj = min(64, c - j0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < nj * (kIndexDim / 4); i += blockDim.x)
+            reinterpret_cast<float4*>(&kb[0][0])[i] = __ldg(pk + size_t(j0) * (kIndexDim / 4) + i);
+        __syncthreads();
+        for (int jj = 0; jj < nj; ++jj) {
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < kIndexDim; i += 4) {
+                const float4 kv = *reinterpret_cast<const float4*>(&kb[jj][i]);
+                acc = fmaf(q[i + 0], kv.x, acc);
+                acc = fmaf(q[i + 1], kv.y, acc);
+                acc = fmaf(q[i + 2], kv.z, acc);
+                acc = fmaf(q[i + 3], kv.w, acc);
+            }
+            if (acc > best[kKeep - 1]) {
+                best[kKeep - 1] = acc; bid[kKeep - 1] = j0 + jj;
+#pragma unroll
+                for (int k = kKeep - 1; k > 0; --k) {
+                    if (best[k] > best[k - 1]) {
+                        float tv = best[k]; best[k] = best[k - 1]; best[k - 1] = tv;
+                        int ti = bid[k]; bid[k] = bid[k - 1]; bid[k - 1] = ti;
+                    }
+                }
+            }
+        }
+    }
+    if (!live) return;
+    int ids[16];
+#pragma unroll
+    for (int k = 0; k < kKeep; ++k) ids[k] = bid[k];
+    ids[15] = c;
+    sort16(ids);
+    int4* o = reinterpret_cast<int4*>(out);
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) o[q4] = make_int4(ids[4 * q4], ids[4 * q4 + 1], ids[4 * q4 + 2], ids[4 * q4 + 3]);
+}
+
+void launch_select_prefill_simt(const void* q_idx, int B, int G, int64_t N, const float* pooled,
+                                int64_t nb_cap, int32_t* sel, cudaStream_t st) {
+    dim3 grid(static_cast<unsigned>((N + kBlock - 1) / kBlock), static_cast<unsigned>(G), static_cast<unsigned>(B));
+    count_launch();
+    select_prefill_simt_kernel<<<grid, 128, 0, st>>>(static_cast<const uint16_t*>(q_idx), N, G, pooled,
+                                                      nb_cap, sel);
+}
+
+// ------------------------------------------------------------------ decode, split + merge
+// One query per (sequence, group); its candidates [0, c) are split into chunks of 128 over
+// CTAs so that the pooled keys (256 B per candidate) stream from HBM on many SMs at once.
+// Each CTA ranks its 128 candidates and leaves its best 15 keys, sorted, in the workspace;
+// the CTA that arrives last for a (sequence, group) merges the sorted lists. The arrival
+// counter wraps to zero by itself (atomicInc), so the workspace is ready for the next call.
+constexpr int kDecChunk = 128;
+
+__global__ void __launch_bounds__(kDecChunk) select_decode_kernel(
+    const uint16_t* __restrict__ q_idx, const int32_t* __restrict__ q_pos, int64_t max_pos, int G,
+    const float* __restrict__ pooled, int64_t nb_cap, int32_t* __restrict__ sel,
+    unsigned long long* __restrict__ cand, unsigned int* __restrict__ ctr, int nchunk_max, WsHeader* hdr) {
+    __shared__ float qs[kIndexDim];
+    __shared__ unsigned long long keys[kDecChunk];
+    __shared__ int heads[1024];
+    __shared__ int last;
+    const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int bg = b * G + g;
+    const int pos = q_pos[b];
+    if (pos < 0 || pos > max_pos || int64_t(pos / kBlock) > nb_cap) {
+        if (ch == 0 && threadIdx.x == 0) record_error(hdr, MSA_ERR_DEVICE_BOUNDS, KID_SELECT_DECODE, bg, 0, pos);
+        return;
+    }
+    const int c = pos / kBlock;
+    int32_t* out = sel + size_t(bg) * kTopK;
+    if (c + 1 <= kTopK) {
+        if (ch == 0 && threadIdx.x == 0) write_all_blocks(out, c);
+        return;
+    }
+    const int nch = (c + kDecChunk - 1) / kDecChunk;
+    if (ch >= nch) return;
+
+    if (threadIdx.x < kIndexDim) qs[threadIdx.x] = bf16_to_f32(q_idx[size_t(bg) * kIndexDim + threadIdx.x]);
+    __syncthreads();
+    const int j = ch * kDecChunk + threadIdx.x;
+    unsigned long long key = 0ull;
+    if (j < c) {
+        const float4* row = reinterpret_cast<const float4*>(pooled + (size_t(bg) * nb_cap + j) * kIndexDim);
+        float4 v[kIndexDim / 4];
+#pragma unroll
+        for (int i = 0; i < kIndexDim / 4; ++i) v[i] = __ldg(row + i);
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < kIndexDim / 4; ++i) {
+            acc = fmaf(qs[4 * i + 0], v[i].x, acc);
+            acc = fmaf(qs[4 * i + 1], v[i].y, acc);
+            acc = fmaf(qs[4 * i + 2], v[i].z, acc);
+            acc = fmaf(qs[4 * i + 3], v[i].w, acc);
+        }
+        key = sel_key(acc, j);
+    }
+    keys[threadIdx.x] = key;
+    __syncthreads();
+    unsigned long long* mine = cand + (size_t(bg) * nchunk_max + ch) * kKeep;
+    if (key != 0ull) {
+        int rank = 0;
+        for (int i = 0; i < kDecChunk; ++i) rank += keys[i] > key;
+        if (rank < kKeep) mine[rank] = key;
+    }
+    const int nvalid = min(kKeep, c - ch * kDecChunk);
+    if (threadIdx.x >= nvalid && threadIdx.x < kKeep) mine[threadIdx.x] = 0ull;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = (atomicInc(ctr + bg, unsigned(nch - 1)) == unsigned(nch - 1));
+    __syncthreads();
+    if (!last || threadIdx.x >= 32) return;
+    __threadfence();
+
+    // warp 0 merges the nch sorted lists: 15 rounds of "best list head"
+    const int lane = threadIdx.x;
+    const unsigned long long* lists = cand + size_t(bg) * nchunk_max * kKeep;
+    for (int l = lane; l < nch; l += 32) heads[l] = 0;
+    __syncwarp();
+    int my_id = c;                                   // lane 15 keeps the diagonal block
+    for (int r = 0; r < kKeep; ++r) {
+        unsigned long long bk = 0ull;
+        int bl = -1;
+        for (int l = lane; l < nch; l += 32) {
+            const int h = heads[l];
+            if (h < kKeep) {
+                const unsigned long long k = __ldcg(lists + size_t(l) * kKeep + h);
+                if (k > bk) { bk = k; bl = l; }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const unsigned long long ok = __shfl_xor_sync(0xffffffffu, bk, off);
+            const int ol = __shfl_xor_sync(0xffffffffu, bl, off);
+            if (ok > bk) { bk = ok; bl = ol; }
+        }
+        if (lane == r) my_id = key_block(bk);
+        if (lane == 0 && bl >= 0) heads[bl] += 1;
+        __syncwarp();
+    }
+    // ascending order of the 16 ids held by lanes 0..15
+    int rank = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int o = __shfl_sync(0xffffffffu, my_id, i);
+        rank += (o < my_id);
+    }
+    if (lane < 16) out[rank] = my_id;
+}
+
+int decode_select_chunks(int64_t max_pos) {
+    const int64_t cmax = max_pos / kBlock;
+    return int(cmax <= 0 ? 1 : (cmax + kDecChunk - 1) / kDecChunk);
+}
+
+size_t decode_select_ws_bytes(int B, int G, int64_t max_pos) {
+    const size_t nbg = size_t(B) * G;
+    size_t bytes = sizeof(WsHeader);
+    bytes += (nbg * sizeof(unsigned int) + 255) / 256 * 256;
+    bytes += nbg * decode_select_chunks(max_pos) * kKeep * sizeof(unsigned long long);
+    return bytes;
+}
+
+void launch_select_decode(const void* q_idx, const int32_t* q_pos, int64_t max_pos, int B, int G,
+                          const float* pooled, int64_t nb_cap, int32_t* sel, void* ws, cudaStream_t st) {
+    const size_t nbg = size_t(B) * G;
+    char* p = static_cast<char*>(ws);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(p);
+    unsigned int* ctr = reinterpret_cast<unsigned int*>(p + sizeof(WsHeader));
+    unsigned long long* cand = reinterpret_cast<unsigned long long*>(
+        p + sizeof(WsHeader) + (nbg * sizeof(unsigned int) + 255) / 256 * 256);
+    const int nchunk = decode_select_chunks(max_pos);
+    dim3 grid(static_cast<unsigned>(nchunk), static_cast<unsigned>(G), static_cast<unsigned>(B));
+    count_launch();
+    select_decode_kernel<<<grid, kDecChunk, 0, st>>>(static_cast<const uint16_t*>(q_idx), q_pos, max_pos,
+                                                     G, pooled, nb_cap, sel, cand, ctr, nchunk, hdr);
+}
+
+}  // namespace msa

@@ -1,0 +1,201 @@
+/*
+ * msa.h -- C ABI of libmsa: MiniMax Sparse Attention (MSA) over grouped query attention,
+ * the data-parallel hot path, for NVIDIA B200 (sm_100a).
+ *
+ * The method (sources, by page title and section):
+ *  - youmind article "MiniMax M3 sparse attention agents", paragraph "The mechanism that
+ *    changes this" and figure 1 caption: before attention a light Index Branch scores the
+ *    key-value context in blocks and keeps the top-k blocks per query and GQA group; the
+ *    main branch attends only to those blocks.
+ *  - same article, bullet "Predictable cost at every length": Bk = 128 tokens per block and
+ *    k = 16 blocks, a fixed budget of 2,048 key-value tokens per query and GQA group.
+ *  - same article, paragraph "Why this comes now": the kernels split the context into blocks
+ *    and read each block once with contiguous memory access.
+ *  - KuCoin flash "MiniMax launches MSA sparse attention method and MiniMax-M3 model",
+ *    summary: MSA is built on GQA; the index branch picks 16 blocks of (default) 128 tokens
+ *    per GQA group, the main branch runs exact softmax attention over those blocks, and the
+ *    top-k selection is exp-free.
+ *
+ * The pages do not give the scoring function. This library computes:
+ *   pooled key of full block j:   kbar_j = mean of the Bk index keys k_I of block j (fp32)
+ *   score of fully-past block j:  s_j = q_I . kbar_j / sqrt(d_I), for j < c = floor(t / Bk)
+ *   selection for the query at t: {c} plus the k-1 best j < c, ordered by (s desc, j asc);
+ *                                 every block 0..c when c + 1 <= k
+ *   output of query head h:       softmax(q_h . k_u / sqrt(d)) weighted sum of v_u over the
+ *                                 keys u <= t of the selected blocks; all heads of a group
+ *                                 share the group's selection; head h is in group h/(Hq/G).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library allocates
+ *    nothing. Tensors are dense row-major with the shapes stated below (innermost last).
+ *    bf16 tensors are passed as void*; 16-byte alignment is required for every pointer.
+ *  - Every call validates its arguments on the host first and returns an error without
+ *    launching anything when they are wrong; otherwise it only enqueues work on `stream`
+ *    (asynchronous, no synchronisation, safe to capture in a CUDA graph).
+ *  - MSA_ERR_CUDA reports a launch error (the CUDA error is kept for msa_last_cuda_error).
+ *  - Problems only the device can see (a selection id out of range, a position beyond the
+ *    cache) are recorded in the workspace's error word and read by msa_get_device_status.
+ *  - Workspaces are device buffers of msa_workspace_size() bytes that must be zero-filled
+ *    before their first use; the library leaves them ready for the next call. Calls that
+ *    share a workspace must be ordered on one stream.
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (NULL = the legacy default stream). */
+typedef struct CUstream_st *msa_stream_t;
+
+typedef enum {
+    MSA_OK = 0,
+    MSA_ERR_INVALID_ARGUMENT = 1, /* null/misaligned pointer, bad size or shape */
+    MSA_ERR_UNSUPPORTED = 2,      /* constants other than d=128, d_I=64, Bk=128, k=16, or Hq/G not in {1,2,4,8,16} */
+    MSA_ERR_WORKSPACE = 3,        /* workspace missing or smaller than msa_workspace_size() */
+    MSA_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed */
+    MSA_ERR_TIMEOUT = 5,          /* (device) a bounded wait expired */
+    MSA_ERR_DEVICE_BOUNDS = 6     /* (device) an index or position was out of range */
+} msa_status_t;
+
+typedef struct {
+    int32_t batch;       /* B: sequences */
+    int32_t n_q_heads;   /* Hq: query heads */
+    int32_t n_kv_groups; /* G: key-value heads (GQA groups); Hq % G == 0 */
+    int32_t head_dim;    /* d: must be 128 */
+    int32_t index_dim;   /* d_I: index-branch dimension per group, must be 64 */
+    int32_t block_size;  /* Bk: must be 128 */
+    int32_t top_k;       /* k: blocks per query and group, must be 16 */
+} msa_shape_t;
+
+/* Operation ids for msa_workspace_size. */
+enum {
+    MSA_OP_INDEX_SELECT_PREFILL = 0,
+    MSA_OP_INDEX_SELECT_DECODE = 1,
+    MSA_OP_ATTN_PREFILL = 2,
+    MSA_OP_ATTN_DECODE = 3
+};
+
+/* Version of this ABI (bumped on any incompatible change). */
+int32_t msa_abi_version(void);
+
+const char *msa_status_string(msa_status_t status);
+
+/* The CUDA error code behind the last MSA_ERR_CUDA returned on this host thread. */
+int32_t msa_last_cuda_error(void);
+
+/* Number of kernels this library has enqueued in this process (all threads), for launch
+ * accounting in benchmarks. Kernels enqueued while a stream is being captured are counted
+ * once, at capture; graph replays are not counted. */
+uint64_t msa_kernel_launches(void);
+
+/*
+ * Workspace bytes needed by one operation.
+ *  op = MSA_OP_INDEX_SELECT_PREFILL: n = number of query tokens per sequence
+ *  op = MSA_OP_INDEX_SELECT_DECODE:  n = max_pos (largest query position)
+ *  op = MSA_OP_ATTN_PREFILL:         n = number of tokens per sequence
+ *  op = MSA_OP_ATTN_DECODE:          n = max_pos
+ * Returns 0 for an invalid shape or op.
+ */
+size_t msa_workspace_size(const msa_shape_t *shape, int32_t op, int64_t n);
+
+/*
+ * Index Branch, step 1 -- block pooling (sources: youmind article, figure 1 caption and
+ * bullet "Predictable cost at every length"; the mean is this library's reading).
+ *   k_idx    bf16 [B, n_tokens, G, d_I]   index keys
+ *   pooled   fp32 [B, G, nb_cap, d_I]     out: pooled[b,g,j] = mean of k_idx[b, j*Bk:(j+1)*Bk, g]
+ *                                         for every full block j < n_tokens / Bk (must be <= nb_cap);
+ *                                         other rows are not touched
+ *   tail_sum fp32 [B, G, d_I] or NULL     out: plain sum of the index keys of the trailing
+ *                                         partial block (zeros when n_tokens % Bk == 0); this is
+ *                                         the running sum msa_pooled_keys_append continues
+ */
+msa_status_t msa_pool_index_keys(const msa_shape_t *shape, const void *k_idx, int64_t n_tokens,
+                                 float *pooled, int64_t nb_cap, float *tail_sum,
+                                 msa_stream_t stream);
+
+/*
+ * Index Branch, steps 2-3 -- block scores and exp-free top-k selection (sources: youmind
+ * article, paragraph "The mechanism that changes this"; KuCoin MSA launch flash, summary).
+ *   q_idx   bf16 [B, n_queries, G, d_I]   index queries
+ *   q_pos   NULL for prefill: query i of every sequence sits at position i;
+ *           else device int32 [B] for decode: the single query (n_queries must be 1) of
+ *           sequence b sits at position q_pos[b] (the position of the new token)
+ *   max_pos host bound on every query position (prefill: n_queries - 1); sizes the grid;
+ *           a q_pos above it is a device bounds error
+ *   pooled  fp32 [B, G, nb_cap, d_I]      pooled keys; rows j < floor(pos / Bk) are read
+ *   sel     int32 [B, n_queries, G, k]    out: selected block ids in ascending order, padded
+ *                                         with -1 (the query's own block is always included)
+ *   workspace of msa_workspace_size(op = MSA_OP_INDEX_SELECT_PREFILL or _DECODE)
+ */
+msa_status_t msa_index_select(const msa_shape_t *shape, const void *q_idx, int64_t n_queries,
+                              const int32_t *q_pos, int64_t max_pos, const float *pooled,
+                              int64_t nb_cap, int32_t *sel, void *workspace,
+                              size_t workspace_bytes, msa_stream_t stream);
+
+/*
+ * Main Branch, prefill -- exact softmax attention over the selected blocks, causal inside
+ * the query's own block (sources: youmind article, figure 1 caption; KuCoin MSA launch
+ * flash, summary: exact softmax attention only over the selected blocks).
+ *   q    bf16 [B, N, Hq, d]     k, v bf16 [B, G, N, d]  (a block of one group is contiguous)
+ *   sel  int32 [B, N, G, k]     from msa_index_select (prefill)
+ *   out  bf16 [B, N, Hq, d]     out
+ *   lse  fp32 [B, N, Hq] or NULL  out: natural log of the softmax denominator of the scaled
+ *                                 scores q.k/sqrt(d)
+ *   workspace of msa_workspace_size(MSA_OP_ATTN_PREFILL, N)
+ */
+msa_status_t msa_sparse_attn_prefill(const msa_shape_t *shape, const void *q, const void *k,
+                                     const void *v, int64_t n_tokens, const int32_t *sel,
+                                     void *out, float *lse, void *workspace,
+                                     size_t workspace_bytes, msa_stream_t stream);
+
+/*
+ * Decode: append the new token to the caches and keep the pooled keys current (the pages
+ * fix only the block size; the incremental update is this library's reading of it).
+ *   ctx_len   device int32 [B]: tokens already cached (L_b); the new token goes to position L_b
+ *   k_idx_new bf16 [B, G, d_I]  the new token's index keys
+ *   k_new, v_new bf16 [B, G, d] or both NULL  -> written to k_cache/v_cache [B, G, l_cap, d]
+ *   tail_sum  fp32 [B, G, d_I]  running sum of the open block: set to k_idx_new when L_b is a
+ *                               multiple of Bk, else incremented by it
+ *   pooled    fp32 [B, G, nb_cap, d_I]: when L_b + 1 completes block j = L_b / Bk,
+ *                               pooled[b,g,j] = tail_sum / Bk
+ */
+msa_status_t msa_pooled_keys_append(const msa_shape_t *shape, const void *k_idx_new,
+                                    const void *k_new, const void *v_new, const int32_t *ctx_len,
+                                    void *k_cache, void *v_cache, int64_t l_cap, float *tail_sum,
+                                    float *pooled, int64_t nb_cap, void *workspace,
+                                    size_t workspace_bytes, msa_stream_t stream);
+
+/*
+ * Main Branch, decode -- one query token per sequence, split over the selected blocks and
+ * merged by log-sum-exp (sources as msa_sparse_attn_prefill).
+ *   q        bf16 [B, Hq, d]
+ *   k_cache, v_cache bf16 [B, G, l_cap, d]; positions 0..q_pos[b] must be filled
+ *   q_pos    device int32 [B]: the query's position (= L_b, after msa_pooled_keys_append)
+ *   max_pos  host bound on q_pos; q_pos[b] must be < l_cap
+ *   sel      int32 [B, G, k]  from msa_index_select (decode)
+ *   out      bf16 [B, Hq, d]  out;   lse fp32 [B, Hq] or NULL
+ *   workspace of msa_workspace_size(MSA_OP_ATTN_DECODE, max_pos)
+ */
+msa_status_t msa_sparse_attn_decode(const msa_shape_t *shape, const void *q, const void *k_cache,
+                                    const void *v_cache, int64_t l_cap, const int32_t *q_pos,
+                                    int64_t max_pos, const int32_t *sel, void *out, float *lse,
+                                    void *workspace, size_t workspace_bytes,
+                                    msa_stream_t stream);
+
+/*
+ * Synchronises `stream`, returns the status recorded in the workspace's error word by the
+ * device (MSA_OK, MSA_ERR_DEVICE_BOUNDS or MSA_ERR_TIMEOUT) and clears it. `info` (nullable,
+ * 4 int32) receives the recorded detail: kernel id, block, index, value.
+ */
+msa_status_t msa_get_device_status(void *workspace, int32_t *info, msa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H */

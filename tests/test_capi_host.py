@@ -1,0 +1,103 @@
+"""The C ABI without a GPU: the library loads, exports what include/msa.h declares, sizes
+workspaces, and rejects bad arguments on the host before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_gqa_branch_b200 as msa
+from block_sparse_gqa_branch_b200 import Shape
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msa.h")
+
+FAKE = 0x10000          # an aligned, never dereferenced address: validation fails before use
+FAKE2 = 0x20000
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_sparse_gqa_branch_b200 import build
+    build.build()
+    return msa.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(msa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(names) == sorted(msa.EXPORTED_SYMBOLS)
+
+
+def test_version_and_status_strings(L):
+    assert msa.msa_abi_version() == 1
+    for code in range(7):
+        assert msa.msa_status_string(code) not in ("", "unknown status")
+    assert msa.msa_status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(L):
+    s = Shape.make(16, 64, 8)
+    assert msa.msa_workspace_size(s, msa.OP_ATTN_DECODE, 131072) >= 256 + 16 * 8 * 16 * 8 * 130 * 4
+    assert msa.msa_workspace_size(s, msa.OP_INDEX_SELECT_DECODE, 131072) > 256
+    assert msa.msa_workspace_size(s, msa.OP_INDEX_SELECT_PREFILL, 4096) >= 256
+    assert msa.msa_workspace_size(s, 17, 10) == 0
+    assert msa.msa_workspace_size(Shape.make(1, 6, 4), msa.OP_ATTN_DECODE, 10) == 0      # Hq % G
+    assert msa.msa_workspace_size(Shape.make(1, 24, 1), msa.OP_ATTN_DECODE, 10) == 0     # Hg = 24
+    assert msa.msa_workspace_size(Shape.make(1, 8, 1, head_dim=64), msa.OP_ATTN_DECODE, 10) == 0
+    assert msa.msa_workspace_size(s, msa.OP_INDEX_SELECT_DECODE, 1 << 25) == 0          # beyond max
+
+
+def _shape(**kw):
+    base = dict(batch=1, n_q_heads=8, n_kv_groups=1)
+    base.update(kw)
+    return Shape.make(**base)
+
+
+def test_validation_errors_before_launch(L):
+    s = _shape()
+    bs = ctypes.byref(s)
+    # null / misaligned pointers
+    assert L.msa_pool_index_keys(bs, None, 256, FAKE, 2, None, None) == 1
+    assert L.msa_pool_index_keys(bs, FAKE + 2, 256, FAKE, 2, None, None) == 1
+    assert L.msa_pool_index_keys(bs, FAKE, 256, FAKE, 1, None, None) == 1            # nb_cap too small
+    assert L.msa_pool_index_keys(None, FAKE, 256, FAKE, 2, None, None) == 1
+    # unsupported constants
+    for bad in (dict(head_dim=64), dict(index_dim=32), dict(block_size=64), dict(top_k=8)):
+        assert L.msa_pool_index_keys(ctypes.byref(_shape(**bad)), FAKE, 256, FAKE, 2, None, None) == 2
+    assert L.msa_pool_index_keys(ctypes.byref(_shape(n_q_heads=12, n_kv_groups=1)), FAKE, 256, FAKE, 2, None, None) == 2
+    assert L.msa_pool_index_keys(ctypes.byref(_shape(n_q_heads=12, n_kv_groups=8)), FAKE, 256, FAKE, 2, None, None) == 1
+    # select: workspace missing / too small; decode with n_queries != 1
+    assert L.msa_index_select(bs, FAKE, 4096, None, 4095, FAKE, 32, FAKE2, None, 0, None) == 3
+    assert L.msa_index_select(bs, FAKE, 4096, None, 4095, FAKE, 32, FAKE2, FAKE, 16, None) == 3
+    assert L.msa_index_select(bs, FAKE, 2, FAKE, 4095, FAKE, 32, FAKE2, FAKE, 1 << 20, None) == 1
+    assert L.msa_index_select(bs, FAKE, 1, FAKE, 1 << 26, FAKE, 1 << 20, FAKE2, FAKE, 1 << 30, None) == 2
+    need = msa.msa_workspace_size(s, msa.OP_INDEX_SELECT_DECODE, 4095)
+    assert L.msa_index_select(bs, FAKE, 1, FAKE, 4095, FAKE, 32, FAKE2, FAKE, need - 16, None) == 3
+    assert L.msa_index_select(bs, FAKE, 1, FAKE, 4095, FAKE, 30, FAKE2, FAKE, need, None) == 1   # nb_cap
+    # prefill attention
+    assert L.msa_sparse_attn_prefill(bs, FAKE, FAKE, None, 100, FAKE, FAKE, None, FAKE, 1 << 20, None) == 1
+    assert L.msa_sparse_attn_prefill(bs, FAKE, FAKE, FAKE, 0, FAKE, FAKE, None, FAKE, 1 << 20, None) == 1
+    assert L.msa_sparse_attn_prefill(bs, FAKE, FAKE, FAKE, 100, FAKE, FAKE, FAKE + 2, FAKE, 1 << 20, None) == 1
+    assert L.msa_sparse_attn_prefill(bs, FAKE, FAKE, FAKE, 100, FAKE, FAKE, None, None, 0, None) == 3
+    # decode attention: position bound beyond the cache, workspace
+    assert L.msa_sparse_attn_decode(bs, FAKE, FAKE, FAKE, 1000, FAKE, 1000, FAKE, FAKE, None, FAKE, 1 << 20, None) == 1
+    assert L.msa_sparse_attn_decode(bs, FAKE, FAKE, FAKE, 1000, FAKE, 999, FAKE, FAKE, None, FAKE, 64, None) == 3
+    # append: k_new without v_new
+    assert L.msa_pooled_keys_append(bs, FAKE, FAKE, None, FAKE, FAKE, FAKE, 10, FAKE, FAKE, 1, FAKE, 256, None) == 1
+    assert L.msa_pooled_keys_append(bs, FAKE, None, None, FAKE, None, None, 0, FAKE, FAKE, 1, FAKE, 16, None) == 3
+
+
+def test_binding_rejects_host_tensors(L):
+    import torch
+    with pytest.raises(ValueError):
+        msa.msa_pool_index_keys(_shape(), torch.zeros(1, 256, 1, 64, dtype=torch.bfloat16), 256,
+                                torch.zeros(1, 1, 2, 64), 2)

@@ -1,0 +1,169 @@
+"""GPU parity of the decode step (append, select, split-KV attention) against the fp64 oracle,
+through the C ABI, plus the cross-path checks decode(L) == prefill row L and 128 appends ==
+block pooling."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from block_sparse_gqa_branch_b200 import (Shape, msa_get_device_status, msa_index_select,
+                                          msa_pool_index_keys, msa_pooled_keys_append, pipeline)
+from tests.gpu_util import check_selection, dev_bf16, f32, host_bits
+from tests.msa_check import assert_close_attention
+
+pytestmark = pytest.mark.gpu
+
+NAN_BF16 = 0x7FC0
+
+
+def build_decode_state(w, l_cap, garbage=True):
+    """Caches holding positions 0..L_b-1 of every sequence (the new token is appended by the
+    step), pooled keys built by the library's pooling kernel, plus the step's inputs."""
+    B, G = w.B, w.G
+    dev = "cuda"
+    k_cache = torch.empty(B, G, l_cap, 128, dtype=torch.bfloat16, device=dev)
+    v_cache = torch.empty_like(k_cache)
+    if garbage:       # positions past the context hold NaNs: they must never reach the output
+        k_cache.view(torch.int16).fill_(NAN_BF16)
+        v_cache.view(torch.int16).fill_(NAN_BF16)
+    nb_cap = l_cap // 128 + 1
+    pooled = torch.full((B, G, nb_cap, 64), float("nan"), device=dev)
+    tail = torch.zeros(B, G, 64, device=dev)
+    q = torch.empty(B, w.Hq, 128, dtype=torch.bfloat16, device=dev)
+    q_idx = torch.empty(B, G, 64, dtype=torch.bfloat16, device=dev)
+    k_idx_new = torch.empty(B, G, 64, dtype=torch.bfloat16, device=dev)
+    k_new = torch.empty(B, G, 128, dtype=torch.bfloat16, device=dev)
+    v_new = torch.empty_like(k_new)
+    for b in range(B):
+        Lb = w.ctx[b]
+        kk = synth.decode_seq_torch(w, b, "k", dev)           # [G, L, d]
+        vv = synth.decode_seq_torch(w, b, "v", dev)
+        ki = synth.decode_seq_torch(w, b, "k_idx", dev)       # [L, G, dI]
+        k_cache[b, :, :Lb] = kk[:, :Lb]
+        v_cache[b, :, :Lb] = vv[:, :Lb]
+        k_new[b], v_new[b], k_idx_new[b] = kk[:, Lb], vv[:, Lb], ki[Lb]
+        q[b] = synth.decode_seq_torch(w, b, "q", dev)
+        q_idx[b] = synth.decode_seq_torch(w, b, "q_idx", dev)
+        if Lb > 0:
+            msa_pool_index_keys(Shape.make(1, w.Hq, G), ki[:Lb].contiguous(), Lb, pooled[b], nb_cap, tail[b])
+    ctx = torch.tensor(list(w.ctx), dtype=torch.int32, device=dev)
+    return dict(k_cache=k_cache, v_cache=v_cache, pooled=pooled, tail=tail, q=q, q_idx=q_idx,
+                k_idx_new=k_idx_new, k_new=k_new, v_new=v_new, ctx=ctx, nb_cap=nb_cap)
+
+
+def run_step(w, st):
+    bufs = pipeline.decode_buffers(w.B, w.Hq, w.G, max(w.ctx), "cuda")
+    out, lse, sel = pipeline.decode_step(st["q"], st["q_idx"], st["k_idx_new"], st["k_new"], st["v_new"],
+                                         st["ctx"], st["k_cache"], st["v_cache"], st["tail"], st["pooled"], bufs)
+    torch.cuda.synchronize()
+    for key in ("ws_append", "ws_select", "ws_attn"):
+        s, info = msa_get_device_status(bufs[key])
+        assert s == 0, (key, s, info)
+    return f32(host_bits(out)), lse.cpu().numpy(), sel.cpu().numpy()
+
+
+def oracle_decode(w, sel_gpu):
+    """Oracle selection and attention (on the GPU's selection) for every (sequence, group)."""
+    res = []
+    for b in range(w.B):
+        Lb = w.ctx[b]
+        ki = synth.decode_seq_np(w, b, "k_idx")               # [L, G, dI]
+        pooled, _ = oracle.pool(ki, 128)
+        qi = synth.decode_seq_np(w, b, "q_idx")
+        q = synth.decode_seq_np(w, b, "q")
+        kk = synth.decode_seq_np(w, b, "k")
+        vv = synth.decode_seq_np(w, b, "v")
+        for g in range(w.G):
+            t = np.array([Lb])
+            s, kth, _ = oracle.select_rows(t, qi[g][None], pooled[g])
+            o, lse, nk = oracle.attend_rows(t, q[None, g * w.Hg:(g + 1) * w.Hg], kk[g], vv[g], sel_gpu[b, g][None])
+            res.append(dict(b=b, g=g, sel=s[0], kth=kth[0], o=o[0], lse=lse[0], pooled=pooled[g], qi=qi[g], t=t))
+    return res
+
+
+@pytest.mark.parametrize("ctx,Hq,G", [((4999, 2048, 127, 255), 16, 2), ((20000,), 64, 8), ((1, 0, 128 * 17), 8, 1),
+                                      ((3000, 70), 4, 4)])
+def test_decode_step_matches_oracle(cuda_ok, ctx, Hq, G):
+    w = synth.Workload(name="t", kind="decode", B=len(ctx), Hq=Hq, G=G, ctx=tuple(ctx), seed=4242 + sum(ctx))
+    l_cap = (max(ctx) + 1 + 127) // 128 * 128 + 128
+    st = build_decode_state(w, l_cap)
+    out, lse, sel = run_step(w, st)
+    ref = oracle_decode(w, sel)
+    for r in ref:
+        b, g = r["b"], r["g"]
+        check_selection(sel[b, g][None], r["sel"][None], np.array([r["kth"]]), r["qi"][None], r["pooled"], r["t"])
+        assert_close_attention(out[b, g * w.Hg:(g + 1) * w.Hg], r["o"], f"decode b={b} g={g}")
+        np.testing.assert_allclose(lse[b, g * w.Hg:(g + 1) * w.Hg], r["lse"], rtol=0, atol=2e-3)
+    # the appended token and the block it closed
+    for b in range(w.B):
+        Lb = w.ctx[b]
+        kk = synth.decode_seq_np(w, b, "k")
+        assert (host_bits(st["k_cache"][b, :, Lb]) == kk[:, Lb]).all()
+        if (Lb + 1) % 128 == 0:
+            ki = synth.decode_seq_np(w, b, "k_idx")
+            ref_pool, _ = oracle.pool(ki, 128)
+            got = st["pooled"][b, :, Lb // 128].cpu().numpy()
+            np.testing.assert_allclose(got, ref_pool[:, Lb // 128], rtol=1e-5, atol=1e-6)
+
+
+def test_decode_is_last_prefill_row(cuda_ok):
+    L = 128 * 19 + 37
+    wp = synth.Workload(name="p", kind="prefill", B=1, N=L + 1, Hq=16, G=2, seed=91)
+    x = synth.prefill_inputs_np(wp)
+    d = {k: dev_bf16(v) for k, v in x.items()}
+    bufs = pipeline.prefill_buffers(1, L + 1, 16, 2, "cuda")
+    out_p, lse_p, sel_p = pipeline.prefill(d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"], bufs)
+    # decode state from the same tensors: cache = first L tokens, the step appends token L
+    l_cap = L + 129
+    kc = torch.zeros(1, 2, l_cap, 128, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    kc[:, :, :L] = d["k"][:, :, :L]
+    vc[:, :, :L] = d["v"][:, :, :L]
+    nb_cap = l_cap // 128 + 1
+    pooled = torch.zeros(1, 2, nb_cap, 64, device="cuda")
+    tail = torch.zeros(1, 2, 64, device="cuda")
+    shape = Shape.make(1, 16, 2)
+    msa_pool_index_keys(shape, d["k_idx"][:, :L].contiguous(), L, pooled, nb_cap, tail)
+    ctx = torch.tensor([L], dtype=torch.int32, device="cuda")
+    dbufs = pipeline.decode_buffers(1, 16, 2, L, "cuda")
+    out_d, lse_d, sel_d = pipeline.decode_step(d["q"][:, L].contiguous(), d["q_idx"][:, L].contiguous(),
+                                               d["k_idx"][:, L].contiguous(), d["k"][:, :, L].contiguous(),
+                                               d["v"][:, :, L].contiguous(), ctx, kc, vc, tail, pooled, dbufs)
+    torch.cuda.synchronize()
+    assert (sel_d[0].cpu() == sel_p[0, L].cpu()).all()
+    a = f32(host_bits(out_d[0]))
+    b = f32(host_bits(out_p[0, L]))
+    assert np.abs(a - b).max() <= 1.6e-2
+    np.testing.assert_allclose(lse_d[0].cpu().numpy(), lse_p[0, L].cpu().numpy(), rtol=0, atol=1e-3)
+
+
+def test_appends_reproduce_block_pooling(cuda_ok):
+    G, n = 2, 128 * 3
+    k_idx = synth.normal_bf16(5, synth.STREAM_KI, (1, n, G, 64))
+    shape = Shape.make(1, 8, G)
+    ref = torch.zeros(1, G, 4, 64, device="cuda")
+    msa_pool_index_keys(shape, dev_bf16(k_idx), n, ref, 4, None)
+    pooled = torch.zeros(1, G, 4, 64, device="cuda")
+    tail = torch.zeros(1, G, 64, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    kd = dev_bf16(k_idx)
+    for pos in range(n):
+        ctx = torch.tensor([pos], dtype=torch.int32, device="cuda")
+        msa_pooled_keys_append(shape, kd[:, pos].contiguous(), None, None, ctx, None, None, 0, tail, pooled, 4, ws)
+    torch.cuda.synchronize()
+    assert msa_get_device_status(ws)[0] == 0
+    np.testing.assert_allclose(pooled[:, :, :3].cpu().numpy(), ref[:, :, :3].cpu().numpy(), rtol=1e-5, atol=1e-6)
+
+
+def test_device_bounds_are_reported_not_faulted(cuda_ok):
+    shape = Shape.make(2, 8, 1)
+    max_pos = 1000
+    bufs = pipeline.decode_buffers(2, 8, 1, max_pos, "cuda")
+    q_idx = torch.zeros(2, 1, 64, dtype=torch.bfloat16, device="cuda")
+    pooled = torch.zeros(2, 1, 8, 64, device="cuda")
+    q_pos = torch.tensor([5, 5000], dtype=torch.int32, device="cuda")   # second is beyond max_pos
+    msa_index_select(shape, q_idx, 1, q_pos, max_pos, pooled, 8, bufs["sel"], bufs["ws_select"])
+    st, info = msa_get_device_status(bufs["ws_select"])
+    assert st == 6 and info[3] == 5000
+    assert msa_get_device_status(bufs["ws_select"])[0] == 0          # cleared after reading
