@@ -20,6 +20,7 @@ __all__ = [
     "msa_abi_version", "msa_status_string", "msa_workspace_size",
     "msa_pool_index_keys", "msa_index_select", "msa_sparse_attn_prefill",
     "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_get_device_status",
+    "msa_index_select_decode_noalloc", "msa_kernel_launches",
     "OP_INDEX_SELECT_PREFILL", "OP_INDEX_SELECT_DECODE", "OP_ATTN_PREFILL", "OP_ATTN_DECODE",
     "EXPORTED_SYMBOLS",
 ]
@@ -39,6 +40,7 @@ EXPORTED_SYMBOLS = [
     "msa_workspace_size",
     "msa_pool_index_keys", "msa_index_select", "msa_sparse_attn_prefill",
     "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_get_device_status",
+    "msa_index_select_decode_noalloc",
 ]
 
 
@@ -91,6 +93,7 @@ def load():
             "msa_pooled_keys_append": [SP, P, P, P, P, P, P, I64, P, P, I64, P, SZ, P],
             "msa_sparse_attn_decode": [SP, P, P, P, I64, P, I64, P, P, P, P, SZ, P],
             "msa_get_device_status": [P, P, P],
+            "msa_index_select_decode_noalloc": [SP, P, P, I64, P, I64, P, P],
         }.items():
             f = getattr(L, name)
             f.restype = ctypes.c_int
@@ -192,3 +195,12 @@ def msa_get_device_status(workspace, stream=None):
     st = load().msa_get_device_status(_ptr(workspace), ctypes.cast(info, ctypes.c_void_p),
                                       _stream(stream))
     return st, list(info)
+
+
+def msa_index_select_decode_noalloc(shape: Shape, q_idx, q_pos, max_pos: int, pooled, nb_cap: int, sel,
+                                    stream=None):
+    """Decode selection that allocates nothing: its scratch is a fixed 2 MiB device array
+    inside libmsa (see include/msa.h). Same results as msa_index_select in decode mode."""
+    _check(load().msa_index_select_decode_noalloc(ctypes.byref(shape), _ptr(q_idx), _ptr(q_pos), max_pos,
+                                                  _ptr(pooled), nb_cap, _ptr(sel), _stream(stream)),
+           "msa_index_select_decode_noalloc")

@@ -26,15 +26,8 @@ void launch_attn_prefill_simt(const void*, const void*, const void*, int64_t, in
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
-}  // namespace msa
-
-using namespace msa;
-
-namespace {
 
 thread_local int g_last_cuda_error = 0;
-
-constexpr int64_t kMaxPos = (int64_t(1) << 24) - 1;   // decode select merge supports 1024 chunks
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -58,6 +51,13 @@ msa_status_t cuda_status() {
     }
     return MSA_OK;
 }
+}  // namespace msa
+
+using namespace msa;
+
+namespace {
+
+constexpr int64_t kMaxPos = kMaxDecodePos;
 
 #define MSA_TRY(x)                            \
     do {                                      \

@@ -15,6 +15,15 @@ namespace msa {
 // host-side count of kernels enqueued by libmsa (see msa_kernel_launches)
 void count_launch(unsigned n = 1);
 
+// host-side argument checks shared by the entry points
+extern thread_local int g_last_cuda_error;
+bool aligned16(const void* p);
+msa_status_t check_shape(const msa_shape_t* s);   // constants and head layout
+msa_status_t cuda_status();                       // MSA_ERR_CUDA if the last launch failed
+
+// largest query position the decode selection supports (its merge handles 1024 chunks)
+constexpr int64_t kMaxDecodePos = (int64_t(1) << 24) - 1;
+
 constexpr int kHeadDim = 128;   // d
 constexpr int kIndexDim = 64;   // d_I
 constexpr int kBlock = 128;     // Bk

@@ -255,3 +255,71 @@ void launch_select_decode(const void* q_idx, const int32_t* q_pos, int64_t max_p
 }
 
 }  // namespace msa
+
+// ------------------------------------------------------------------ allocation-free variant
+// Some callers cannot allocate device memory when they select blocks: a serving engine that
+// hands all device memory to its own pool at start-up and forbids allocation per step, or a
+// host thread that must not block on the allocator while the GPU runs. For them the decode
+// selection can keep its scratch (the arrival counters and the per-chunk candidate lists of
+// select_decode_kernel) in this file-scope device array instead of a caller workspace.
+// Every GPU that loads libmsa holds the array until the process exits.
+#include <mutex>
+
+namespace msa {
+
+constexpr size_t kNoAllocSelectScratch = size_t(2) << 20;   // 2 MiB per GPU
+static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocSelectScratch];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// The device address of g_select_scratch on the current device. The host-side name of the
+// array is only a stand-in, so the address is looked up once per device, with that device
+// current, and cached.
+msa_status_t scratch_on_current_device(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) { g_last_cuda_error = int(e); return MSA_ERR_CUDA; }
+    if (dev < 0 || dev >= kMaxDevices) return MSA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_select_scratch);
+        if (e != cudaSuccess || p == nullptr) { g_last_cuda_error = int(e); return MSA_ERR_CUDA; }
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return MSA_OK;
+}
+}  // namespace
+}  // namespace msa
+
+extern "C" msa_status_t msa_index_select_decode_noalloc(const msa_shape_t* shape, const void* q_idx,
+                                                        const int32_t* q_pos, int64_t max_pos,
+                                                        const float* pooled, int64_t nb_cap, int32_t* sel,
+                                                        msa_stream_t stream) {
+    using namespace msa;
+    msa_status_t s = check_shape(shape);
+    if (s != MSA_OK) return s;
+    if (q_idx == nullptr || !aligned16(q_idx) || q_pos == nullptr || sel == nullptr || !aligned16(sel) ||
+        pooled == nullptr || !aligned16(pooled) || max_pos < 0 || nb_cap < max_pos / kBlock)
+        return MSA_ERR_INVALID_ARGUMENT;
+    if (max_pos > kMaxDecodePos) return MSA_ERR_UNSUPPORTED;
+    const int B = shape->batch, G = shape->n_kv_groups;
+    if (decode_select_ws_bytes(B, G, max_pos) > kNoAllocSelectScratch) return MSA_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    s = scratch_on_current_device(&scratch);
+    if (s != MSA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // The array keeps the previous call's contents: the error word and the arrival counters
+    // must start at zero. Rows are preset to -1 so that a query whose position the device finds
+    // out of range is left all -1 (this variant has no workspace to report it in).
+    const size_t zero_bytes = sizeof(WsHeader) + (size_t(B) * G * sizeof(unsigned int) + 255) / 256 * 256;
+    cudaError_t e = cudaMemsetAsync(scratch, 0, zero_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(sel, 0xFF, size_t(B) * G * kTopK * sizeof(int32_t), st);
+    if (e != cudaSuccess) { g_last_cuda_error = int(e); return MSA_ERR_CUDA; }
+    launch_select_decode(q_idx, q_pos, max_pos, B, G, pooled, nb_cap, sel, scratch, st);
+    return cuda_status();
+}

@@ -138,6 +138,30 @@ msa_status_t msa_index_select(const msa_shape_t *shape, const void *q_idx, int64
                               size_t workspace_bytes, msa_stream_t stream);
 
 /*
+ * Decode selection without a workspace. The paper has no counterpart: this is an interface
+ * for callers that cannot allocate device memory when they select blocks -- a serving
+ * engine that gives all device memory to its own pool at start-up and allows no allocation
+ * per step, or a host thread that must not wait on the allocator. It computes exactly what
+ * msa_index_select computes in decode mode (same arguments, n_queries = 1), but keeps its
+ * scratch in a 2 MiB array that libmsa holds on every GPU that loads it, until exit.
+ *  - Limit: B * G * (ceil((max_pos / 128) / 128) * 120 + 4) bytes plus at most 512 must fit
+ *    in the 2 MiB: B = 16, G = 8 fits up to max_pos = 2,228,351; B = 4, G = 8 up to four
+ *    times that. Larger problems return MSA_ERR_WORKSPACE without launching.
+ *  - The first call on a device looks up the array's device address (once per device); make
+ *    that first call before any stream capture.
+ *  - Every call shares the one array: calls that may overlap on the GPU (other streams,
+ *    other host threads on the same device) race and must be serialised by the caller.
+ *  - sel rows are preset to -1; a row left all -1 means the device found its q_pos out of
+ *    range (this variant has no workspace error word).
+ *  - Allocates nothing: no cudaMalloc/cudaFree; two cudaMemsetAsync calls and one kernel on
+ *    `stream`.
+ */
+msa_status_t msa_index_select_decode_noalloc(const msa_shape_t *shape, const void *q_idx,
+                                             const int32_t *q_pos, int64_t max_pos,
+                                             const float *pooled, int64_t nb_cap, int32_t *sel,
+                                             msa_stream_t stream);
+
+/*
  * Main Branch, prefill -- exact softmax attention over the selected blocks, causal inside
  * the query's own block (sources: youmind article, figure 1 caption; KuCoin MSA launch
  * flash, summary: exact softmax attention only over the selected blocks).
