@@ -21,8 +21,9 @@ size_t decode_select_ws_bytes(int, int, int64_t);
 void launch_attn_decode(const CUtensorMap&, const CUtensorMap&, const void*, int64_t, const int32_t*, int64_t,
                         const int32_t*, int, int, int, void*, float*, void*, cudaStream_t);
 size_t decode_attn_ws_bytes(int, int, int);
-void launch_attn_prefill_simt(const void*, const void*, const void*, int64_t, int, int, int, const int32_t*,
-                              void*, float*, cudaStream_t);
+size_t prefill_attn_ws_bytes(int, int64_t, int, int);
+void launch_attn_prefill_tc(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, int64_t, int, int, int,
+                            const int32_t*, void*, float*, void*, cudaStream_t);
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
@@ -80,7 +81,9 @@ size_t ws_size(const msa_shape_t* s, int32_t op, int64_t n) {
         case MSA_OP_INDEX_SELECT_DECODE:
             if (n > kMaxPos) return 0;
             return decode_select_ws_bytes(s->batch, s->n_kv_groups, n);
-        case MSA_OP_ATTN_PREFILL: return header_only();
+        case MSA_OP_ATTN_PREFILL:
+            if (n < 1) return 0;
+            return prefill_attn_ws_bytes(s->batch, n, s->n_kv_groups, hg);
         case MSA_OP_ATTN_DECODE: return decode_attn_ws_bytes(s->batch, s->n_kv_groups, hg);
         default: return 0;
     }
@@ -191,11 +194,20 @@ msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const void* q, co
     MSA_REQ(q && k && v && sel && out && aligned16(q) && aligned16(k) && aligned16(v) && aligned16(sel) &&
                 aligned16(out) && (lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u) == 0),
             MSA_ERR_INVALID_ARGUMENT);
+    const int B = shape->batch, G = shape->n_kv_groups, Hq = shape->n_q_heads, hg = Hq / G;
+    // int32 device indexing: list entries, TMA row coordinates, per-block histogram in shared memory
+    MSA_REQ(int64_t(B) * n_tokens * G * (kTopK - 1) < (int64_t(1) << 31) &&
+                int64_t(B) * n_tokens * Hq < (int64_t(1) << 31) && int64_t(B) * G * n_tokens + kBlock < (int64_t(1) << 31) &&
+                (n_tokens + kBlock - 1) / kBlock <= 48 * 1024,
+            MSA_ERR_UNSUPPORTED);
     const size_t need = ws_size(shape, MSA_OP_ATTN_PREFILL, n_tokens);
-    MSA_REQ(workspace != nullptr && workspace_bytes >= need, MSA_ERR_WORKSPACE);
-    const int hg = shape->n_q_heads / shape->n_kv_groups;
-    launch_attn_prefill_simt(q, k, v, n_tokens, shape->batch, shape->n_kv_groups, hg, sel, out, lse,
-                             reinterpret_cast<cudaStream_t>(stream));
+    MSA_REQ(workspace != nullptr && aligned16(workspace) && need > 0 && workspace_bytes >= need, MSA_ERR_WORKSPACE);
+    CUtensorMap tmQ, tmK, tmV;
+    MSA_TRY(make_tmap_bf16(&tmQ, q, uint64_t(B) * n_tokens * Hq, kHeadDim, 64, uint32_t(hg)));
+    MSA_TRY(make_tmap_bf16(&tmK, k, uint64_t(B) * G * n_tokens, kHeadDim, 64, 128));
+    MSA_TRY(make_tmap_bf16(&tmV, v, uint64_t(B) * G * n_tokens, kHeadDim, 64, 128));
+    launch_attn_prefill_tc(tmQ, tmK, tmV, n_tokens, B, G, hg, sel, out, lse, workspace,
+                           reinterpret_cast<cudaStream_t>(stream));
     return cuda_status();
 }
 
