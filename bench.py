@@ -214,7 +214,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_tok * PREFILL.N * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded SplitMix64 -> N(0,1) quantiles -> bf16)",
-            "config": config_block(),
+            "config": config_block(PREFILL, DECODE),
             "cpu_baseline": {"value": value, "unit": "tok/s", "cores": oracle.default_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -222,12 +222,24 @@ def run_reference(args):
     return 0
 
 
-def config_block():
-    return {"workload": f"{PREFILL.name} + {DECODE.name}",
-            "prefill": {"batch": PREFILL.B, "seq_len": PREFILL.N, "q_heads": PREFILL.Hq, "kv_groups": PREFILL.G,
-                        "head_dim": PREFILL.d, "index_dim": PREFILL.dI, "block": PREFILL.Bk, "top_k": PREFILL.topk},
-            "decode": {"batch": DECODE.B, "ctx_len": DECODE.ctx[0], "q_heads": DECODE.Hq, "kv_groups": DECODE.G,
-                       "head_dim": DECODE.d, "index_dim": DECODE.dI, "block": DECODE.Bk, "top_k": DECODE.topk},
+def workloads(args):
+    """The benchmark workloads, or smaller ones of the same structure for a profiler capture."""
+    import dataclasses
+    wp, wd = PREFILL, DECODE
+    if args.prefill_tokens:
+        wp = dataclasses.replace(wp, N=args.prefill_tokens, name=f"prefill_{args.prefill_tokens}_h64g8")
+    if args.decode_batch:
+        wd = dataclasses.replace(wd, B=args.decode_batch, ctx=wd.ctx[:1] * args.decode_batch,
+                                 name=f"decode_128k_b{args.decode_batch}_h64g8")
+    return wp, wd
+
+
+def config_block(wp, wd):
+    return {"workload": f"{wp.name} + {wd.name}",
+            "prefill": {"batch": wp.B, "seq_len": wp.N, "q_heads": wp.Hq, "kv_groups": wp.G,
+                        "head_dim": wp.d, "index_dim": wp.dI, "block": wp.Bk, "top_k": wp.topk},
+            "decode": {"batch": wd.B, "ctx_len": wd.ctx[0], "q_heads": wd.Hq, "kv_groups": wd.G,
+                       "head_dim": wd.d, "index_dim": wd.dI, "block": wd.Bk, "top_k": wd.topk},
             "l2": "flushed before every timed step (256 MiB write)",
             "parallelism": "replicas (one independent problem per GPU)"}
 
@@ -298,11 +310,12 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    wp, wd = PREFILL, DECODE
+    wp, wd = workloads(args)
+    do_prefill, do_decode = args.only in (None, "prefill"), args.only in (None, "decode")
     x = synth.prefill_inputs_torch(wp, dev)
     pbufs = pipeline.prefill_buffers(wp.B, wp.N, wp.Hq, wp.G, dev)
-    ds = build_decode_state(wd, dev)
-    dbufs = pipeline.decode_buffers(wd.B, wd.Hq, wd.G, max(wd.ctx), dev)
+    ds = build_decode_state(wd, dev) if do_decode else None
+    dbufs = pipeline.decode_buffers(wd.B, wd.Hq, wd.G, max(wd.ctx), dev) if do_decode else None
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -311,12 +324,15 @@ def run_ours(args):
                              ds["k_cache"], ds["v_cache"], ds["tail"], ds["pooled"], dbufs)
 
     # eager warm-up (sets kernel attributes), then capture the decode step in a CUDA graph
-    pipeline.prefill(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], pbufs)
-    decode_call()
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
+    graph = None
+    if do_prefill:
+        pipeline.prefill(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], pbufs)
+    if do_decode:
         decode_call()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            decode_call()
     torch.cuda.synchronize()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
@@ -327,13 +343,16 @@ def run_ours(args):
         flush.zero_()
         e0, e1, e2, e3, e4 = ev(), ev(), ev(), ev(), ev()
         e0.record(stream)
-        pipeline.prefill_index(x["q_idx"], x["k_idx"], pbufs)
+        if do_prefill:
+            pipeline.prefill_index(x["q_idx"], x["k_idx"], pbufs)
         e1.record(stream)
-        pipeline.prefill_main(x["q"], x["k"], x["v"], pbufs)
+        if do_prefill:
+            pipeline.prefill_main(x["q"], x["k"], x["v"], pbufs)
         e2.record(stream)
         flush.zero_()
         e3.record(stream)
-        graph.replay()
+        if do_decode:
+            graph.replay()
         e4.record(stream)
         return (e0, e1, e2, e3, e4) if record else None
 
@@ -353,7 +372,7 @@ def run_ours(args):
         t_index.append(e0.elapsed_time(e1) * 1e-3)
         t_main.append(e1.elapsed_time(e2) * 1e-3)
         t_dec.append(e3.elapsed_time(e4) * 1e-3)
-    decode_graph_kernels = 3
+    decode_graph_kernels = 3 if do_decode else 0
     gpu_launches = launches_eager + decode_graph_kernels * args.steps
 
     # check the device error words after the timed region
@@ -361,7 +380,7 @@ def run_ours(args):
         st_, info = msa.msa_get_device_status(pbufs[key])
         if st_ != 0:
             raise SystemExit(f"device status {st_} in prefill {key}: {info}")
-    for key in ("ws_append", "ws_select", "ws_attn"):
+    for key in (("ws_append", "ws_select", "ws_attn") if do_decode else ()):
         st_, info = msa.msa_get_device_status(dbufs[key])
         if st_ != 0:
             raise SystemExit(f"device status {st_} in decode {key}: {info}")
@@ -378,7 +397,7 @@ def run_ours(args):
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and do_prefill and do_decode:
         host_in = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in x.items()}
         for k in x:
             host_in[k].copy_(x[k])
@@ -423,7 +442,7 @@ def run_ours(args):
         return 0
 
     cpu = None
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and args.only is None:
         try:
             cpu = cpu_baseline(wp, budget_s=args.cpu_budget)
         except Exception as exc:  # reported, never fatal for the GPU number
@@ -443,7 +462,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded SplitMix64 -> N(0,1) quantiles -> bf16), generated on the device",
-        "config": config_block(),
+        "config": config_block(wp, wd),
         "prefill_ms": tp * 1e3,
         "prefill_index_ms": tidx * 1e3,
         "prefill_main_ms": tmain * 1e3,
@@ -474,6 +493,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="run one half of the step (profiler captures; not a benchmark value)")
+    ap.add_argument("--prefill-tokens", type=int, default=0, help="smaller prefill for profiler captures")
+    ap.add_argument("--decode-batch", type=int, default=0, help="smaller decode batch for profiler captures")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

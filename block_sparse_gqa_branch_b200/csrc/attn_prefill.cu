@@ -29,7 +29,7 @@ constexpr int kMaxTilesPerItem = 32;    // tiles per work item (K/V loaded once 
 constexpr int kSlots = 16;              // partial slots per (token, group); slot 15 = diagonal block
 constexpr int kDiagSlot = 15;
 constexpr int kDiagFlag = int(0x40000000);
-constexpr int kKvThreads = 384;         // warp 0 TMA, warp 1 MMA, warps 4-7 and 8-11 softmax/epilogue
+constexpr int kKvThreads = 384;         // warps 0-7 softmax/epilogue, 8 and 11 Q loads, 9 MMA, 10 K/V loads
 
 static_assert(kRange % kCountChunk == 0 && kRange % kBlock == 0, "range must hold whole chunks and blocks");
 
@@ -159,7 +159,10 @@ __global__ void __launch_bounds__(1024) csr_scan_kernel(int* __restrict__ counts
                 items[ioff++] = make_int4(bg, c | kDiagFlag, c * kBlock, int(imin64(kBlock, N - int64_t(c) * kBlock)));
         }
     }
-    if (threadIdx.x == 1023) n_items[0] = int(ioff);
+    if (threadIdx.x == 1023) {
+        n_items[0] = int(ioff);
+        n_items[1] = 0;                                   // work-item counter of the tensor-core kernel
+    }
 }
 
 // ------------------------------------------------------------------ CSR: fill
@@ -193,11 +196,19 @@ __global__ void __launch_bounds__(256) csr_fill_kernel(const int32_t* __restrict
 }
 
 // ------------------------------------------------------------------ the tensor-core kernel
+constexpr int kQStages = 2;
+constexpr int kRing = 8;           // work items handed from the scheduler to the other roles
+constexpr int kRingReaders = 11;   // 2 Q warps, MMA thread, 8 softmax warps
+
 struct __align__(1024) KvSmem {
-    uint8_t kv[2][2][32768];   // [K/V buffer][K, V][d half][128 rows][128 B], 128B swizzle
-    uint8_t q[2][32768];       // [stage][d half][128 rows][128 B], 128B swizzle
-    uint64_t kv_full[2], kv_empty[2], q_full[2], q_empty[2];
+    uint8_t k[2][32768];          // K_j, double-buffered: [d half][128 rows][128 B], 128B swizzle
+    uint8_t v[32768];             // V_j: [d half][128 rows][128 B], 128B swizzle
+    uint8_t q[kQStages][32768];   // gathered query rows: [d half][128 rows][128 B], 128B swizzle
+    uint8_t o_stage[8][8192];     // per softmax warp: [d half][32 output rows][128 B] (bf16), 128B swizzle
+    uint64_t k_full[2], k_empty[2], v_full, v_empty, q_full[kQStages], q_empty[kQStages];
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+    uint64_t item_full[kRing], item_empty[kRing];
+    volatile int item_ring[kRing];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -205,18 +216,113 @@ struct __align__(1024) KvSmem {
 struct PrefillArgs {
     int64_t N;
     int G, Hg, Hq, tpt;
-    const int* n_items;
+    int* n_items;                  // [0] = number of work items, [1] = next item to hand out
     const int4* items;
     const int* list;
     float* part_lse;
     uint16_t* part_o;
+    const uint16_t* q;
     WsHeader* hdr;
     float scale_log2;
 };
 
+// packed fp32x2 arithmetic (one instruction for two lanes of data)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// Work-item decoding shared by every role: all roles walk items blockIdx.x, +gridDim.x, ...
+struct Item {
+    int bg, b, g, j, first, n, ntiles;
+    bool diag;
+};
+__device__ __forceinline__ Item load_item(const PrefillArgs a, int k) {
+    const int4 v = a.items[k];
+    Item it;
+    it.bg = v.x; it.b = v.x / a.G; it.g = v.x % a.G;
+    it.diag = (v.y & kDiagFlag) != 0;
+    it.j = v.y & ~kDiagFlag;
+    it.first = v.z; it.n = v.w;
+    it.ntiles = (v.w + a.tpt - 1) / a.tpt;
+    return it;
+}
+
+// O = P V for a tile whose S was issued earlier (MMA-issuing thread only). The first tile of an
+// item waits for the item's V; the last one releases V when its MMAs complete.
+struct PendO { int it, ic; bool first, last; };
+__device__ __forceinline__ bool issue_o(KvSmem& sm, const PrefillArgs a, uint32_t tmem, uint32_t vbase,
+                                        uint32_t idesc_o, const PendO& p) {
+    const int buf = p.it & 1;
+    if (p.first && !mbar_wait(&sm.v_full, p.ic & 1, a.hdr, KID_ATTN_PREFILL)) return false;
+    if (!mbar_wait(&sm.p_full[buf], (p.it >> 1) & 1, a.hdr, KID_ATTN_PREFILL)) return false;
+    if (!mbar_wait(&sm.o_free[buf], ((p.it >> 1) & 1) ^ 1, a.hdr, KID_ATTN_PREFILL)) return false;
+    tc_fence_after();
+    const uint32_t tS = tmem + buf * 128, tO = tmem + 256 + buf * 128;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks)
+        tc_mma_ts(tO, tS + ks * 8, sdesc_sw128(vbase + ks * 2048, 16384, 1024), idesc_o, ks > 0);
+    tc_commit(&sm.o_full[buf]);
+    if (p.last) tc_commit(&sm.v_empty);
+    return true;
+}
+
+// A bounded wait by every lane of a warp whose outcome is the same for the whole warp (a lane
+// that timed out makes all lanes fail), so the warp's collective instructions stay converged.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, WsHeader* hdr) {
+    const bool ok = mbar_wait(bar, parity, hdr, KID_ATTN_PREFILL);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Next work item of a role's sequence s (-1 = no more work, -2 = timeout). With whole_warp,
+// every lane of the warp calls this, reads the slot, and lane 0 releases it after the warp has
+// read it; otherwise a single thread calls it and releases the slot itself.
+__device__ __forceinline__ int ring_take(KvSmem& sm, int s, WsHeader* hdr, bool whole_warp) {
+    const int slot = s % kRing;
+    const bool got = whole_warp ? warp_wait(&sm.item_full[slot], (s / kRing) & 1, hdr)
+                                : mbar_wait(&sm.item_full[slot], (s / kRing) & 1, hdr, KID_ATTN_PREFILL);
+    if (!got) return -2;
+    const int k = sm.item_ring[slot];
+    if (whole_warp) {
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.item_empty[slot]);
+    } else {
+        mbar_arrive(&sm.item_empty[slot]);
+    }
+    return k;
+}
+
+// token of row group r of tile tt of an item (0 when r is past the item's end)
+__device__ __forceinline__ int fetch_token(const PrefillArgs a, const Item item, int tt, int r) {
+    const int e = tt * a.tpt + r;
+    if (r >= a.tpt || tt >= item.ntiles || e >= item.n) return 0;
+    return item.diag ? item.first + e : (__ldg(a.list + item.first + e) / kSlots);
+}
+
 __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                      const __grid_constant__ CUtensorMap tmK,
                                                                      const __grid_constant__ CUtensorMap tmV,
+                                                                     const __grid_constant__ CUtensorMap tmO,
                                                                      const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     KvSmem& sm = *reinterpret_cast<KvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -226,22 +332,31 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&sm.kv_full[i], 1);
-            mbar_init(&sm.kv_empty[i], 1);
-            mbar_init(&sm.q_full[i], 1);
-            mbar_init(&sm.q_empty[i], 1);
+            mbar_init(&sm.k_full[i], 1);
+            mbar_init(&sm.k_empty[i], 1);
             mbar_init(&sm.s_full[i], 1);
             mbar_init(&sm.p_full[i], 128);
             mbar_init(&sm.o_full[i], 1);
             mbar_init(&sm.o_free[i], 128);
+        }
+        for (int i = 0; i < kQStages; ++i) {
+            mbar_init(&sm.q_full[i], 1);
+            mbar_init(&sm.q_empty[i], 1);
+        }
+        mbar_init(&sm.v_full, 1);
+        mbar_init(&sm.v_empty, 1);
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(&sm.item_full[i], 1);
+            mbar_init(&sm.item_empty[i], kRingReaders);
         }
         sm.abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmO);
     }
-    if (warp == 1) {
+    if (warp == 9) {
         tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
     }
@@ -250,195 +365,278 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0) {
-        // ---------------------------------------------------------------- TMA producer
-        int it = 0, ic = 0;
-        for (int k = blockIdx.x; k < n_items; k += gridDim.x, ++ic) {
-            const int4 item = a.items[k];
-            const int bg = item.x, b = bg / a.G, g = bg % a.G;
-            const bool diag = (item.y & kDiagFlag) != 0;
-            const int j = item.y & ~kDiagFlag;
-            const int kvb = ic & 1;
-            bool ok = true;
-            if (lane == 0) {
-                ok = mbar_wait(&sm.kv_empty[kvb], ((ic >> 1) & 1) ^ 1, a.hdr, KID_ATTN_PREFILL);
-                if (ok) {
-                    mbar_arrive_expect_tx(&sm.kv_full[kvb], 65536);
-                    const int row0 = int(int64_t(bg) * a.N + int64_t(j) * kBlock);
-                    for (int h = 0; h < 2; ++h) {
-                        tma_load_2d(sm.kv[kvb][0] + h * 16384, &tmK, h * 64, row0, &sm.kv_full[kvb]);
-                        tma_load_2d(sm.kv[kvb][1] + h * 16384, &tmV, h * 64, row0, &sm.kv_full[kvb]);
-                    }
-                }
-            }
-            if (!__shfl_sync(0xffffffffu, ok, 0)) { sm.abort_flag = 1; break; }
-            const int n = item.w;
-            const int ntiles = (n + tpt - 1) / tpt;
-            for (int tt = 0; tt < ntiles; ++tt, ++it) {
-                const int buf = it & 1;
-                const int nv = min(tpt, n - tt * tpt);
+    if (warp == 8 || warp == 11) {
+        // ---------------------------------------------------------------- Q gather (TMA)
+        // Warp 8 loads the even tiles (stage 0), warp 11 the odd ones (stage 1); lane r issues
+        // the copies of the tile's tokens r, r + 32, ... For Hg >= 8 one 3-D box brings 8 head rows
+        // of a token with both d halves (2 KB): the stage is laid out as 8-row groups of 2 KB
+        // ([half][8 rows][128 B], 128B swizzle). For Hg < 8 a token's Hg rows come as two 2-D boxes
+        // into [half][128 rows][128 B]. List entries of a loader's next tile are fetched ahead.
+        const int mine = warp == 8 ? 0 : 1;
+        const uint64_t keep = l2_evict_last();          // query rows are re-read ~15 times per range
+        int it = 0;
+        for (int sq = 0;; ++sq) {
+            const int k = ring_take(sm, sq, a.hdr, true);
+            if (k < 0) { if (k == -2) sm.abort_flag = 1; break; }
+            const Item item = load_item(a, k);
+            const int t0 = (it & 1) == mine ? 0 : 1;                      // this warp's first tile
+            int tok[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tok[i] = fetch_token(a, item, t0, lane + 32 * i);
+            for (int tt = 0; tt < item.ntiles; ++tt, ++it) {
+                if ((it & 1) != mine) continue;
+                const int use = it >> 1;
+                const int nv = min(tpt, item.n - tt * tpt);
+                bool ok = true;
                 if (lane == 0) {
-                    ok = mbar_wait(&sm.q_empty[buf], ((it >> 1) & 1) ^ 1, a.hdr, KID_ATTN_PREFILL);
-                    if (ok) mbar_arrive_expect_tx(&sm.q_full[buf], uint32_t(nv) * Hg * 256u);
+                    ok = mbar_wait(&sm.q_empty[mine], (use & 1) ^ 1, a.hdr, KID_ATTN_PREFILL);
+                    if (ok) mbar_arrive_expect_tx(&sm.q_full[mine], uint32_t(nv) * Hg * 256u);
                 }
                 if (!__shfl_sync(0xffffffffu, ok, 0)) { sm.abort_flag = 1; break; }
-                for (int r = lane; r < nv; r += 32) {
-                    const int e = tt * tpt + r;
-                    const int t = diag ? item.z + e : (a.list[item.z + e] / kSlots);
-                    const int qrow = int((int64_t(b) * a.N + t) * a.Hq + int64_t(g) * Hg);
-                    tma_load_2d(sm.q[buf] + r * Hg * 128, &tmQ, 0, qrow, &sm.q_full[buf]);
-                    tma_load_2d(sm.q[buf] + 16384 + r * Hg * 128, &tmQ, 64, qrow, &sm.q_full[buf]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = lane + 32 * i;
+                    if (r < nv) {
+                        const int qrow = int((int64_t(item.b) * a.N + tok[i]) * a.Hq + int64_t(item.g) * Hg);
+                        if (Hg >= 8) {
+                            for (int h8 = 0; h8 < Hg; h8 += 8)
+                                tma_load_3d_hint(sm.q[mine] + (r * Hg + h8) * 256, &tmQ, 0, qrow + h8, 0, &sm.q_full[mine], keep);
+                        } else {
+                            tma_load_2d_hint(sm.q[mine] + r * Hg * 128, &tmQ, 0, qrow, &sm.q_full[mine], keep);
+                            tma_load_2d_hint(sm.q[mine] + 16384 + r * Hg * 128, &tmQ, 64, qrow, &sm.q_full[mine], keep);
+                        }
+                    }
                 }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) tok[i] = fetch_token(a, item, tt + 2, lane + 32 * i);
                 __syncwarp();
             }
-            if (sm.abort_flag) break;
+            if (__any_sync(0xffffffffu, sm.abort_flag != 0)) break;
         }
-    } else if (warp == 1) {
+    } else if (warp == 10) {
+        // ---------------------------------------------------------------- scheduler + K/V loads (TMA)
+        // Items are handed out in list order through a global counter, so all CTAs stay within a
+        // narrow window of the work order (the window's query rows stay in L2).
+        if (lane == 0) {
+            const uint64_t stream = l2_evict_first();   // a key/value block serves one work item
+            for (int ic = 0;; ++ic) {
+                const int slot = ic % kRing;
+                if (!mbar_wait(&sm.item_empty[slot], ((ic / kRing) & 1) ^ 1, a.hdr, KID_ATTN_PREFILL)) {
+                    sm.abort_flag = 1;
+                    break;
+                }
+                int k = atomicAdd(a.n_items + 1, 1);
+                if (k >= n_items) k = -1;
+                sm.item_ring[slot] = k;
+                mbar_arrive(&sm.item_full[slot]);
+                if (k < 0) break;
+                const Item item = load_item(a, k);
+                if (!item.diag) {                           // warm L2 with the item's list entries
+                    const uint64_t lo = (uint64_t(reinterpret_cast<uintptr_t>(a.list + item.first))) & ~uint64_t(15);
+                    const uint64_t hi = (uint64_t(reinterpret_cast<uintptr_t>(a.list + item.first + item.n)) + 15) & ~uint64_t(15);
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(lo), "r"(uint32_t(hi - lo)) : "memory");
+                }
+                const int row0 = int(int64_t(item.bg) * a.N + int64_t(item.j) * kBlock);
+                const int kb = ic & 1;
+                if (!mbar_wait(&sm.k_empty[kb], ((ic >> 1) & 1) ^ 1, a.hdr, KID_ATTN_PREFILL)) { sm.abort_flag = 1; break; }
+                mbar_arrive_expect_tx(&sm.k_full[kb], 32768);
+                tma_load_2d_hint(sm.k[kb], &tmK, 0, row0, &sm.k_full[kb], stream);
+                tma_load_2d_hint(sm.k[kb] + 16384, &tmK, 64, row0, &sm.k_full[kb], stream);
+                if (!mbar_wait(&sm.v_empty, (ic & 1) ^ 1, a.hdr, KID_ATTN_PREFILL)) { sm.abort_flag = 1; break; }
+                mbar_arrive_expect_tx(&sm.v_full, 32768);
+                tma_load_2d_hint(sm.v, &tmV, 0, row0, &sm.v_full, stream);
+                tma_load_2d_hint(sm.v + 16384, &tmV, 64, row0, &sm.v_full, stream);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);   // Q (K-major) x K_j (K-major)
+            // Q stage layout (see the Q gather): d-half offset and 8-row-group stride
+            const uint32_t q_half = Hg >= 8 ? 1024u : 16384u, q_sbo = Hg >= 8 ? 2048u : 1024u;
             const uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);   // P (TMEM) x V_j (MN-major)
-            int it = 0, ic = 0;
-            int prev_it = -1, prev_kvb = 0;
-            bool prev_last = false, ok = true;
-            auto issue_o = [&](int pit, int pkvb, bool plast) -> bool {
-                const int pbuf = pit & 1;
-                if (!mbar_wait(&sm.p_full[pbuf], (pit >> 1) & 1, a.hdr, KID_ATTN_PREFILL)) return false;
-                if (!mbar_wait(&sm.o_free[pbuf], ((pit >> 1) & 1) ^ 1, a.hdr, KID_ATTN_PREFILL)) return false;
+            const uint32_t vbase = smem_u32(sm.v);
+            PendO pend{-1, 0, false, false};
+            bool ok = true;
+            int it = 0;
+            for (int ic = 0; ok; ++ic) {
+                const int k = ring_take(sm, ic, a.hdr, false);
+                if (k < 0) { ok = (k == -1); break; }
+                const Item item = load_item(a, k);
+                const int kb = ic & 1;
+                // finish the previous item's last tile before waiting for this item's keys
+                if (pend.it >= 0) {
+                    if (!issue_o(sm, a, tmem, vbase, idesc_o, pend)) { ok = false; break; }
+                    pend.it = -1;
+                }
+                if (!mbar_wait(&sm.k_full[kb], (ic >> 1) & 1, a.hdr, KID_ATTN_PREFILL)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t tS = tmem + pbuf * 128, tO = tmem + 256 + pbuf * 128;
-                const uint32_t vbase = smem_u32(sm.kv[pkvb][1]);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    tc_mma_ts(tO, tS + ks * 8, sdesc_sw128(vbase + ks * 2048, 16384, 1024), idesc_o, ks > 0);
-                tc_commit(&sm.o_full[pbuf]);
-                if (plast) tc_commit(&sm.kv_empty[pkvb]);
-                return true;
-            };
-            for (int k = blockIdx.x; k < n_items && ok; k += gridDim.x, ++ic) {
-                const int4 item = a.items[k];
-                const int n = item.w;
-                const int ntiles = (n + tpt - 1) / tpt;
-                const int kvb = ic & 1;
-                if (!mbar_wait(&sm.kv_full[kvb], (ic >> 1) & 1, a.hdr, KID_ATTN_PREFILL)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t kbase = smem_u32(sm.kv[kvb][0]);
-                for (int tt = 0; tt < ntiles; ++tt, ++it) {
-                    const int buf = it & 1;
-                    if (!mbar_wait(&sm.q_full[buf], (it >> 1) & 1, a.hdr, KID_ATTN_PREFILL)) { ok = false; break; }
+                const uint32_t kbase = smem_u32(sm.k[kb]);
+                for (int tt = 0; tt < item.ntiles; ++tt, ++it) {
+                    const int buf = it & 1, stage = it % kQStages;
+                    if (!mbar_wait(&sm.q_full[stage], (it / kQStages) & 1, a.hdr, KID_ATTN_PREFILL)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t qbase = smem_u32(sm.q[buf]);
+                    const uint32_t qbase = smem_u32(sm.q[stage]);
                     const uint32_t tS = tmem + buf * 128;
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        tc_mma_ss(tS, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
+                        const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        const uint32_t qoff = (ks >> 2) * q_half + (ks & 3) * 32;
+                        tc_mma_ss(tS, sdesc_sw128(qbase + qoff, 16, q_sbo), sdesc_sw128(kbase + koff, 16, 1024),
                                   idesc_s, ks > 0);
                     }
                     tc_commit(&sm.s_full[buf]);
-                    tc_commit(&sm.q_empty[buf]);
-                    if (prev_it >= 0 && !issue_o(prev_it, prev_kvb, prev_last)) { ok = false; break; }
-                    prev_it = it;
-                    prev_kvb = kvb;
-                    prev_last = (tt == ntiles - 1);
+                    tc_commit(&sm.q_empty[stage]);
+                    if (tt == item.ntiles - 1) tc_commit(&sm.k_empty[kb]);
+                    if (pend.it >= 0 && !issue_o(sm, a, tmem, vbase, idesc_o, pend)) { ok = false; break; }
+                    pend = PendO{it, ic, tt == 0, tt == item.ntiles - 1};
                 }
             }
-            if (ok && prev_it >= 0) issue_o(prev_it, prev_kvb, prev_last);
+            if (ok && pend.it >= 0) issue_o(sm, a, tmem, vbase, idesc_o, pend);
+            if (!ok) sm.abort_flag = 1;
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    } else if (warp < 8) {
         // ---------------------------------------------------------------- softmax + epilogue
-        const int w = (warp - 4) >> 2;                      // warpgroup: tiles with it % 2 == w
+        const int w = warp >> 2;                            // warpgroup w takes the tiles with it % 2 == w
         const int row = (warp & 3) * 32 + lane;             // TMEM lane = tile row
         const int r = row / Hg, h = row % Hg;
         const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_off + w * 128;
         const uint32_t tO = tmem + lane_off + 256 + w * 128;
         const float sl2 = a.scale_log2;
+        const float2 sc = make_float2(sl2, sl2);
+        uint8_t* stg = sm.o_stage[warp];
+        const uint64_t stream = l2_evict_first();       // partial outputs are read once, much later
         int it = 0;
-        for (int k = blockIdx.x; k < n_items; k += gridDim.x) {
-            const int4 item = a.items[k];
-            const int bg = item.x, b = bg / a.G, g = bg % a.G;
-            const bool diag = (item.y & kDiagFlag) != 0;
-            const int j = item.y & ~kDiagFlag;
-            const int n = item.w;
-            const int ntiles = (n + tpt - 1) / tpt;
-            bool ok = true;
-            for (int tt = 0; tt < ntiles; ++tt, ++it) {
+        bool ok = true;
+        for (int si = 0; ok; ++si) {
+            const int k = ring_take(sm, si, a.hdr, true);
+            if (k < 0) { ok = (k == -1); break; }
+            const Item item = load_item(a, k);
+            for (int tt = 0; tt < item.ntiles; ++tt, ++it) {
                 if ((it & 1) != w) continue;
                 const int use = it >> 1;
                 const int e = tt * tpt + r;
-                const bool valid = e < n;
+                const bool valid = e < item.n;
                 int t = 0, slot = kDiagSlot;
                 if (valid) {
-                    if (diag) t = item.z + e;
-                    else { const int v = a.list[item.z + e]; t = v / kSlots; slot = v % kSlots; }
+                    if (item.diag) t = item.first + e;
+                    else { const int v = __ldg(a.list + item.first + e); t = v / kSlots; slot = v % kSlots; }
                 }
-                const int lim = diag ? (t - j * kBlock) : (kBlock - 1);      // last visible key column
-                if (!mbar_wait(&sm.s_full[w], use & 1, a.hdr, KID_ATTN_PREFILL)) { ok = false; break; }
+                // columns past lim are masked (causal mask of the diagonal block)
+                const int lim = item.diag ? t - item.j * kBlock : kBlock - 1;
+                if (!warp_wait(&sm.s_full[w], use & 1, a.hdr)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t v[32];
-                float mx = -INFINITY;
+                uint32_t va[32], vb[32];
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld32(tS + c * 32, v);
+                for (int p = 0; p < 2; ++p) {                       // row max, 64 columns per TMEM wait
+                    tmem_ld32(tS + p * 64, va);
+                    tmem_ld32(tS + p * 64 + 32, vb);
                     tmem_wait_ld();
+                    if (!item.diag) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (c * 32 + i <= lim) mx = fmaxf(mx, __uint_as_float(v[i]));
-                }
-                const float ms = (mx == -INFINITY) ? 0.f : mx * sl2;
-                float l = 0.f;
+                        for (int i = 0; i < 32; ++i) {
+                            m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(va[i]));
+                            m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(vb[i]));
+                        }
+                    } else {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld32(tS + c * 32, v);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int col = c * 32 + 2 * i;
-                        const float p0 = col <= lim ? fast_exp2(fmaf(__uint_as_float(v[2 * i]), sl2, -ms)) : 0.f;
-                        const float p1 = col + 1 <= lim ? fast_exp2(fmaf(__uint_as_float(v[2 * i + 1]), sl2, -ms)) : 0.f;
-                        l += p0 + p1;
-                        pk[i] = pack_bf16x2(p0, p1);
+                        for (int i = 0; i < 32; ++i) {
+                            if (p * 64 + i <= lim) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(va[i]));
+                            if (p * 64 + 32 + i <= lim) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(vb[i]));
+                        }
                     }
-                    tmem_st16(tS + c * 16, pk);
+                }
+                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                const float ms = (mx == -INFINITY) ? 0.f : mx * sl2;
+                const float2 nm = make_float2(-ms, -ms);
+                float2 l2 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {                       // p = 2^(s*scale - m), P -> TMEM as bf16
+                    tmem_ld32(tS + p * 64, va);
+                    tmem_ld32(tS + p * 64 + 32, vb);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const uint32_t x0 = q == 0 ? va[2 * i] : vb[2 * i];
+                            const uint32_t x1 = q == 0 ? va[2 * i + 1] : vb[2 * i + 1];
+                            const float2 x = ffma2(make_float2(__uint_as_float(x0), __uint_as_float(x1)), sc, nm);
+                            const int col = p * 64 + q * 32 + 2 * i;
+                            float2 pv = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                            if (item.diag) {
+                                pv.x = col <= lim ? pv.x : 0.f;
+                                pv.y = col + 1 <= lim ? pv.y : 0.f;
+                            }
+                            l2 = fadd2(l2, pv);
+                            pk[i] = pack_bf16x2(pv.x, pv.y);
+                        }
+                        tmem_st16(tS + p * 32 + q * 16, pk);
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.p_full[w]);
+                const float l = l2.x + l2.y;
 
-                if (!mbar_wait(&sm.o_full[w], use & 1, a.hdr, KID_ATTN_PREFILL)) { ok = false; break; }
+                if (!warp_wait(&sm.o_full[w], use & 1, a.hdr)) { ok = false; break; }
                 tc_fence_after();
                 const float inv_l = 1.f / l;
-                const size_t prow = ((((size_t(b) * a.N + t) * a.G + g) * kSlots + slot) * Hg + h);
-                uint4* dst = reinterpret_cast<uint4*>(a.part_o + prow * kHeadDim);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld32(tO + c * 32, v);
+                const float2 il = make_float2(inv_l, inv_l);
+                const size_t prow = ((((size_t(item.b) * a.N + t) * a.G + item.g) * kSlots + slot) * Hg + h);
+                // this warp's 32 rows hold 32 / Hg whole tokens; lane i stores token i's Hg rows
+                const int ntok_w = 32 / Hg;
+                const int src_lane = (lane * Hg) & 31;
+                const int tok_prow = __shfl_sync(0xffffffffu, int(prow - h), src_lane);   // row of head 0
+                const bool tok_valid = __shfl_sync(0xffffffffu, valid, src_lane) && lane < ntok_w;
+                bulk_wait_read0();                  // the previous tile's stores have read the staging
+                __syncwarp();
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    tmem_ld32(tO + half * 64, va);
+                    tmem_ld32(tO + half * 64 + 32, vb);
                     tmem_wait_ld();
-                    if (valid) {
+                    if (half == 1) {
+                        tc_fence_before();
+                        mbar_arrive(&sm.o_free[w]);                // O of this buffer fully read
+                    }
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv_l, __uint_as_float(v[8 * q + 1]) * inv_l);
-                            o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv_l, __uint_as_float(v[8 * q + 3]) * inv_l);
-                            o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv_l, __uint_as_float(v[8 * q + 5]) * inv_l);
-                            o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv_l, __uint_as_float(v[8 * q + 7]) * inv_l);
-                            __stcs(dst + c * 4 + q, o);
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t o[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int i0 = (8 * c + 2 * e2) & 31;
+                            const uint32_t x0 = c < 4 ? va[i0] : vb[i0];
+                            const uint32_t x1 = c < 4 ? va[i0 + 1] : vb[i0 + 1];
+                            const float2 y = fmul2(make_float2(__uint_as_float(x0), __uint_as_float(x1)), il);
+                            o[e2] = pack_bf16x2(y.x, y.y);
                         }
+                        *reinterpret_cast<uint4*>(stg + half * 4096 + sw128(lane, c)) = make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(&sm.o_free[w]);
+                fence_proxy_async();
+                __syncwarp();
+                if (tok_valid) {
+                    tma_store_2d_hint(&tmO, 0, tok_prow, stg + lane * Hg * 128, stream);
+                    tma_store_2d_hint(&tmO, 64, tok_prow, stg + 4096 + lane * Hg * 128, stream);
+                    bulk_commit();
+                }
                 if (valid) __stcs(a.part_lse + prow, ms + __log2f(l));
             }
-            if (!ok || sm.abort_flag) { sm.abort_flag = 1; break; }
+            if (__any_sync(0xffffffffu, sm.abort_flag != 0)) ok = false;
         }
+        bulk_wait0();                               // this warp's stores are complete before exit
+        __syncwarp();
+        if (!ok) sm.abort_flag = 1;
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -523,7 +721,7 @@ int num_sms() {
     return n[dev] > 0 ? n[dev] : 148;
 }
 
-void launch_attn_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, int64_t N,
+msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, const CUtensorMap& tmK, const CUtensorMap& tmV, int64_t N,
                             int B, int G, int Hg, const int32_t* sel, void* out, float* lse, void* ws,
                             cudaStream_t st) {
     const PrefillLayout L = prefill_layout(B, N, G, Hg);
@@ -559,6 +757,7 @@ void launch_attn_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, cons
         PrefillArgs a;
         a.N = N; a.G = G; a.Hg = Hg; a.Hq = G * Hg; a.tpt = L.tpt;
         a.n_items = nitems; a.items = items; a.list = list; a.part_lse = part_lse; a.part_o = part_o;
+        a.q = static_cast<const uint16_t*>(q);
         a.hdr = hdr;
         a.scale_log2 = 1.4426950408889634f / sqrtf(float(kHeadDim));
         const int smem = int(sizeof(KvSmem)) + 1024;
@@ -569,8 +768,13 @@ void launch_attn_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, cons
             cudaFuncSetAttribute(attn_kvmajor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             attr_set[dev] = true;
         }
+        CUtensorMap tmO, tmQ3;
+        msa_status_t st_map = make_tmap_bf16(&tmO, part_o, uint64_t(B) * N * G * kSlots * Hg, kHeadDim, 64, uint32_t(Hg));
+        if (st_map == MSA_OK && Hg >= 8) st_map = make_tmap_q_rows(&tmQ3, q, uint64_t(B) * N * G * Hg);
+        if (st_map != MSA_OK) return st_map;
+        const CUtensorMap& tmQ = Hg >= 8 ? tmQ3 : tmQ2;
         count_launch();
-        attn_kvmajor_kernel<<<num_sms(), kKvThreads, smem, st>>>(tmQ, tmK, tmV, a);
+        attn_kvmajor_kernel<<<num_sms(), kKvThreads, smem, st>>>(tmQ, tmK, tmV, tmO, a);
     }
     {
         const int64_t total = int64_t(B) * N * G * Hg * 4;
@@ -579,6 +783,6 @@ void launch_attn_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, cons
                                                                                   static_cast<uint16_t*>(out), lse,
                                                                                   total);
     }
+    return MSA_OK;
 }
-
 }  // namespace msa

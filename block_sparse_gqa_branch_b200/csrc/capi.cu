@@ -22,13 +22,26 @@ void launch_attn_decode(const CUtensorMap&, const CUtensorMap&, const void*, int
                         const int32_t*, int, int, int, void*, float*, void*, cudaStream_t);
 size_t decode_attn_ws_bytes(int, int, int);
 size_t prefill_attn_ws_bytes(int, int64_t, int, int);
-void launch_attn_prefill_tc(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, int64_t, int, int, int,
-                            const int32_t*, void*, float*, void*, cudaStream_t);
+msa_status_t launch_attn_prefill_tc(const void*, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, int64_t, int,
+                                    int, int, const int32_t*, void*, float*, void*, cudaStream_t);
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 thread_local int g_last_cuda_error = 0;
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda)
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -48,6 +61,40 @@ msa_status_t cuda_status() {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         g_last_cuda_error = int(e);
+        return MSA_ERR_CUDA;
+    }
+    return MSA_OK;
+}
+// bf16 matrix of `rows` x `cols` (row stride = cols), box = box_cols x box_rows, 128B swizzle
+msa_status_t make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                            uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return MSA_ERR_CUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error = int(r);
+        return MSA_ERR_CUDA;
+    }
+    return MSA_OK;
+}
+msa_status_t make_tmap_q_rows(CUtensorMap* m, const void* base, uint64_t rows) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return MSA_ERR_CUDA;
+    cuuint64_t dims[3] = {64, rows, 2};
+    cuuint64_t strides[2] = {uint64_t(kHeadDim) * 2, 128};      // bytes: next row, next d half
+    cuuint32_t box[3] = {64, 8, 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error = int(r);
         return MSA_ERR_CUDA;
     }
     return MSA_OK;
@@ -87,38 +134,6 @@ size_t ws_size(const msa_shape_t* s, int32_t op, int64_t n) {
         case MSA_OP_ATTN_DECODE: return decode_attn_ws_bytes(s->batch, s->n_kv_groups, hg);
         default: return 0;
     }
-}
-
-// ---------------------------------------------------------------- TMA descriptors
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-// bf16 matrix of `rows` x `cols` (row stride = cols), box = box_cols x box_rows, 128B swizzle
-msa_status_t make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                            uint32_t box_rows) {
-    auto fn = encode_fn();
-    if (fn == nullptr) return MSA_ERR_CUDA;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-        g_last_cuda_error = int(r);
-        return MSA_ERR_CUDA;
-    }
-    return MSA_OK;
 }
 
 }  // namespace
@@ -206,8 +221,8 @@ msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const void* q, co
     MSA_TRY(make_tmap_bf16(&tmQ, q, uint64_t(B) * n_tokens * Hq, kHeadDim, 64, uint32_t(hg)));
     MSA_TRY(make_tmap_bf16(&tmK, k, uint64_t(B) * G * n_tokens, kHeadDim, 64, 128));
     MSA_TRY(make_tmap_bf16(&tmV, v, uint64_t(B) * G * n_tokens, kHeadDim, 64, 128));
-    launch_attn_prefill_tc(tmQ, tmK, tmV, n_tokens, B, G, hg, sel, out, lse, workspace,
-                           reinterpret_cast<cudaStream_t>(stream));
+    MSA_TRY(launch_attn_prefill_tc(q, tmQ, tmK, tmV, n_tokens, B, G, hg, sel, out, lse, workspace,
+                                   reinterpret_cast<cudaStream_t>(stream)));
     return cuda_status();
 }
 
