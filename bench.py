@@ -6,7 +6,7 @@ One step = one pass of the whole hot path on synthetic inputs already resident i
     exp-free top-16 selection, main-branch sparse attention), and
   * one decode step of a batch of 16 sequences at 131,072 cached tokens (append + pooled-key
     update, selection, split-KV attention), replayed from a CUDA graph.
-L2 is flushed (256 MiB write) before every timed step, outside the events.
+L2 is flushed (256 MiB write, then 256 MiB read) before every timed step, outside the events.
 
 Printed value: prefill tokens/s over all ranks (131,072 x N / slowest rank's prefill time).
 The same line carries the decode step latency, the index-select and main-branch split, the
@@ -240,7 +240,7 @@ def config_block(wp, wd):
                         "head_dim": wp.d, "index_dim": wp.dI, "block": wp.Bk, "top_k": wp.topk},
             "decode": {"batch": wd.B, "ctx_len": wd.ctx[0], "q_heads": wd.Hq, "kv_groups": wd.G,
                        "head_dim": wd.d, "index_dim": wd.dI, "block": wd.Bk, "top_k": wd.topk},
-            "l2": "flushed before every timed step (256 MiB write)",
+            "l2": "flushed before every timed step and before the decode half (256 MiB write, then 256 MiB read)",
             "parallelism": "replicas (one independent problem per GPU)"}
 
 
@@ -316,7 +316,15 @@ def run_ours(args):
     pbufs = pipeline.prefill_buffers(wp.B, wp.N, wp.Hq, wp.G, dev)
     ds = build_decode_state(wd, dev) if do_decode else None
     dbufs = pipeline.decode_buffers(wd.B, wd.Hq, wd.G, max(wd.ctx), dev) if do_decode else None
+    # L2 flush between timed steps: write a buffer larger than L2 (126 MB), then read another
+    # one, so that the written lines are written back before the timed region (a write alone
+    # leaves ~126 MB of dirty lines whose write-back would land inside the next step)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        flush_rd.sum()
     stream = torch.cuda.current_stream()
 
     def decode_call():
@@ -340,7 +348,7 @@ def run_ours(args):
     launches0 = msa.msa_kernel_launches()
 
     def one_step(record: bool):
-        flush.zero_()
+        flush_l2()
         e0, e1, e2, e3, e4 = ev(), ev(), ev(), ev(), ev()
         e0.record(stream)
         if do_prefill:
@@ -349,7 +357,7 @@ def run_ours(args):
         if do_prefill:
             pipeline.prefill_main(x["q"], x["k"], x["v"], pbufs)
         e2.record(stream)
-        flush.zero_()
+        flush_l2()
         e3.record(stream)
         if do_decode:
             graph.replay()
@@ -413,7 +421,7 @@ def run_ours(args):
         d2h = host_out.numel() * host_out.element_size() + dhost_out.numel() * dhost_out.element_size()
         times = []
         for s in range(max(1, args.warmup // 2) + args.steps):
-            flush.zero_()
+            flush_l2()
             torch.cuda.synchronize()
             e0, e1 = ev(), ev()
             e0.record(stream)

@@ -18,8 +18,8 @@ void launch_select_prefill_simt(const void*, int, int, int64_t, const float*, in
 void launch_select_decode(const void*, const int32_t*, int64_t, int, int, const float*, int64_t, int32_t*,
                           void*, cudaStream_t);
 size_t decode_select_ws_bytes(int, int, int64_t);
-void launch_attn_decode(const CUtensorMap&, const CUtensorMap&, const void*, int64_t, const int32_t*, int64_t,
-                        const int32_t*, int, int, int, void*, float*, void*, cudaStream_t);
+msa_status_t launch_attn_decode(const void*, const void*, const void*, int64_t, const int32_t*, int64_t, const int32_t*,
+                                int, int, int, void*, float*, void*, cudaStream_t);
 size_t decode_attn_ws_bytes(int, int, int);
 size_t prefill_attn_ws_bytes(int, int64_t, int, int);
 msa_status_t launch_attn_prefill_tc(const void*, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, int64_t, int,
@@ -261,12 +261,8 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const void* q, con
     MSA_REQ(int64_t(B) * G * l_cap + kBlock < (int64_t(1) << 31), MSA_ERR_UNSUPPORTED);
     const size_t need = ws_size(shape, MSA_OP_ATTN_DECODE, max_pos);
     MSA_REQ(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need, MSA_ERR_WORKSPACE);
-    CUtensorMap tmK, tmV;
-    const uint64_t rows = uint64_t(B) * G * uint64_t(l_cap);
-    MSA_TRY(make_tmap_bf16(&tmK, k_cache, rows, kHeadDim, 64, 32));
-    MSA_TRY(make_tmap_bf16(&tmV, v_cache, rows, kHeadDim, 64, 32));
-    launch_attn_decode(tmK, tmV, q, l_cap, q_pos, max_pos, sel, B, G, shape->n_q_heads / G, out, lse, workspace,
-                       reinterpret_cast<cudaStream_t>(stream));
+    MSA_TRY(launch_attn_decode(k_cache, v_cache, q, l_cap, q_pos, max_pos, sel, B, G, shape->n_q_heads / G, out, lse,
+                               workspace, reinterpret_cast<cudaStream_t>(stream)));
     return cuda_status();
 }
 

@@ -92,6 +92,7 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t* __restrict_
                                                      float* __restrict__ tail_sum,
                                                      float* __restrict__ pooled, int64_t nb_cap,
                                                      WsHeader* hdr) {
+    grid_dep_launch();                 // the selection may start: it does not read what this writes
     const int b = blockIdx.x;
     const int pos = ctx_len[b];
     const int64_t j = pos / kBlock;

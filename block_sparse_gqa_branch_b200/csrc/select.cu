@@ -129,50 +129,67 @@ void launch_select_prefill_simt(const void* q_idx, int B, int G, int64_t N, cons
 // the CTA that arrives last for a (sequence, group) merges the sorted lists. The arrival
 // counter wraps to zero by itself (atomicInc), so the workspace is ready for the next call.
 constexpr int kDecChunk = 128;
+constexpr int kDecSmemChunks = 64;    // merges of up to 64 chunks run from shared memory
 
 __global__ void __launch_bounds__(kDecChunk) select_decode_kernel(
     const uint16_t* __restrict__ q_idx, const int32_t* __restrict__ q_pos, int64_t max_pos, int G,
     const float* __restrict__ pooled, int64_t nb_cap, int32_t* __restrict__ sel,
     unsigned long long* __restrict__ cand, unsigned int* __restrict__ ctr, int nchunk_max, WsHeader* hdr) {
-    __shared__ float qs[kIndexDim];
+    __shared__ __align__(16) float qs[kIndexDim];
+    __shared__ float sc[kDecChunk];
     __shared__ unsigned long long keys[kDecChunk];
+    __shared__ unsigned long long lst[kDecSmemChunks * kKeep];
     __shared__ int heads[1024];
     __shared__ int last;
+    grid_dep_launch();                 // the attention kernel may start its prologue
     const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int bg = b * G + g;
     const int pos = q_pos[b];
     if (pos < 0 || pos > max_pos || int64_t(pos / kBlock) > nb_cap) {
         if (ch == 0 && threadIdx.x == 0) record_error(hdr, MSA_ERR_DEVICE_BOUNDS, KID_SELECT_DECODE, bg, 0, pos);
+        grid_dep_wait();
         return;
     }
     const int c = pos / kBlock;
     int32_t* out = sel + size_t(bg) * kTopK;
     if (c + 1 <= kTopK) {
         if (ch == 0 && threadIdx.x == 0) write_all_blocks(out, c);
+        grid_dep_wait();
         return;
     }
     const int nch = (c + kDecChunk - 1) / kDecChunk;
-    if (ch >= nch) return;
+    if (ch >= nch) { grid_dep_wait(); return; }
 
     if (threadIdx.x < kIndexDim) qs[threadIdx.x] = bf16_to_f32(q_idx[size_t(bg) * kIndexDim + threadIdx.x]);
     __syncthreads();
+    // Coalesced scoring: each warp instruction reads two whole 256-byte candidate rows (lane l
+    // takes float4 (l mod 16) of row 2i + l / 16); 16-lane shuffles finish each dot product.
+    const int ln = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int part = ln & 15, half = ln >> 4;
+    const float4 qv = *reinterpret_cast<const float4*>(&qs[4 * part]);
+    const float4* rows = reinterpret_cast<const float4*>(pooled + (size_t(bg) * nb_cap + size_t(ch) * kDecChunk) * kIndexDim);
+    const int nrow = min(kDecChunk, c - ch * kDecChunk);      // candidates in this chunk
+    float4 v[kDecChunk / 4 / 2];                                 // this warp's 32 rows, 2 per load
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int r = wid * 32 + 2 * i + half;
+        v[i] = r < nrow ? __ldg(rows + size_t(r) * (kIndexDim / 4) + part) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        // fixed order: x, y, z, w, then a butterfly over the 16 lanes of this half-warp
+        float d = fmaf(qv.x, v[i].x, 0.f);
+        d = fmaf(qv.y, v[i].y, d);
+        d = fmaf(qv.z, v[i].z, d);
+        d = fmaf(qv.w, v[i].w, d);
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+        if (part == 0) sc[wid * 32 + 2 * i + half] = d;
+    }
+    __syncthreads();
     const int j = ch * kDecChunk + threadIdx.x;
     unsigned long long key = 0ull;
-    if (j < c) {
-        const float4* row = reinterpret_cast<const float4*>(pooled + (size_t(bg) * nb_cap + j) * kIndexDim);
-        float4 v[kIndexDim / 4];
-#pragma unroll
-        for (int i = 0; i < kIndexDim / 4; ++i) v[i] = __ldg(row + i);
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < kIndexDim / 4; ++i) {
-            acc = fmaf(qs[4 * i + 0], v[i].x, acc);
-            acc = fmaf(qs[4 * i + 1], v[i].y, acc);
-            acc = fmaf(qs[4 * i + 2], v[i].z, acc);
-            acc = fmaf(qs[4 * i + 3], v[i].w, acc);
-        }
-        key = sel_key(acc, j);
-    }
+    if (j < c) key = sel_key(sc[threadIdx.x], j);
     keys[threadIdx.x] = key;
     __syncthreads();
     unsigned long long* mine = cand + (size_t(bg) * nchunk_max + ch) * kKeep;
@@ -187,12 +204,22 @@ __global__ void __launch_bounds__(kDecChunk) select_decode_kernel(
     __syncthreads();
     if (threadIdx.x == 0) last = (atomicInc(ctr + bg, unsigned(nch - 1)) == unsigned(nch - 1));
     __syncthreads();
-    if (!last || threadIdx.x >= 32) return;
+    // The selection does not read what the preceding append writes (only fully-past pooled
+    // rows), so it waits for that kernel only before finishing: the attention kernel that waits
+    // for this grid then also sees the appended token.
+    grid_dep_wait();
+    if (!last) return;
     __threadfence();
-
-    // warp 0 merges the nch sorted lists: 15 rounds of "best list head"
+    // stage the nch sorted lists in shared memory with one coalesced pass (global fallback for
+    // more than kDecSmemChunks chunks), then warp 0 merges: 15 rounds of "best list head"
+    const unsigned long long* glists = cand + size_t(bg) * nchunk_max * kKeep;
+    const bool in_smem = nch <= kDecSmemChunks;
+    if (in_smem)
+        for (int i = threadIdx.x; i < nch * kKeep; i += kDecChunk) lst[i] = __ldcg(glists + i);
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
     const int lane = threadIdx.x;
-    const unsigned long long* lists = cand + size_t(bg) * nchunk_max * kKeep;
+    const unsigned long long* lists = in_smem ? lst : glists;
     for (int l = lane; l < nch; l += 32) heads[l] = 0;
     __syncwarp();
     int my_id = c;                                   // lane 15 keeps the diagonal block
@@ -202,7 +229,7 @@ __global__ void __launch_bounds__(kDecChunk) select_decode_kernel(
         for (int l = lane; l < nch; l += 32) {
             const int h = heads[l];
             if (h < kKeep) {
-                const unsigned long long k = __ldcg(lists + size_t(l) * kKeep + h);
+                const unsigned long long k = in_smem ? lists[size_t(l) * kKeep + h] : __ldcg(lists + size_t(l) * kKeep + h);
                 if (k > bk) { bk = k; bl = l; }
             }
         }
@@ -248,10 +275,18 @@ void launch_select_decode(const void* q_idx, const int32_t* q_pos, int64_t max_p
     unsigned long long* cand = reinterpret_cast<unsigned long long*>(
         p + sizeof(WsHeader) + (nbg * sizeof(unsigned int) + 255) / 256 * 256);
     const int nchunk = decode_select_chunks(max_pos);
-    dim3 grid(static_cast<unsigned>(nchunk), static_cast<unsigned>(G), static_cast<unsigned>(B));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(nchunk), static_cast<unsigned>(G), static_cast<unsigned>(B));
+    cfg.blockDim = dim3(kDecChunk);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap with the append's tail
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     count_launch();
-    select_decode_kernel<<<grid, kDecChunk, 0, st>>>(static_cast<const uint16_t*>(q_idx), q_pos, max_pos,
-                                                     G, pooled, nb_cap, sel, cand, ctr, nchunk, hdr);
+    cudaLaunchKernelEx(&cfg, select_decode_kernel, static_cast<const uint16_t*>(q_idx), q_pos, max_pos, G, pooled,
+                       nb_cap, sel, cand, ctr, nchunk, hdr);
 }
 
 }  // namespace msa
