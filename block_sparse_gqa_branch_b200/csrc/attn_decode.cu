@@ -9,25 +9,30 @@
 //
 // Design (HBM-bound, 8 FLOP per byte read). The work items (sequence, group, selected block)
 // are laid out in order and cut into one contiguous range per CTA (one persistent CTA per SM),
-// so every CTA streams the same number of 64 KB K+V blocks. A loader warp walks the range and
-// streams each item's K and V block -- two contiguous 32 KB ranges of the head-major cache --
-// and the group's query rows with TMA into a 3-deep ring of stages, so several items' loads
-// are in flight while the 8 compute warps work on another. For an item, warp w scores keys
-// 16w..16w+15 for all Hg heads with warp MMAs; the row max is combined across warps in shared
-// memory, P goes to shared memory as bf16, and warp w then accumulates output columns
-// 16w..16w+15 over all 128 keys with an online softmax that runs across the items of one
-// (sequence, group). A (sequence, group) whose items all lie in one CTA is written out
-// directly; otherwise each CTA leaves an unnormalised partial (max, sum, o) and the last to
-// finish merges them.
+// so every CTA streams the same number of 64 KB K+V blocks. Warp roles:
+//   * loader (warp 8): streams each item's K and V block -- two contiguous 32 KB ranges of the
+//     head-major cache -- and the group's query rows with TMA into a 3-deep ring of stages;
+//   * compute (warps 0-7): warp w owns keys 16w..16w+15 of every block. It scores them for all
+//     Hg heads with warp MMAs, turns them into probabilities in registers (the accumulator
+//     layout of S is the A-operand layout of P) and accumulates all 128 output columns with
+//     its own online softmax, so the warps never wait for one another. At the last item of a
+//     group in this CTA each warp parks its state in its own 16 rows of the stage;
+//   * epilogue (warp 9): folds the 8 parked states by log-sum-exp, releases the stage, and
+//     either writes the output (the group lies in this CTA) or deals with the other CTAs that
+//     hold parts of the group: if all of them are in it merges their partials (max, sum, o)
+//     into its registers, otherwise it leaves its own partial for the last one to arrive.
+//     None of this global-memory traffic stalls the compute warps.
 #include "msa_common.cuh"
 
 namespace msa {
 
-constexpr int kDecWarps = 8;           // compute warps; warp 8 loads
-constexpr int kDecThreads = (kDecWarps + 1) * 32;
+constexpr int kDecWarps = 8;           // compute warps; warp 8 loads, warp 9 finishes groups
+constexpr int kDecLoader = kDecWarps, kDecEpi = kDecWarps + 1;
+constexpr int kDecThreads = (kDecWarps + 2) * 32;
 constexpr int kDecStages = 3;
 constexpr int kDecDiagRows = 32;       // row granularity of the diagonal block's loads
-constexpr int kPRow = 136;             // bf16 elements per P / Q row in shared memory (padded)
+constexpr int kQRow = 136;             // bf16 elements per query row in shared memory (padded)
+constexpr int kRowCache = 8;           // selection rows the loader fetches per round trip
 
 // A partial is [max: Hg][sum: Hg][pad to 4 floats][o: Hg x 128] fp32; o is 16-byte aligned.
 __host__ __device__ inline int dec_part_ooff(int Hg) { return (2 * Hg + 3) / 4 * 4; }
@@ -45,15 +50,18 @@ struct DecMaps {
 
 struct __align__(1024) DecSmem {
     uint8_t kv[kDecStages][2][32768];           // [stage][K, V][d half][128 rows][128 B]
-    uint16_t q[kDecStages][kMaxHg][kPRow];      // the item's query heads (rows padded)
-    uint16_t p[kMaxHg][kPRow];                  // probabilities of the current item, bf16
-    float red_m[kDecWarps][kMaxHg], red_l[kDecWarps][kMaxHg];
-    float wts[kTopK][kMaxHg], ls[kTopK][kMaxHg], mrg_m[kMaxHg], mrg_l[kMaxHg];
+    uint16_t q[kDecStages][kMaxHg][kQRow];      // the item's query heads (rows padded)
+    float pm[kDecStages][kDecWarps][kMaxHg];    // parked warp states: max and sum per head
+    float pl[kDecStages][kDecWarps][kMaxHg];
+    float4 ot[16][32];                          // epilogue: other CTAs' parts of its last group
+    float om[kMaxHg], ol[kMaxHg];
     uint64_t full_k[kDecStages], full_v[kDecStages], empty[kDecStages];
+    uint64_t parked[kDecStages];                // 8 warp states parked (queue of group ends)
     int meta_bg[kDecStages], meta_ntok[kDecStages], meta_fin[kDecStages], meta_nfrag[kDecStages],
         meta_frag[kDecStages];
-    int ld_row[kTopK];                          // loader: selection row of the current group
-    int is_last;
+    int park_stage[kDecStages];                 // stage holding the parked states (-1 = end)
+    int row_sel[kRowCache][kTopK];              // loader: selection rows and positions
+    int row_pos[kRowCache];
 };
 
 struct DecArgs {
@@ -68,33 +76,114 @@ struct DecArgs {
     unsigned int* ctr;
     WsHeader* hdr;
     float scale_log2;
+    double inv_grid, inv_items;                 // 1 / gridDim.x, 1 / (B G 16)
 };
 
-// barrier among the compute warps only (the loader warp never joins it)
-__device__ __forceinline__ void compute_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32) : "memory");
+// first item of CTA c when n items are cut into `grid` contiguous ranges: floor(c * n / grid)
+__device__ __forceinline__ int range_begin(int c, int n, int grid, double inv_grid) {
+    const long long t = (long long)c * n;
+    int b = int(double(t) * inv_grid);
+    while ((long long)(b + 1) * grid <= t) ++b;
+    while ((long long)b * grid > t) --b;
+    return b;
 }
 
-// the same barrier, returning whether any compute thread passed a nonzero flag
-__device__ __forceinline__ bool compute_sync_or(bool flag) {
-    uint32_t r;
-    asm volatile(
-        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}"
-        : "=r"(r)
-        : "r"(uint32_t(flag)), "n"(kDecWarps * 32)
-        : "memory");
-    return r != 0;
+// the CTA whose range holds item k: the largest c with c * n < (k + 1) * grid
+__device__ __forceinline__ int range_owner(int k, int n, int grid, double inv_n) {
+    const long long t = (long long)(k + 1) * grid - 1;
+    int c = int(double(t) * inv_n);
+    while ((long long)(c + 1) * n <= t) ++c;
+    while ((long long)c * n > t) --c;
+    return c < grid - 1 ? c : grid - 1;
 }
 
-// first item of CTA c when n items are cut into `grid` contiguous ranges
-__device__ __forceinline__ int64_t range_begin(int c, int64_t n, int grid) { return int64_t(c) * n / grid; }
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 
-// the CTA whose range holds item k
-__device__ __forceinline__ int range_owner(int64_t k, int64_t n, int grid) {
-    int c = int(k * grid / n);
-    while (c + 1 < grid && range_begin(c + 1, n, grid) <= k) ++c;
-    while (c > 0 && range_begin(c, n, grid) > k) --c;
-    return c;
+// raise the transaction count of the current phase without arriving
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
+}
+
+// bounded wait by every lane of a warp, with one outcome for the whole warp
+__device__ __forceinline__ bool warp_wait_all(uint64_t* bar, uint32_t parity, WsHeader* hdr) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, hdr, KID_ATTN_DECODE));
+}
+
+// log-sum-exp weights of two states with maxima m (own) and mo (other), log2 units
+__device__ __forceinline__ void lse_weights(float m, float mo, float& mn, float& wa, float& wb) {
+    mn = fmaxf(m, mo);
+    wa = m == -INFINITY ? 0.f : fast_exp2(m - mn);
+    wb = mo == -INFINITY ? 0.f : fast_exp2(mo - mn);
+}
+
+// A warp's part of an (unnormalised) attention state, in the accumulator layout of m16n8:
+// rows (heads) gq and gq + 8, columns 8 nt + 2 tq + {0, 1}.
+struct WarpState {
+    float o[16][4];
+    float m0, m1;        // maxima of rows gq, gq + 8 (log2 units)
+    float l0, l1;        // sums
+};
+
+// Accumulators of a lane in groups of four: group g < 8 holds row gq, columns 16 g + 2 tq +
+// {0, 1, 8, 9} (o[2g][0..1], o[2g+1][0..1]); group g >= 8 the same for row gq + 8.
+__device__ __forceinline__ float4 acc_group(const WarpState& st, int g) {
+    const int e = (g >> 3) << 1, nt = (g & 7) << 1;
+    return make_float4(st.o[nt][e], st.o[nt][e + 1], st.o[nt + 1][e], st.o[nt + 1][e + 1]);
+}
+__device__ __forceinline__ void set_acc_group(WarpState& st, int g, float4 x) {
+    const int e = (g >> 3) << 1, nt = (g & 7) << 1;
+    st.o[nt][e] = x.x; st.o[nt][e + 1] = x.y; st.o[nt + 1][e] = x.z; st.o[nt + 1][e + 1] = x.w;
+}
+
+// Parked state of warp w in stage s: group g of lane l sits in the warp's own K rows (g < 8)
+// or V rows (g >= 8), 512 B (32 lanes x 16 B) per group.
+__device__ __forceinline__ float4* park_addr(DecSmem& sm, int s, int w, int g, int lane) {
+    uint8_t* chunk = sm.kv[s][g >> 3] + ((g >> 2) & 1) * 16384 + w * 2048 + (g & 3) * 512;
+    return reinterpret_cast<float4*>(chunk) + lane;
+}
+
+// Fold the partial of another CTA (max, sum, o of rows gq, gq + 8) into st.
+__device__ __forceinline__ void merge_partial(WarpState& st, const float* pf, int Hg, int ooff, int gq, int tq) {
+    float wa0 = 1.f, wb0 = 0.f, wa1 = 1.f, wb1 = 0.f, mn;
+    if (gq < Hg) {
+        lse_weights(st.m0, __ldcg(pf + gq), mn, wa0, wb0);
+        st.l0 = st.l0 * wa0 + __ldcg(pf + Hg + gq) * wb0;
+        st.m0 = mn;
+    }
+    if (gq + 8 < Hg) {
+        lse_weights(st.m1, __ldcg(pf + gq + 8), mn, wa1, wb1);
+        st.l1 = st.l1 * wa1 + __ldcg(pf + Hg + gq + 8) * wb1;
+        st.m1 = mn;
+    }
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+        const int col = nt * 8 + 2 * tq;
+        if (gq < Hg) {
+            const float2 x = __ldcg(reinterpret_cast<const float2*>(pf + ooff + gq * kHeadDim + col));
+            st.o[nt][0] = st.o[nt][0] * wa0 + x.x * wb0;
+            st.o[nt][1] = st.o[nt][1] * wa0 + x.y * wb0;
+        }
+        if (gq + 8 < Hg) {
+            const float2 x = __ldcg(reinterpret_cast<const float2*>(pf + ooff + (gq + 8) * kHeadDim + col));
+            st.o[nt][2] = st.o[nt][2] * wa1 + x.x * wb1;
+            st.o[nt][3] = st.o[nt][3] * wa1 + x.y * wb1;
+        }
+    }
+}
+
+__device__ __forceinline__ void clear_state(WarpState& st) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) st.o[i][0] = st.o[i][1] = st.o[i][2] = st.o[i][3] = 0.f;
+    st.m0 = st.m1 = -INFINITY;
+    st.l0 = st.l1 = 0.f;
 }
 
 __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __grid_constant__ DecMaps maps,
@@ -104,134 +193,333 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gq = lane >> 2, tq = lane & 3;
     const int Hg = a.Hg, G = a.G;
-    const int stride = dec_part_stride(Hg), ooff = dec_part_ooff(Hg);
+    const int n_items = a.B * G * kTopK;
 
     if (tid == 0) {
         for (int s = 0; s < kDecStages; ++s) {
             mbar_init(&sm.full_k[s], 1);
             mbar_init(&sm.full_v[s], 1);
             mbar_init(&sm.empty[s], kDecWarps);
+            mbar_init(&sm.parked[s], kDecWarps);
         }
         fence_barrier_init();
     }
-    for (int i = tid; i < kMaxHg * kPRow; i += kDecThreads) {      // rows >= Hg stay 0
-        (&sm.p[0][0])[i] = 0;
-        for (int s = 0; s < kDecStages; ++s) (&sm.q[s][0][0])[i] = 0;
-    }
+    for (int i = tid; i < kDecStages * kMaxHg * kQRow; i += kDecThreads) (&sm.q[0][0][0])[i] = 0;   // rows >= Hg stay 0
     __syncthreads();
     grid_dep_wait();                   // the selection and the appended token are ready from here on
 
-    if (warp == kDecWarps) {
-        // ---------------------------------------------------------------- loader warp (lane 0)
-        // Streams the items of this CTA's range into the ring, skipping empty slots, and ends
-        // with an end marker (bg = -1).
-        if (lane != 0) return;
-        const int64_t n_items = int64_t(a.B) * G * kTopK;
-        const int64_t kend = range_begin(blockIdx.x + 1, n_items, gridDim.x);
+    if (warp == kDecLoader) {
+        // ---------------------------------------------------------------- loader warp
+        // Streams the items of this CTA's range into the ring (lane 0 issues the copies),
+        // skipping empty slots, and ends with an end marker (bg = -1).
+        const int kbeg = range_begin(blockIdx.x, n_items, gridDim.x, a.inv_grid);
+        const int kend = range_begin(blockIdx.x + 1, n_items, gridDim.x, a.inv_grid);
         const uint64_t pol = l2_evict_first();               // K and V are read once
         const uint32_t qrow = kHeadDim * 2u;
+        int cache0 = 0, cachen = 0;                           // groups [cache0, cache0 + cachen) fetched
         int cur_bg = -1, pos = 0, nsel = 0, nfrag = 1, frag = 0;
+        bool need_frag = false;
         int n = 0;
         bool ok = true;
-        for (int64_t k = range_begin(blockIdx.x, n_items, gridDim.x); k < kend; ++k) {
-            const int bg = int(k / kTopK), slot = int(k % kTopK);
+        for (int k = kbeg; k < kend; ++k) {
+            const int bg = k / kTopK, slot = k % kTopK;
             if (bg != cur_bg) {
                 cur_bg = bg;
-                nsel = 0;
-                pos = a.q_pos[bg / G];
-                if (pos < 0 || pos > a.max_pos || pos >= a.l_cap) {
-                    if (slot == 0) record_error(a.hdr, MSA_ERR_DEVICE_BOUNDS, KID_ATTN_DECODE, bg, 0, pos);
-                } else {
-                    const int4* srow = reinterpret_cast<const int4*>(a.sel + size_t(bg) * kTopK);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int4 v = __ldcg(srow + q4);
-                        sm.ld_row[4 * q4] = v.x; sm.ld_row[4 * q4 + 1] = v.y;
-                        sm.ld_row[4 * q4 + 2] = v.z; sm.ld_row[4 * q4 + 3] = v.w;
-                        nsel += (v.x >= 0) + (v.y >= 0) + (v.z >= 0) + (v.w >= 0);
+                if (bg >= cache0 + cachen) {                  // fetch the next rows in one round trip
+                    const int left = (kend - 1) / kTopK - bg + 1;
+                    cache0 = bg;
+                    cachen = left < kRowCache ? left : kRowCache;
+                    __syncwarp();
+                    if (lane < cachen * 4) {
+                        const int4 v = __ldcg(reinterpret_cast<const int4*>(a.sel + size_t(bg) * kTopK) + lane);
+                        int* d = &sm.row_sel[lane >> 2][(lane & 3) * 4];
+                        d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
                     }
-                    if (nsel > 0) {
-                        const int c0 = range_owner(int64_t(bg) * kTopK, n_items, gridDim.x);
-                        const int c1 = range_owner(int64_t(bg) * kTopK + nsel - 1, n_items, gridDim.x);
-                        nfrag = c1 - c0 + 1;
-                        frag = int(blockIdx.x) - c0;
-                    }
+                    if (lane < cachen) sm.row_pos[lane] = __ldcg(a.q_pos + (bg + lane) / G);
+                    __syncwarp();
                 }
+                const int r = bg - cache0;
+                pos = sm.row_pos[r];
+                nsel = 0;
+#pragma unroll
+                for (int i = 0; i < kTopK; ++i) nsel += sm.row_sel[r][i] >= 0;
+                if (pos < 0 || pos > a.max_pos || pos >= a.l_cap) {
+                    if (lane == 0 && slot == 0) record_error(a.hdr, MSA_ERR_DEVICE_BOUNDS, KID_ATTN_DECODE, bg, 0, pos);
+                    nsel = 0;
+                }
+                need_frag = nsel > 0;
             }
             if (slot >= nsel) {                               // the row's tail is empty
-                k = int64_t(bg + 1) * kTopK - 1;
+                k = bg * kTopK + kTopK - 1;
                 continue;
             }
             const int stage = n % kDecStages;
-            if (n >= kDecStages && !mbar_wait(&sm.empty[stage], ((n / kDecStages) - 1) & 1, a.hdr, KID_ATTN_DECODE)) {
-                ok = false;
-                break;
+            if (n >= kDecStages) {
+                bool w = true;
+                if (lane == 0) w = mbar_wait(&sm.empty[stage], ((n / kDecStages) - 1) & 1, a.hdr, KID_ATTN_DECODE);
+                if (!__shfl_sync(0xffffffffu, w, 0)) {
+                    ok = false;
+                    break;
+                }
             }
-            const int c = pos / kBlock;
-            int j = sm.ld_row[slot];
-            if (j > c || j < 0) {
-                record_error(a.hdr, MSA_ERR_DEVICE_BOUNDS, KID_ATTN_DECODE, bg, slot, j);
-                j = -1;
-            }
-            const int ntok = j < 0 ? 0 : (j == c ? pos - c * kBlock + 1 : kBlock);
-            sm.meta_bg[stage] = bg;
-            sm.meta_ntok[stage] = ntok;
-            sm.meta_fin[stage] = (slot == nsel - 1 || k + 1 == kend);
-            sm.meta_nfrag[stage] = nfrag;
-            sm.meta_frag[stage] = frag;
-            const bool full = ntok == kBlock;
-            const int nload = full ? kBlock : (ntok + kDecDiagRows - 1) / kDecDiagRows * kDecDiagRows;
-            mbar_arrive_expect_tx(&sm.full_k[stage], uint32_t(nload) * 256u + uint32_t(Hg) * qrow);
-            mbar_arrive_expect_tx(&sm.full_v[stage], uint32_t(nload) * 256u);
-            const uint16_t* qg = a.q + size_t(bg) * Hg * kHeadDim;
-            for (int h = 0; h < Hg; ++h) bulk_load(sm.q[stage][h], qg + h * kHeadDim, qrow, &sm.full_k[stage]);
-            const int row0 = int(int64_t(bg) * a.l_cap + int64_t(j < 0 ? 0 : j) * kBlock);
-            uint8_t* ks = sm.kv[stage][0];
-            uint8_t* vs = sm.kv[stage][1];
-            if (full) {
-                for (int h = 0; h < 2; ++h)
-                    tma_load_2d_hint(ks + h * 16384, &maps.k128, h * 64, row0, &sm.full_k[stage], pol);
-                for (int h = 0; h < 2; ++h)
-                    tma_load_2d_hint(vs + h * 16384, &maps.v128, h * 64, row0, &sm.full_v[stage], pol);
-            } else {
-                for (int r0 = 0; r0 < nload; r0 += kDecDiagRows)
+            // The copies go out first; the item's description and the arrivals that complete the
+            // stage follow (the phase cannot complete before those arrivals).
+            int ntok = 0;
+            if (lane == 0) {
+                const int c = pos / kBlock;
+                int j = sm.row_sel[bg - cache0][slot];
+                if (j > c || j < 0) {
+                    record_error(a.hdr, MSA_ERR_DEVICE_BOUNDS, KID_ATTN_DECODE, bg, slot, j);
+                    j = -1;
+                }
+                ntok = j < 0 ? 0 : (j == c ? pos - c * kBlock + 1 : kBlock);
+                const bool full = ntok == kBlock;
+                const int nload = full ? kBlock : (ntok + kDecDiagRows - 1) / kDecDiagRows * kDecDiagRows;
+                mbar_expect_tx(&sm.full_k[stage], uint32_t(nload) * 256u + uint32_t(Hg) * qrow);
+                mbar_expect_tx(&sm.full_v[stage], uint32_t(nload) * 256u);
+                const int row0 = int(int64_t(bg) * a.l_cap + int64_t(j < 0 ? 0 : j) * kBlock);
+                uint8_t* ks = sm.kv[stage][0];
+                uint8_t* vs = sm.kv[stage][1];
+                if (full) {
                     for (int h = 0; h < 2; ++h)
-                        tma_load_2d_hint(ks + h * 16384 + r0 * 128, &maps.k32, h * 64, row0 + r0, &sm.full_k[stage], pol);
-                for (int r0 = 0; r0 < nload; r0 += kDecDiagRows)
+                        tma_load_2d_hint(ks + h * 16384, &maps.k128, h * 64, row0, &sm.full_k[stage], pol);
+                } else {
+                    for (int r0 = 0; r0 < nload; r0 += kDecDiagRows)
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_2d_hint(ks + h * 16384 + r0 * 128, &maps.k32, h * 64, row0 + r0, &sm.full_k[stage], pol);
+                }
+                const uint16_t* qg = a.q + size_t(bg) * Hg * kHeadDim;
+                for (int h = 0; h < Hg; ++h) bulk_load(sm.q[stage][h], qg + h * kHeadDim, qrow, &sm.full_k[stage]);
+                if (full) {
                     for (int h = 0; h < 2; ++h)
-                        tma_load_2d_hint(vs + h * 16384 + r0 * 128, &maps.v32, h * 64, row0 + r0, &sm.full_v[stage], pol);
+                        tma_load_2d_hint(vs + h * 16384, &maps.v128, h * 64, row0, &sm.full_v[stage], pol);
+                } else {
+                    for (int r0 = 0; r0 < nload; r0 += kDecDiagRows)
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_2d_hint(vs + h * 16384 + r0 * 128, &maps.v32, h * 64, row0 + r0, &sm.full_v[stage], pol);
+                }
             }
+            if (need_frag) {                                  // parts of this group in other CTAs
+                const int c0 = range_owner(bg * kTopK, n_items, gridDim.x, a.inv_items);
+                const int c1 = range_owner(bg * kTopK + nsel - 1, n_items, gridDim.x, a.inv_items);
+                nfrag = c1 - c0 + 1;
+                frag = int(blockIdx.x) - c0;
+                need_frag = false;
+            }
+            if (lane == 0) {
+                sm.meta_bg[stage] = bg;
+                sm.meta_ntok[stage] = ntok;
+                sm.meta_fin[stage] = (slot == nsel - 1 || k + 1 == kend);
+                sm.meta_nfrag[stage] = nfrag;
+                sm.meta_frag[stage] = frag;
+                mbar_arrive(&sm.full_k[stage]);
+                mbar_arrive(&sm.full_v[stage]);
+            }
+            __syncwarp();
             ++n;
         }
-        // end marker; after a wait that gave up the compute warps stop on their own bounded waits
-        const int stage = n % kDecStages;
-        if (ok && n >= kDecStages) mbar_wait(&sm.empty[stage], ((n / kDecStages) - 1) & 1, a.hdr, KID_ATTN_DECODE);
-        sm.meta_bg[stage] = -1;
-        mbar_arrive(&sm.full_k[stage]);
+        if (lane == 0) {
+            // end marker; after a wait that gave up the other warps stop on their own bounded waits
+            const int stage = n % kDecStages;
+            if (ok && n >= kDecStages) mbar_wait(&sm.empty[stage], ((n / kDecStages) - 1) & 1, a.hdr, KID_ATTN_DECODE);
+            sm.meta_bg[stage] = -1;
+            mbar_arrive(&sm.full_k[stage]);
+        }
+        return;
+    }
+
+    if (warp == kDecEpi) {
+        // ---------------------------------------------------------------- epilogue warp
+        const int stride = dec_part_stride(Hg), ooff = dec_part_ooff(Hg);
+        const int ngroups = Hg > 8 ? 16 : 8;
+        // This CTA's last group: when its other parts live in later CTAs (which reach them at the
+        // start of their ranges), merge those partials while the compute warps still work, so
+        // that the group's output leaves without further global round trips.
+        int tgt_bg = -1, tgt_nfrag = 1, tgt_frag = 0;
+        {
+            const int kend = range_begin(blockIdx.x + 1, n_items, gridDim.x, a.inv_grid);
+            const int bgl = (kend - 1) / kTopK;
+            const int v = lane < kTopK ? __ldcg(a.sel + size_t(bgl) * kTopK + lane) : -1;
+            const int nsel = __popc(__ballot_sync(0xffffffffu, v >= 0));
+            const int pos = __ldcg(a.q_pos + bgl / G);
+            if (!(pos < 0 || pos > a.max_pos || pos >= a.l_cap) && nsel > 0) {
+                const int c0 = range_owner(bgl * kTopK, n_items, gridDim.x, a.inv_items);
+                const int c1 = range_owner(bgl * kTopK + nsel - 1, n_items, gridDim.x, a.inv_items);
+                if (int(blockIdx.x) >= c0 && int(blockIdx.x) <= c1 && c1 > c0) {
+                    tgt_bg = bgl;
+                    tgt_nfrag = c1 - c0 + 1;
+                    tgt_frag = int(blockIdx.x) - c0;
+                }
+            }
+        }
+        int pre = tgt_bg >= 0 ? 1 : 0;                        // 1: others pending, 2: merged in ot
+        WarpState st;
+        for (int f = 0;; ++f) {
+            const int qs = f % kDecStages;
+            const uint32_t par = (f / kDecStages) & 1;
+            bool got = false;
+            const long long t0 = clock64();
+            while (true) {
+                got = __all_sync(0xffffffffu, mbar_try_wait(&sm.parked[qs], par));
+                if (got) break;
+                if (pre == 1) {
+                    unsigned cnt = 0;
+                    if (lane == 0) cnt = ld_acquire_gpu(a.ctr + tgt_bg);
+                    if (__shfl_sync(0xffffffffu, cnt, 0) == unsigned(tgt_nfrag - 1)) {
+                        clear_state(st);
+                        for (int fo = 0; fo < tgt_nfrag; ++fo)
+                            if (fo != tgt_frag)
+                                merge_partial(st, a.part + (size_t(tgt_bg) * kTopK + fo) * stride, Hg, ooff, gq, tq);
+#pragma unroll
+                        for (int g = 0; g < 16; ++g)
+                            if (g < ngroups) sm.ot[g][lane] = acc_group(st, g);
+                        if (tq == 0) {
+                            sm.om[gq] = st.m0; sm.om[gq + 8] = st.m1;
+                            sm.ol[gq] = st.l0; sm.ol[gq + 8] = st.l1;
+                        }
+                        __syncwarp();
+                        pre = 2;
+                    } else {
+                        __nanosleep(500);
+                    }
+                }
+                if (clock64() - t0 > kWaitCycles) {
+                    if (lane == 0) record_error(a.hdr, MSA_ERR_TIMEOUT, KID_ATTN_DECODE, blockIdx.x, threadIdx.x, int(par));
+                    break;
+                }
+            }
+            if (!got) break;
+            const int stage = sm.park_stage[qs];
+            if (stage < 0) break;
+            const int bg = sm.meta_bg[stage], nfrag = sm.meta_nfrag[stage], frag = sm.meta_frag[stage];
+            const bool premerged = pre == 2 && bg == tgt_bg;
+            // fold the 8 parked warp states (and the pre-merged other parts)
+            float mw0[kDecWarps + 1], mw1[kDecWarps + 1];
+            st.m0 = st.m1 = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kDecWarps + 1; ++w) {
+                mw0[w] = w < kDecWarps ? sm.pm[stage][w][gq] : (premerged ? sm.om[gq] : -INFINITY);
+                mw1[w] = w < kDecWarps ? sm.pm[stage][w][gq + 8] : (premerged ? sm.om[gq + 8] : -INFINITY);
+                st.m0 = fmaxf(st.m0, mw0[w]);
+                st.m1 = fmaxf(st.m1, mw1[w]);
+            }
+            st.l0 = st.l1 = 0.f;
+#pragma unroll
+            for (int w = 0; w < kDecWarps + 1; ++w) {
+                mw0[w] = mw0[w] == -INFINITY ? 0.f : fast_exp2(mw0[w] - st.m0);
+                mw1[w] = mw1[w] == -INFINITY ? 0.f : fast_exp2(mw1[w] - st.m1);
+                st.l0 += (w < kDecWarps ? sm.pl[stage][w][gq] : (premerged ? sm.ol[gq] : 0.f)) * mw0[w];
+                st.l1 += (w < kDecWarps ? sm.pl[stage][w][gq + 8] : (premerged ? sm.ol[gq + 8] : 0.f)) * mw1[w];
+            }
+#pragma unroll
+            for (int g = 0; g < 16; ++g) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (g < ngroups) {
+#pragma unroll
+                    for (int w = 0; w < kDecWarps; ++w) {
+                        const float4 x = *park_addr(sm, stage, w, g, lane);
+                        const float wt = g >= 8 ? mw1[w] : mw0[w];
+                        acc.x += x.x * wt; acc.y += x.y * wt; acc.z += x.z * wt; acc.w += x.w * wt;
+                    }
+                    if (premerged) {
+                        const float4 x = sm.ot[g][lane];
+                        const float wt = g >= 8 ? mw1[kDecWarps] : mw0[kDecWarps];
+                        acc.x += x.x * wt; acc.y += x.y * wt; acc.z += x.z * wt; acc.w += x.w * wt;
+                    }
+                }
+                set_acc_group(st, g, acc);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_n(&sm.empty[stage], kDecWarps);   // the stage may be refilled
+
+            const int b = bg / G, g = bg % G;
+            const size_t orow = size_t(b) * G * Hg + size_t(g) * Hg;
+            bool last = nfrag == 1 || premerged;
+            if (premerged && lane == 0) *reinterpret_cast<volatile unsigned*>(a.ctr + bg) = 0u;   // ready for the next call
+            if (!last) {
+                // Parts of a split group: if all the others are in, merge them into these
+                // registers; otherwise leave this one for the last to arrive.
+                unsigned cnt = 0;
+                if (lane == 0) cnt = ld_acquire_gpu(a.ctr + bg);
+                cnt = __shfl_sync(0xffffffffu, cnt, 0);
+                if (cnt == unsigned(nfrag - 1)) {
+                    last = true;
+                    if (lane == 0) *reinterpret_cast<volatile unsigned*>(a.ctr + bg) = 0u;
+                } else {
+                    float* mypart = a.part + (size_t(bg) * kTopK + frag) * stride;
+                    if (tq == 0) {
+                        if (gq < Hg) { mypart[gq] = st.m0; mypart[Hg + gq] = st.l0; }
+                        if (gq + 8 < Hg) { mypart[gq + 8] = st.m1; mypart[Hg + gq + 8] = st.l1; }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < 16; ++nt) {
+                        const int col = nt * 8 + 2 * tq;
+                        if (gq < Hg)
+                            *reinterpret_cast<float2*>(mypart + ooff + gq * kHeadDim + col) = make_float2(st.o[nt][0], st.o[nt][1]);
+                        if (gq + 8 < Hg)
+                            *reinterpret_cast<float2*>(mypart + ooff + (gq + 8) * kHeadDim + col) =
+                                make_float2(st.o[nt][2], st.o[nt][3]);
+                    }
+                    __syncwarp();
+                    unsigned old = 0;
+                    if (lane == 0) {
+                        __threadfence();
+                        old = atomicInc(a.ctr + bg, unsigned(nfrag - 1));
+                    }
+                    last = __shfl_sync(0xffffffffu, old, 0) == unsigned(nfrag - 1);
+                }
+                if (last) {
+                    __threadfence();
+                    for (int fo = 0; fo < nfrag; ++fo)
+                        if (fo != frag) merge_partial(st, a.part + (size_t(bg) * kTopK + fo) * stride, Hg, ooff, gq, tq);
+                }
+            }
+            if (last) {
+                const float inv0 = 1.f / st.l0, inv1 = 1.f / st.l1;
+#pragma unroll
+                for (int nt = 0; nt < 16; ++nt) {
+                    const int col = nt * 8 + 2 * tq;
+                    if (gq < Hg)
+                        *reinterpret_cast<uint32_t*>(a.out + (orow + gq) * kHeadDim + col) =
+                            pack_bf16x2(st.o[nt][0] * inv0, st.o[nt][1] * inv0);
+                    if (gq + 8 < Hg)
+                        *reinterpret_cast<uint32_t*>(a.out + (orow + gq + 8) * kHeadDim + col) =
+                            pack_bf16x2(st.o[nt][2] * inv1, st.o[nt][3] * inv1);
+                }
+                if (a.lse != nullptr && tq == 0) {
+                    if (gq < Hg) a.lse[orow + gq] = (st.m0 + log2f(st.l0)) * 0.69314718055994530942f;
+                    if (gq + 8 < Hg) a.lse[orow + gq + 8] = (st.m1 + log2f(st.l1)) * 0.69314718055994530942f;
+                }
+            }
+        }
         return;
     }
 
     // -------------------------------------------------------------------- compute warps
-    const uint32_t psm = smem_u32(&sm.p[0][0]);
-    float o[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};   // heads gq, gq + 8 x 4 columns
-    float lsum0 = 0.f, lsum1 = 0.f;                                 // this thread's share of the sums
-    float Mrun0 = -INFINITY, Mrun1 = -INFINITY;                      // running maxima (log2 units)
+    // Every wait below is bounded; a warp whose wait gives up leaves the loop, and the others
+    // then give up at their next wait for it.
+    const int kbase = warp * 16;
+    WarpState st;
+    clear_state(st);
+    int nfin = 0;                                       // group ends parked so far
     for (int n = 0;; ++n) {
         const int stage = n % kDecStages;
         const uint32_t ph = (n / kDecStages) & 1;
-        // A wait that gives up, or the loader's end marker, stops every compute warp at barrier
-        // (A) below, so that no warp is left waiting at a barrier the others have left.
-        const bool okk = mbar_wait(&sm.full_k[stage], ph, a.hdr, KID_ATTN_DECODE);
+        if (!warp_wait_all(&sm.full_k[stage], ph, a.hdr)) break;
         const int bg = sm.meta_bg[stage];
-        const bool stop = !okk || bg < 0;
-        int ntok = stop ? 0 : sm.meta_ntok[stage];
-        const int fin = sm.meta_fin[stage], nfrag = sm.meta_nfrag[stage], frag = sm.meta_frag[stage];
-        const uint8_t* Ks = sm.kv[stage][0];
-        // ---- scores of keys 16w .. 16w + 15 (two n-tiles) for all heads (rows of the MMA)
+        if (bg < 0) {                                   // end: tell the epilogue warp
+            const int qs = nfin % kDecStages;
+            if (warp == 0 && lane == 0) sm.park_stage[qs] = -1;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.parked[qs]);
+            break;
+        }
+        const int ntok = sm.meta_ntok[stage], fin = sm.meta_fin[stage];
+        const bool active = kbase < ntok;
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        const int kbase = warp * 16;
-        if (kbase < ntok) {
-            const uint16_t* q0 = sm.q[stage][gq];
+        if (active) {
+            const uint8_t* Ks = sm.kv[stage][0];
+            const uint16_t* q0 = sm.q[stage][gq];       // query rows gq, gq + 8 (A fragments)
             const uint16_t* q1 = sm.q[stage][gq + 8];
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
@@ -250,6 +538,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
                 }
             }
         }
+        // ---- online softmax of this warp's 16 keys (rows gq, gq + 8 of the accumulators)
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -262,184 +551,86 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
                 mx1 = fmaxf(mx1, s[nt][2 + e]);
             }
         }
-#pragma unroll
-        for (int off = 1; off <= 2; off <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-        }
-        if (tq == 0) {
-            sm.red_m[warp][gq] = mx0;
-            sm.red_m[warp][gq + 8] = mx1;
-        }
-        if (compute_sync_or(stop)) break;                 // (A) per-warp maxima visible
-        float Mi0 = -INFINITY, Mi1 = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kDecWarps; ++w) {
-            Mi0 = fmaxf(Mi0, sm.red_m[w][gq]);
-            Mi1 = fmaxf(Mi1, sm.red_m[w][gq + 8]);
-        }
-        const float Mn0 = fmaxf(Mrun0, Mi0), Mn1 = fmaxf(Mrun1, Mi1);
-        const float base0 = Mn0 == -INFINITY ? 0.f : Mn0, base1 = Mn1 == -INFINITY ? 0.f : Mn1;
-        const float al0 = Mrun0 == -INFINITY ? 0.f : fast_exp2(Mrun0 - Mn0);
-        const float al1 = Mrun1 == -INFINITY ? 0.f : fast_exp2(Mrun1 - Mn1);
-        Mrun0 = Mn0;
-        Mrun1 = Mn1;
-        float l0 = 0.f, l1 = 0.f;
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        float mn0, mn1, al0, al1, dummy;
+        lse_weights(st.m0, mx0, mn0, al0, dummy);
+        lse_weights(st.m1, mx1, mn1, al1, dummy);
+        const float base0 = mn0 == -INFINITY ? 0.f : mn0, base1 = mn1 == -INFINITY ? 0.f : mn1;
+        st.m0 = mn0;
+        st.m1 = mn1;
+        float p[2][4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-            const float p0 = fast_exp2(s[nt][0] - base0), p1 = fast_exp2(s[nt][1] - base0);
-            const float p2 = fast_exp2(s[nt][2] - base1), p3 = fast_exp2(s[nt][3] - base1);
-            l0 += p0 + p1;
-            l1 += p2 + p3;
-            const int col = kbase + nt * 8 + 2 * tq;
-            *reinterpret_cast<uint32_t*>(&sm.p[gq][col]) = pack_bf16x2(p0, p1);
-            *reinterpret_cast<uint32_t*>(&sm.p[gq + 8][col]) = pack_bf16x2(p2, p3);
-            o[nt][0] *= al0; o[nt][1] *= al0;
-            o[nt][2] *= al1; o[nt][3] *= al1;
+            p[nt][0] = fast_exp2(s[nt][0] - base0);
+            p[nt][1] = fast_exp2(s[nt][1] - base0);
+            p[nt][2] = fast_exp2(s[nt][2] - base1);
+            p[nt][3] = fast_exp2(s[nt][3] - base1);
         }
-        lsum0 = lsum0 * al0 + l0;
-        lsum1 = lsum1 * al1 + l1;
-        // ---- V (rows past the query in the diagonal block must be finite: zero them)
-        if (ntok > 0 && !mbar_wait(&sm.full_v[stage], ph, a.hdr, KID_ATTN_DECODE)) ntok = 0;
-        if (ntok < kBlock) {
-            uint8_t* vw = sm.kv[stage][1];
-            const int nload = (ntok + kDecDiagRows - 1) / kDecDiagRows * kDecDiagRows;
-            for (int i = tid; i < (nload - ntok) * 16; i += kDecWarps * 32) {
-                const int row = ntok + i / 16, ch = i % 16;
-                *reinterpret_cast<uint4*>(vw + (ch >> 3) * 16384 + sw128(row, ch & 7)) = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async();                          // ordered before the stage's next TMA fill
-        }
-        compute_sync();                                   // (B) P and zeroed V rows visible
-        // ---- o[:, 16w .. 16w + 15] += P V over the block's keys
-        const int nks = (ntok + 15) / 16;
-        const uint32_t vsm = smem_u32(sm.kv[stage][1]);
-        for (int kk = 0; kk < nks; ++kk) {
-            uint32_t a0, a1, a2, a3;                      // P rows 0-15 x keys 16kk .. 16kk + 15
-            {
-                const int prow = lane & 15, pcol = kk * 16 + (lane >> 4) * 8;
-                asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
-                             : "r"(psm + uint32_t(prow * kPRow + pcol) * 2u));
-            }
-            uint32_t v0, v1, v2, v3;
-            const int row = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            const int col = warp * 16 + (lane >> 4) * 8;
-            ldsm_x4_trans(vsm + kv_off(row, col), v0, v1, v2, v3);
-            mma_bf16_16816(o[0], a0, a1, a2, a3, v0, v1);
-            mma_bf16_16816(o[1], a0, a1, a2, a3, v2, v3);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.empty[stage]);    // this warp is done with the stage
-        if (!fin) continue;
-
-        // ---- end of this CTA's share of (b, g): combine the warps' sums
-        const int b = bg / G, g = bg % G;
-        float L0 = lsum0, L1 = lsum1;
+        st.l0 = st.l0 * al0 + (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+        st.l1 = st.l1 * al1 + (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
+        if (!__all_sync(0xffffffffu, al0 == 1.f && al1 == 1.f)) {
 #pragma unroll
-        for (int off = 1; off <= 2; off <<= 1) {
-            L0 += __shfl_xor_sync(0xffffffffu, L0, off);
-            L1 += __shfl_xor_sync(0xffffffffu, L1, off);
+            for (int i = 0; i < 16; ++i) {
+                st.o[i][0] *= al0; st.o[i][1] *= al0;
+                st.o[i][2] *= al1; st.o[i][3] *= al1;
+            }
         }
+        // ---- o += P V over this warp's 16 keys: the accumulator layout of S is the A layout of P
+        if (active) {
+            if (!warp_wait_all(&sm.full_v[stage], ph, a.hdr)) break;
+            uint8_t* Vs = sm.kv[stage][1];
+            if (ntok < kbase + 16) {                    // rows past the query must be finite: zero them
+                const int r0 = ntok - kbase;             // 1 .. 15
+                for (int i = lane; i < (16 - r0) * 16; i += 32) {
+                    const int row = kbase + r0 + i / 16, ch = i % 16;
+                    *reinterpret_cast<uint4*>(Vs + (ch >> 3) * 16384 + sw128(row, ch & 7)) = make_uint4(0, 0, 0, 0);
+                }
+                __syncwarp();
+            }
+            const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]), pa1 = pack_bf16x2(p[0][2], p[0][3]);
+            const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]), pa3 = pack_bf16x2(p[1][2], p[1][3]);
+            const uint32_t vrow = smem_u32(Vs);
+            const int row = kbase + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+            for (int dn = 0; dn < 8; ++dn) {
+                uint32_t v0, v1, v2, v3;
+                ldsm_x4_trans(vrow + kv_off(row, dn * 16 + (lane >> 4) * 8), v0, v1, v2, v3);
+                mma_bf16_16816(st.o[2 * dn], pa0, pa1, pa2, pa3, v0, v1);
+                mma_bf16_16816(st.o[2 * dn + 1], pa0, pa1, pa2, pa3, v2, v3);
+            }
+        }
+        if (!fin) {
+            if (active && ntok < kbase + 16) fence_proxy_async();   // zeroed rows before the next TMA fill
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[stage]);   // this warp is done with the stage
+            continue;
+        }
+        // ---- end of this CTA's share of the group: park the state in this warp's own rows of
+        // the stage (no other warp reads them) and hand the stage to the epilogue warp
+        st.l0 += __shfl_xor_sync(0xffffffffu, st.l0, 1);
+        st.l1 += __shfl_xor_sync(0xffffffffu, st.l1, 1);
+        st.l0 += __shfl_xor_sync(0xffffffffu, st.l0, 2);
+        st.l1 += __shfl_xor_sync(0xffffffffu, st.l1, 2);
+        __syncwarp();                                   // every lane is done reading its rows
+#pragma unroll
+        for (int g = 0; g < 16; ++g)
+            if (g < 8 || Hg > 8) *park_addr(sm, stage, warp, g, lane) = acc_group(st, g);
         if (tq == 0) {
-            sm.red_l[warp][gq] = L0;
-            sm.red_l[warp][gq + 8] = L1;
+            sm.pm[stage][warp][gq] = st.m0;
+            sm.pm[stage][warp][gq + 8] = st.m1;
+            sm.pl[stage][warp][gq] = st.l0;
+            sm.pl[stage][warp][gq + 8] = st.l1;
         }
-        compute_sync();                                   // (C)
-        L0 = 0.f;
-        L1 = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDecWarps; ++w) {
-            L0 += sm.red_l[w][gq];
-            L1 += sm.red_l[w][gq + 8];
-        }
-        const size_t orow = size_t(b) * G * Hg + size_t(g) * Hg;
-        if (nfrag == 1) {
-            const float inv0 = 1.f / L0, inv1 = 1.f / L1;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int col = warp * 16 + nt * 8 + 2 * tq;
-                if (gq < Hg)
-                    *reinterpret_cast<uint32_t*>(a.out + (orow + gq) * kHeadDim + col) =
-                        pack_bf16x2(o[nt][0] * inv0, o[nt][1] * inv0);
-                if (gq + 8 < Hg)
-                    *reinterpret_cast<uint32_t*>(a.out + (orow + gq + 8) * kHeadDim + col) =
-                        pack_bf16x2(o[nt][2] * inv1, o[nt][3] * inv1);
-            }
-            if (a.lse != nullptr && warp == 0 && tq == 0) {
-                if (gq < Hg) a.lse[orow + gq] = (Mrun0 + log2f(L0)) * 0.69314718055994530942f;
-                if (gq + 8 < Hg) a.lse[orow + gq + 8] = (Mrun1 + log2f(L1)) * 0.69314718055994530942f;
-            }
-        } else {
-            float* mypart = a.part + (size_t(bg) * kTopK + frag) * stride;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int col = warp * 16 + nt * 8 + 2 * tq;
-                if (gq < Hg) *reinterpret_cast<float2*>(mypart + ooff + gq * kHeadDim + col) = make_float2(o[nt][0], o[nt][1]);
-                if (gq + 8 < Hg)
-                    *reinterpret_cast<float2*>(mypart + ooff + (gq + 8) * kHeadDim + col) = make_float2(o[nt][2], o[nt][3]);
-            }
-            if (warp == 0 && tq == 0) {
-                if (gq < Hg) { mypart[gq] = Mrun0; mypart[Hg + gq] = L0; }
-                if (gq + 8 < Hg) { mypart[gq + 8] = Mrun1; mypart[Hg + gq + 8] = L1; }
-            }
-            __threadfence();
-            compute_sync();                               // (D) the partial is written
-            if (tid == 0) sm.is_last = (atomicInc(a.ctr + bg, unsigned(nfrag - 1)) == unsigned(nfrag - 1));
-            compute_sync();                               // (E)
-            if (sm.is_last) {
-                __threadfence();
-                // merge the nfrag partials: stage (max, sum) pairs, then thread t produces 8 columns
-                const float* pbase = a.part + size_t(bg) * kTopK * stride;
-                for (int i = tid; i < nfrag * Hg; i += kDecWarps * 32) {
-                    const int f = i / Hg, h = i % Hg;
-                    sm.wts[f][h] = __ldcg(pbase + f * stride + h);
-                    sm.ls[f][h] = __ldcg(pbase + f * stride + Hg + h);
-                }
-                compute_sync();
-                if (tid < Hg) {
-                    float M = -INFINITY;
-                    for (int f = 0; f < nfrag; ++f) M = fmaxf(M, sm.wts[f][tid]);
-                    float L = 0.f;
-                    for (int f = 0; f < nfrag; ++f) {
-                        const float m = sm.wts[f][tid];
-                        const float wf = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
-                        L += sm.ls[f][tid] * wf;
-                        sm.wts[f][tid] = wf;
-                    }
-                    sm.mrg_m[tid] = M;
-                    sm.mrg_l[tid] = L;
-                }
-                compute_sync();
-                for (int base = tid * 8; base < Hg * kHeadDim; base += kDecWarps * 32 * 8) {
-                    const int h = base / kHeadDim, col = base % kHeadDim;
-                    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-                    for (int f = 0; f < nfrag; ++f) {
-                        const float4* src = reinterpret_cast<const float4*>(pbase + f * stride + ooff + h * kHeadDim + col);
-                        const float4 x = __ldcg(src), y = __ldcg(src + 1);
-                        const float wf = sm.wts[f][h];
-                        acc[0] = fmaf(wf, x.x, acc[0]); acc[1] = fmaf(wf, x.y, acc[1]);
-                        acc[2] = fmaf(wf, x.z, acc[2]); acc[3] = fmaf(wf, x.w, acc[3]);
-                        acc[4] = fmaf(wf, y.x, acc[4]); acc[5] = fmaf(wf, y.y, acc[5]);
-                        acc[6] = fmaf(wf, y.z, acc[6]); acc[7] = fmaf(wf, y.w, acc[7]);
-                    }
-                    const float inv = 1.f / sm.mrg_l[h];
-                    uint4 ov;
-                    ov.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-                    ov.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-                    ov.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-                    ov.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-                    *reinterpret_cast<uint4*>(a.out + (orow + h) * kHeadDim + col) = ov;
-                    if (a.lse != nullptr && col == 0)
-                        a.lse[orow + h] = (sm.mrg_m[h] + log2f(sm.mrg_l[h])) * 0.69314718055994530942f;
-                }
-                compute_sync();                           // merge buffers free for the next group
-            }
-        }
-        o[0][0] = o[0][1] = o[0][2] = o[0][3] = 0.f;
-        o[1][0] = o[1][1] = o[1][2] = o[1][3] = 0.f;
-        lsum0 = lsum1 = 0.f;
-        Mrun0 = Mrun1 = -INFINITY;
+        fence_proxy_async();                            // smem writes before the stage's next TMA fill
+        const int qs = nfin % kDecStages;
+        if (warp == 0 && lane == 0) sm.park_stage[qs] = stage;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.parked[qs]);
+        ++nfin;
+        clear_state(st);
     }
 }
 
@@ -482,6 +673,8 @@ msa_status_t launch_attn_decode(const void* k_cache, const void* v_cache, const 
     }
     const int64_t n_items = int64_t(B) * G * kTopK;
     const int grid = int(n_items < num_sms() ? n_items : num_sms());   // persistent: one CTA per SM
+    a.inv_grid = 1.0 / double(grid);
+    a.inv_items = 1.0 / double(n_items);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kDecThreads);
