@@ -129,7 +129,23 @@ void launch_select_prefill_simt(const void* q_idx, int B, int G, int64_t N, cons
 // the CTA that arrives last for a (sequence, group) merges the sorted lists. The arrival
 // counter wraps to zero by itself (atomicInc), so the workspace is ready for the next call.
 constexpr int kDecChunk = 128;
-constexpr int kDecSmemChunks = 64;    // merges of up to 64 chunks run from shared memory
+constexpr int kMaxSurvivors = 1024;   // merge keys ranked in shared memory
+
+__device__ __forceinline__ unsigned long long umax64(unsigned long long x, unsigned long long y) { return x > y ? x : y; }
+
+// Bitonic sort of one key per lane, descending across the warp's lanes.
+__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
+            const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+            x = keep_max ? umax64(x, y) : (x < y ? x : y);
+        }
+    }
+    return x;
+}
 
 __global__ void __launch_bounds__(kDecChunk) select_decode_kernel(
     const uint16_t* __restrict__ q_idx, const int32_t* __restrict__ q_pos, int64_t max_pos, int G,
@@ -137,13 +153,16 @@ __global__ void __launch_bounds__(kDecChunk) select_decode_kernel(
     unsigned long long* __restrict__ cand, unsigned int* __restrict__ ctr, int nchunk_max, WsHeader* hdr) {
     __shared__ __align__(16) float qs[kIndexDim];
     __shared__ float sc[kDecChunk];
-    __shared__ unsigned long long keys[kDecChunk];
-    __shared__ unsigned long long lst[kDecSmemChunks * kKeep];
-    __shared__ int heads[1024];
+    __shared__ unsigned long long wl[4 * kKeep];          // the warps' best 15 keys
+    __shared__ unsigned long long surv[kMaxSurvivors];    // merge: keys that may be in the top 15
+    __shared__ unsigned long long top[kKeep];
+    __shared__ int nsurv;
     __shared__ int last;
     grid_dep_launch();                 // the attention kernel may start its prologue
     const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int bg = b * G + g;
+    // the query row does not depend on the position: load both at once
+    const float qx = threadIdx.x < kIndexDim ? bf16_to_f32(q_idx[size_t(bg) * kIndexDim + threadIdx.x]) : 0.f;
     const int pos = q_pos[b];
     if (pos < 0 || pos > max_pos || int64_t(pos / kBlock) > nb_cap) {
         if (ch == 0 && threadIdx.x == 0) record_error(hdr, MSA_ERR_DEVICE_BOUNDS, KID_SELECT_DECODE, bg, 0, pos);
@@ -160,7 +179,7 @@ __global__ void __launch_bounds__(kDecChunk) select_decode_kernel(
     const int nch = (c + kDecChunk - 1) / kDecChunk;
     if (ch >= nch) { grid_dep_wait(); return; }
 
-    if (threadIdx.x < kIndexDim) qs[threadIdx.x] = bf16_to_f32(q_idx[size_t(bg) * kIndexDim + threadIdx.x]);
+    if (threadIdx.x < kIndexDim) qs[threadIdx.x] = qx;
     __syncthreads();
     // Coalesced scoring: each warp instruction reads two whole 256-byte candidate rows (lane l
     // takes float4 (l mod 16) of row 2i + l / 16); 16-lane shuffles finish each dot product.
@@ -190,13 +209,21 @@ __global__ void __launch_bounds__(kDecChunk) select_decode_kernel(
     const int j = ch * kDecChunk + threadIdx.x;
     unsigned long long key = 0ull;
     if (j < c) key = sel_key(sc[threadIdx.x], j);
-    keys[threadIdx.x] = key;
+    // Chunk top-15: each warp sorts its 32 keys; the chunk's best 15 are among the warps' best
+    // 15, and none of them is below the largest of the warps' 15th keys.
+    key = warp_sort_desc(key, ln);
+    if (ln < kKeep) wl[wid * kKeep + ln] = key;
     __syncthreads();
     unsigned long long* mine = cand + (size_t(bg) * nchunk_max + ch) * kKeep;
-    if (key != 0ull) {
-        int rank = 0;
-        for (int i = 0; i < kDecChunk; ++i) rank += keys[i] > key;
-        if (rank < kKeep) mine[rank] = key;
+    if (threadIdx.x < 4 * kKeep) {
+        const unsigned long long k = wl[threadIdx.x];
+        const unsigned long long t = umax64(umax64(wl[kKeep - 1], wl[2 * kKeep - 1]), umax64(wl[3 * kKeep - 1], wl[4 * kKeep - 1]));
+        if (k != 0ull && k >= t) {
+            int rank = 0;
+#pragma unroll 4
+            for (int i = 0; i < 4 * kKeep; ++i) rank += wl[i] > k;
+            if (rank < kKeep) mine[rank] = k;
+        }
     }
     const int nvalid = min(kKeep, c - ch * kDecChunk);
     if (threadIdx.x >= nvalid && threadIdx.x < kKeep) mine[threadIdx.x] = 0ull;
@@ -210,40 +237,50 @@ __global__ void __launch_bounds__(kDecChunk) select_decode_kernel(
     grid_dep_wait();
     if (!last) return;
     __threadfence();
-    // stage the nch sorted lists in shared memory with one coalesced pass (global fallback for
-    // more than kDecSmemChunks chunks), then warp 0 merges: 15 rounds of "best list head"
+    // Merge the nch sorted lists. The 15th key of every list is a lower bound of the overall
+    // 15th key, so only keys at or above the largest of them (the survivors, usually a few
+    // dozen) are ranked against each other.
     const unsigned long long* glists = cand + size_t(bg) * nchunk_max * kKeep;
-    const bool in_smem = nch <= kDecSmemChunks;
-    if (in_smem)
-        for (int i = threadIdx.x; i < nch * kKeep; i += kDecChunk) lst[i] = __ldcg(glists + i);
+    const int ncand = nch * kKeep;
+    unsigned long long t = 0ull;
+    for (int l = threadIdx.x; l < nch; l += kDecChunk) t = umax64(t, __ldcg(glists + size_t(l) * kKeep + kKeep - 1));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) t = umax64(t, __shfl_xor_sync(0xffffffffu, t, off));
+    if (ln == 0) wl[wid] = t;
+    if (threadIdx.x == 0) nsurv = 0;
+    __syncthreads();
+    t = umax64(umax64(wl[0], wl[1]), umax64(wl[2], wl[3]));
+    for (int i = threadIdx.x; i < ncand; i += kDecChunk) {
+        const unsigned long long k = __ldcg(glists + i);
+        if (k != 0ull && k >= t) {
+            const int at = atomicAdd(&nsurv, 1);
+            if (at < kMaxSurvivors) surv[at] = k;
+        }
+    }
+    __syncthreads();
+    const int ns = nsurv;
+    if (ns > kMaxSurvivors) {
+        // more survivors than the buffer holds (many near-equal lists): rank every candidate
+        for (int i = threadIdx.x; i < ncand; i += kDecChunk) {
+            const unsigned long long k = __ldcg(glists + i);
+            if (k == 0ull || k < t) continue;
+            int rank = 0;
+            for (int q = 0; q < ncand && rank < kKeep; ++q) rank += __ldcg(glists + q) > k;
+            if (rank < kKeep) top[rank] = k;
+        }
+    } else {
+        for (int i = threadIdx.x; i < ns; i += kDecChunk) {
+            const unsigned long long k = surv[i];
+            int rank = 0;
+            for (int q = 0; q < ns; ++q) rank += surv[q] > k;
+            if (rank < kKeep) top[rank] = k;
+        }
+    }
     __syncthreads();
     if (threadIdx.x >= 32) return;
+    // ascending order of the 15 selected ids and the diagonal block c (lane 15)
     const int lane = threadIdx.x;
-    const unsigned long long* lists = in_smem ? lst : glists;
-    for (int l = lane; l < nch; l += 32) heads[l] = 0;
-    __syncwarp();
-    int my_id = c;                                   // lane 15 keeps the diagonal block
-    for (int r = 0; r < kKeep; ++r) {
-        unsigned long long bk = 0ull;
-        int bl = -1;
-        for (int l = lane; l < nch; l += 32) {
-            const int h = heads[l];
-            if (h < kKeep) {
-                const unsigned long long k = in_smem ? lists[size_t(l) * kKeep + h] : __ldcg(lists + size_t(l) * kKeep + h);
-                if (k > bk) { bk = k; bl = l; }
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const unsigned long long ok = __shfl_xor_sync(0xffffffffu, bk, off);
-            const int ol = __shfl_xor_sync(0xffffffffu, bl, off);
-            if (ok > bk) { bk = ok; bl = ol; }
-        }
-        if (lane == r) my_id = key_block(bk);
-        if (lane == 0 && bl >= 0) heads[bl] += 1;
-        __syncwarp();
-    }
-    // ascending order of the 16 ids held by lanes 0..15
+    const int my_id = lane < kKeep ? key_block(top[lane]) : c;
     int rank = 0;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {

@@ -167,3 +167,43 @@ def test_device_bounds_are_reported_not_faulted(cuda_ok):
     st, info = msa_get_device_status(bufs["ws_select"])
     assert st == 6 and info[3] == 5000
     assert msa_get_device_status(bufs["ws_select"])[0] == 0          # cleared after reading
+
+
+@pytest.mark.parametrize("case", ["many_survivors", "all_equal", "random"])
+def test_decode_select_long_context_merge(cuda_ok, case):
+    """Selection over 10,240 candidate blocks (80 chunks of 128 per query): the merge of the
+    chunks' best-15 lists against the oracle, including lists built so that more than a
+    thousand keys tie with or exceed the largest 15th key (the merge's slow path) and pooled
+    keys that are all equal (ties to the lower id everywhere)."""
+    c = 10240
+    pos = c * 128 + 5
+    nb_cap = c + 1
+    q_bits = np.zeros((1, 1, 64), np.uint16)
+    pooled = np.zeros((1, 1, nb_cap, 64), np.float32)
+    if case == "random":
+        q_bits = synth.normal_bf16(77, synth.STREAM_QI, (1, 1, 64))
+        pooled[..., :] = synth.bf16_bits_to_f32(synth.normal_bf16(78, synth.STREAM_KI, (1, 1, nb_cap, 64)))
+    else:
+        q_bits[..., 0] = 0x3F80                       # q_I = e_0: the score of block j is pooled[j, 0] / 8
+        if case == "many_survivors":
+            # chunk 0: 15 blocks at 5; chunks 1..79: 14 blocks at 10 and the rest at 0, so every
+            # list but the first has its 15th key at score 0 and ~1,100 keys survive the bound
+            pooled[0, 0, :15, 0] = 5.0
+            for ch in range(1, c // 128):
+                pooled[0, 0, ch * 128:ch * 128 + 14, 0] = 10.0
+        else:
+            pooled[..., 0] = 1.0
+    shape = Shape.make(1, 4, 1)
+    bufs = pipeline.decode_buffers(1, 4, 1, pos, "cuda")
+    q_pos = torch.tensor([pos], dtype=torch.int32, device="cuda")
+    msa_index_select(shape, dev_bf16(q_bits), 1, q_pos, pos, torch.from_numpy(pooled).cuda(), nb_cap,
+                     bufs["sel"], bufs["ws_select"])
+    torch.cuda.synchronize()
+    assert msa_get_device_status(bufs["ws_select"])[0] == 0
+    sel = bufs["sel"].cpu().numpy()[0, 0]
+    ref, kth, _ = oracle.select_rows(np.array([pos]), q_bits[0], pooled[0, 0].astype(np.float64))
+    check_selection(sel[None], ref, kth, q_bits[0], pooled[0, 0].astype(np.float64), np.array([pos]))
+    if case != "random":
+        assert (sel == ref[0]).all(), (case, sel, ref[0])
+    if case == "many_survivors":
+        assert list(sel) == list(range(128, 142)) + [256, c]
