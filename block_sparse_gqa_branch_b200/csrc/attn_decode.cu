@@ -221,12 +221,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
         bool need_frag = false;
         int n = 0;
         bool ok = true;
-        for (int k = kbeg; k < kend; ++k) {
+        // The range is walked rotated: first the part of its last group (the next CTA finishes
+        // that group last), then from its first item on. So this CTA ends with the tail of a
+        // group whose head the previous CTA took first, and its epilogue warp has usually
+        // merged that head before the tail arrives.
+        const int kmid = max(kbeg, (kend - 1) / kTopK * kTopK);
+        for (int idx = 0; idx < kend - kbeg; ++idx) {
+            const bool first_seg = idx < kend - kmid;
+            const int k = first_seg ? kmid + idx : kbeg + (idx - (kend - kmid));
+            const int seg_end = first_seg ? kend : kmid;
             const int bg = k / kTopK, slot = k % kTopK;
             if (bg != cur_bg) {
                 cur_bg = bg;
-                if (bg >= cache0 + cachen) {                  // fetch the next rows in one round trip
-                    const int left = (kend - 1) / kTopK - bg + 1;
+                if (bg < cache0 || bg >= cache0 + cachen) {   // fetch the next rows in one round trip
+                    const int left = (seg_end - 1) / kTopK - bg + 1;
                     cache0 = bg;
                     cachen = left < kRowCache ? left : kRowCache;
                     __syncwarp();
@@ -249,10 +257,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
                 }
                 need_frag = nsel > 0;
             }
-            if (slot >= nsel) {                               // the row's tail is empty
-                k = bg * kTopK + kTopK - 1;
-                continue;
-            }
+            if (slot >= nsel) continue;                       // the row's tail is empty
             const int stage = n % kDecStages;
             if (n >= kDecStages) {
                 bool w = true;
@@ -309,7 +314,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
             if (lane == 0) {
                 sm.meta_bg[stage] = bg;
                 sm.meta_ntok[stage] = ntok;
-                sm.meta_fin[stage] = (slot == nsel - 1 || k + 1 == kend);
+                sm.meta_fin[stage] = (slot == nsel - 1 || k + 1 == seg_end);
                 sm.meta_nfrag[stage] = nfrag;
                 sm.meta_frag[stage] = frag;
                 mbar_arrive(&sm.full_k[stage]);
@@ -332,13 +337,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
         // ---------------------------------------------------------------- epilogue warp
         const int stride = dec_part_stride(Hg), ooff = dec_part_ooff(Hg);
         const int ngroups = Hg > 8 ? 16 : 8;
-        // This CTA's last group: when its other parts live in later CTAs (which reach them at the
-        // start of their ranges), merge those partials while the compute warps still work, so
-        // that the group's output leaves without further global round trips.
+        // The last group this CTA works on: when its other parts live in other CTAs (which reach
+        // them first), merge those partials while the compute warps still work, so that the
+        // group's output leaves without further global round trips.
         int tgt_bg = -1, tgt_nfrag = 1, tgt_frag = 0;
         {
+            // the group the loader walks last (see the rotated walk above)
+            const int kbeg = range_begin(blockIdx.x, n_items, gridDim.x, a.inv_grid);
             const int kend = range_begin(blockIdx.x + 1, n_items, gridDim.x, a.inv_grid);
-            const int bgl = (kend - 1) / kTopK;
+            const int kmid = max(kbeg, (kend - 1) / kTopK * kTopK);
+            const int bgl = kmid > kbeg ? (kmid - 1) / kTopK : (kend - 1) / kTopK;
             const int v = lane < kTopK ? __ldcg(a.sel + size_t(bgl) * kTopK + lane) : -1;
             const int nsel = __popc(__ballot_sync(0xffffffffu, v >= 0));
             const int pos = __ldcg(a.q_pos + bgl / G);

@@ -27,7 +27,7 @@ msa_status_t make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uin
 // halves as [half][8 rows][128 B] (128B swizzle)
 msa_status_t make_tmap_q_rows(CUtensorMap* m, const void* base, uint64_t rows);
 
-// largest query position the decode selection supports (its merge handles 1024 chunks)
+// largest query position the decode path supports (bounds its workspaces and row indices)
 constexpr int64_t kMaxDecodePos = (int64_t(1) << 24) - 1;
 
 constexpr int kHeadDim = 128;   // d

@@ -9,6 +9,8 @@
 // and cannot change the order, so it is not applied). Ranking uses only compares: the
 // running top-15 keeps the earlier (lower) block on equal scores, which is the order
 // (score desc, id asc). The query's own block is added and the ids are written ascending.
+#include <cooperative_groups.h>
+
 #include "msa_common.cuh"
 
 namespace msa {
@@ -123,15 +125,26 @@ void launch_select_prefill_simt(const void* q_idx, int B, int G, int64_t N, cons
 }
 
 // ------------------------------------------------------------------ decode, split + merge
-// One query per (sequence, group); its candidates [0, c) are split into chunks of 128 over
-// CTAs so that the pooled keys (256 B per candidate) stream from HBM on many SMs at once.
-// Each CTA ranks its 128 candidates and leaves its best 15 keys, sorted, in the workspace;
-// the CTA that arrives last for a (sequence, group) merges the sorted lists. The arrival
-// counter wraps to zero by itself (atomicInc), so the workspace is ready for the next call.
-constexpr int kDecChunk = 128;
-constexpr int kMaxSurvivors = 1024;   // merge keys ranked in shared memory
+// One query per (sequence, group); its candidates [0, c) are split over 8 k CTAs that form k
+// thread-block clusters of 8. A CTA of 4 warps scores its span 128 candidates per pass (each
+// warp instruction reads two whole 256-byte pooled rows; 16 loads per lane are in flight), and
+// every warp keeps a running best-16 list: the pass's 32 keys are sorted in registers
+// (bitonic) and merged into the list (a bitonic merge). The CTA's 4 lists are merged into one
+// in shared memory; after a cluster barrier the cluster's first CTA reads the 8 lists over
+// distributed shared memory and merges them (3 rounds of pairwise merges). With one cluster
+// per (sequence, group) -- the case whenever the batch fills the GPU -- that CTA writes the
+// selection; with several, each cluster leaves its best 15 in the workspace and the cluster
+// that arrives last merges those lists the same way (the arrival counter wraps to zero by
+// itself, so the workspace is ready for the next call). No step depends on the data.
+int num_sms();
+
+constexpr int kSelThreads = 128;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelCluster = 8;                    // CTAs per cluster
+constexpr int kSelMaxClusters = 64;               // clusters per (sequence, group)
 
 __device__ __forceinline__ unsigned long long umax64(unsigned long long x, unsigned long long y) { return x > y ? x : y; }
+__device__ __forceinline__ unsigned long long umin64(unsigned long long x, unsigned long long y) { return x < y ? x : y; }
 
 // Bitonic sort of one key per lane, descending across the warp's lanes.
 __device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
@@ -140,147 +153,32 @@ __device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long 
 #pragma unroll
         for (int j = k >> 1; j > 0; j >>= 1) {
             const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
-            const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
-            x = keep_max ? umax64(x, y) : (x < y ? x : y);
+            x = (((lane & j) == 0) == ((lane & k) == 0)) ? umax64(x, y) : umin64(x, y);
         }
     }
     return x;
 }
 
-__global__ void __launch_bounds__(kDecChunk) select_decode_kernel(
-    const uint16_t* __restrict__ q_idx, const int32_t* __restrict__ q_pos, int64_t max_pos, int G,
-    const float* __restrict__ pooled, int64_t nb_cap, int32_t* __restrict__ sel,
-    unsigned long long* __restrict__ cand, unsigned int* __restrict__ ctr, int nchunk_max, WsHeader* hdr) {
-    __shared__ __align__(16) float qs[kIndexDim];
-    __shared__ float sc[kDecChunk];
-    __shared__ unsigned long long wl[4 * kKeep];          // the warps' best 15 keys
-    __shared__ unsigned long long surv[kMaxSurvivors];    // merge: keys that may be in the top 15
-    __shared__ unsigned long long top[kKeep];
-    __shared__ int nsurv;
-    __shared__ int last;
-    grid_dep_launch();                 // the attention kernel may start its prologue
-    const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int bg = b * G + g;
-    // the query row does not depend on the position: load both at once
-    const float qx = threadIdx.x < kIndexDim ? bf16_to_f32(q_idx[size_t(bg) * kIndexDim + threadIdx.x]) : 0.f;
-    const int pos = q_pos[b];
-    if (pos < 0 || pos > max_pos || int64_t(pos / kBlock) > nb_cap) {
-        if (ch == 0 && threadIdx.x == 0) record_error(hdr, MSA_ERR_DEVICE_BOUNDS, KID_SELECT_DECODE, bg, 0, pos);
-        grid_dep_wait();
-        return;
+// Lanes 0-15 hold a descending list, lanes 16-31 another one in ascending order (a bitonic
+// sequence): after the half-cleaners lanes 0-15 hold the 16 largest keys, descending.
+__device__ __forceinline__ unsigned long long warp_merge_desc(unsigned long long x, int lane) {
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) {
+        const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
+        x = ((lane & j) == 0) ? umax64(x, y) : umin64(x, y);
     }
-    const int c = pos / kBlock;
-    int32_t* out = sel + size_t(bg) * kTopK;
-    if (c + 1 <= kTopK) {
-        if (ch == 0 && threadIdx.x == 0) write_all_blocks(out, c);
-        grid_dep_wait();
-        return;
-    }
-    const int nch = (c + kDecChunk - 1) / kDecChunk;
-    if (ch >= nch) { grid_dep_wait(); return; }
+    return x;
+}
 
-    if (threadIdx.x < kIndexDim) qs[threadIdx.x] = qx;
-    __syncthreads();
-    // Coalesced scoring: each warp instruction reads two whole 256-byte candidate rows (lane l
-    // takes float4 (l mod 16) of row 2i + l / 16); 16-lane shuffles finish each dot product.
-    const int ln = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int part = ln & 15, half = ln >> 4;
-    const float4 qv = *reinterpret_cast<const float4*>(&qs[4 * part]);
-    const float4* rows = reinterpret_cast<const float4*>(pooled + (size_t(bg) * nb_cap + size_t(ch) * kDecChunk) * kIndexDim);
-    const int nrow = min(kDecChunk, c - ch * kDecChunk);      // candidates in this chunk
-    float4 v[kDecChunk / 4 / 2];                                 // this warp's 32 rows, 2 per load
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int r = wid * 32 + 2 * i + half;
-        v[i] = r < nrow ? __ldg(rows + size_t(r) * (kIndexDim / 4) + part) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        // fixed order: x, y, z, w, then a butterfly over the 16 lanes of this half-warp
-        float d = fmaf(qv.x, v[i].x, 0.f);
-        d = fmaf(qv.y, v[i].y, d);
-        d = fmaf(qv.z, v[i].z, d);
-        d = fmaf(qv.w, v[i].w, d);
-#pragma unroll
-        for (int off = 8; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-        if (part == 0) sc[wid * 32 + 2 * i + half] = d;
-    }
-    __syncthreads();
-    const int j = ch * kDecChunk + threadIdx.x;
-    unsigned long long key = 0ull;
-    if (j < c) key = sel_key(sc[threadIdx.x], j);
-    // Chunk top-15: each warp sorts its 32 keys; the chunk's best 15 are among the warps' best
-    // 15, and none of them is below the largest of the warps' 15th keys.
-    key = warp_sort_desc(key, ln);
-    if (ln < kKeep) wl[wid * kKeep + ln] = key;
-    __syncthreads();
-    unsigned long long* mine = cand + (size_t(bg) * nchunk_max + ch) * kKeep;
-    if (threadIdx.x < 4 * kKeep) {
-        const unsigned long long k = wl[threadIdx.x];
-        const unsigned long long t = umax64(umax64(wl[kKeep - 1], wl[2 * kKeep - 1]), umax64(wl[3 * kKeep - 1], wl[4 * kKeep - 1]));
-        if (k != 0ull && k >= t) {
-            int rank = 0;
-#pragma unroll 4
-            for (int i = 0; i < 4 * kKeep; ++i) rank += wl[i] > k;
-            if (rank < kKeep) mine[rank] = k;
-        }
-    }
-    const int nvalid = min(kKeep, c - ch * kDecChunk);
-    if (threadIdx.x >= nvalid && threadIdx.x < kKeep) mine[threadIdx.x] = 0ull;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) last = (atomicInc(ctr + bg, unsigned(nch - 1)) == unsigned(nch - 1));
-    __syncthreads();
-    // The selection does not read what the preceding append writes (only fully-past pooled
-    // rows), so it waits for that kernel only before finishing: the attention kernel that waits
-    // for this grid then also sees the appended token.
-    grid_dep_wait();
-    if (!last) return;
-    __threadfence();
-    // Merge the nch sorted lists. The 15th key of every list is a lower bound of the overall
-    // 15th key, so only keys at or above the largest of them (the survivors, usually a few
-    // dozen) are ranked against each other.
-    const unsigned long long* glists = cand + size_t(bg) * nchunk_max * kKeep;
-    const int ncand = nch * kKeep;
-    unsigned long long t = 0ull;
-    for (int l = threadIdx.x; l < nch; l += kDecChunk) t = umax64(t, __ldcg(glists + size_t(l) * kKeep + kKeep - 1));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) t = umax64(t, __shfl_xor_sync(0xffffffffu, t, off));
-    if (ln == 0) wl[wid] = t;
-    if (threadIdx.x == 0) nsurv = 0;
-    __syncthreads();
-    t = umax64(umax64(wl[0], wl[1]), umax64(wl[2], wl[3]));
-    for (int i = threadIdx.x; i < ncand; i += kDecChunk) {
-        const unsigned long long k = __ldcg(glists + i);
-        if (k != 0ull && k >= t) {
-            const int at = atomicAdd(&nsurv, 1);
-            if (at < kMaxSurvivors) surv[at] = k;
-        }
-    }
-    __syncthreads();
-    const int ns = nsurv;
-    if (ns > kMaxSurvivors) {
-        // more survivors than the buffer holds (many near-equal lists): rank every candidate
-        for (int i = threadIdx.x; i < ncand; i += kDecChunk) {
-            const unsigned long long k = __ldcg(glists + i);
-            if (k == 0ull || k < t) continue;
-            int rank = 0;
-            for (int q = 0; q < ncand && rank < kKeep; ++q) rank += __ldcg(glists + q) > k;
-            if (rank < kKeep) top[rank] = k;
-        }
-    } else {
-        for (int i = threadIdx.x; i < ns; i += kDecChunk) {
-            const unsigned long long k = surv[i];
-            int rank = 0;
-            for (int q = 0; q < ns; ++q) rank += surv[q] > k;
-            if (rank < kKeep) top[rank] = k;
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x >= 32) return;
-    // ascending order of the 15 selected ids and the diagonal block c (lane 15)
+// warp: the best 16 of two descending lists a, b of 16 (lanes 0-15 of the result)
+__device__ __forceinline__ unsigned long long merge2(const unsigned long long* a, const unsigned long long* b, int lane) {
+    return warp_merge_desc(lane < 16 ? a[lane] : b[31 - lane], lane);
+}
+
+// warp 0: write the 15 best ids of `best` and the diagonal block c in ascending order
+__device__ __forceinline__ void write_selection(const unsigned long long* best, int32_t* out, int c) {
     const int lane = threadIdx.x;
-    const int my_id = lane < kKeep ? key_block(top[lane]) : c;
+    const int my_id = lane < kKeep ? key_block(best[lane]) : c;
     int rank = 0;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -290,9 +188,153 @@ __global__ void __launch_bounds__(kDecChunk) select_decode_kernel(
     if (lane < 16) out[rank] = my_id;
 }
 
+// Merge n <= 8 descending lists of 16 in `l` (n rows of 16) into l[0] with the CTA's warps.
+__device__ __forceinline__ void merge8(unsigned long long (*l)[16], int n) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    while (n > 1) {
+        const int npairs = n >> 1;
+        unsigned long long x = 0ull;
+        if (wid < npairs) x = merge2(l[2 * wid], l[2 * wid + 1], lane);
+        __syncthreads();
+        if (wid < npairs && lane < 16) l[wid][lane] = x;
+        if ((n & 1) && wid == kSelWarps - 1 && lane < 16) l[npairs][lane] = l[n - 1][lane];
+        __syncthreads();
+        n = (n + 1) >> 1;
+    }
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_decode_kernel(
+    const uint16_t* __restrict__ q_idx, const int32_t* __restrict__ q_pos, int64_t max_pos, int G,
+    const float* __restrict__ pooled, int64_t nb_cap, int32_t* __restrict__ sel,
+    unsigned long long* __restrict__ cand, unsigned int* __restrict__ ctr, WsHeader* hdr) {
+    __shared__ __align__(16) float qs[kIndexDim];
+    __shared__ float sc[kSelThreads];
+    __shared__ unsigned long long lists[kSelCluster][16];     // rank 0 of the cluster uses all 8
+    __shared__ int last;
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    grid_dep_launch();                 // the attention kernel may start its prologue
+    const int split = blockIdx.x, nsplit = gridDim.x, g = blockIdx.y, b = blockIdx.z;
+    const int rank = int(cluster.block_rank()), cl = split / kSelCluster, ncl = nsplit / kSelCluster;
+    const int bg = b * G + g;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    // the query row does not depend on the position: load both at once
+    const float qx = tid < kIndexDim ? bf16_to_f32(q_idx[size_t(bg) * kIndexDim + tid]) : 0.f;
+    const int pos = q_pos[b];
+    // every CTA of a cluster belongs to the same (sequence, group): the early exits below are
+    // taken by the whole cluster, before its barriers
+    if (pos < 0 || pos > max_pos || int64_t(pos / kBlock) > nb_cap) {
+        if (split == 0 && tid == 0) record_error(hdr, MSA_ERR_DEVICE_BOUNDS, KID_SELECT_DECODE, bg, 0, pos);
+        grid_dep_wait();
+        return;
+    }
+    const int c = pos / kBlock;
+    int32_t* out = sel + size_t(bg) * kTopK;
+    if (c + 1 <= kTopK) {
+        if (split == 0 && tid == 0) write_all_blocks(out, c);
+        grid_dep_wait();
+        return;
+    }
+    const int span = ((c + nsplit - 1) / nsplit + 31) / 32 * 32;
+    const int lo = min(c, split * span), hi = min(c, lo + span);   // may be empty
+
+    if (tid < kIndexDim) qs[tid] = qx;
+    __syncthreads();
+    const int part = lane & 15, half = lane >> 4;
+    const float4 qv = *reinterpret_cast<const float4*>(&qs[4 * part]);
+    const float4* rows = reinterpret_cast<const float4*>(pooled + size_t(bg) * nb_cap * kIndexDim);
+    unsigned long long best = 0ull;                      // lanes 0-15: this warp's best 16
+    for (int base = lo; base < hi; base += kSelThreads) {
+        const int r0 = base + wid * 32;                  // this warp's 32 rows
+        float4 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = r0 + 2 * i + half;
+            v[i] = r < hi ? __ldg(rows + size_t(r) * (kIndexDim / 4) + part) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            // fixed order: x, y, z, w, then a butterfly over the 16 lanes of this half-warp
+            float d = fmaf(qv.x, v[i].x, 0.f);
+            d = fmaf(qv.y, v[i].y, d);
+            d = fmaf(qv.z, v[i].z, d);
+            d = fmaf(qv.w, v[i].w, d);
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+            if (part == 0) sc[wid * 32 + 2 * i + half] = d;
+        }
+        __syncwarp();
+        const int j = r0 + lane;
+        unsigned long long key = j < hi ? sel_key(sc[wid * 32 + lane], j) : 0ull;
+        __syncwarp();
+        key = warp_sort_desc(key, lane);
+        const unsigned long long top16 = __shfl_sync(0xffffffffu, key, 31 - lane);   // lanes 16-31: ascending
+        best = warp_merge_desc(lane < 16 ? best : top16, lane);
+    }
+    if (lane < 16) lists[wid][lane] = best;
+    __syncthreads();
+    merge8(lists, kSelWarps);                            // this CTA's best 16 in lists[0]
+    cluster.sync();                                      // every CTA's list is ready
+    if (rank == 0) {
+        if (wid == 0) {
+            for (int r = 1; r < kSelCluster; ++r) {
+                const unsigned long long* rl = cluster.map_shared_rank(&lists[0][0], r);
+                if (lane < 16) lists[r][lane] = rl[lane];
+            }
+        }
+        __syncthreads();
+        merge8(lists, kSelCluster);                      // the cluster's best 16 in lists[0]
+    }
+    cluster.sync();                                      // the other CTAs' lists have been read
+    grid_dep_wait();
+    // The selection does not read what the preceding append writes (only fully-past pooled
+    // rows), so it waits for that kernel only before finishing: the attention kernel that waits
+    // for this grid then also sees the appended token.
+    if (rank != 0) return;
+    if (ncl == 1) {                                      // the whole pair in this cluster
+        if (wid == 0) write_selection(lists[0], out, c);
+        return;
+    }
+    unsigned long long* mine = cand + (size_t(bg) * ncl + cl) * kKeep;
+    if (tid < kKeep) mine[tid] = lists[0][tid];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last = (atomicInc(ctr + bg, unsigned(ncl - 1)) == unsigned(ncl - 1));
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    // merge the ncl cluster lists, 8 at a time, keeping a running best 16 in lists[0]
+    const unsigned long long* glists = cand + size_t(bg) * ncl * kKeep;
+    for (int l0 = 0; l0 < ncl; l0 += kSelCluster - 1) {
+        const int n = min(kSelCluster - 1, ncl - l0);
+        for (int i = tid; i < n * 16; i += kSelThreads) {
+            const int l = i >> 4, e = i & 15;
+            lists[1 + l][e] = e < kKeep ? __ldcg(glists + (l0 + l) * kKeep + e) : 0ull;
+        }
+        if (l0 == 0 && tid < 16) lists[0][tid] = 0ull;
+        __syncthreads();
+        merge8(lists, 1 + n);
+    }
+    if (wid == 0) write_selection(lists[0], out, c);
+}
+
+// Clusters per (sequence, group): enough CTAs for about 7 per SM when the batch is small, at
+// most one CTA per 128 candidates.
+int decode_select_clusters(int B, int G, int64_t max_pos) {
+    const int64_t cmax = max_pos / kBlock;
+    const int64_t nbg = int64_t(B) * G;
+    int64_t n = (int64_t(num_sms()) * 7 + nbg * kSelCluster - 1) / (nbg * kSelCluster);
+    const int64_t cap = (cmax + kSelCluster * 128 - 1) / (kSelCluster * 128);
+    if (n > cap) n = cap;
+    if (n > kSelMaxClusters) n = kSelMaxClusters;
+    return int(n < 1 ? 1 : n);
+}
+
+// workspace bound, independent of the device: one list per cluster at most
 int decode_select_chunks(int64_t max_pos) {
     const int64_t cmax = max_pos / kBlock;
-    return int(cmax <= 0 ? 1 : (cmax + kDecChunk - 1) / kDecChunk);
+    const int64_t n = cmax <= 0 ? 1 : (cmax + kSelCluster * 128 - 1) / (kSelCluster * 128);
+    return int(n < kSelMaxClusters ? (n < 1 ? 1 : n) : kSelMaxClusters);
 }
 
 size_t decode_select_ws_bytes(int B, int G, int64_t max_pos) {
@@ -311,19 +353,23 @@ void launch_select_decode(const void* q_idx, const int32_t* q_pos, int64_t max_p
     unsigned int* ctr = reinterpret_cast<unsigned int*>(p + sizeof(WsHeader));
     unsigned long long* cand = reinterpret_cast<unsigned long long*>(
         p + sizeof(WsHeader) + (nbg * sizeof(unsigned int) + 255) / 256 * 256);
-    const int nchunk = decode_select_chunks(max_pos);
+    const int ncl = decode_select_clusters(B, G, max_pos);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(nchunk), static_cast<unsigned>(G), static_cast<unsigned>(B));
-    cfg.blockDim = dim3(kDecChunk);
+    cfg.gridDim = dim3(static_cast<unsigned>(ncl * kSelCluster), static_cast<unsigned>(G), static_cast<unsigned>(B));
+    cfg.blockDim = dim3(kSelThreads);
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap with the append's tail
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = kSelCluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     count_launch();
     cudaLaunchKernelEx(&cfg, select_decode_kernel, static_cast<const uint16_t*>(q_idx), q_pos, max_pos, G, pooled,
-                       nb_cap, sel, cand, ctr, nchunk, hdr);
+                       nb_cap, sel, cand, ctr, hdr);
 }
 
 }  // namespace msa

@@ -144,9 +144,10 @@ msa_status_t msa_index_select(const msa_shape_t *shape, const void *q_idx, int64
  * per step, or a host thread that must not wait on the allocator. It computes exactly what
  * msa_index_select computes in decode mode (same arguments, n_queries = 1), but keeps its
  * scratch in a 2 MiB array that libmsa holds on every GPU that loads it, until exit.
- *  - Limit: B * G * (ceil((max_pos / 128) / 128) * 120 + 4) bytes plus at most 512 must fit
- *    in the 2 MiB: B = 16, G = 8 fits up to max_pos = 2,228,351; B = 4, G = 8 up to four
- *    times that. Larger problems return MSA_ERR_WORKSPACE without launching.
+ *  - Limit: B * G * (min(ceil((max_pos / 128) / 1024), 64) * 120 + 4) bytes plus at most
+ *    512 must fit in the 2 MiB: any B * G <= 272 fits at every supported max_pos (B = 16,
+ *    G = 8 included); B * G = 1024 fits up to max_pos = 2,228,351. Larger problems return
+ *    MSA_ERR_WORKSPACE without launching.
  *  - The first call on a device looks up the array's device address (once per device); make
  *    that first call before any stream capture.
  *  - Every call shares the one array: calls that may overlap on the GPU (other streams,
