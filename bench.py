@@ -475,14 +475,16 @@ def run_ours(args):
         "prefill_index_ms": tidx * 1e3,
         "prefill_main_ms": tmain * 1e3,
         "decode_step_us": tdec * 1e6,
-        "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"], "traffic": None,
-                     "kernel": "prefill main branch (msa_sparse_attn_prefill, all its kernels)",
-                     "algorithmic": f"{flops:.4e} FLOP per launch", "peak_source": f"{peak_src} burst bf16"},
-        "roofline_decode": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": dec_gbs / peaks["hbm_gbs"], "traffic": None,
-                            "kernel": "decode step (append + select + attention, one graph replay)",
-                            "algorithmic": f"{dbytes['total']} B per step", "peak_source": f"{peak_src} copy"},
+        "roofline": ({"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
+                      "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"], "traffic": None,
+                      "kernel": "prefill main branch (msa_sparse_attn_prefill, all its kernels)",
+                      "algorithmic": f"{flops:.4e} FLOP per launch", "peak_source": f"{peak_src} burst bf16"}
+                     if do_prefill else None),
+        "roofline_decode": ({"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": dec_gbs / peaks["hbm_gbs"], "traffic": None,
+                             "kernel": "decode step (append + select + attention, one graph replay)",
+                             "algorithmic": f"{dbytes['total']} B per step", "peak_source": f"{peak_src} copy"}
+                            if do_decode else None),
         "clocks": clocks,
         "gpu_launches": int(gpu_launches),
         "e2e": e2e,
