@@ -20,7 +20,7 @@ __all__ = [
     "msa_abi_version", "msa_status_string", "msa_workspace_size",
     "msa_pool_index_keys", "msa_index_select", "msa_sparse_attn_prefill",
     "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_get_device_status",
-    "msa_index_select_decode_noalloc", "msa_kernel_launches",
+    "msa_index_select_decode_noalloc", "msa_selftest_wait_timeout", "msa_kernel_launches",
     "OP_INDEX_SELECT_PREFILL", "OP_INDEX_SELECT_DECODE", "OP_ATTN_PREFILL", "OP_ATTN_DECODE",
     "EXPORTED_SYMBOLS",
 ]
@@ -40,7 +40,7 @@ EXPORTED_SYMBOLS = [
     "msa_workspace_size",
     "msa_pool_index_keys", "msa_index_select", "msa_sparse_attn_prefill",
     "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_get_device_status",
-    "msa_index_select_decode_noalloc",
+    "msa_index_select_decode_noalloc", "msa_selftest_wait_timeout",
 ]
 
 
@@ -94,6 +94,7 @@ def load():
             "msa_sparse_attn_decode": [SP, P, P, P, I64, P, I64, P, P, P, P, SZ, P],
             "msa_get_device_status": [P, P, P],
             "msa_index_select_decode_noalloc": [SP, P, P, I64, P, I64, P, P],
+            "msa_selftest_wait_timeout": [P, SZ, P],
         }.items():
             f = getattr(L, name)
             f.restype = ctypes.c_int
@@ -195,6 +196,13 @@ def msa_get_device_status(workspace, stream=None):
     st = load().msa_get_device_status(_ptr(workspace), ctypes.cast(info, ctypes.c_void_p),
                                       _stream(stream))
     return st, list(info)
+
+
+def msa_selftest_wait_timeout(workspace, stream=None):
+    """Runs the failure-path self-test (see include/msa.h): a wait that expires after about
+    2 s and is recorded as MSA_ERR_TIMEOUT in `workspace` (>= 256 zeroed bytes)."""
+    _check(load().msa_selftest_wait_timeout(_ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "msa_selftest_wait_timeout")
 
 
 def msa_index_select_decode_noalloc(shape: Shape, q_idx, q_pos, max_pos: int, pooled, nb_cap: int, sel,

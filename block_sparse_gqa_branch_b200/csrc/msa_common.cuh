@@ -48,7 +48,7 @@ static_assert(sizeof(WsHeader) == 256, "workspace header must be 256 bytes");
 
 enum KernelId : int {
     KID_POOL = 1, KID_SELECT_PREFILL = 2, KID_SELECT_DECODE = 3, KID_APPEND = 4,
-    KID_ATTN_DECODE = 5, KID_ATTN_PREFILL = 6, KID_CSR = 7, KID_COMBINE = 8
+    KID_ATTN_DECODE = 5, KID_ATTN_PREFILL = 6, KID_CSR = 7, KID_COMBINE = 8, KID_SELFTEST = 9
 };
 
 __device__ __forceinline__ void record_error(WsHeader* h, unsigned code, int kid, int blk,

@@ -219,6 +219,18 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t *shape, const void *q, con
  */
 msa_status_t msa_get_device_status(void *workspace, int32_t *info, msa_stream_t stream);
 
+/*
+ * Self-test of the device failure path. The paper has no counterpart: it lets a caller, and
+ * the tests, check that an expired wait is reported rather than hung. One CTA of 32 threads
+ * is launched on `stream`; lane 0 waits on a shared-memory barrier that nothing completes,
+ * with the same bounded wait every kernel of the library uses (about 2 s of SM clocks), then
+ * records MSA_ERR_TIMEOUT with kernel id 9 in the workspace's error word and the kernel ends;
+ * the context stays usable. Read the result with msa_get_device_status.
+ *   workspace  device, >= 256 bytes, zero before the call (its error word is written)
+ * Returns MSA_ERR_WORKSPACE for a null or short workspace (nothing launched).
+ */
+msa_status_t msa_selftest_wait_timeout(void *workspace, size_t workspace_bytes, msa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

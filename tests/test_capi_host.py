@@ -56,6 +56,12 @@ def test_workspace_sizes(L):
     assert msa.msa_workspace_size(s, msa.OP_INDEX_SELECT_DECODE, 1 << 25) == 0          # beyond max
 
 
+def test_selftest_validates_its_workspace(L):
+    assert L.msa_selftest_wait_timeout(None, 256, None) == 3                 # MSA_ERR_WORKSPACE
+    assert L.msa_selftest_wait_timeout(FAKE, 100, None) == 3                  # too small
+    assert L.msa_selftest_wait_timeout(FAKE + 2, 256, None) == 3              # misaligned
+
+
 def _shape(**kw):
     base = dict(batch=1, n_q_heads=8, n_kv_groups=1)
     base.update(kw)
