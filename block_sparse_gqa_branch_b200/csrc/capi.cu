@@ -15,6 +15,7 @@ void launch_pool(const void*, int, int, int64_t, float*, int64_t, float*, cudaSt
 void launch_append(const void*, const void*, const void*, const int32_t*, int, int, void*, void*, int64_t,
                    float*, float*, int64_t, void*, cudaStream_t);
 void launch_select_prefill_simt(const void*, int, int, int64_t, const float*, int64_t, int32_t*, cudaStream_t);
+void launch_select_prefill_mma(const void*, int, int, int64_t, const float*, int64_t, int32_t*, cudaStream_t);
 void launch_select_decode(const void*, const int32_t*, int64_t, int, int, const float*, int64_t, int32_t*,
                           void*, cudaStream_t);
 size_t decode_select_ws_bytes(int, int, int64_t);
@@ -189,7 +190,7 @@ msa_status_t msa_index_select(const msa_shape_t* shape, const void* q_idx, int64
         MSA_REQ(nb_cap >= (n_queries - 1) / kBlock, MSA_ERR_INVALID_ARGUMENT);
         const size_t need = ws_size(shape, MSA_OP_INDEX_SELECT_PREFILL, n_queries);
         MSA_REQ(workspace != nullptr && workspace_bytes >= need, MSA_ERR_WORKSPACE);
-        launch_select_prefill_simt(q_idx, B, G, n_queries, pooled, nb_cap, sel, st);
+        launch_select_prefill_mma(q_idx, B, G, n_queries, pooled, nb_cap, sel, st);
     } else {                                       // decode: one query per sequence at q_pos[b]
         MSA_REQ(n_queries == 1, MSA_ERR_INVALID_ARGUMENT);
         MSA_REQ(max_pos <= kMaxPos, MSA_ERR_UNSUPPORTED);

@@ -131,11 +131,23 @@ def test_decode_is_last_prefill_row(cuda_ok):
                                                d["k_idx"][:, L].contiguous(), d["k"][:, :, L].contiguous(),
                                                d["v"][:, :, L].contiguous(), ctx, kc, vc, tail, pooled, dbufs)
     torch.cuda.synchronize()
-    assert (sel_d[0].cpu() == sel_p[0, L].cpu()).all()
-    a = f32(host_bits(out_d[0]))
-    b = f32(host_bits(out_p[0, L]))
+    # The two paths score in different fp32 orders (fma chains vs tensor-core sums), so their
+    # sets may differ only where the oracle's fp64 scores make a near-tie; both must be valid.
+    pooled_o, _ = oracle.pool(x["k_idx"][0, :L], 128)
+    t = np.array([L])
+    sd, sp = sel_d[0].cpu().numpy(), sel_p[0, L].cpu().numpy()
+    for g in range(2):
+        qi = x["q_idx"][0, L, g][None]
+        ref, kth, _ = oracle.select_rows(t, qi, pooled_o[g])
+        check_selection(sd[g][None], ref, kth, qi, pooled_o[g], t)
+        check_selection(sp[g][None], ref, kth, qi, pooled_o[g], t)
+    same = (sd == sp).all(axis=1)
+    assert same.any()
+    a = f32(host_bits(out_d[0])).reshape(2, 8, 128)[same]
+    b = f32(host_bits(out_p[0, L])).reshape(2, 8, 128)[same]
     assert np.abs(a - b).max() <= 1.6e-2
-    np.testing.assert_allclose(lse_d[0].cpu().numpy(), lse_p[0, L].cpu().numpy(), rtol=0, atol=1e-3)
+    np.testing.assert_allclose(lse_d[0].cpu().numpy().reshape(2, 8)[same], lse_p[0, L].cpu().numpy().reshape(2, 8)[same],
+                               rtol=0, atol=1e-3)
 
 
 def test_appends_reproduce_block_pooling(cuda_ok):
