@@ -319,6 +319,63 @@ __device__ __forceinline__ int fetch_token(const PrefillArgs a, const Item item,
     return item.diag ? item.first + e : (__ldg(a.list + item.first + e) / kSlots);
 }
 
+// Epilogue of a softmax warpgroup's tile: O from tensor memory, divided by the row sums, to
+// bf16, staged per warp and stored with TMA, plus the rows' log2-sum-exp.
+struct PendEpi {
+    int use;                 // the tile's use of its S/O buffer pair (-1: none)
+    size_t prow;             // partial row of this thread's (token, head)
+    bool valid;
+    float l, ms;             // row sum and scaled row max
+};
+__device__ __forceinline__ bool epilogue_tile(KvSmem& sm, const PrefillArgs& a, const CUtensorMap* tmO, uint32_t tO,
+                                  uint8_t* stg, uint64_t stream, int w, int lane, int Hg, int h,
+                                  const PendEpi& p) {
+    uint32_t va[32], vb[32];
+    if (!warp_wait(&sm.o_full[w], p.use & 1, a.hdr)) return false;
+    tc_fence_after();
+    const float inv_l = 1.f / p.l;
+    const float2 il = make_float2(inv_l, inv_l);
+    // this warp's 32 rows hold 32 / Hg whole tokens; lane i stores token i's Hg rows
+    const int ntok_w = 32 / Hg;
+    const int src_lane = (lane * Hg) & 31;
+    const int tok_prow = __shfl_sync(0xffffffffu, int(p.prow - h), src_lane);   // row of head 0
+    const bool tok_valid = __shfl_sync(0xffffffffu, p.valid, src_lane) && lane < ntok_w;
+    bulk_wait_read0();                  // the previous tile's stores have read the staging
+    __syncwarp();
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+        tmem_ld32(tO + half * 64, va);
+        tmem_ld32(tO + half * 64 + 32, vb);
+        tmem_wait_ld();
+        if (half == 1) {
+            tc_fence_before();
+            mbar_arrive(&sm.o_free[w]);                // O of this buffer fully read
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t o[4];
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+                const int i0 = (8 * c + 2 * e2) & 31;
+                const uint32_t x0 = c < 4 ? va[i0] : vb[i0];
+                const uint32_t x1 = c < 4 ? va[i0 + 1] : vb[i0 + 1];
+                const float2 y = fmul2(make_float2(__uint_as_float(x0), __uint_as_float(x1)), il);
+                o[e2] = pack_bf16x2(y.x, y.y);
+            }
+            *reinterpret_cast<uint4*>(stg + half * 4096 + sw128(lane, c)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+    fence_proxy_async();
+    __syncwarp();
+    if (tok_valid) {
+        tma_store_2d_hint(tmO, 0, tok_prow, stg + lane * Hg * 128, stream);
+        tma_store_2d_hint(tmO, 64, tok_prow, stg + 4096 + lane * Hg * 128, stream);
+        bulk_commit();
+    }
+    if (p.valid) __stcs(a.part_lse + p.prow, p.ms + __log2f(p.l));
+    return true;
+}
+
 __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                      const __grid_constant__ CUtensorMap tmK,
                                                                      const __grid_constant__ CUtensorMap tmV,
@@ -509,6 +566,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
         const float2 sc = make_float2(sl2, sl2);
         uint8_t* stg = sm.o_stage[warp];
         const uint64_t stream = l2_evict_first();       // partial outputs are read once, much later
+        PendEpi pend{-1, 0, false, 1.f, 0.f};
         int it = 0;
         bool ok = true;
         for (int si = 0; ok; ++si) {
@@ -584,52 +642,18 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
                 mbar_arrive(&sm.p_full[w]);
                 const float l = l2.x + l2.y;
 
-                if (!warp_wait(&sm.o_full[w], use & 1, a.hdr)) { ok = false; break; }
-                tc_fence_after();
-                const float inv_l = 1.f / l;
-                const float2 il = make_float2(inv_l, inv_l);
                 const size_t prow = ((((size_t(item.b) * a.N + t) * a.G + item.g) * kSlots + slot) * Hg + h);
-                // this warp's 32 rows hold 32 / Hg whole tokens; lane i stores token i's Hg rows
-                const int ntok_w = 32 / Hg;
-                const int src_lane = (lane * Hg) & 31;
-                const int tok_prow = __shfl_sync(0xffffffffu, int(prow - h), src_lane);   // row of head 0
-                const bool tok_valid = __shfl_sync(0xffffffffu, valid, src_lane) && lane < ntok_w;
-                bulk_wait_read0();                  // the previous tile's stores have read the staging
-                __syncwarp();
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tO + half * 64, va);
-                    tmem_ld32(tO + half * 64 + 32, vb);
-                    tmem_wait_ld();
-                    if (half == 1) {
-                        tc_fence_before();
-                        mbar_arrive(&sm.o_free[w]);                // O of this buffer fully read
-                    }
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t o[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int i0 = (8 * c + 2 * e2) & 31;
-                            const uint32_t x0 = c < 4 ? va[i0] : vb[i0];
-                            const uint32_t x1 = c < 4 ? va[i0 + 1] : vb[i0 + 1];
-                            const float2 y = fmul2(make_float2(__uint_as_float(x0), __uint_as_float(x1)), il);
-                            o[e2] = pack_bf16x2(y.x, y.y);
-                        }
-                        *reinterpret_cast<uint4*>(stg + half * 4096 + sw128(lane, c)) = make_uint4(o[0], o[1], o[2], o[3]);
-                    }
+                // the epilogue of this warpgroup's previous tile: its O was computed while this
+                // tile's S and softmax ran, so nothing waits here for the tensor cores
+                if (pend.use >= 0 && !epilogue_tile(sm, a, &tmO, tO, stg, stream, w, lane, Hg, h, pend)) {
+                    ok = false;
+                    break;
                 }
-                fence_proxy_async();
-                __syncwarp();
-                if (tok_valid) {
-                    tma_store_2d_hint(&tmO, 0, tok_prow, stg + lane * Hg * 128, stream);
-                    tma_store_2d_hint(&tmO, 64, tok_prow, stg + 4096 + lane * Hg * 128, stream);
-                    bulk_commit();
-                }
-                if (valid) __stcs(a.part_lse + prow, ms + __log2f(l));
+                pend = PendEpi{use, prow, valid, l, ms};
             }
             if (__any_sync(0xffffffffu, sm.abort_flag != 0)) ok = false;
         }
+        if (ok && pend.use >= 0) ok = epilogue_tile(sm, a, &tmO, tO, stg, stream, w, lane, Hg, h, pend);
         bulk_wait0();                               // this warp's stores are complete before exit
         __syncwarp();
         if (!ok) sm.abort_flag = 1;
