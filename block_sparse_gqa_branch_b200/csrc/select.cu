@@ -42,80 +42,6 @@ __device__ __forceinline__ void write_all_blocks(int32_t* out, int c) {
     }
 }
 
-// ------------------------------------------------------------------ prefill, CUDA cores
-// grid (ceil(N / 128), G, B), 128 threads: thread i owns query t = 128 * blockIdx.x + i.
-// All queries of one 128-token block share the candidate set [0, c), c = blockIdx.x, so the
-// CTA stages the pooled keys through shared memory 64 candidates at a time.
-__global__ void __launch_bounds__(128) select_prefill_simt_kernel(const uint16_t* __restrict__ q_idx,
-                                                                  int64_t N, int G,
-                                                                  const float* __restrict__ pooled,
-                                                                  int64_t nb_cap, int32_t* __restrict__ sel) {
-    __shared__ __align__(16) float kb[64][kIndexDim];
-    const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int64_t t = int64_t(c) * kBlock + threadIdx.x;
-    const bool live = t < N;
-    int32_t* out = sel + ((size_t(b) * N + t) * G + g) * kTopK;
-    if (c + 1 <= kTopK) {
-        if (live) write_all_blocks(out, c);
-        return;
-    }
-    float q[kIndexDim];
-    {
-        const uint4* src = reinterpret_cast<const uint4*>(q_idx + ((size_t(b) * N + (live ? t : 0)) * G + g) * kIndexDim);
-#pragma unroll
-        for (int v = 0; v < kIndexDim / 8; ++v) {
-            uint4 w = __ldg(src + v);
-            q[8 * v + 0] = bf16_lo(w.x); q[8 * v + 1] = bf16_hi(w.x);
-            q[8 * v + 2] = bf16_lo(w.y); q[8 * v + 3] = bf16_hi(w.y);
-            q[8 * v + 4] = bf16_lo(w.z); q[8 * v + 5] = bf16_hi(w.z);
-            q[8 * v + 6] = bf16_lo(w.w); q[8 * v + 7] = bf16_hi(w.w);
-        }
-    }
-    float best[kKeep];
-    int bid[kKeep];
-#pragma unroll
-    for (int k = 0; k < kKeep; ++k) { best[k] = -INFINITY; bid[k] = 0x7fffffff; }
-
-    const float4* pk = reinterpret_cast<const float4*>(pooled + (size_t(b) * G + g) * nb_cap * kIndexDim);
-    for (int j0 = 0; j0 < c; j0 += 64) {
-        const int nj = min(64, c - j0);
-        __syncthreads();
-        for (int i = threadIdx.x; i < nj * (kIndexDim / 4); i += blockDim.x)
-            reinterpret_cast<float4*>(&kb[0][0])[i] = __ldg(pk + size_t(j0) * (kIndexDim / 4) + i);
-        __syncthreads();
-        for (int jj = 0; jj < nj; ++jj) {
-            float acc = 0.f;
-#pragma unroll
-            for (int i = 0; i < kIndexDim; i += 4) {
-                const float4 kv = *reinterpret_cast<const float4*>(&kb[jj][i]);
-                acc = fmaf(q[i + 0], kv.x, acc);
-                acc = fmaf(q[i + 1], kv.y, acc);
-                acc = fmaf(q[i + 2], kv.z, acc);
-                acc = fmaf(q[i + 3], kv.w, acc);
-            }
-            if (acc > best[kKeep - 1]) {
-                best[kKeep - 1] = acc; bid[kKeep - 1] = j0 + jj;
-#pragma unroll
-                for (int k = kKeep - 1; k > 0; --k) {
-                    if (best[k] > best[k - 1]) {
-                        float tv = best[k]; best[k] = best[k - 1]; best[k - 1] = tv;
-                        int ti = bid[k]; bid[k] = bid[k - 1]; bid[k - 1] = ti;
-                    }
-                }
-            }
-        }
-    }
-    if (!live) return;
-    int ids[16];
-#pragma unroll
-    for (int k = 0; k < kKeep; ++k) ids[k] = bid[k];
-    ids[15] = c;
-    sort16(ids);
-    int4* o = reinterpret_cast<int4*>(out);
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) o[q4] = make_int4(ids[4 * q4], ids[4 * q4 + 1], ids[4 * q4 + 2], ids[4 * q4 + 3]);
-}
-
 // ------------------------------------------------------------------ prefill, warp MMAs
 // The same selection with the scores of a 128-token query block as one dense contraction
 // S = Q_I (128 x 64, bf16) x Kbar^T (64 x c) on the tensor cores (mma.sync m16n8k16, fp32
@@ -256,13 +182,6 @@ void launch_select_prefill_mma(const void* q_idx, int B, int G, int64_t N, const
     select_prefill_mma_kernel<<<grid, 128, 0, st>>>(static_cast<const uint16_t*>(q_idx), N, G, pooled, nb_cap, sel);
 }
 
-void launch_select_prefill_simt(const void* q_idx, int B, int G, int64_t N, const float* pooled,
-                                int64_t nb_cap, int32_t* sel, cudaStream_t st) {
-    dim3 grid(static_cast<unsigned>((N + kBlock - 1) / kBlock), static_cast<unsigned>(G), static_cast<unsigned>(B));
-    count_launch();
-    select_prefill_simt_kernel<<<grid, 128, 0, st>>>(static_cast<const uint16_t*>(q_idx), N, G, pooled,
-                                                      nb_cap, sel);
-}
 
 // ------------------------------------------------------------------ decode, split + merge
 // One query per (sequence, group); its candidates [0, c) are split over 8 k CTAs that form k
