@@ -5,7 +5,7 @@ One step = one pass of the whole hot path on synthetic inputs already resident i
   * prefill of 131,072 tokens, batch 1, 64 query heads / 8 KV groups (pooling, block scoring +
     exp-free top-16 selection, main-branch sparse attention), and
   * one decode step of a batch of 16 sequences at 131,072 cached tokens (append + pooled-key
-    update, selection, split-KV attention), replayed from a CUDA graph.
+    update, selection, attention split over the selected blocks), replayed from a CUDA graph.
 L2 is flushed (256 MiB write, then 256 MiB read) before every timed step, outside the events.
 
 Printed value: prefill tokens/s over all ranks (131,072 x N / slowest rank's prefill time).

@@ -437,8 +437,9 @@ void launch_select_decode(const void* q_idx, const int32_t* q_pos, int64_t max_p
 // Some callers cannot allocate device memory when they select blocks: a serving engine that
 // hands all device memory to its own pool at start-up and forbids allocation per step, or a
 // host thread that must not block on the allocator while the GPU runs. For them the decode
-// selection can keep its scratch (the arrival counters and the per-chunk candidate lists of
-// select_decode_kernel) in this file-scope device array instead of a caller workspace.
+// selection can keep its scratch (the error word, the arrival counters and the per-cluster
+// candidate lists of select_decode_kernel) in this file-scope device array instead of a
+// caller workspace.
 // Every GPU that loads libmsa holds the array until the process exits.
 #include <mutex>
 
