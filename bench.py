@@ -39,6 +39,14 @@ DECODE = synth.WORKLOADS["decode_128k_b16_h64g8"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture) of one decode
+# step of batch 16 at 131,072 tokens: select_decode_kernel 8,430,080 B and attn_decode_kernel
+# 32,128,000 B captured at batch 4 (same contexts), times 4 (both kernels' work is per
+# (sequence, group)); the append kernel's few KB are left out. Re-capture when those kernels
+# change.
+DECODE_STEP_DRAM_BYTES = 4 * (8_430_080 + 32_116_736 + 11_264)
+
+
 # ----------------------------------------------------------------------------- work counts
 def attended_pairs(N: int, Bk: int = 128, k: int = 16) -> int:
     """(query, key) pairs a causal MSA prefill of N tokens attends per (head): a query at t in
@@ -481,7 +489,8 @@ def run_ours(args):
                       "algorithmic": f"{flops:.4e} FLOP per launch", "peak_source": f"{peak_src} burst bf16"}
                      if do_prefill else None),
         "roofline_decode": ({"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                             "frac": dec_gbs / peaks["hbm_gbs"], "traffic": None,
+                             "frac": dec_gbs / peaks["hbm_gbs"],
+                             "traffic": DECODE_STEP_DRAM_BYTES if (wd.B, wd.ctx) == (16, (131072,) * 16) else None,
                              "kernel": "decode step (append + select + attention, one graph replay)",
                              "algorithmic": f"{dbytes['total']} B per step", "peak_source": f"{peak_src} copy"}
                             if do_decode else None),
