@@ -289,6 +289,17 @@ def build_decode_state(w, device):
     return {"k_cache": k_cache, "v_cache": v_cache, "pooled": pooled, "tail": tail, "ctx": ctx, **new}
 
 
+def reduce_max(x: float, world: int, device) -> float:
+    """The largest of the ranks' values (every rank calls it; one collective when world > 1)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -312,11 +323,7 @@ def run_ours(args):
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     wp, wd = workloads(args)
     do_prefill, do_decode = args.only in (None, "prefill"), args.only in (None, "decode")
