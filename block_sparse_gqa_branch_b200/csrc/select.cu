@@ -149,7 +149,18 @@ __global__ void __launch_bounds__(128, 2) select_prefill_mma_kernel(const uint16
                 scs[r + 8][col + 1] = acc[m][n][3];
             }
         __syncwarp();                                    // a warp's rows are its own lanes' queries
-        for (int jj = 0; jj < nj; ++jj) {
+        // Mark the pass's candidates above the current 15th score (no branches), then insert
+        // only those, in id order: the warp runs as many insertion rounds as its busiest lane.
+        unsigned msk = 0u;
+        {
+            const float thr = best[kKeep - 1];
+#pragma unroll
+            for (int jj = 0; jj < kSelPass; ++jj)
+                msk |= (jj < nj && scs[tid][jj] > thr) ? (1u << jj) : 0u;
+        }
+        while (msk != 0u) {
+            const int jj = __ffs(msk) - 1;
+            msk &= msk - 1u;
             const float sc = scs[tid][jj];
             if (sc > best[kKeep - 1]) {
                 best[kKeep - 1] = sc; bid[kKeep - 1] = j0 + jj;
