@@ -29,7 +29,7 @@ constexpr int kMaxTilesPerItem = 32;    // tiles per work item (K/V loaded once 
 constexpr int kSlots = 16;              // partial slots per (token, group); slot 15 = diagonal block
 constexpr int kDiagSlot = 15;
 constexpr int kDiagFlag = int(0x40000000);
-constexpr int kKvThreads = 384;         // warps 0-7 softmax/epilogue, 8 and 11 Q loads, 9 MMA, 10 K/V loads
+constexpr int kKvThreads = 352;         // warps 0-7 softmax/epilogue, 8 Q loads, 9 MMA, 10 K/V loads
 
 static_assert(kRange % kCountChunk == 0 && kRange % kBlock == 0, "range must hold whole chunks and blocks");
 
@@ -196,15 +196,15 @@ __global__ void __launch_bounds__(256) csr_fill_kernel(const int32_t* __restrict
 }
 
 // ------------------------------------------------------------------ the tensor-core kernel
-constexpr int kQStages = 2;
+constexpr int kQStages = 3;
 constexpr int kRing = 8;           // work items handed from the scheduler to the other roles
-constexpr int kRingReaders = 11;   // 2 Q warps, MMA thread, 8 softmax warps
+constexpr int kRingReaders = 10;   // Q warp, MMA thread, 8 softmax warps
 
 struct __align__(1024) KvSmem {
     uint8_t k[2][32768];          // K_j, double-buffered: [d half][128 rows][128 B], 128B swizzle
     uint8_t v[32768];             // V_j: [d half][128 rows][128 B], 128B swizzle
     uint8_t q[kQStages][32768];   // gathered query rows: [d half][128 rows][128 B], 128B swizzle
-    uint8_t o_stage[8][8192];     // per softmax warp: [d half][32 output rows][128 B] (bf16), 128B swizzle
+    uint8_t o_stage[8][4096];     // per softmax warp, one d half at a time: [32 output rows][128 B] (bf16), 128B swizzle
     uint64_t k_full[2], k_empty[2], v_full, v_empty, q_full[kQStages], q_empty[kQStages];
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
     uint64_t item_full[kRing], item_empty[kRing];
@@ -340,8 +340,6 @@ __device__ __forceinline__ bool epilogue_tile(KvSmem& sm, const PrefillArgs& a, 
     const int src_lane = (lane * Hg) & 31;
     const int tok_prow = __shfl_sync(0xffffffffu, int(p.prow - h), src_lane);   // row of head 0
     const bool tok_valid = __shfl_sync(0xffffffffu, p.valid, src_lane) && lane < ntok_w;
-    bulk_wait_read0();                  // the previous tile's stores have read the staging
-    __syncwarp();
 #pragma unroll 1
     for (int half = 0; half < 2; ++half) {
         tmem_ld32(tO + half * 64, va);
@@ -351,26 +349,29 @@ __device__ __forceinline__ bool epilogue_tile(KvSmem& sm, const PrefillArgs& a, 
             tc_fence_before();
             mbar_arrive(&sm.o_free[w]);                // O of this buffer fully read
         }
+        uint32_t o[8][4];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            uint32_t o[4];
 #pragma unroll
             for (int e2 = 0; e2 < 4; ++e2) {
                 const int i0 = (8 * c + 2 * e2) & 31;
                 const uint32_t x0 = c < 4 ? va[i0] : vb[i0];
                 const uint32_t x1 = c < 4 ? va[i0 + 1] : vb[i0 + 1];
                 const float2 y = fmul2(make_float2(__uint_as_float(x0), __uint_as_float(x1)), il);
-                o[e2] = pack_bf16x2(y.x, y.y);
+                o[c][e2] = pack_bf16x2(y.x, y.y);
             }
-            *reinterpret_cast<uint4*>(stg + half * 4096 + sw128(lane, c)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
-    }
-    fence_proxy_async();
-    __syncwarp();
-    if (tok_valid) {
-        tma_store_2d_hint(tmO, 0, tok_prow, stg + lane * Hg * 128, stream);
-        tma_store_2d_hint(tmO, 64, tok_prow, stg + 4096 + lane * Hg * 128, stream);
-        bulk_commit();
+        bulk_wait_read0();              // the staging's earlier stores have read it
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(stg + sw128(lane, c)) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+        fence_proxy_async();
+        __syncwarp();
+        if (tok_valid) {
+            tma_store_2d_hint(tmO, half * 64, tok_prow, stg + lane * Hg * 128, stream);
+            bulk_commit();
+        }
     }
     if (p.valid) __stcs(a.part_lse + p.prow, p.ms + __log2f(p.l));
     return true;
@@ -422,32 +423,30 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 8 || warp == 11) {
+    if (warp == 8) {
         // ---------------------------------------------------------------- Q gather (TMA)
-        // Warp 8 loads the even tiles (stage 0), warp 11 the odd ones (stage 1); lane r issues
-        // the copies of the tile's tokens r, r + 32, ... For Hg >= 8 one 3-D box brings 8 head rows
-        // of a token with both d halves (2 KB): the stage is laid out as 8-row groups of 2 KB
-        // ([half][8 rows][128 B], 128B swizzle). For Hg < 8 a token's Hg rows come as two 2-D boxes
-        // into [half][128 rows][128 B]. List entries of a loader's next tile are fetched ahead.
-        const int mine = warp == 8 ? 0 : 1;
+        // Tile it goes to stage it % kQStages; lane r issues the copies of the tile's tokens r,
+        // r + 32, ... For Hg >= 8 one 3-D box brings 8 head rows of a token with both d halves
+        // (2 KB): the stage is laid out as 8-row groups of 2 KB ([half][8 rows][128 B], 128B
+        // swizzle). For Hg < 8 a token's Hg rows come as two 2-D boxes into [half][128 rows][128 B].
+        // List entries of the next tile are fetched ahead. One warp produces every stage, so each
+        // stage's uses are waited for in order.
         const uint64_t keep = l2_evict_last();          // query rows are re-read ~15 times per range
         int it = 0;
         for (int sq = 0;; ++sq) {
             const int k = ring_take(sm, sq, a.hdr, true);
             if (k < 0) { if (k == -2) sm.abort_flag = 1; break; }
             const Item item = load_item(a, k);
-            const int t0 = (it & 1) == mine ? 0 : 1;                      // this warp's first tile
             int tok[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) tok[i] = fetch_token(a, item, t0, lane + 32 * i);
+            for (int i = 0; i < 4; ++i) tok[i] = fetch_token(a, item, 0, lane + 32 * i);
             for (int tt = 0; tt < item.ntiles; ++tt, ++it) {
-                if ((it & 1) != mine) continue;
-                const int use = it >> 1;
+                const int stage = it % kQStages, use = it / kQStages;
                 const int nv = min(tpt, item.n - tt * tpt);
                 bool ok = true;
                 if (lane == 0) {
-                    ok = mbar_wait(&sm.q_empty[mine], (use & 1) ^ 1, a.hdr, KID_ATTN_PREFILL);
-                    if (ok) mbar_arrive_expect_tx(&sm.q_full[mine], uint32_t(nv) * Hg * 256u);
+                    ok = mbar_wait(&sm.q_empty[stage], (use & 1) ^ 1, a.hdr, KID_ATTN_PREFILL);
+                    if (ok) mbar_arrive_expect_tx(&sm.q_full[stage], uint32_t(nv) * Hg * 256u);
                 }
                 if (!__shfl_sync(0xffffffffu, ok, 0)) { sm.abort_flag = 1; break; }
 #pragma unroll
@@ -457,15 +456,15 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
                         const int qrow = int((int64_t(item.b) * a.N + tok[i]) * a.Hq + int64_t(item.g) * Hg);
                         if (Hg >= 8) {
                             for (int h8 = 0; h8 < Hg; h8 += 8)
-                                tma_load_3d_hint(sm.q[mine] + (r * Hg + h8) * 256, &tmQ, 0, qrow + h8, 0, &sm.q_full[mine], keep);
+                                tma_load_3d_hint(sm.q[stage] + (r * Hg + h8) * 256, &tmQ, 0, qrow + h8, 0, &sm.q_full[stage], keep);
                         } else {
-                            tma_load_2d_hint(sm.q[mine] + r * Hg * 128, &tmQ, 0, qrow, &sm.q_full[mine], keep);
-                            tma_load_2d_hint(sm.q[mine] + 16384 + r * Hg * 128, &tmQ, 64, qrow, &sm.q_full[mine], keep);
+                            tma_load_2d_hint(sm.q[stage] + r * Hg * 128, &tmQ, 0, qrow, &sm.q_full[stage], keep);
+                            tma_load_2d_hint(sm.q[stage] + 16384 + r * Hg * 128, &tmQ, 64, qrow, &sm.q_full[stage], keep);
                         }
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) tok[i] = fetch_token(a, item, tt + 2, lane + 32 * i);
+                for (int i = 0; i < 4; ++i) tok[i] = fetch_token(a, item, tt + 1, lane + 32 * i);
                 __syncwarp();
             }
             if (__any_sync(0xffffffffu, sm.abort_flag != 0)) break;
