@@ -340,7 +340,10 @@ __device__ __forceinline__ bool epilogue_tile(KvSmem& sm, const PrefillArgs& a, 
     const int src_lane = (lane * Hg) & 31;
     const int tok_prow = __shfl_sync(0xffffffffu, int(p.prow - h), src_lane);   // row of head 0
     const bool tok_valid = __shfl_sync(0xffffffffu, p.valid, src_lane) && lane < ntok_w;
-#pragma unroll 1
+    // both d halves leave tensor memory first (packed to bf16 in registers), so the O buffer is
+    // free for the next tile's P V before any staging or store
+    uint32_t o[2][8][4];
+#pragma unroll
     for (int half = 0; half < 2; ++half) {
         tmem_ld32(tO + half * 64, va);
         tmem_ld32(tO + half * 64 + 32, vb);
@@ -349,7 +352,6 @@ __device__ __forceinline__ bool epilogue_tile(KvSmem& sm, const PrefillArgs& a, 
             tc_fence_before();
             mbar_arrive(&sm.o_free[w]);                // O of this buffer fully read
         }
-        uint32_t o[8][4];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
 #pragma unroll
@@ -358,14 +360,18 @@ __device__ __forceinline__ bool epilogue_tile(KvSmem& sm, const PrefillArgs& a, 
                 const uint32_t x0 = c < 4 ? va[i0] : vb[i0];
                 const uint32_t x1 = c < 4 ? va[i0 + 1] : vb[i0 + 1];
                 const float2 y = fmul2(make_float2(__uint_as_float(x0), __uint_as_float(x1)), il);
-                o[c][e2] = pack_bf16x2(y.x, y.y);
+                o[half][c][e2] = pack_bf16x2(y.x, y.y);
             }
         }
+    }
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
         bulk_wait_read0();              // the staging's earlier stores have read it
         __syncwarp();
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(stg + sw128(lane, c)) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+            *reinterpret_cast<uint4*>(stg + sw128(lane, c)) =
+                make_uint4(o[half][c][0], o[half][c][1], o[half][c][2], o[half][c][3]);
         fence_proxy_async();
         __syncwarp();
         if (tok_valid) {
