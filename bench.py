@@ -510,6 +510,65 @@ def run_ours(args):
     return 0
 
 
+def run_topk(args):
+    """Exp-free top-k micro-benchmark (one GPU): msa_topk_rows against torch.topk on the block
+    scores of 8 groups at 131,072 tokens, [1,048,576, 1024] fp32 with k = 15 (the fully-past
+    blocks a query keeps besides its own). The scores are seeded normal values generated on the
+    device; at 4.3 GB they are larger than L2, so no flush is needed between iterations."""
+    import torch
+    import block_sparse_gqa_branch_b200 as msa
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    msa.load()
+    rows, n, k = 8 * 131072, 1024, 15
+    s = torch.randn(rows, n, device=dev, generator=torch.Generator(device=dev).manual_seed(0x4D5341))
+    idx = torch.empty(rows, k, dtype=torch.int32, device=dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e-3)
+        return statistics.median(ts)
+
+    t_ref = timed(lambda: torch.topk(s, k, dim=1))
+    launches0 = msa.msa_kernel_launches()
+    with ClockSampler(local) as clk:
+        t = timed(lambda: msa.msa_topk_rows(s, k, idx))
+    launches = msa.msa_kernel_launches() - launches0
+    peaks, peak_src = load_peaks()
+    nbytes = rows * n * 4 + rows * k * 4
+    gbs = nbytes / t / 1e9
+    line = {
+        "metric": "exp-free top-k rows/s (k = 15 of 1,024 fp32 block scores per row)",
+        "value": rows / t, "unit": "rows/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded normal scores generated on the device)",
+        "config": {"workload": "topk_rows_1048576x1024_k15", "rows": rows, "n": n, "k": k,
+                   "l2": "inputs (4.3 GB) larger than L2, no flush"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "topk_rows_kernel",
+                     "algorithmic": f"{nbytes} B per launch (scores read once, ids written)",
+                     "peak_source": f"{peak_src} copy"},
+        "torch_topk_ms": t_ref * 1e3, "speedup_vs_torch_topk": t_ref / t,
+        "clocks": clk.summary(), "gpu_launches": int(launches),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -523,9 +582,13 @@ def main():
                     help="run one half of the step (profiler captures; not a benchmark value)")
     ap.add_argument("--prefill-tokens", type=int, default=0, help="smaller prefill for profiler captures")
     ap.add_argument("--decode-batch", type=int, default=0, help="smaller decode batch for profiler captures")
+    ap.add_argument("--topk", action="store_true",
+                    help="the exp-free top-k micro-benchmark against torch.topk instead of the step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.topk:
+        return run_topk(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

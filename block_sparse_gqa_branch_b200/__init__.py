@@ -21,6 +21,7 @@ __all__ = [
     "msa_pool_index_keys", "msa_index_select", "msa_sparse_attn_prefill",
     "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_get_device_status",
     "msa_index_select_decode_noalloc", "msa_selftest_wait_timeout", "msa_kernel_launches",
+    "msa_topk_rows",
     "OP_INDEX_SELECT_PREFILL", "OP_INDEX_SELECT_DECODE", "OP_ATTN_PREFILL", "OP_ATTN_DECODE",
     "EXPORTED_SYMBOLS",
 ]
@@ -40,7 +41,7 @@ EXPORTED_SYMBOLS = [
     "msa_workspace_size",
     "msa_pool_index_keys", "msa_index_select", "msa_sparse_attn_prefill",
     "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_get_device_status",
-    "msa_index_select_decode_noalloc", "msa_selftest_wait_timeout",
+    "msa_index_select_decode_noalloc", "msa_selftest_wait_timeout", "msa_topk_rows",
 ]
 
 
@@ -95,6 +96,7 @@ def load():
             "msa_get_device_status": [P, P, P],
             "msa_index_select_decode_noalloc": [SP, P, P, I64, P, I64, P, P],
             "msa_selftest_wait_timeout": [P, SZ, P],
+            "msa_topk_rows": [P, I64, I64, I32, P, P, P],
         }.items():
             f = getattr(L, name)
             f.restype = ctypes.c_int
@@ -212,3 +214,13 @@ def msa_index_select_decode_noalloc(shape: Shape, q_idx, q_pos, max_pos: int, po
     _check(load().msa_index_select_decode_noalloc(ctypes.byref(shape), _ptr(q_idx), _ptr(q_pos), max_pos,
                                                   _ptr(pooled), nb_cap, _ptr(sel), _stream(stream)),
            "msa_index_select_decode_noalloc")
+
+
+def msa_topk_rows(scores, k: int, idx, val=None, stream=None):
+    """Exp-free top-k of every row of scores (fp32 [rows, n]) into idx (int32 [rows, k]) and,
+    when given, val (fp32 [rows, k])."""
+    if scores.dim() != 2:
+        raise ValueError("msa_topk_rows takes scores of shape [rows, n]")
+    rows, n = scores.shape
+    _check(load().msa_topk_rows(_ptr(scores), rows, n, k, _ptr(idx), _ptr(val), _stream(stream)),
+           "msa_topk_rows")

@@ -213,33 +213,6 @@ constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelCluster = 8;                    // CTAs per cluster
 constexpr int kSelMaxClusters = 64;               // clusters per (sequence, group)
 
-__device__ __forceinline__ unsigned long long umax64(unsigned long long x, unsigned long long y) { return x > y ? x : y; }
-__device__ __forceinline__ unsigned long long umin64(unsigned long long x, unsigned long long y) { return x < y ? x : y; }
-
-// Bitonic sort of one key per lane, descending across the warp's lanes.
-__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
-#pragma unroll
-    for (int k = 2; k <= 32; k <<= 1) {
-#pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
-            x = (((lane & j) == 0) == ((lane & k) == 0)) ? umax64(x, y) : umin64(x, y);
-        }
-    }
-    return x;
-}
-
-// Lanes 0-15 hold a descending list, lanes 16-31 another one in ascending order (a bitonic
-// sequence): after the half-cleaners lanes 0-15 hold the 16 largest keys, descending.
-__device__ __forceinline__ unsigned long long warp_merge_desc(unsigned long long x, int lane) {
-#pragma unroll
-    for (int j = 16; j > 0; j >>= 1) {
-        const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
-        x = ((lane & j) == 0) ? umax64(x, y) : umin64(x, y);
-    }
-    return x;
-}
-
 // warp: the best 16 of two descending lists a, b of 16 (lanes 0-15 of the result)
 __device__ __forceinline__ unsigned long long merge2(const unsigned long long* a, const unsigned long long* b, int lane) {
     return warp_merge_desc(lane < 16 ? a[lane] : b[31 - lane], lane);

@@ -220,6 +220,26 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t *shape, const void *q, con
 msa_status_t msa_get_device_status(void *workspace, int32_t *info, msa_stream_t stream);
 
 /*
+ * Exp-free top-k of every row of a score matrix: the Index Branch's selection step on its
+ * own, for block scores computed elsewhere. Sources: KuCoin flash "MiniMax launches MSA
+ * sparse attention method and MiniMax-M3 model", "ME AI News" paragraph (the top-k is
+ * exp-free and is compared with torch.topk at 128K context); youmind article "MiniMax M3
+ * sparse attention agents", bullet "Fast in production".
+ *   scores  device fp32 [rows, n], row-major; rows of n >= k values, n <= 2^30
+ *   k       1..16
+ *   idx     device int32 [rows, k]: the k best columns of each row, best first, under the
+ *           total order (score descending, column ascending); every NaN ranks above +inf
+ *           (NaNs tie with each other) and -0 ties with +0
+ *   val     device fp32 [rows, k] or NULL: the scores at idx (the stored values, bit for bit)
+ * Only integer compares of order-preserving codes are used (no exponential, no float
+ * arithmetic), so the result is exact. No workspace; rows == 0 launches nothing.
+ * Returns MSA_ERR_INVALID_ARGUMENT (nothing launched) for rows < 0, k outside 1..16, n < k,
+ * n > 2^30, or a null or non-16-byte-aligned scores/idx/val pointer.
+ */
+msa_status_t msa_topk_rows(const float *scores, int64_t rows, int64_t n, int32_t k, int32_t *idx, float *val,
+                           msa_stream_t stream);
+
+/*
  * Self-test of the device failure path. The paper has no counterpart: it lets a caller, and
  * the tests, check that an expired wait is reported rather than hung. One CTA of 32 threads
  * is launched on `stream`; lane 0 waits on a shared-memory barrier that nothing completes,

@@ -51,6 +51,7 @@ def lib():
         _lib.oracle_select_from_scores.argtypes = [P, I64, I64, P, P]
         _lib.oracle_select_fullsort.restype = I64
         _lib.oracle_select_fullsort.argtypes = [P, I64, I64, P]
+        _lib.oracle_topk_rows.argtypes = [P, I64, I64, I64, P]
         _lib.oracle_attend_row.restype = I64
         _lib.oracle_attend_row.argtypes = [P, P, P, I64, I64, P, I64, I64, P, P]
         _lib.oracle_select_rows.argtypes = [I64, P, P, P, I64, I64, I64, INT, P, P, P]
@@ -105,6 +106,18 @@ def select_fullsort(s: np.ndarray, c: int, topk: int = 16):
     sel = np.zeros(topk, np.int32)
     n = lib().oracle_select_fullsort(_p(s), c, topk, _p(sel))
     return sel, int(n)
+
+
+def topk_rows(scores: np.ndarray, k: int) -> np.ndarray:
+    """Exp-free top-k of every row of fp32 scores [rows, n]: int32 [rows, k], best first
+    (score descending, column ascending; NaN above +inf; -0 == +0)."""
+    s = _c(scores, np.float32)
+    rows, n = s.shape
+    if not 1 <= k <= n:
+        raise ValueError("topk_rows needs 1 <= k <= n")
+    idx = np.zeros((rows, k), np.int32)
+    lib().oracle_topk_rows(_p(s), rows, n, k, _p(idx))
+    return idx
 
 
 def select_rows(t: np.ndarray, q_idx_rows: np.ndarray, pooled_g: np.ndarray, Bk: int = 128,

@@ -164,6 +164,38 @@ int64_t oracle_select_fullsort(const double *s, int64_t c, int64_t topk, int32_t
     return n;
 }
 
+/* ---------------------------------------------------------------- exp-free top-k of score rows */
+/* The selection step on its own, for rows of n given fp32 scores (KuCoin flash "MiniMax
+ * launches MSA sparse attention method and MiniMax-M3 model", "ME AI News" paragraph: the
+ * index branch's top-k is exp-free). Order: higher score first, then lower column; every NaN
+ * ranks above +inf and NaNs tie with each other; -0 and +0 are equal (as C's == has it). */
+static int topk_before(float a, int64_t ja, float b, int64_t jb)
+{
+    const int na = isnan(a) != 0, nb = isnan(b) != 0;
+    if (na != nb) return na;
+    if (!na && a != b) return a > b;
+    return ja < jb;
+}
+
+/* idx[row][r] = the r-th best column of the row: k rounds of "take the best column not yet
+ * taken". Requires 1 <= k <= n. */
+void oracle_topk_rows(const float *scores, int64_t rows, int64_t n, int64_t k, int32_t *idx)
+{
+    char *taken = (char *)malloc((size_t)n);
+    for (int64_t row = 0; row < rows; ++row) {
+        const float *s = scores + row * n;
+        memset(taken, 0, (size_t)n);
+        for (int64_t r = 0; r < k; ++r) {
+            int64_t best = -1;
+            for (int64_t j = 0; j < n; ++j)
+                if (!taken[j] && (best < 0 || topk_before(s[j], j, s[best], best))) best = j;
+            taken[best] = 1;
+            idx[row * k + r] = (int32_t)best;
+        }
+    }
+    free(taken);
+}
+
 /* ---------------------------------------------------------------- step 4: attention */
 static int block_selected(int64_t j, const int32_t *sel, int64_t nsel)
 {

@@ -107,3 +107,18 @@ def test_binding_rejects_host_tensors(L):
     with pytest.raises(ValueError):
         msa.msa_pool_index_keys(_shape(), torch.zeros(1, 256, 1, 64, dtype=torch.bfloat16), 256,
                                 torch.zeros(1, 1, 2, 64), 2)
+
+
+def test_topk_validation_before_launch(L):
+    ok = (FAKE, 100, 1024, 15, FAKE2, None, None)
+    for bad in ((None,) + ok[1:],                       # null scores
+                (FAKE + 4,) + ok[1:],                   # misaligned scores
+                ok[:4] + (None,) + ok[5:],              # null idx
+                ok[:4] + (FAKE2 + 8,) + ok[5:],         # misaligned idx
+                ok[:5] + (FAKE + 2,) + ok[6:],          # misaligned val
+                ok[:1] + (-1,) + ok[2:],                # rows < 0
+                ok[:3] + (0,) + ok[4:], ok[:3] + (17,) + ok[4:],     # k outside 1..16
+                ok[:2] + (14,) + ok[3:],                # n < k
+                ok[:2] + ((1 << 30) + 4,) + ok[3:]):    # n too large
+        assert L.msa_topk_rows(*bad) == 1, bad
+    assert L.msa_topk_rows(None, 0, 1024, 15, None, None, None) == 0    # no rows: nothing to do

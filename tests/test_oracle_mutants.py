@@ -27,6 +27,9 @@ MUTANTS = {
     "causal_self_excluded": ("use[u] = (sel == NULL) || block_selected(u / Bk, sel, nsel);",
                              "use[u] = (u < t || t == 0) && ((sel == NULL) || block_selected(u / Bk, sel, nsel));"),
     "pv_uses_keys": ("o[i] += p * oracle_bf16_to_f64(V[u * d + i]);", "o[i] += p * oracle_bf16_to_f64(K[u * d + i]);"),
+    "topk_ties_to_higher_column": ("    return ja < jb;\n}\n\n/* idx[row][r]", "    return ja > jb;\n}\n\n/* idx[row][r]"),
+    "topk_nan_ranked_low": ("    if (na != nb) return na;", "    if (na != nb) return nb;"),
+    "topk_ascending": ("    if (!na && a != b) return a > b;", "    if (!na && a != b) return a < b;"),
     "score_sign": ("dot += oracle_bf16_to_f64(q_idx_row[i]) * pooled_g[j * dI + i];",
                    "dot -= oracle_bf16_to_f64(q_idx_row[i]) * pooled_g[j * dI + i];"),
 }

@@ -246,3 +246,41 @@ def test_oracle_key_counts_match_closed_form():
     assert int(nk.sum()) == closed_form_total_keys(4096) == 6162432
     for tt in [2048, 2049, 3000, 4095]:
         assert nk[tt] == 1920 + tt % 128 + 1
+
+
+# ----------------------------------------------------------------------------- top-k of score rows
+# The selection step on its own (KuCoin flash "MiniMax launches MSA sparse attention method and
+# MiniMax-M3 model", "ME AI News" paragraph: exp-free top-k, compared with torch.topk).
+@pytest.mark.parametrize("seed", [0, 1])
+def test_topk_rows_match_lexsort_with_ties(seed):
+    rng = np.random.default_rng(seed)
+    rows, n, k = 40, 97, 15
+    s = (np.round(rng.standard_normal((rows, n)) * 2.0) / 2.0).astype(np.float32)   # many exact ties
+    got = oracle.topk_rows(s, k)
+    cols = np.arange(n)
+    for i in range(rows):
+        want = np.lexsort((cols, -s[i].astype(np.float64)))[:k]     # score desc, then column asc
+        assert got[i].tolist() == want.tolist()
+
+
+def test_topk_rows_distinct_values_match_torch_topk():
+    g = torch.Generator().manual_seed(5)
+    s = torch.randn(64, 1024, generator=g)
+    want = torch.topk(s, 16, dim=1, largest=True, sorted=True).indices.numpy()
+    assert (oracle.topk_rows(s.numpy(), 16) == want).all()
+
+
+def test_topk_rows_special_values():
+    nan, inf = float("nan"), float("inf")
+    row = np.array([[1.0, nan, -inf, inf, -0.0, 0.0, nan, -1.0, 2.0]], np.float32)
+    # NaNs first (lower column first), then +inf, 2, 1, the two zeros by column, -1, -inf
+    assert oracle.topk_rows(row, 9)[0].tolist() == [1, 6, 3, 8, 0, 4, 5, 7, 2]
+    assert oracle.topk_rows(row, 3)[0].tolist() == [1, 6, 3]
+
+
+def test_topk_rows_constant_and_descending_rows():
+    assert (oracle.topk_rows(np.full((3, 50), 0.25, np.float32), 16) == np.arange(16)).all()
+    desc = -np.arange(33, dtype=np.float32)[None, :].repeat(2, axis=0)
+    assert (oracle.topk_rows(desc, 16) == np.arange(16)).all()
+    asc = np.arange(33, dtype=np.float32)[None, :]
+    assert oracle.topk_rows(asc, 4)[0].tolist() == [32, 31, 30, 29]
