@@ -12,6 +12,7 @@ Printed value: prefill tokens/s over all ranks (131,072 x N / slowest rank's pre
 The same line carries the decode step latency, the index-select and main-branch split, the
 roofline fractions, the end-to-end figure through host buffers, the clocks seen, and the CPU
 oracle baseline. ``--impl reference`` times the fp64 CPU oracle instead (the reference arm).
+``--topk`` runs the exp-free top-k micro-benchmark against torch.topk instead of the step.
 """
 from __future__ import annotations
 
