@@ -83,7 +83,8 @@ def oracle_decode(w, sel_gpu):
 
 
 @pytest.mark.parametrize("ctx,Hq,G", [((4999, 2048, 127, 255), 16, 2), ((20000,), 64, 8), ((1, 0, 128 * 17), 8, 1),
-                                      ((3000, 70), 4, 4)])
+                                      ((3000, 70), 4, 4), ((3000, 129), 8, 4), ((2500, 40), 16, 4),
+                                      ((2900, 1), 16, 1)])
 def test_decode_step_matches_oracle(cuda_ok, ctx, Hq, G):
     w = synth.Workload(name="t", kind="decode", B=len(ctx), Hq=Hq, G=G, ctx=tuple(ctx), seed=4242 + sum(ctx))
     l_cap = (max(ctx) + 1 + 127) // 128 * 128 + 128

@@ -43,7 +43,7 @@ def test_pool_matches_oracle(cuda_ok, N, G):
 
 
 @pytest.mark.parametrize("N,Hq,G,planted", [(4096, 4, 1, 0), (2500, 8, 2, 0), (128 * 40 + 77, 16, 2, 8),
-                                            (3000, 16, 1, 0), (2177, 2, 2, 0), (640, 4, 4, 0)])
+                                            (3000, 16, 1, 0), (2177, 2, 2, 0), (640, 4, 4, 0), (1500, 4, 2, 0)])
 def test_prefill_matches_oracle(cuda_ok, N, Hq, G, planted):
     w = synth.Workload(name="t", kind="prefill", B=1, N=N, Hq=Hq, G=G, seed=1000 + N, planted=planted)
     x = synth.prefill_inputs_np(w)
