@@ -210,10 +210,12 @@ msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const void* q, co
                 aligned16(out) && (lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u) == 0),
             MSA_ERR_INVALID_ARGUMENT);
     const int B = shape->batch, G = shape->n_kv_groups, Hq = shape->n_q_heads, hg = Hq / G;
-    // int32 device indexing: list entries, TMA row coordinates, per-block histogram in shared memory
+    // int32 device indexing: list entries, TMA row coordinates (query rows, key/value rows, and
+    // the partial rows: one per token, query head and selected block), per-block histogram in
+    // shared memory
     MSA_REQ(int64_t(B) * n_tokens * G * (kTopK - 1) < (int64_t(1) << 31) &&
-                int64_t(B) * n_tokens * Hq < (int64_t(1) << 31) && int64_t(B) * G * n_tokens + kBlock < (int64_t(1) << 31) &&
-                (n_tokens + kBlock - 1) / kBlock <= 48 * 1024,
+                int64_t(B) * n_tokens * Hq * kTopK < (int64_t(1) << 31) &&
+                int64_t(B) * G * n_tokens + kBlock < (int64_t(1) << 31) && (n_tokens + kBlock - 1) / kBlock <= 48 * 1024,
             MSA_ERR_UNSUPPORTED);
     const size_t need = ws_size(shape, MSA_OP_ATTN_PREFILL, n_tokens);
     MSA_REQ(workspace != nullptr && aligned16(workspace) && need > 0 && workspace_bytes >= need, MSA_ERR_WORKSPACE);

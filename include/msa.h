@@ -172,6 +172,9 @@ msa_status_t msa_index_select_decode_noalloc(const msa_shape_t *shape, const voi
  *   lse  fp32 [B, N, Hq] or NULL  out: natural log of the softmax denominator of the scaled
  *                                 scores q.k/sqrt(d)
  *   workspace of msa_workspace_size(MSA_OP_ATTN_PREFILL, N)
+ * Size limits (device indices are 32-bit): B*N*Hq*k < 2^31 (one partial row per token, query
+ * head and selected block), B*N*G*(k-1) < 2^31, B*G*N + Bk < 2^31 and N/Bk <= 49152, else
+ * MSA_ERR_UNSUPPORTED before any launch.
  */
 msa_status_t msa_sparse_attn_prefill(const msa_shape_t *shape, const void *q, const void *k,
                                      const void *v, int64_t n_tokens, const int32_t *sel,

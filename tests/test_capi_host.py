@@ -94,6 +94,10 @@ def test_validation_errors_before_launch(L):
     assert L.msa_sparse_attn_prefill(bs, FAKE, FAKE, FAKE, 0, FAKE, FAKE, None, FAKE, 1 << 20, None) == 1
     assert L.msa_sparse_attn_prefill(bs, FAKE, FAKE, FAKE, 100, FAKE, FAKE, FAKE + 2, FAKE, 1 << 20, None) == 1
     assert L.msa_sparse_attn_prefill(bs, FAKE, FAKE, FAKE, 100, FAKE, FAKE, None, None, 0, None) == 3
+    # 32-bit device indices: B*N*Hq*16 partial rows must stay below 2^31 (here exactly 2^31)
+    big = ctypes.byref(_shape(n_q_heads=64, n_kv_groups=8))
+    assert L.msa_sparse_attn_prefill(big, FAKE, FAKE, FAKE, 1 << 21, FAKE, FAKE, None, FAKE, 1 << 62, None) == 2
+    assert L.msa_sparse_attn_prefill(big, FAKE, FAKE, FAKE, 1 << 20, FAKE, FAKE, None, FAKE, 16, None) == 3
     # decode attention: position bound beyond the cache, workspace
     assert L.msa_sparse_attn_decode(bs, FAKE, FAKE, FAKE, 1000, FAKE, 1000, FAKE, FAKE, None, FAKE, 1 << 20, None) == 1
     assert L.msa_sparse_attn_decode(bs, FAKE, FAKE, FAKE, 1000, FAKE, 999, FAKE, FAKE, None, FAKE, 64, None) == 3
