@@ -22,6 +22,8 @@
 //     hold parts of the group: if all of them are in it merges their partials (max, sum, o)
 //     into its registers, otherwise it leaves its own partial for the last one to arrive.
 //     None of this global-memory traffic stalls the compute warps.
+#include <atomic>
+
 #include "msa_common.cuh"
 
 namespace msa {
@@ -672,12 +674,12 @@ msa_status_t launch_attn_decode(const void* k_cache, const void* v_cache, const 
     a.part = reinterpret_cast<float*>(p + sizeof(WsHeader) + (nbg * sizeof(unsigned int) + 255) / 256 * 256);
     a.scale_log2 = 1.4426950408889634f / sqrtf(float(kHeadDim));
     const int smem = int(sizeof(DecSmem)) + 1024;
-    static bool attr_set[64] = {false};
+    static std::atomic<bool> attr_set[64];          // per device; setting it twice is harmless
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
         cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_relaxed);
     }
     const int64_t n_items = int64_t(B) * G * kTopK;
     const int grid = int(n_items < num_sms() ? n_items : num_sms());   // persistent: one CTA per SM

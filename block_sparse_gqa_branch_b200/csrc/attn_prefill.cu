@@ -19,6 +19,8 @@
 // Work order. Lists are keyed by (sequence, group, range of kRange query tokens, block), and
 // the persistent CTAs walk the work in that order, so the query rows gathered at any moment
 // come from one 16K-token range of one group (32 MB at Hg = 8) and stay in L2.
+#include <atomic>
+
 #include "msa_common.cuh"
 
 namespace msa {
@@ -742,12 +744,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict_
 
 // ------------------------------------------------------------------ host launcher
 int num_sms() {
-    static int n[64] = {0};
+    static std::atomic<int> n[64];                  // per device, filled on first use
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
-    if (n[dev] == 0) cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
-    return n[dev] > 0 ? n[dev] : 148;
+    int v = n[dev].load(std::memory_order_relaxed);
+    if (v == 0 && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+        n[dev].store(v, std::memory_order_relaxed);
+    return v > 0 ? v : 148;
 }
 
 msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, const CUtensorMap& tmK, const CUtensorMap& tmV, int64_t N,
@@ -790,12 +794,12 @@ msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, cons
         a.hdr = hdr;
         a.scale_log2 = 1.4426950408889634f / sqrtf(float(kHeadDim));
         const int smem = int(sizeof(KvSmem)) + 1024;
-        static bool attr_set[64] = {false};
+        static std::atomic<bool> attr_set[64];      // per device; setting it twice is harmless
         int dev = 0;
         cudaGetDevice(&dev);
-        if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
             cudaFuncSetAttribute(attn_kvmajor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            attr_set[dev] = true;
+            attr_set[dev].store(true, std::memory_order_relaxed);
         }
         CUtensorMap tmO, tmQ3;
         msa_status_t st_map = make_tmap_bf16(&tmO, part_o, uint64_t(B) * N * G * kSlots * Hg, kHeadDim, 64, uint32_t(Hg));

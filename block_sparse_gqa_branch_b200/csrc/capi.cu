@@ -32,13 +32,16 @@ thread_local int g_last_cuda_error = 0;
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda)
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> cached{nullptr};
+    PFN_cuTensorMapEncodeTiled_v12000 fn = cached.load(std::memory_order_acquire);
     if (fn == nullptr) {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
+            q == cudaDriverEntryPointSuccess) {
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+            cached.store(fn, std::memory_order_release);
+        }
     }
     return fn;
 }
