@@ -65,8 +65,11 @@ def prefill_main_flops(w) -> float:
 
 
 def prefill_index_flops(w) -> float:
-    cand = sum(min(t // w.Bk, 10 ** 12) for t in range(0, w.N, 1)) if w.N <= 0 else \
-        w.Bk * sum(c for c in range(w.N // w.Bk)) + (w.N % w.Bk) * (w.N // w.Bk)
+    """2 * d_I FLOP per (query, group, candidate): a query at t scores its t // Bk fully-past
+    blocks, so a full block c contributes Bk * c candidates and the ragged tail (N mod Bk) *
+    (N // Bk)."""
+    nbf = w.N // w.Bk
+    cand = w.Bk * (nbf * (nbf - 1) // 2) + (w.N % w.Bk) * nbf
     return 2.0 * w.dI * w.G * w.B * cand
 
 

@@ -1,0 +1,62 @@
+"""The benchmark's work counts (the numerators of its roofline fractions) against the golden
+key counts and closed forms, on the CPU. Sources: youmind article "MiniMax M3 sparse attention
+agents", bullet "Predictable cost at every length" (Bk = 128, k = 16: 2,048 key-value tokens
+per query and GQA group)."""
+import json
+import os
+
+import pytest
+
+import bench
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "key_counts.json")
+
+
+def test_attended_pairs_match_golden_totals():
+    totals = json.load(open(GOLDEN))["totals"]
+    for n, want in totals.items():
+        assert bench.attended_pairs(int(n)) == want
+
+
+@pytest.mark.parametrize("N,Bk,k", [(1000, 16, 4), (77, 8, 3), (64, 16, 4)])
+def test_attended_pairs_by_explicit_key_sets(N, Bk, k):
+    # every query keeps its own block plus up to k-1 full past blocks: count the keys of an
+    # explicit selection (the first k-1 past blocks) one by one
+    total = 0
+    for t in range(N):
+        c = t // Bk
+        sel = set(range(c + 1)) if c + 1 <= k else set(range(k - 1)) | {c}
+        total += sum(1 for u in range(t + 1) if u // Bk in sel)
+    assert bench.attended_pairs(N, Bk, k) == total
+
+
+def test_prefill_flop_counts():
+    w = bench.PREFILL
+    assert (w.N, w.Hq, w.G, w.d, w.dI) == (131072, 64, 8, 128, 64)
+    assert bench.prefill_main_flops(w) == 4 * 128 * 64 * 258146304          # 8.459e12
+    nb = 131072 // 128                                                        # 1,024 blocks
+    assert bench.prefill_index_flops(w) == 2 * 64 * 8 * 128 * (nb * (nb - 1) // 2)   # 6.87e10
+
+
+def test_prefill_index_flops_ragged_tail_by_enumeration():
+    import dataclasses
+    w = dataclasses.replace(bench.PREFILL, N=128 * 5 + 37)
+    cand = sum(t // 128 for t in range(w.N))
+    assert bench.prefill_index_flops(w) == 2 * 64 * w.G * w.B * cand
+
+
+def test_decode_step_bytes_closed_form():
+    w = bench.DECODE
+    assert (w.B, w.Hq, w.G) == (16, 64, 8) and set(w.ctx) == {131072}
+    d = bench.decode_step_bytes(w)
+    per_bg_pooled = 1024 * 64 * 4                          # every fully-past block's pooled key
+    per_bg_kv = (15 * 128 + 1) * 128 * 2 * 2               # 15 full blocks + the new token, K and V
+    small = 16 * (64 * 128 * 2 * 2 + 8 * 64 * 2 * 2 + 8 * 128 * 2 * 2 * 2 + 8 * 64 * 4 * 2 + 8 * 16 * 4)
+    assert d["pooled"] == 128 * per_bg_pooled
+    assert d["kv"] == 128 * per_bg_kv
+    assert d["total"] == 128 * (per_bg_pooled + per_bg_kv) + small == 160210944
+
+
+def test_captured_decode_traffic_is_close_to_the_algorithmic_bytes():
+    ratio = bench.DECODE_STEP_DRAM_BYTES / bench.decode_step_bytes(bench.DECODE)["total"]
+    assert 1.0 <= ratio < 1.03
