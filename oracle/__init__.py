@@ -52,6 +52,14 @@ def lib():
         _lib.oracle_select_fullsort.restype = I64
         _lib.oracle_select_fullsort.argtypes = [P, I64, I64, P]
         _lib.oracle_topk_rows.argtypes = [P, I64, I64, I64, P]
+        _lib.oracle_e4m3_to_f64.restype = ctypes.c_double
+        _lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        _lib.oracle_e4m3_from_f32.restype = ctypes.c_uint8
+        _lib.oracle_e4m3_from_f32.argtypes = [ctypes.c_float]
+        _lib.oracle_fp8_quantize_block.restype = ctypes.c_float
+        _lib.oracle_fp8_quantize_block.argtypes = [P, I64, P]
+        _lib.oracle_attend_row_fp8.restype = I64
+        _lib.oracle_attend_row_fp8.argtypes = [P, P, P, P, P, P, P, I64, I64, P, I64, I64, P, P]
         _lib.oracle_attend_row.restype = I64
         _lib.oracle_attend_row.argtypes = [P, P, P, I64, I64, P, I64, I64, P, P]
         _lib.oracle_select_rows.argtypes = [I64, P, P, P, I64, I64, I64, INT, P, P, P]
@@ -118,6 +126,59 @@ def topk_rows(scores: np.ndarray, k: int) -> np.ndarray:
     idx = np.zeros((rows, k), np.int32)
     lib().oracle_topk_rows(_p(s), rows, n, k, _p(idx))
     return idx
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Values of e4m3 codes (uint8), by the format's definition."""
+    c = np.asarray(codes, np.uint8)
+    return np.array([lib().oracle_e4m3_to_f64(int(v)) for v in c.ravel()], np.float64).reshape(c.shape)
+
+
+def e4m3_from_f32(x) -> np.ndarray:
+    """Nearest e4m3 codes of fp32 values (ties to even mantissa, saturating at +-448)."""
+    a = np.asarray(x, np.float32)
+    return np.array([lib().oracle_e4m3_from_f32(float(v)) for v in a.ravel()], np.uint8).reshape(a.shape)
+
+
+def fp8_quantize_blocks(x_bits: np.ndarray, Bk: int = 128):
+    """Per-block e4m3 quantisation of bf16 rows [L, d]: (codes [L, d] uint8, scales [ceil(L/Bk)]
+    fp32), one scale per block of Bk rows."""
+    x = _c(x_bits, np.uint16)
+    L, d = x.shape
+    codes = np.zeros((L, d), np.uint8)
+    nb = (L + Bk - 1) // Bk
+    scales = np.zeros(nb, np.float32)
+    for j in range(nb):
+        blk = np.ascontiguousarray(x[j * Bk:(j + 1) * Bk])
+        out = np.zeros(blk.shape, np.uint8)
+        scales[j] = lib().oracle_fp8_quantize_block(_p(blk), blk.size, _p(out))
+        codes[j * Bk:(j + 1) * Bk] = out
+    return codes, scales
+
+
+def attend_row_fp8(t: int, q_rows: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, ks: np.ndarray,
+                   vs: np.ndarray, K: np.ndarray, V: np.ndarray, sel: Optional[np.ndarray] = None,
+                   Bk: int = 128):
+    """Attention of the query heads q_rows [Hg, d] (bf16 bits) at position t over the FP8 cache
+    (codes Kc, Vc [L, d], scales ks, vs per block) with the query's own block from the bf16 rows
+    K, V [L, d]. Returns (o [Hg, d], lse [Hg], keys attended)."""
+    q = _c(q_rows, np.uint16)
+    Kc, Vc = _c(Kc, np.uint8), _c(Vc, np.uint8)
+    ks, vs = _c(ks, np.float32), _c(vs, np.float32)
+    K, V = _c(K, np.uint16), _c(V, np.uint16)
+    Hg, d = q.shape
+    s = None if sel is None else _c(sel, np.int32)
+    ns = 0 if s is None else int((s >= 0).sum())
+    o = np.zeros((Hg, d), np.float64)
+    lse = np.zeros(Hg, np.float64)
+    nk = 0
+    for h in range(Hg):
+        oh = np.zeros(d, np.float64)
+        lh = np.zeros(1, np.float64)
+        nk = lib().oracle_attend_row_fp8(_p(np.ascontiguousarray(q[h])), _p(Kc), _p(Vc), _p(ks), _p(vs),
+                                         _p(K), _p(V), d, t, _p(s), ns, Bk, _p(oh), _p(lh))
+        o[h], lse[h] = oh, lh[0]
+    return o, lse, int(nk)
 
 
 def select_rows(t: np.ndarray, q_idx_rows: np.ndarray, pooled_g: np.ndarray, Bk: int = 128,

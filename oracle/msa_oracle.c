@@ -240,6 +240,107 @@ int64_t oracle_attend_row(const uint16_t *q_row, const uint16_t *K, const uint16
     return nk;
 }
 
+/* ---------------------------------------------------------------- FP8 (e4m3) key-value cache */
+/* The compressed cache of the decode variant (KuCoin flash "MiniMax launches MSA sparse
+ * attention method and MiniMax-M3 model", "ME AI News" paragraph: the SM100 kernel also
+ * takes FP8 inputs). Reading taken: every closed block of Bk keys (or values) of one group
+ * is stored as e4m3 codes with one fp32 scale per block; the open block, which is also the
+ * newest query's own block, stays in bf16 until it fills.
+ *
+ * e4m3 ("E4M3FN"): sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities, the
+ * pattern S.1111.111 is NaN, largest finite value 448, subnormals m * 2^-9. */
+double oracle_e4m3_to_f64(uint8_t c)
+{
+    const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* The e4m3 code nearest to x (ties to the code with an even mantissa), |x| > 448 saturating
+ * to +-448: a search over the 127 non-negative finite codes, ascending. */
+uint8_t oracle_e4m3_from_f32(float x)
+{
+    const int s = signbit(x) ? 1 : 0;
+    const double a = fabs((double)x);
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c <= 126; ++c) {
+        const double dist = fabs(oracle_e4m3_to_f64((uint8_t)c) - a);
+        if (dist < bd || (dist == bd && (c & 1) == 0)) { bd = dist; best = c; }
+    }
+    if (a > 448.0) best = 126;
+    return (uint8_t)(best | (s << 7));
+}
+
+/* One block of n bf16 values: scale = amax / 448 in fp32 (1 for an all-zero block), and
+ * codes[i] = e4m3(x_i / scale) with the division in fp32 (the precision that decides the
+ * code on both sides). Returns the scale. */
+float oracle_fp8_quantize_block(const uint16_t *x, int64_t n, uint8_t *codes)
+{
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        const float v = (float)fabs(oracle_bf16_to_f64(x[i]));
+        if (v > amax) amax = v;
+    }
+    const float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        const float q = (float)oracle_bf16_to_f64(x[i]) / scale;
+        codes[i] = oracle_e4m3_from_f32(q);
+    }
+    return scale;
+}
+
+/* Step 4 over the FP8 cache: keys and values of the fully-past blocks j < floor(t / Bk) are
+ * code * scale (exact in fp64), those of the query's own block come from the bf16 rows;
+ * everything else as in oracle_attend_row. Kc, Vc [L][d] codes; ks, vs one scale per block. */
+int64_t oracle_attend_row_fp8(const uint16_t *q_row, const uint8_t *Kc, const uint8_t *Vc, const float *ks,
+                              const float *vs, const uint16_t *K, const uint16_t *V, int64_t d, int64_t t,
+                              const int32_t *sel, int64_t nsel, int64_t Bk, double *o, double *lse)
+{
+    const double scale = 1.0 / sqrt((double)d);
+    const int64_t c = t / Bk;
+    double *qd = (double *)malloc((size_t)d * sizeof(double));
+    double *z = (double *)malloc((size_t)(t + 1) * sizeof(double));
+    char *use = (char *)malloc((size_t)(t + 1));
+    for (int64_t i = 0; i < d; ++i) qd[i] = oracle_bf16_to_f64(q_row[i]);
+    int64_t nk = 0;
+    double m = -INFINITY;
+    for (int64_t u = 0; u <= t; ++u) {
+        use[u] = (sel == NULL) || block_selected(u / Bk, sel, nsel);
+        if (!use[u]) continue;
+        const int64_t j = u / Bk;
+        double dot = 0.0;
+        for (int64_t i = 0; i < d; ++i) {
+            const double k = j < c ? oracle_e4m3_to_f64(Kc[u * d + i]) * (double)ks[j]
+                                   : oracle_bf16_to_f64(K[u * d + i]);
+            dot += qd[i] * k;
+        }
+        z[u] = dot * scale;
+        if (z[u] > m) m = z[u];
+        ++nk;
+    }
+    double den = 0.0;
+    for (int64_t i = 0; i < d; ++i) o[i] = 0.0;
+    for (int64_t u = 0; u <= t; ++u) {
+        if (!use[u]) continue;
+        const int64_t j = u / Bk;
+        const double p = exp(z[u] - m);
+        den += p;
+        for (int64_t i = 0; i < d; ++i) {
+            const double v = j < c ? oracle_e4m3_to_f64(Vc[u * d + i]) * (double)vs[j]
+                                   : oracle_bf16_to_f64(V[u * d + i]);
+            o[i] += p * v;
+        }
+    }
+    for (int64_t i = 0; i < d; ++i) o[i] /= den;
+    if (lse) *lse = m + log(den);
+    free(qd); free(z); free(use);
+    return nk;
+}
+
 /* ---------------------------------------------------------------- row batches (threads) */
 typedef struct {
     int kind;   /* 0 = select, 1 = attend */

@@ -30,6 +30,10 @@ MUTANTS = {
     "topk_ties_to_higher_column": ("    return ja < jb;\n}\n\n/* idx[row][r]", "    return ja > jb;\n}\n\n/* idx[row][r]"),
     "topk_nan_ranked_low": ("    if (na != nb) return na;", "    if (na != nb) return nb;"),
     "topk_ascending": ("    if (!na && a != b) return a > b;", "    if (!na && a != b) return a < b;"),
+    "e4m3_bias": ("    else v = ldexp(1.0 + m / 8.0, e - 7);", "    else v = ldexp(1.0 + m / 8.0, e - 8);"),
+    "e4m3_ties_to_odd": ("if (dist < bd || (dist == bd && (c & 1) == 0))", "if (dist < bd || (dist == bd && (c & 1) == 1))"),
+    "fp8_scale_divisor": ("amax > 0.0f ? amax / 448.0f : 1.0f", "amax > 0.0f ? amax / 240.0f : 1.0f"),
+    "fp8_open_block_from_codes": ("            const double k = j < c ?", "            const double k = j <= c ?"),
     "score_sign": ("dot += oracle_bf16_to_f64(q_idx_row[i]) * pooled_g[j * dI + i];",
                    "dot -= oracle_bf16_to_f64(q_idx_row[i]) * pooled_g[j * dI + i];"),
 }

@@ -284,3 +284,93 @@ def test_topk_rows_constant_and_descending_rows():
     assert (oracle.topk_rows(desc, 16) == np.arange(16)).all()
     asc = np.arange(33, dtype=np.float32)[None, :]
     assert oracle.topk_rows(asc, 4)[0].tolist() == [32, 31, 30, 29]
+
+
+# ----------------------------------------------------------------------------- FP8 (e4m3) key-value cache
+# The compressed cache of the decode variant (KuCoin flash "MiniMax launches MSA sparse attention
+# method and MiniMax-M3 model", "ME AI News" paragraph: the SM100 kernel also takes FP8 inputs).
+def test_e4m3_decode_matches_torch_float8():
+    codes = torch.arange(256, dtype=torch.uint8)
+    want = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.e4m3_to_f64(codes.numpy())
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert (got[ok] == want[ok]).all() and (np.signbit(got[ok]) == np.signbit(want[ok])).all()
+
+
+def test_e4m3_encode_matches_torch_rounding():
+    # every finite code, every midpoint between neighbouring codes (the ties), random values;
+    # |x| <= 464, where torch's cast and a saturating one agree
+    grid = oracle.e4m3_to_f64(np.arange(127, dtype=np.uint8))
+    mids = (grid[:-1] + grid[1:]) / 2
+    rng = np.random.default_rng(0)
+    rnd = rng.uniform(-464, 464, 20000) * 10.0 ** rng.uniform(-6, 0, 20000)
+    x = np.concatenate([grid, -grid[1:], mids, -mids, rnd, [464.0, -464.0]]).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert (oracle.e4m3_from_f32(x) == want).all()
+
+
+def test_e4m3_saturates_beyond_448():
+    x = np.array([448.5, 463.9, 465.0, 1e6, 3e38, -500.0], np.float32)
+    assert oracle.e4m3_from_f32(x).tolist() == [126, 126, 126, 126, 126, 254]
+
+
+def test_fp8_block_quantisation_bounds():
+    rng = np.random.default_rng(1)
+    xb = synth.f64_to_bf16_bits(rng.standard_normal((300, 128)) * 3.0)
+    codes, scales = oracle.fp8_quantize_blocks(xb, 128)
+    assert len(scales) == 3
+    x = f32(xb)
+    for j in range(3):
+        blk = x[j * 128:(j + 1) * 128]
+        amax = np.abs(blk).max()
+        assert abs(scales[j] - amax / 448.0) <= amax / 448.0 * 2.0 ** -23
+        cv = oracle.e4m3_to_f64(codes[j * 128:(j + 1) * 128])
+        assert np.abs(cv).max() == 448.0                    # the largest magnitude maps to 448
+        # 3 mantissa bits: half a unit in the last place is at most 2^-4 of |x|; the subnormal
+        # spacing 2^-9 leaves at most 2^-10 absolute; both in units of the scale
+        err = np.abs(cv * float(scales[j]) - blk)
+        assert (err <= (np.abs(blk) * 2.0 ** -4 + 2.0 ** -10 * float(scales[j])) * (1 + 1e-6)).all()
+    zc, zs = oracle.fp8_quantize_blocks(np.zeros((5, 128), np.uint16), 128)
+    assert zs.tolist() == [1.0] and not zc.any()
+
+
+def test_fp8_quantisation_commutes_with_powers_of_two():
+    rng = np.random.default_rng(2)
+    xb = synth.f64_to_bf16_bits(rng.standard_normal((128, 128)))
+    c1, s1 = oracle.fp8_quantize_blocks(xb)
+    c2, s2 = oracle.fp8_quantize_blocks(synth.f64_to_bf16_bits(f32(xb) * 2.0 ** 5))
+    assert (c1 == c2).all() and s2[0] == s1[0] * 2.0 ** 5
+
+
+def test_fp8_attention_equals_bf16_attention_on_a_representable_cache():
+    # closed blocks hold exactly code * 2^e with a +-448 in every block, so quantisation gives
+    # back the same codes and scales 2^e, and attention over the FP8 cache must equal step 4 on
+    # the bf16 cache bit for bit; the open block holds arbitrary bf16 values, which only the
+    # bf16 rows carry exactly
+    rng = np.random.default_rng(3)
+    L, d, Bk, Hg = 128 * 20 + 17, 128, 128, 4
+    nb_closed = L // Bk
+    finite = np.array([c for c in range(1, 255) if c not in (127, 128)], np.uint8)
+
+    def cache():
+        codes = rng.choice(finite, size=(L, d))
+        vals = oracle.e4m3_to_f64(codes)
+        for j in range(nb_closed):
+            vals[j * Bk, 0] = 448.0
+            vals[j * Bk:(j + 1) * Bk] *= 2.0 ** int(rng.integers(-9, -3))
+        vals[nb_closed * Bk:] = rng.standard_normal((L - nb_closed * Bk, d))
+        return synth.f64_to_bf16_bits(vals)
+
+    K, V = cache(), cache()
+    Kc, ks = oracle.fp8_quantize_blocks(K, Bk)
+    Vc, vs = oracle.fp8_quantize_blocks(V, Bk)
+    assert (oracle.e4m3_to_f64(Kc[:nb_closed * Bk]) * np.repeat(ks[:nb_closed], Bk)[:, None]
+            == f32(K[:nb_closed * Bk])).all()
+    q = synth.f64_to_bf16_bits(rng.standard_normal((Hg, d)))
+    t = L - 1
+    sel = np.array([0, 1, 2, 3, 5, 6, 7, 9, 10, 11, 13, 14, 15, 17, 19, t // Bk], np.int32)
+    o8, l8, n8 = oracle.attend_row_fp8(t, q, Kc, Vc, ks, vs, K, V, sel, Bk)
+    o, l, n = oracle.attend_rows(np.array([t]), q[None], K, V, sel[None], Bk)
+    assert n8 == n[0] == 15 * Bk + (t % Bk) + 1
+    assert np.array_equal(o8, o[0]) and np.array_equal(l8, l[0])
