@@ -23,9 +23,9 @@ MUTANTS = {
     "one_block_too_few": ("for (int64_t r = 0; r < topk - 1; ++r) {\n            int64_t best",
                           "for (int64_t r = 0; r < topk - 2; ++r) {\n            int64_t best"),
     "diagonal_dropped": ("        free(taken);\n        sel[n++] = (int32_t)c;", "        free(taken);"),
-    "softmax_scale": ("double scale = 1.0 / sqrt((double)d);", "double scale = 1.0 / sqrt((double)d * 2.0);"),
-    "causal_self_excluded": ("use[u] = (sel == NULL) || block_selected(u / Bk, sel, nsel);",
-                             "use[u] = (u < t || t == 0) && ((sel == NULL) || block_selected(u / Bk, sel, nsel));"),
+    "softmax_scale": ("    double scale = 1.0 / sqrt((double)d);", "    double scale = 1.0 / sqrt((double)d * 2.0);"),
+    "causal_self_excluded": ("use[u] = (sel == NULL) || block_selected(u / Bk, sel, nsel);\n        if (!use[u]) continue;\n        double dot",
+                             "use[u] = (u < t || t == 0) && ((sel == NULL) || block_selected(u / Bk, sel, nsel));\n        if (!use[u]) continue;\n        double dot"),
     "pv_uses_keys": ("o[i] += p * oracle_bf16_to_f64(V[u * d + i]);", "o[i] += p * oracle_bf16_to_f64(K[u * d + i]);"),
     "topk_ties_to_higher_column": ("    return ja < jb;\n}\n\n/* idx[row][r]", "    return ja > jb;\n}\n\n/* idx[row][r]"),
     "topk_nan_ranked_low": ("    if (na != nb) return na;", "    if (na != nb) return nb;"),
