@@ -52,6 +52,7 @@ def lib():
         _lib.oracle_select_fullsort.restype = I64
         _lib.oracle_select_fullsort.argtypes = [P, I64, I64, P]
         _lib.oracle_topk_rows.argtypes = [P, I64, I64, I64, P]
+        _lib.oracle_attend_row_grad.argtypes = [P, P, P, I64, I64, P, I64, I64, P, P, P, P]
         _lib.oracle_e4m3_to_f64.restype = ctypes.c_double
         _lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         _lib.oracle_e4m3_from_f32.restype = ctypes.c_uint8
@@ -126,6 +127,31 @@ def topk_rows(scores: np.ndarray, k: int) -> np.ndarray:
     idx = np.zeros((rows, k), np.int32)
     lib().oracle_topk_rows(_p(s), rows, n, k, _p(idx))
     return idx
+
+
+def attend_grad(t: np.ndarray, q_rows: np.ndarray, K: np.ndarray, V: np.ndarray, sel: Optional[np.ndarray],
+                dO: np.ndarray, Bk: int = 128):
+    """Gradient of step 4 for queries of one (sequence, group), the selection held fixed.
+    q_rows [n, Hg, d] (bf16 bits), K, V [L, d] (bf16 bits), sel [n, k] or None (every key u <= t),
+    dO [n, Hg, d] (float64). Returns (dQ [n, Hg, d], dK [L, d], dV [L, d]) in float64, dK and dV
+    summed over every row and head."""
+    t = _c(t, np.int64)
+    q = _c(q_rows, np.uint16)
+    K, V = _c(K, np.uint16), _c(V, np.uint16)
+    g = _c(dO, np.float64)
+    n, Hg, d = q.shape
+    dQ = np.zeros((n, Hg, d), np.float64)
+    dK = np.zeros(K.shape, np.float64)
+    dV = np.zeros(V.shape, np.float64)
+    for r in range(n):
+        s = None if sel is None else _c(sel[r], np.int32)
+        ns = 0 if s is None else int((s >= 0).sum())
+        for h in range(Hg):
+            out = np.zeros(d, np.float64)
+            lib().oracle_attend_row_grad(_p(np.ascontiguousarray(q[r, h])), _p(K), _p(V), d, int(t[r]), _p(s), ns,
+                                         Bk, _p(np.ascontiguousarray(g[r, h])), _p(out), _p(dK), _p(dV))
+            dQ[r, h] = out
+    return dQ, dK, dV
 
 
 def e4m3_to_f64(codes) -> np.ndarray:

@@ -240,6 +240,58 @@ int64_t oracle_attend_row(const uint16_t *q_row, const uint16_t *K, const uint16
     return nk;
 }
 
+/* ---------------------------------------------------------------- step 4, gradient */
+/* Gradient of step 4 for one query head at position t, the selection held fixed (it is a
+ * discrete choice), given the upstream gradient dO of the output o: writes dQ[d] and adds
+ * this row's contributions to dK[u][d] and dV[u][d] for the keys u it attends. With
+ * z_u = s q.k_u (s = 1/sqrt(d)), p = softmax(z) and o = sum_u p_u v_u:
+ *   dV_u += p_u dO,   dp_u = dO.v_u,   dz_u = p_u (dp_u - dO.o),
+ *   dQ = s sum_u dz_u k_u,   dK_u += s dz_u q.                                              */
+void oracle_attend_row_grad(const uint16_t *q_row, const uint16_t *K, const uint16_t *V, int64_t d,
+                            int64_t t, const int32_t *sel, int64_t nsel, int64_t Bk, const double *dO,
+                            double *dQ, double *dK, double *dV)
+{
+    const double s = 1.0 / sqrt((double)d);
+    double *qd = (double *)malloc((size_t)d * sizeof(double));
+    double *o = (double *)malloc((size_t)d * sizeof(double));
+    double *p = (double *)malloc((size_t)(t + 1) * sizeof(double));
+    char *use = (char *)malloc((size_t)(t + 1));
+    for (int64_t i = 0; i < d; ++i) qd[i] = oracle_bf16_to_f64(q_row[i]);
+    double m = -INFINITY;
+    for (int64_t u = 0; u <= t; ++u) {
+        use[u] = (sel == NULL) || block_selected(u / Bk, sel, nsel);
+        if (!use[u]) continue;
+        double dot = 0.0;
+        for (int64_t i = 0; i < d; ++i) dot += qd[i] * oracle_bf16_to_f64(K[u * d + i]);
+        p[u] = dot * s;
+        if (p[u] > m) m = p[u];
+    }
+    double den = 0.0;
+    for (int64_t u = 0; u <= t; ++u)
+        if (use[u]) { p[u] = exp(p[u] - m); den += p[u]; }
+    for (int64_t i = 0; i < d; ++i) o[i] = 0.0;
+    for (int64_t u = 0; u <= t; ++u) {
+        if (!use[u]) continue;
+        p[u] /= den;
+        for (int64_t i = 0; i < d; ++i) o[i] += p[u] * oracle_bf16_to_f64(V[u * d + i]);
+    }
+    double dOo = 0.0;
+    for (int64_t i = 0; i < d; ++i) dOo += dO[i] * o[i];
+    for (int64_t i = 0; i < d; ++i) dQ[i] = 0.0;
+    for (int64_t u = 0; u <= t; ++u) {
+        if (!use[u]) continue;
+        double dp = 0.0;
+        for (int64_t i = 0; i < d; ++i) dp += dO[i] * oracle_bf16_to_f64(V[u * d + i]);
+        const double dz = p[u] * (dp - dOo);
+        for (int64_t i = 0; i < d; ++i) {
+            dV[u * d + i] += p[u] * dO[i];
+            dQ[i] += s * dz * oracle_bf16_to_f64(K[u * d + i]);
+            dK[u * d + i] += s * dz * qd[i];
+        }
+    }
+    free(qd); free(o); free(p); free(use);
+}
+
 /* ---------------------------------------------------------------- FP8 (e4m3) key-value cache */
 /* The compressed cache of the decode variant (KuCoin flash "MiniMax launches MSA sparse
  * attention method and MiniMax-M3 model", "ME AI News" paragraph: the SM100 kernel also

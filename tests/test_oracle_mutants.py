@@ -24,8 +24,12 @@ MUTANTS = {
                           "for (int64_t r = 0; r < topk - 2; ++r) {\n            int64_t best"),
     "diagonal_dropped": ("        free(taken);\n        sel[n++] = (int32_t)c;", "        free(taken);"),
     "softmax_scale": ("    double scale = 1.0 / sqrt((double)d);", "    double scale = 1.0 / sqrt((double)d * 2.0);"),
-    "causal_self_excluded": ("use[u] = (sel == NULL) || block_selected(u / Bk, sel, nsel);\n        if (!use[u]) continue;\n        double dot",
-                             "use[u] = (u < t || t == 0) && ((sel == NULL) || block_selected(u / Bk, sel, nsel));\n        if (!use[u]) continue;\n        double dot"),
+    "causal_self_excluded": ("use[u] = (sel == NULL) || block_selected(u / Bk, sel, nsel);\n        if (!use[u]) continue;\n"
+                             "        double dot = 0.0;\n        for (int64_t i = 0; i < d; ++i) dot += qd[i] * oracle_bf16_to_f64(K[u * d + i]);\n"
+                             "        z[u] = dot * scale;",
+                             "use[u] = (u < t || t == 0) && ((sel == NULL) || block_selected(u / Bk, sel, nsel));\n        if (!use[u]) continue;\n"
+                             "        double dot = 0.0;\n        for (int64_t i = 0; i < d; ++i) dot += qd[i] * oracle_bf16_to_f64(K[u * d + i]);\n"
+                             "        z[u] = dot * scale;"),
     "pv_uses_keys": ("o[i] += p * oracle_bf16_to_f64(V[u * d + i]);", "o[i] += p * oracle_bf16_to_f64(K[u * d + i]);"),
     "topk_ties_to_higher_column": ("    return ja < jb;\n}\n\n/* idx[row][r]", "    return ja > jb;\n}\n\n/* idx[row][r]"),
     "topk_nan_ranked_low": ("    if (na != nb) return na;", "    if (na != nb) return nb;"),
@@ -34,6 +38,9 @@ MUTANTS = {
     "e4m3_ties_to_odd": ("if (dist < bd || (dist == bd && (c & 1) == 0))", "if (dist < bd || (dist == bd && (c & 1) == 1))"),
     "fp8_scale_divisor": ("amax > 0.0f ? amax / 448.0f : 1.0f", "amax > 0.0f ? amax / 240.0f : 1.0f"),
     "fp8_open_block_from_codes": ("            const double k = j < c ?", "            const double k = j <= c ?"),
+    "grad_dz_sign": ("const double dz = p[u] * (dp - dOo);", "const double dz = p[u] * (dp + dOo);"),
+    "grad_dq_unscaled": ("dQ[i] += s * dz * oracle_bf16_to_f64(K[u * d + i]);", "dQ[i] += dz * oracle_bf16_to_f64(K[u * d + i]);"),
+    "grad_dk_uses_keys": ("dK[u * d + i] += s * dz * qd[i];", "dK[u * d + i] += s * dz * oracle_bf16_to_f64(K[u * d + i]);"),
     "score_sign": ("dot += oracle_bf16_to_f64(q_idx_row[i]) * pooled_g[j * dI + i];",
                    "dot -= oracle_bf16_to_f64(q_idx_row[i]) * pooled_g[j * dI + i];"),
 }

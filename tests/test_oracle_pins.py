@@ -374,3 +374,61 @@ def test_fp8_attention_equals_bf16_attention_on_a_representable_cache():
     o, l, n = oracle.attend_rows(np.array([t]), q[None], K, V, sel[None], Bk)
     assert n8 == n[0] == 15 * Bk + (t % Bk) + 1
     assert np.array_equal(o8, o[0]) and np.array_equal(l8, l[0])
+
+
+# ----------------------------------------------------------------------------- step 4, gradient
+# The main branch's backward pass (dQ, dK, dV over the selected blocks, the selection held
+# fixed), the oracle of a later kernel: torch fp64 autograd of the equivalent masked dense
+# attention, and identities of the softmax gradient.
+def _grad_case(seed, N=150, Hg=2, d=32, Bk=16, k=4, grid=None):
+    rng = np.random.default_rng(seed)
+    vals = lambda shape: (np.round(rng.standard_normal(shape) * 16) / 16).clip(-4, 4) if grid else rng.standard_normal(shape)
+    q = synth.f64_to_bf16_bits(vals((N, Hg, d)))
+    K = synth.f64_to_bf16_bits(vals((N, d)))
+    V = synth.f64_to_bf16_bits(vals((N, d)))
+    sel = np.full((N, k), -1, np.int32)
+    for t in range(N):
+        c = t // Bk
+        ids = list(range(c + 1)) if c + 1 <= k else sorted(rng.choice(c, k - 1, replace=False).tolist()) + [c]
+        sel[t, :len(ids)] = ids
+    dO = rng.standard_normal((N, Hg, d))
+    return q, K, V, sel, dO
+
+
+def test_attention_grad_matches_torch_autograd():
+    N, Hg, d, Bk, k = 150, 2, 32, 16, 4
+    q, K, V, sel, dO = _grad_case(0, N, Hg, d, Bk, k)
+    dQ, dK, dV = oracle.attend_grad(np.arange(N), q, K, V, sel, dO, Bk)
+    qt = torch.tensor(f32(q), requires_grad=True)
+    kt = torch.tensor(f32(K), requires_grad=True)
+    vt = torch.tensor(f32(V), requires_grad=True)
+    u = torch.arange(N)
+    mask = (u[None, :] <= u[:, None]) & torch.tensor(
+        [[(j // Bk) in set(sel[t][sel[t] >= 0].tolist()) for j in range(N)] for t in range(N)])
+    z = torch.einsum("thd,ud->thu", qt, kt) / np.sqrt(d)
+    z = z.masked_fill(~mask[:, None, :], float("-inf"))
+    o = torch.einsum("thu,ud->thd", torch.softmax(z, dim=-1), vt)
+    (o * torch.tensor(dO)).sum().backward()
+    np.testing.assert_allclose(dQ, qt.grad.numpy(), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(dK, kt.grad.numpy(), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(dV, vt.grad.numpy(), rtol=0, atol=1e-10)
+
+
+def test_attention_grad_identities():
+    N, Hg, d, Bk, k = 120, 2, 32, 16, 4
+    q, K, V, sel, dO = _grad_case(1, N, Hg, d, Bk, k, grid=True)
+    t = np.arange(N)
+    dQ, dK, dV = oracle.attend_grad(t, q, K, V, sel, dO, Bk)
+    # the softmax gradient sums to zero over a row's keys, so the keys' gradients sum to zero
+    assert np.abs(dK.sum(axis=0)).max() < 1e-9
+    # shifting every key by one vector shifts all of a row's scores equally: nothing changes
+    K2 = synth.f64_to_bf16_bits(f32(K) + 0.25)
+    assert (f32(K2) == f32(K) + 0.25).all()                # exact on the 1/16 grid
+    dQ2, dK2, dV2 = oracle.attend_grad(t, q, K2, V, sel, dO, Bk)
+    for a, b in ((dQ, dQ2), (dK, dK2), (dV, dV2)):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-9)
+    # a query that attends one key (position 0): dQ = 0, dK_0 = 0, dV_0 = dO summed over heads
+    g0Q, g0K, g0V = oracle.attend_grad(np.array([0]), q[:1], K, V, sel[:1], dO[:1], Bk)
+    assert not g0Q.any() and not g0K.any()
+    np.testing.assert_array_equal(g0V[0], dO[0].sum(axis=0))
+    assert not g0V[1:].any()
