@@ -41,10 +41,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture) of one decode
-# step of batch 16 at 131,072 tokens: select_decode_kernel 8,430,080 B and attn_decode_kernel
-# 32,128,000 B captured at batch 4 (same contexts), times 4 (both kernels' work is per
-# (sequence, group)); the append kernel's few KB are left out. Re-capture when those kernels
-# change.
+# step of batch 16 at 131,072 tokens: select_decode_kernel 8,430,080 B read and
+# attn_decode_kernel 32,116,736 B read + 11,264 B written, captured at batch 4 (same contexts),
+# times 4 (both kernels' work is per (sequence, group)); the append kernel's few KB are left
+# out. Re-capture when those kernels change.
 DECODE_STEP_DRAM_BYTES = 4 * (8_430_080 + 32_116_736 + 11_264)
 
 
