@@ -37,15 +37,36 @@ import synth  # noqa: E402
 METRIC = "MSA prefill tok/s & decode step µs at 128K ctx; % of HBM/tensor roofline"
 PREFILL = synth.WORKLOADS["prefill_128k_h64g8"]
 DECODE = synth.WORKLOADS["decode_128k_b16_h64g8"]
+PREFILL_32K = synth.WORKLOADS["prefill_32k_h64g8_planted"]
+DECODE_1M = synth.WORKLOADS["decode_1m_ragged_b4_h64g8"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CSRC = os.path.join(ROOT, "block_sparse_gqa_branch_b200", "csrc")
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) from ncu captures of the kernels
+# behind each roofline, with the hash of the CUDA sources the captured build was made from
+# (source_sha16 of the listed files). A capture stands only while those sources are unchanged:
+# when any of them changes, the bench reports traffic null until the capture is taken again.
+# Each entry says which workload was captured and how it is scaled to the bench's workload.
+CAPTURES = {}
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture) of one decode
-# step of batch 16 at 131,072 tokens: select_decode_kernel 8,430,080 B read and
-# attn_decode_kernel 32,116,736 B read + 11,264 B written, captured at batch 4 (same contexts),
-# times 4 (both kernels' work is per (sequence, group)); the append kernel's few KB are left
-# out. Re-capture when those kernels change.
-DECODE_STEP_DRAM_BYTES = 4 * (8_430_080 + 32_116_736 + 11_264)
+def source_sha16(files) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def captured_traffic(name: str, scale: float):
+    """(bytes per launch of the bench workload, note) from CAPTURES, or (None, why)."""
+    c = CAPTURES.get(name)
+    if c is None:
+        return None, "no capture recorded"
+    if source_sha16(c["sources"]) != c["sha16"]:
+        return None, "kernel sources changed since the capture (" + c["profile"] + ")"
+    return int(round(c["bytes"] * scale)), c["note"] + " (" + c["profile"] + ")"
 
 
 # ----------------------------------------------------------------------------- work counts
@@ -86,6 +107,46 @@ def decode_step_bytes(w) -> dict:
                    + w.G * w.d * 2 * 2 * 2                          # k_new, v_new read + cache write
                    + w.G * w.dI * 4 * 2 + w.G * w.topk * 4)         # running sum, sel
     return {"kv": kv, "pooled": pooled, "small": small, "total": kv + pooled + small}
+
+
+def _per_block_counts(N: int, Bk: int, k: int):
+    """(tokens, fully-past blocks kept per token) for every query block of an N-token prefill."""
+    for c in range((N + Bk - 1) // Bk):
+        yield min(Bk, N - c * Bk), min(c, k - 1)
+
+
+def prefill_main_bytes(w, range_tokens: int = 16384) -> dict:
+    """Bytes of the main-branch call (inverted index, attention, merge) of a prefill.
+
+    algorithmic: what the definition must touch once -- q, the selection, K and V, out and lse.
+    model: what this build moves to or from DRAM when the re-reads of query rows and of key /
+    value blocks within one 16K-token range hit L2: the selection read three times (count,
+    fill, merge), the inverted-index entries written and read, q once, K and V once per
+    (range, group, block) below the range's end plus once per diagonal item, one partial per
+    (token, head, selected block) -- 256 B of bf16 o and a 4 B log-sum-exp -- written by the
+    attention and read by the merge, then out and lse written."""
+    B, N, G, Hq, d, Bk, k = w.B, w.N, w.G, w.Hq, w.d, w.Bk, w.topk
+    nb = (N + Bk - 1) // Bk
+    entries = sum(n * kept for n, kept in _per_block_counts(N, Bk, k)) * B * G
+    rows = sum(n * (kept + 1) for n, kept in _per_block_counts(N, Bk, k)) * B * Hq
+    q = B * N * Hq * d * 2
+    out = q + B * N * Hq * 4
+    sel = B * N * G * k * 4
+    kv_once = B * G * N * d * 2 * 2
+    n_ranges = (N + range_tokens - 1) // range_tokens
+    kv_tiles = sum(min(nb, (r + 1) * (range_tokens // Bk)) for r in range(n_ranges)) + nb
+    kv_model = B * G * kv_tiles * Bk * d * 2 * 2
+    partials = rows * (d * 2 + 4)
+    model = 3 * sel + 2 * entries * 4 + q + kv_model + 2 * partials + out
+    return {"algorithmic": q + sel + kv_once + out, "model": model, "partial_rows": rows,
+            "partials": partials}
+
+
+def prefill_index_bytes(w) -> int:
+    """Compulsory bytes of the index branch: k_I and q_I read, the pooled keys written and read
+    back once, the selection written."""
+    nb = w.N // w.Bk
+    return w.B * (w.N * w.G * w.dI * 2 * 2 + w.G * nb * w.dI * 4 * 2 + w.N * w.G * w.topk * 4)
 
 
 def load_peaks():
@@ -156,7 +217,8 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_prefill_sample(w, n_rows: int, g: int, seed: int = 7, cache: dict = None):
     """Time the oracle on n_rows (token, group g) rows of a prefill workload, uniformly sampled.
-    Returns seconds per token (all G groups), including the group's pooling."""
+    Returns (seconds per token over all G groups including the group's pooling, seconds of
+    oracle work this sample took)."""
     import oracle
     cache = {} if cache is None else cache
     key = ("grp", g)
@@ -203,7 +265,73 @@ def cpu_baseline(w, budget_s: float = 15.0):
                       f"scaled to whole tokens (x{w.G} groups); {el:.1f} s of CPU time"}
 
 
+def oracle_decode_step(w):
+    """The oracle's decode step over EVERY (sequence, group) pair of a decode workload: the
+    selection of the new token's blocks from the pooled cache and the attention of its Hg heads
+    over them. The pooled cache (built from all earlier tokens) and the K/V rows of the
+    selected blocks are prepared first and not timed. Pairs run concurrently, one oracle thread
+    each. Returns (seconds, threads used)."""
+    import concurrent.futures
+    import oracle
+    threads = min(oracle.default_threads(), w.B * w.G)
+    work = []
+    for b in range(w.B):
+        Lb = w.ctx[b]
+        ki = synth.decode_seq_np(w, b, "k_idx")
+        pooled, _ = oracle.pool(ki, w.Bk)
+        del ki
+        qi = synth.decode_seq_np(w, b, "q_idx")
+        q = synth.decode_seq_np(w, b, "q")
+        for g in range(w.G):
+            work.append((b, g, Lb, np.ascontiguousarray(pooled[g]), qi[g][None].copy(),
+                         q[g * w.Hg:(g + 1) * w.Hg][None].copy()))
+        del pooled
+    t = np.zeros(1)
+
+    def select(item):
+        b, g, Lb, pooled_g, qi, _ = item
+        sel, _, _ = oracle.select_rows(np.array([Lb]), qi, pooled_g, w.Bk, w.topk, nthreads=1)
+        return sel
+
+    wall0 = time.perf_counter()
+    with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+        sels = list(ex.map(select, work))
+    t[0] = time.perf_counter() - wall0
+    # K / V rows of the selected blocks only (not timed)
+    kv = []
+    for (b, g, Lb, _, _, _), sel in zip(work, sels):
+        K = np.zeros((Lb + 1, w.d), np.uint16)
+        V = np.zeros((Lb + 1, w.d), np.uint16)
+        for j in sel[0]:
+            if j >= 0:
+                lo, hi = j * w.Bk, min((j + 1) * w.Bk, Lb + 1)
+                K[lo:hi] = synth.decode_seq_np(w, b, "k", lo, hi, g=g)
+                V[lo:hi] = synth.decode_seq_np(w, b, "v", lo, hi, g=g)
+        kv.append((K, V))
+
+    def attend(i):
+        b, g, Lb, _, _, q = work[i]
+        K, V = kv[i]
+        oracle.attend_rows(np.array([Lb]), q, K, V, sels[i], w.Bk, w.topk, nthreads=1)
+
+    wall0 = time.perf_counter()
+    with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(attend, range(len(work))))
+    t[0] += time.perf_counter() - wall0
+    return float(t[0]), threads
+
+
+def cpu_baseline_decode(w):
+    sec, threads = oracle_decode_step(w)
+    return {"value": sec * 1e6, "unit": "us per step", "cores": threads, "kind": "oracle",
+            "sample": f"whole step of {w.name}: all {w.B * w.G} (sequence, group) pairs, selection over "
+                      f"the pooled cache + attention of {w.Hg} heads over the selected blocks "
+                      f"(pooled cache and K/V rows prepared beforehand, not timed)"}
+
+
 def run_reference(args):
+    """The reference arm: the fp64 oracle as it stands on the host cores, on a bounded sample of
+    the prefill workload per step (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
@@ -212,18 +340,24 @@ def run_reference(args):
     cache = {}
     n = 64
     _, el = oracle_prefill_sample(PREFILL, n, 0, cache=cache)
-    n_step = int(max(32, min(20000, n * 8.0 / max(el, 1e-3))))
-    times = []
+    n_step = int(max(32, min(20000, n * 4.0 / max(el, 1e-3))))
+    per_tok_l, step_s = [], []
     for s in range(args.warmup + args.steps):
-        per_tok, el = oracle_prefill_sample(PREFILL, n_step, 0, seed=100 + s, cache=cache)
+        t0 = time.perf_counter()
+        per_tok, _ = oracle_prefill_sample(PREFILL, n_step, 0, seed=100 + s, cache=cache)
+        dt = time.perf_counter() - t0
         if s >= args.warmup:
-            times.append(per_tok)
-    per_tok = statistics.mean(times)
+            per_tok_l.append(per_tok)
+            step_s.append(dt)
+    per_tok = statistics.mean(per_tok_l)
     value = 1.0 / per_tok
     sample = (f"each step: {n_step} (token, group 0) rows of {PREFILL.name} drawn uniformly, "
-              f"selection + attention, plus group 0's pooling, scaled to whole tokens (x{PREFILL.G})")
+              f"selection + attention, plus group 0's pooling; value scaled to whole tokens (x{PREFILL.G})")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_tok * PREFILL.N * 1e3,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": statistics.mean(step_s) * 1e3,
+            "ms_per_step_note": "measured seconds of one step's sample (rows drawn, oracle run)",
+            "extrapolated_full_prefill_ms": per_tok * PREFILL.N * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded SplitMix64 -> N(0,1) quantiles -> bf16)",
             "config": config_block(PREFILL, DECODE),
@@ -304,6 +438,242 @@ def reduce_max(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def make_flusher(torch, dev):
+    """L2 flush between timed steps: write a buffer larger than L2 (126 MB), then read another
+    one, so that the written lines are written back before the timed region (a write alone
+    leaves ~126 MB of dirty lines whose write-back would land inside the next step)."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        flush_rd.sum()
+    return flush_l2
+
+
+def time_prefill(torch, w, dev, steps, warmup, flush_l2):
+    """Prefill of workload w (inputs resident in HBM): per-step (index, main) device seconds."""
+    from block_sparse_gqa_branch_b200 import msa_get_device_status, msa_kernel_launches, pipeline
+    x = synth.prefill_inputs_torch(w, dev)
+    bufs = pipeline.prefill_buffers(w.B, w.N, w.Hq, w.G, dev)
+    stream = torch.cuda.current_stream()
+    pipeline.prefill(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], bufs)
+    ti, tm = [], []
+    for s in range(warmup + steps):
+        flush_l2()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        if s == warmup:
+            torch.cuda.synchronize()
+            l0 = msa_kernel_launches()
+        e[0].record(stream)
+        pipeline.prefill_index(x["q_idx"], x["k_idx"], bufs)
+        e[1].record(stream)
+        pipeline.prefill_main(x["q"], x["k"], x["v"], bufs)
+        e[2].record(stream)
+        if s >= warmup:
+            ti.append(e)
+    torch.cuda.synchronize()
+    launches = msa_kernel_launches() - l0
+    for key in ("ws_select", "ws_attn"):
+        st_, info = msa_get_device_status(bufs[key])
+        if st_ != 0:
+            raise SystemExit(f"device status {st_} in {w.name} {key}: {info}")
+    t_index = [a.elapsed_time(b) * 1e-3 for a, b, _ in ti]
+    t_main = [b.elapsed_time(c) * 1e-3 for _, b, c in ti]
+    return t_index, t_main, launches
+
+
+def time_decode(torch, w, dev, steps, warmup, flush_l2):
+    """Decode step of workload w replayed from a CUDA graph: per-step device seconds."""
+    from block_sparse_gqa_branch_b200 import msa_get_device_status, pipeline
+    ds = build_decode_state(w, dev)
+    bufs = pipeline.decode_buffers(w.B, w.Hq, w.G, max(w.ctx), dev)
+
+    def call():
+        pipeline.decode_step(ds["q"], ds["q_idx"], ds["k_idx_new"], ds["k_new"], ds["v_new"], ds["ctx"],
+                             ds["k_cache"], ds["v_cache"], ds["tail"], ds["pooled"], bufs)
+    call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    stream = torch.cuda.current_stream()
+    ts = []
+    for s in range(warmup + steps):
+        flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        if s >= warmup:
+            ts.append((e0, e1))
+    torch.cuda.synchronize()
+    for key in ("ws_append", "ws_select", "ws_attn"):
+        st_, info = msa_get_device_status(bufs[key])
+        if st_ != 0:
+            raise SystemExit(f"device status {st_} in {w.name} {key}: {info}")
+    del graph
+    return [a.elapsed_time(b) * 1e-3 for a, b in ts], 3 * steps
+
+
+def prefill_report(w, t_index, t_main, peaks, peak_src, world, launches, traffic_name=None, scale=1.0):
+    tidx, tmain = statistics.mean(t_index), statistics.mean(t_main)
+    flops = prefill_main_flops(w)
+    ach = flops / tmain / 1e12
+    mb = prefill_main_bytes(w)
+    traffic, tnote = captured_traffic(traffic_name, scale) if traffic_name else (None, "not captured")
+    idx_flops = prefill_index_flops(w)
+    idx_bytes = prefill_index_bytes(w)
+    return {
+        "workload": w.name, "value": w.N * w.B * world / (tidx + tmain), "unit": "tok/s",
+        "prefill_ms": (tidx + tmain) * 1e3, "prefill_index_ms": tidx * 1e3, "prefill_main_ms": tmain * 1e3,
+        "gpu_launches": int(launches),
+        "roofline": {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": ach / peaks["bf16_tflops"], "traffic": traffic,
+                     "traffic_note": tnote,
+                     "kernel": "prefill main branch (msa_sparse_attn_prefill: inverted index, attention, merge)",
+                     "algorithmic": f"{flops:.4e} FLOP per launch", "peak_source": f"{peak_src} burst bf16"},
+        "hbm": {"algorithmic_bytes": mb["algorithmic"], "model_bytes": mb["model"],
+                "achieved_gbs": mb["algorithmic"] / tmain / 1e9,
+                "frac": mb["algorithmic"] / tmain / 1e9 / peaks["hbm_gbs"],
+                "model_frac": mb["model"] / tmain / 1e9 / peaks["hbm_gbs"],
+                "note": "main branch: algorithmic = q, sel, K, V read once and out, lse written; model = "
+                        "this build's DRAM bytes (partials written and read back dominate)"},
+        "roofline_index": {"bound": "tensor", "achieved": idx_flops / tidx / 1e12, "peak": peaks["bf16_tflops"],
+                           "unit": "TFLOP/s", "frac": idx_flops / tidx / 1e12 / peaks["bf16_tflops"],
+                           "executed_frac": 3 * idx_flops / tidx / 1e12 / peaks["bf16_tflops"],
+                           "hbm_frac": idx_bytes / tidx / 1e9 / peaks["hbm_gbs"],
+                           "kernel": "index branch (pooling + scores + exp-free top-15)",
+                           "algorithmic": f"{idx_flops:.4e} FLOP (2 d_I per query, group and candidate; "
+                                          f"executed 3x by the exact three-term bf16 split), {idx_bytes} B compulsory"},
+    }
+
+
+def decode_report(w, t_dec, peaks, peak_src, launches, traffic_name=None, scale=1.0):
+    tdec = statistics.mean(t_dec)
+    dbytes = decode_step_bytes(w)
+    gbs = dbytes["total"] / tdec / 1e9
+    traffic, tnote = captured_traffic(traffic_name, scale) if traffic_name else (None, "not captured")
+    return {
+        "workload": w.name, "decode_step_us": tdec * 1e6, "gpu_launches": int(launches),
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, "traffic_note": tnote,
+                     "kernel": "decode step (append + select + attention, one graph replay)",
+                     "algorithmic": f"{dbytes['total']} B per step", "peak_source": f"{peak_src} copy"},
+    }
+
+
+def topk_report(torch, dev, steps, warmup, peaks, peak_src, with_torch=True):
+    """Exp-free top-k (msa_topk_rows) on the block scores of 8 groups at 131,072 tokens:
+    [1,048,576, 1024] fp32 seeded normal values on the device, k = 15; 4.3 GB exceed L2."""
+    import block_sparse_gqa_branch_b200 as msa
+    rows, n, k = 8 * 131072, 1024, 15
+    s = torch.randn(rows, n, device=dev, generator=torch.Generator(device=dev).manual_seed(0x4D5341))
+    idx = torch.empty(rows, k, dtype=torch.int32, device=dev)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e-3)
+        return statistics.median(ts)
+
+    t_ref = timed(lambda: torch.topk(s, k, dim=1)) if with_torch else None
+    l0 = msa.msa_kernel_launches()
+    t = timed(lambda: msa.msa_topk_rows(s, k, idx))
+    launches = (msa.msa_kernel_launches() - l0) * steps // (steps + warmup)
+    nbytes = rows * n * 4 + rows * k * 4
+    gbs = nbytes / t / 1e9
+    traffic, tnote = captured_traffic("topk_rows", rows / CAPTURES["topk_rows"]["rows"]) \
+        if "topk_rows" in CAPTURES else (None, "no capture recorded")
+    del s
+    return {"workload": "topk_rows_1048576x1024_k15", "metric": "exp-free top-k rows/s (k = 15 of 1,024 fp32)",
+            "value": rows / t, "unit": "rows/s", "ms": t * 1e3, "gpu_launches": int(launches),
+            "torch_topk_ms": None if t_ref is None else t_ref * 1e3,
+            "speedup_vs_torch_topk": None if t_ref is None else t_ref / t,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, "traffic_note": tnote,
+                         "kernel": "topk_rows_kernel",
+                         "algorithmic": f"{nbytes} B per launch (scores read once, ids written)",
+                         "peak_source": f"{peak_src} copy"}}
+
+
+def e2e_pipelined(torch, pipeline, x, pbufs, ds, dbufs, graph, steps, warmup, dev):
+    """The step end to end through the public API with host buffers: every step copies its
+    prefill inputs and its decode-token inputs from pinned host memory, runs the prefill pass and
+    the decode step, and copies the prefill output and the decode output back. Copies of step
+    i + 1's inputs and of step i - 1's outputs run on their own streams (one per direction)
+    while step i computes; inputs and outputs are double-buffered on the device. Time = first
+    input copy to last output copy, divided by the steps."""
+    names = list(x.keys())
+    host_in = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in x.items()}
+    for k in names:
+        host_in[k].copy_(x[k])
+    dev_in = [{k: torch.empty_like(v) for k, v in x.items()} for _ in range(2)]
+    outs = [pbufs["out"], torch.empty_like(pbufs["out"])]
+    host_out = [torch.empty(pbufs["out"].shape, dtype=pbufs["out"].dtype, pin_memory=True) for _ in range(2)]
+    dnames = ("q", "q_idx", "k_idx_new", "k_new", "v_new")
+    dhost = {k: torch.empty(ds[k].shape, dtype=ds[k].dtype, pin_memory=True) for k in dnames}
+    for k in dnames:
+        dhost[k].copy_(ds[k])
+    dhost_out = [torch.empty(dbufs["out"].shape, dtype=dbufs["out"].dtype, pin_memory=True) for _ in range(2)]
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values()) + \
+        sum(v.numel() * v.element_size() for v in dhost.values())
+    d2h = host_out[0].numel() * host_out[0].element_size() + dhost_out[0].numel() * dhost_out[0].element_size()
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def run(n):
+        in_ready, comp_done, out_done = [], [], []
+        start = ev()
+        start.record(s_in)
+        for i in range(n):
+            buf = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(comp_done[i - 2])          # the compute that read dev_in[buf] is done
+                for k in names:
+                    dev_in[buf][k].copy_(host_in[k], non_blocking=True)
+                e = ev()
+                e.record(s_in)
+                in_ready.append(e)
+            comp.wait_event(in_ready[i])
+            if i >= 2:
+                comp.wait_event(out_done[i - 2])               # outs[buf] has been copied out
+            d = dev_in[buf]
+            bufs = dict(pbufs, out=outs[buf])
+            pipeline.prefill(d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"], bufs, comp)
+            for k in dnames:
+                ds[k].copy_(dhost[k], non_blocking=True)
+            graph.replay()
+            e = ev()
+            e.record(comp)
+            comp_done.append(e)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[i])
+                host_out[buf].copy_(outs[buf], non_blocking=True)
+                dhost_out[buf].copy_(dbufs["out"], non_blocking=True)
+                e = ev()
+                e.record(s_out)
+                out_done.append(e)
+        end = ev()
+        end.record(s_out)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) * 1e-3 / n
+
+    run(max(2, warmup))
+    t = run(steps)
+    return t, int(h2d), int(d2h)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -335,15 +705,7 @@ def run_ours(args):
     pbufs = pipeline.prefill_buffers(wp.B, wp.N, wp.Hq, wp.G, dev)
     ds = build_decode_state(wd, dev) if do_decode else None
     dbufs = pipeline.decode_buffers(wd.B, wd.Hq, wd.G, max(wd.ctx), dev) if do_decode else None
-    # L2 flush between timed steps: write a buffer larger than L2 (126 MB), then read another
-    # one, so that the written lines are written back before the timed region (a write alone
-    # leaves ~126 MB of dirty lines whose write-back would land inside the next step)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
-
-    def flush_l2():
-        flush.zero_()
-        flush_rd.sum()
+    flush_l2 = make_flusher(torch, dev)
     stream = torch.cuda.current_stream()
 
     def decode_call():
@@ -364,7 +726,6 @@ def run_ours(args):
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     t_index, t_main, t_dec = [], [], []
-    launches0 = msa.msa_kernel_launches()
 
     def one_step(record: bool):
         flush_l2()
@@ -417,50 +778,52 @@ def run_ours(args):
     tidx = max_over_ranks(statistics.mean(t_index))
     tdec = max_over_ranks(statistics.mean(t_dec))
     peaks, peak_src = load_peaks()
-    flops = prefill_main_flops(wp)
-    achieved_tf = flops / tmain / 1e12
-    dbytes = decode_step_bytes(wd)
-    dec_gbs = dbytes["total"] / tdec / 1e9
+    pre = prefill_report(wp, [tidx], [tmain], peaks, peak_src, world, launches_eager,
+                         traffic_name="prefill_main",
+                         scale=(prefill_main_bytes(wp)["model"] / CAPTURES["prefill_main"]["model_bytes"]
+                                if "prefill_main" in CAPTURES else 1.0))
+    dec = decode_report(wd, [tdec], peaks, peak_src, decode_graph_kernels * args.steps,
+                        traffic_name="decode_step",
+                        scale=(decode_step_bytes(wd)["total"] / CAPTURES["decode_step"]["algorithmic_bytes"]
+                               if "decode_step" in CAPTURES else 1.0))
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
     if not args.no_e2e and do_prefill and do_decode:
-        host_in = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in x.items()}
-        for k in x:
-            host_in[k].copy_(x[k])
-        dev_in = {k: torch.empty_like(v) for k, v in x.items()}
-        host_out = torch.empty(pbufs["out"].shape, dtype=pbufs["out"].dtype, pin_memory=True)
-        dnames = ("q", "q_idx", "k_idx_new", "k_new", "v_new")
-        dhost = {k: torch.empty(ds[k].shape, dtype=ds[k].dtype, pin_memory=True) for k in dnames}
-        for k in dnames:
-            dhost[k].copy_(ds[k])
-        dhost_out = torch.empty(dbufs["out"].shape, dtype=dbufs["out"].dtype, pin_memory=True)
-        h2d = sum(v.numel() * v.element_size() for v in host_in.values()) + \
-            sum(v.numel() * v.element_size() for v in dhost.values())
-        d2h = host_out.numel() * host_out.element_size() + dhost_out.numel() * dhost_out.element_size()
-        times = []
-        for s in range(max(1, args.warmup // 2) + args.steps):
-            flush_l2()
-            torch.cuda.synchronize()
-            e0, e1 = ev(), ev()
-            e0.record(stream)
-            for k in x:
-                dev_in[k].copy_(host_in[k], non_blocking=True)
-            pipeline.prefill(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["q_idx"], dev_in["k_idx"], pbufs)
-            host_out.copy_(pbufs["out"], non_blocking=True)
-            for k in dnames:
-                ds[k].copy_(dhost[k], non_blocking=True)
-            graph.replay()
-            dhost_out.copy_(dbufs["out"], non_blocking=True)
-            e1.record(stream)
-            torch.cuda.synchronize()
-            if s >= max(1, args.warmup // 2):
-                times.append(e0.elapsed_time(e1) * 1e-3)
-        te = max_over_ranks(statistics.mean(times))
-        e2e = {"value": wp.N * wp.B * world / te, "unit": "tok/s", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": te * 1e3,
-               "note": "prefill inputs and decode-token inputs copied from pinned host memory, prefill output "
-                       "and decode output copied back, every step; value counts prefill tokens"}
+        te, h2d, d2h = e2e_pipelined(torch, pipeline, x, pbufs, ds, dbufs, graph, args.steps, args.warmup, dev)
+        te = max_over_ranks(te)
+        e2e = {"value": wp.N * wp.B * world / te, "unit": "tok/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": te * 1e3,
+               "note": "through the public API: prefill inputs and decode-token inputs copied from pinned host "
+                       "memory and the prefill and decode outputs copied back every step; copies of the next "
+                       "step's inputs and the previous step's outputs overlap this step's compute (one stream "
+                       "per direction, double-buffered); value counts prefill tokens"}
+
+    # ---------------------------------------------------------------- the other workloads
+    extra = {}
+    if not args.no_extra and args.only is None and not (args.prefill_tokens or args.decode_batch):
+        graph = None
+        del x, pbufs, ds, dbufs
+        torch.cuda.empty_cache()
+        n_x, w_x = min(args.steps, 10), 3
+        ti2, tm2, l2 = time_prefill(torch, PREFILL_32K, dev, n_x, w_x, flush_l2)
+        r = prefill_report(PREFILL_32K, [max_over_ranks(statistics.mean(ti2))], [max_over_ranks(statistics.mean(tm2))],
+                           peaks, peak_src, world, l2, traffic_name="prefill_main",
+                           scale=(prefill_main_bytes(PREFILL_32K)["model"] / CAPTURES["prefill_main"]["model_bytes"]
+                                  if "prefill_main" in CAPTURES else 1.0))
+        extra[PREFILL_32K.name] = r
+        torch.cuda.empty_cache()
+        td5, l5 = time_decode(torch, DECODE_1M, dev, n_x, w_x, flush_l2)
+        extra[DECODE_1M.name] = decode_report(
+            DECODE_1M, [max_over_ranks(statistics.mean(td5))], peaks, peak_src, l5, traffic_name="decode_step",
+            scale=(decode_step_bytes(DECODE_1M)["total"] / CAPTURES["decode_step"]["algorithmic_bytes"]
+                   if "decode_step" in CAPTURES else 1.0))
+        torch.cuda.empty_cache()
+        tk = topk_report(torch, dev, n_x, w_x, peaks, peak_src)
+        tk["ms"] = max_over_ranks(tk["ms"])
+        tk["value"] = 8 * 131072 * world / (tk["ms"] * 1e-3)
+        extra[tk["workload"]] = tk
+        torch.cuda.empty_cache()
 
     if world > 1:
         graph = None
@@ -468,13 +831,19 @@ def run_ours(args):
     if rank != 0:
         return 0
 
-    cpu = None
+    cpu = cpu_dec = None
     if not args.no_cpu_baseline and args.only is None:
         try:
             cpu = cpu_baseline(wp, budget_s=args.cpu_budget)
         except Exception as exc:  # reported, never fatal for the GPU number
             cpu = {"value": None, "unit": "tok/s", "cores": os.cpu_count(), "kind": "oracle",
                    "sample": f"failed: {exc!r}"}
+        try:
+            cpu_dec = {DECODE.name: cpu_baseline_decode(DECODE)}
+            if not args.no_extra:
+                cpu_dec[DECODE_1M.name] = cpu_baseline_decode(DECODE_1M)
+        except Exception as exc:
+            cpu_dec = {"failed": repr(exc)}
     clocks = clk.summary()
     line = {
         "metric": METRIC,
@@ -494,31 +863,23 @@ def run_ours(args):
         "prefill_index_ms": tidx * 1e3,
         "prefill_main_ms": tmain * 1e3,
         "decode_step_us": tdec * 1e6,
-        "roofline": ({"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
-                      "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"], "traffic": None,
-                      "kernel": "prefill main branch (msa_sparse_attn_prefill, all its kernels)",
-                      "algorithmic": f"{flops:.4e} FLOP per launch", "peak_source": f"{peak_src} burst bf16"}
-                     if do_prefill else None),
-        "roofline_decode": ({"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                             "frac": dec_gbs / peaks["hbm_gbs"],
-                             "traffic": DECODE_STEP_DRAM_BYTES if (wd.B, wd.ctx) == (16, (131072,) * 16) else None,
-                             "kernel": "decode step (append + select + attention, one graph replay)",
-                             "algorithmic": f"{dbytes['total']} B per step", "peak_source": f"{peak_src} copy"}
-                            if do_decode else None),
+        "roofline": pre["roofline"] if do_prefill else None,
+        "prefill_hbm": pre["hbm"] if do_prefill else None,
+        "roofline_index": pre["roofline_index"] if do_prefill else None,
+        "roofline_decode": dec["roofline"] if do_decode else None,
         "clocks": clocks,
         "gpu_launches": int(gpu_launches),
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "cpu_baseline_decode": cpu_dec,
+        "workloads": extra,
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
 def run_topk(args):
-    """Exp-free top-k micro-benchmark (one GPU): msa_topk_rows against torch.topk on the block
-    scores of 8 groups at 131,072 tokens, [1,048,576, 1024] fp32 with k = 15 (the fully-past
-    blocks a query keeps besides its own). The scores are seeded normal values generated on the
-    device; at 4.3 GB they are larger than L2, so no flush is needed between iterations."""
+    """The exp-free top-k micro-benchmark alone (one GPU), as one JSON line."""
     import torch
     import block_sparse_gqa_branch_b200 as msa
     if int(os.environ.get("RANK", "0")) != 0:
@@ -529,46 +890,17 @@ def run_topk(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     msa.load()
-    rows, n, k = 8 * 131072, 1024, 15
-    s = torch.randn(rows, n, device=dev, generator=torch.Generator(device=dev).manual_seed(0x4D5341))
-    idx = torch.empty(rows, k, dtype=torch.int32, device=dev)
-
-    def timed(fn):
-        for _ in range(args.warmup):
-            fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(args.steps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            torch.cuda.synchronize()
-            ts.append(e0.elapsed_time(e1) * 1e-3)
-        return statistics.median(ts)
-
-    t_ref = timed(lambda: torch.topk(s, k, dim=1))
-    launches0 = msa.msa_kernel_launches()
-    with ClockSampler(local) as clk:
-        t = timed(lambda: msa.msa_topk_rows(s, k, idx))
-    launches = msa.msa_kernel_launches() - launches0
     peaks, peak_src = load_peaks()
-    nbytes = rows * n * 4 + rows * k * 4
-    gbs = nbytes / t / 1e9
-    line = {
-        "metric": "exp-free top-k rows/s (k = 15 of 1,024 fp32 block scores per row)",
-        "value": rows / t, "unit": "rows/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic (seeded normal scores generated on the device)",
-        "config": {"workload": "topk_rows_1048576x1024_k15", "rows": rows, "n": n, "k": k,
-                   "l2": "inputs (4.3 GB) larger than L2, no flush"},
-        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "topk_rows_kernel",
-                     "algorithmic": f"{nbytes} B per launch (scores read once, ids written)",
-                     "peak_source": f"{peak_src} copy"},
-        "torch_topk_ms": t_ref * 1e3, "speedup_vs_torch_topk": t_ref / t,
-        "clocks": clk.summary(), "gpu_launches": int(launches),
-    }
+    with ClockSampler(local) as clk:
+        r = topk_report(torch, dev, args.steps, args.warmup, peaks, peak_src)
+    line = {"metric": r["metric"], "value": r["value"], "unit": r["unit"], "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded normal scores generated on the device)",
+            "config": {"workload": r["workload"], "rows": 8 * 131072, "n": 1024, "k": 15,
+                       "l2": "inputs (4.3 GB) larger than L2, no flush"},
+            "roofline": r["roofline"], "torch_topk_ms": r["torch_topk_ms"],
+            "speedup_vs_torch_topk": r["speedup_vs_torch_topk"], "clocks": clk.summary(),
+            "gpu_launches": r["gpu_launches"]}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -581,6 +913,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads (32K planted prefill, 1M ragged decode, top-k)")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one half of the step (profiler captures; not a benchmark value)")

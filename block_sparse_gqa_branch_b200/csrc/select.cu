@@ -266,16 +266,18 @@ __global__ void __launch_bounds__(kSelThreads) select_decode_kernel(
     const int pos = q_pos[b];
     // every CTA of a cluster belongs to the same (sequence, group): the early exits below are
     // taken by the whole cluster, before its barriers
+    // (the writes of these exits wait for the preceding kernel like every other write of sel
+    // and of the error word below, whatever that kernel is)
     if (pos < 0 || pos > max_pos || int64_t(pos / kBlock) > nb_cap) {
-        if (split == 0 && tid == 0) record_error(hdr, MSA_ERR_DEVICE_BOUNDS, KID_SELECT_DECODE, bg, 0, pos);
         grid_dep_wait();
+        if (split == 0 && tid == 0) record_error(hdr, MSA_ERR_DEVICE_BOUNDS, KID_SELECT_DECODE, bg, 0, pos);
         return;
     }
     const int c = pos / kBlock;
     int32_t* out = sel + size_t(bg) * kTopK;
     if (c + 1 <= kTopK) {
-        if (split == 0 && tid == 0) write_all_blocks(out, c);
         grid_dep_wait();
+        if (split == 0 && tid == 0) write_all_blocks(out, c);
         return;
     }
     const int span = ((c + nsplit - 1) / nsplit + 31) / 32 * 32;

@@ -149,7 +149,10 @@ msa_status_t msa_index_select(const msa_shape_t *shape, const void *q_idx, int64
  *    G = 8 included); B * G = 1024 fits up to max_pos = 2,228,351. Larger problems return
  *    MSA_ERR_WORKSPACE without launching.
  *  - The first call on a device looks up the array's device address (once per device); make
- *    that first call before any stream capture.
+ *    that first call before any stream capture. The address is kept for the life of the
+ *    process: do not call this entry point after a cudaDeviceReset (or any other teardown of
+ *    the device's primary context) in the same process, since the array may then live
+ *    elsewhere.
  *  - Every call shares the one array: calls that may overlap on the GPU (other streams,
  *    other host threads on the same device) race and must be serialised by the caller.
  *  - sel rows are preset to -1; a row left all -1 means the device found its q_pos out of

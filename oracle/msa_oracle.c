@@ -312,12 +312,14 @@ double oracle_e4m3_to_f64(uint8_t c)
 }
 
 /* The e4m3 code nearest to x (ties to the code with an even mantissa), |x| > 448 saturating
- * to +-448: a search over the 127 non-negative finite codes, ascending. */
+ * to +-448: a search over the 127 non-negative finite codes, ascending. NaN maps to the
+ * NaN pattern with the input's sign. */
 uint8_t oracle_e4m3_from_f32(float x)
 {
     const int s = signbit(x) ? 1 : 0;
     const double a = fabs((double)x);
     int best = 0;
+    if (isnan(x)) return (uint8_t)(0x7F | (s << 7));   /* NaN keeps its sign, S.1111.111 */
     double bd = INFINITY;
     for (int c = 0; c <= 126; ++c) {
         const double dist = fabs(oracle_e4m3_to_f64((uint8_t)c) - a);

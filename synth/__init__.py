@@ -107,13 +107,25 @@ def normal_bf16_at(seed: int, stream: int, idx: np.ndarray) -> np.ndarray:
 
 
 def normal_bf16(seed: int, stream: int, shape: Sequence[int], start: int = 0) -> np.ndarray:
-    """A whole tensor of bf16 bits: element with row-major offset i uses counter start + i."""
+    """A whole tensor of bf16 bits: element with row-major offset i uses counter start + i.
+    Large tensors are generated in 4M-element chunks on a thread pool (numpy releases the
+    interpreter lock inside its array operations); the result does not depend on it."""
     n = int(np.prod(shape)) if len(shape) else 1
     out = np.empty(n, dtype=np.uint16)
-    step = 1 << 24
-    for lo in range(0, n, step):
+    step = 1 << 22
+
+    def fill(lo):
         hi = min(n, lo + step)
         out[lo:hi] = normal_bf16_at(seed, stream, np.arange(start + lo, start + hi, dtype=np.uint64))
+
+    chunks = list(range(0, n, step))
+    if len(chunks) > 1:
+        import concurrent.futures
+        import os
+        with concurrent.futures.ThreadPoolExecutor(max_workers=min(len(chunks), os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, chunks))
+    elif chunks:
+        fill(0)
     return out.reshape(shape)
 
 
@@ -327,9 +339,8 @@ def decode_seq_np(w: Workload, b: int, what: str, pos_lo: int = 0, pos_hi: Optio
         return np.stack(out) if g is None else out[0]
     if what == "k_idx":
         pos = np.arange(pos_lo, pos_hi, dtype=np.uint64)
-        if g is None:
-            idx = (pos[:, None, None] * np.uint64(w.G) + np.arange(w.G, dtype=np.uint64)[None, :, None]) \
-                * np.uint64(w.dI) + np.arange(w.dI, dtype=np.uint64)[None, None, :]
+        if g is None:                    # whole rows: a contiguous range of counters
+            return normal_bf16(s, STREAM_KI, (pos_hi - pos_lo, w.G, w.dI), start=pos_lo * w.G * w.dI)
         else:
             idx = (pos[:, None] * np.uint64(w.G) + np.uint64(g)) * np.uint64(w.dI) \
                 + np.arange(w.dI, dtype=np.uint64)[None, :]

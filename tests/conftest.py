@@ -13,6 +13,18 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: long-running (full-size workloads)")
 
 
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Selection near-ties per workload, as the parity rule requires them logged and counted."""
+    from tests.msa_check import TIE_LOG
+    if not TIE_LOG:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "selection near-ties (rows checked / rows differing / near-ties / cancellation near-ties)")
+    for label in sorted(TIE_LOG):
+        e = TIE_LOG[label]
+        tr.write_line(f"{label}: {e['rows']} / {e['differing_rows']} / {e['near_ties']} / {e['cancel_ties']}")
+
+
 @pytest.fixture(scope="session")
 def cuda_ok():
     import torch

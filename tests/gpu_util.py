@@ -5,7 +5,7 @@ import numpy as np
 import torch
 
 import oracle
-from tests.msa_check import compare_selection_row, sel_sorted_ok
+from tests.msa_check import compare_selection_row, log_ties, sel_sorted_ok_rows
 
 
 def dev_bf16(bits: np.ndarray) -> torch.Tensor:
@@ -20,13 +20,17 @@ def f32(bits):
     return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
-def check_selection(gpu_sel, ora_sel, kth, q_idx_rows, pooled_g, t):
-    """Compare selections of rows (one group). Returns (n_near, n_cancel); asserts validity."""
+def check_selection(gpu_sel, ora_sel, kth, q_idx_rows, pooled_g, t, label="unlabelled"):
+    """Compare the selections of rows of one group under the near-tie rule; logs the counts
+    under `label` and returns (n_near, n_cancel). Asserts that every GPU row is a valid,
+    ascending, -1 padded set and that every difference is an allowed near-tie."""
+    gpu_sel = np.asarray(gpu_sel)
+    ora_sel = np.asarray(ora_sel)
+    assert sel_sorted_ok_rows(gpu_sel).all(), "GPU selection rows not ascending / -1 padded"
+    differ = np.nonzero((gpu_sel != ora_sel).any(axis=1))[0]
     near = cancel = 0
     bad = []
-    for r in range(len(t)):
-        if (gpu_sel[r] == ora_sel[r]).all():
-            continue
+    for r in differ:
         c = int(t[r]) // 128
         s = oracle.block_scores(q_idx_rows[r], pooled_g, c)
         absscale = (np.abs(f32(q_idx_rows[r]).astype(np.float64)[None, :] * pooled_g[:c]).sum(1) / 8.0
@@ -36,7 +40,6 @@ def check_selection(gpu_sel, ora_sel, kth, q_idx_rows, pooled_g, t):
             bad.append((int(t[r]), list(gpu_sel[r]), list(ora_sel[r])))
         near += n1
         cancel += n2
+    log_ties(label, len(t), len(differ), near, cancel)
     assert not bad, f"{len(bad)} selection mismatches beyond near-ties, first: {bad[:3]}"
-    for r in range(len(t)):
-        assert sel_sorted_ok(gpu_sel[r])
     return near, cancel

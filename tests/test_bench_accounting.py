@@ -57,6 +57,33 @@ def test_decode_step_bytes_closed_form():
     assert d["total"] == 128 * (per_bg_pooled + per_bg_kv) + small == 160210944
 
 
-def test_captured_decode_traffic_is_close_to_the_algorithmic_bytes():
-    ratio = bench.DECODE_STEP_DRAM_BYTES / bench.decode_step_bytes(bench.DECODE)["total"]
-    assert 1.0 <= ratio < 1.03
+def test_partial_rows_by_enumeration():
+    # one partial per (token, head, selected block): the own block plus min(c, k - 1) past ones
+    import dataclasses
+    for N in (77, 128 * 3, 128 * 20 + 5):
+        w = dataclasses.replace(bench.PREFILL, N=N, Hq=4, G=1)
+        want = sum(min(t // 128, 15) + 1 for t in range(N)) * 4
+        assert bench.prefill_main_bytes(w)["partial_rows"] == want
+    w = bench.PREFILL
+    rows = bench.prefill_main_bytes(w)["partial_rows"]
+    assert rows == (128 * sum(c + 1 for c in range(16)) + (131072 - 2048) * 16) * 64 == 133234688
+
+
+def test_captured_traffic_is_dropped_when_sources_change(monkeypatch):
+    files = ["select.cu"]
+    good = {"sources": files, "sha16": bench.source_sha16(files), "bytes": 1000, "note": "n", "profile": "p.md"}
+    monkeypatch.setitem(bench.CAPTURES, "probe", good)
+    assert bench.captured_traffic("probe", 2.0)[0] == 2000
+    monkeypatch.setitem(bench.CAPTURES, "probe", dict(good, sha16="0" * 16))
+    got, why = bench.captured_traffic("probe", 2.0)
+    assert got is None and "changed" in why
+    assert bench.captured_traffic("absent", 1.0)[0] is None
+
+
+def test_recorded_captures_are_close_to_their_models():
+    # every recorded capture: traffic within a few percent above the model it is scaled by
+    c = bench.CAPTURES
+    if "decode_step" in c:
+        assert 1.0 <= c["decode_step"]["bytes"] / c["decode_step"]["algorithmic_bytes"] < 1.05
+    if "prefill_main" in c:
+        assert 0.9 <= c["prefill_main"]["bytes"] / c["prefill_main"]["model_bytes"] < 1.2

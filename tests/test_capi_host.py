@@ -126,3 +126,23 @@ def test_topk_validation_before_launch(L):
                 ok[:2] + ((1 << 30) + 4,) + ok[3:]):    # n too large
         assert L.msa_topk_rows(*bad) == 1, bad
     assert L.msa_topk_rows(None, 0, 1024, 15, None, None, None) == 0    # no rows: nothing to do
+
+
+def test_no_alloc_select_rejects_problems_beyond_its_scratch(L):
+    # msa_index_select_decode_noalloc keeps its scratch in a fixed 2 MiB device array; a
+    # problem whose scratch would not fit returns MSA_ERR_WORKSPACE on the host, before any
+    # CUDA call, so the fake pointers are never touched
+    shape = ctypes.byref(Shape.make(64, 512, 64))
+    max_pos = 4_000_000
+    assert L.msa_index_select_decode_noalloc(shape, FAKE, FAKE2, max_pos, FAKE, max_pos // 128 + 1, FAKE,
+                                             None) == 3
+    # B * G = 272 fits at the largest supported position; B * G = 1024 only up to 2,228,351
+    ok_shape = ctypes.byref(Shape.make(34, 8 * 8, 8))
+    assert L.msa_index_select_decode_noalloc(ok_shape, FAKE, FAKE2, (1 << 24) - 1, FAKE, 1 << 17, FAKE + 2,
+                                             None) == 1      # misaligned sel: rejected as an argument
+    big = ctypes.byref(Shape.make(128, 8 * 8, 8))
+    assert L.msa_index_select_decode_noalloc(big, FAKE, FAKE2, 2_228_352 + 128 * 1024 * 8, FAKE, 1 << 17, FAKE,
+                                             None) == 3
+    # invalid arguments come first
+    assert L.msa_index_select_decode_noalloc(shape, None, FAKE2, 100, FAKE, 1, FAKE, None) == 1
+    assert L.msa_index_select_decode_noalloc(shape, FAKE, FAKE2, 1 << 25, FAKE, 1 << 18, FAKE, None) == 2

@@ -93,7 +93,8 @@ def test_decode_step_matches_oracle(cuda_ok, ctx, Hq, G):
     ref = oracle_decode(w, sel)
     for r in ref:
         b, g = r["b"], r["g"]
-        check_selection(sel[b, g][None], r["sel"][None], np.array([r["kth"]]), r["qi"][None], r["pooled"], r["t"])
+        check_selection(sel[b, g][None], r["sel"][None], np.array([r["kth"]]), r["qi"][None], r["pooled"], r["t"],
+                        label=f"decode ctx={ctx} Hq={Hq} G={G}")
         assert_close_attention(out[b, g * w.Hg:(g + 1) * w.Hg], r["o"], f"decode b={b} g={g}")
         np.testing.assert_allclose(lse[b, g * w.Hg:(g + 1) * w.Hg], r["lse"], rtol=0, atol=2e-3)
     # the appended token and the block it closed
@@ -140,8 +141,8 @@ def test_decode_is_last_prefill_row(cuda_ok):
     for g in range(2):
         qi = x["q_idx"][0, L, g][None]
         ref, kth, _ = oracle.select_rows(t, qi, pooled_o[g])
-        check_selection(sd[g][None], ref, kth, qi, pooled_o[g], t)
-        check_selection(sp[g][None], ref, kth, qi, pooled_o[g], t)
+        check_selection(sd[g][None], ref, kth, qi, pooled_o[g], t, label="decode(L) vs prefill row L: decode")
+        check_selection(sp[g][None], ref, kth, qi, pooled_o[g], t, label="decode(L) vs prefill row L: prefill")
     same = (sd == sp).all(axis=1)
     assert same.any()
     a = f32(host_bits(out_d[0])).reshape(2, 8, 128)[same]
@@ -215,7 +216,8 @@ def test_decode_select_long_context_merge(cuda_ok, case):
     assert msa_get_device_status(bufs["ws_select"])[0] == 0
     sel = bufs["sel"].cpu().numpy()[0, 0]
     ref, kth, _ = oracle.select_rows(np.array([pos]), q_bits[0], pooled[0, 0].astype(np.float64))
-    check_selection(sel[None], ref, kth, q_bits[0], pooled[0, 0].astype(np.float64), np.array([pos]))
+    check_selection(sel[None], ref, kth, q_bits[0], pooled[0, 0].astype(np.float64), np.array([pos]),
+                    label=f"decode 10,240 candidates ({case})")
     if case != "random":
         assert (sel == ref[0]).all(), (case, sel, ref[0])
     if case == "many_survivors":

@@ -53,7 +53,7 @@ def test_prefill_matches_oracle(cuda_ok, N, Hq, G, planted):
     t = np.arange(N)
     for g in range(G):
         check_selection(r["sel"][0, :, g], o["sel"][0, :, g], o["kth"][0, :, g], x["q_idx"][0, :, g],
-                        o["pooled"][0, g], t)
+                        o["pooled"][0, g], t, label=f"prefill N={N} Hq={Hq} G={G} planted={planted}")
     # pooled keys
     nb = N // 128
     np.testing.assert_allclose(r["pooled"][0, :, :nb], o["pooled"][0], rtol=1e-6, atol=1e-7)
@@ -93,5 +93,5 @@ def test_prefill_batch_of_two(cuda_ok):
     for b in range(2):
         for g in range(2):
             check_selection(r["sel"][b, :, g], o["sel"][b, :, g], o["kth"][b, :, g], x["q_idx"][b, :, g],
-                            o["pooled"][b, g], np.arange(2400))
+                            o["pooled"][b, g], np.arange(2400), label="prefill batch 2 N=2400")
     assert_close_attention(r["out"], o["out"], "batch 2")

@@ -53,3 +53,21 @@ def test_reference_arm_runs_on_rank_zero_only():
                        cwd=ROOT)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_reference_arm_step_time_is_measured():
+    # rank 0 prints one line whose ms_per_step is the measured time of a step's sample, so that
+    # steps x ms_per_step fits inside the run's own wall clock
+    import json
+    import time
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    t0 = time.perf_counter()
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "2",
+                        "--warmup", "3"], env=env, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    wall = time.perf_counter() - t0
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 2
+    assert 0 < line["ms_per_step"] * line["steps"] / 1e3 < wall
+    assert line["extrapolated_full_prefill_ms"] > line["ms_per_step"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"

@@ -130,6 +130,23 @@ def test_near_tie_rule():
     assert compare_selection_row([2, 3, 3], [2, 3, -1], s, kth)[0] is False
 
 
+def test_cancellation_window_only_when_the_kth_score_is_near_zero():
+    # block 1 differs from the 15th score by 3e-6: outside 1e-5 * |kth|, inside 1e-5 * its
+    # term magnitude (0.5). Accepted as a cancellation near-tie only when |kth| < 0.1 * 0.5.
+    absscale = np.array([0.5, 0.5, 0.5, 0.5])
+    s = np.array([1.0, 0.01 + 3e-6, 0.01, -1.0])
+    assert compare_selection_row([1, 3, -1], [2, 3, -1], s, 0.01, absscale) == (True, 1, 1)
+    s = np.array([1.0, 0.2 + 3e-6, 0.2, -1.0])
+    assert compare_selection_row([1, 3, -1], [2, 3, -1], s, 0.2, absscale)[0] is False
+
+
+def test_vectorised_row_validity():
+    from tests.msa_check import sel_sorted_ok_rows
+    rows = np.array([[0, 3, 9, -1], [0, 3, 3, -1], [0, -1, 2, -1], [5, 2, -1, -1], [1, 2, 3, 4], [-1, -1, -1, -1]])
+    want = [sel_sorted_ok(r) for r in rows]
+    assert list(sel_sorted_ok_rows(rows)) == want == [True, False, False, False, True, True]
+
+
 # ----------------------------------------------------------------------------- attention
 def _sdpa_masked(qf, kf, vf, mask):
     """torch fp64 attention. qf [H, T, d], kf/vf [U, d], mask [T, U] bool (True = attend)."""
@@ -308,6 +325,14 @@ def test_e4m3_encode_matches_torch_rounding():
     x = np.concatenate([grid, -grid[1:], mids, -mids, rnd, [464.0, -464.0]]).astype(np.float32)
     want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert (oracle.e4m3_from_f32(x) == want).all()
+
+
+def test_e4m3_encodes_nan_as_nan():
+    x = np.array([np.nan, -np.nan], np.float32)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = oracle.e4m3_from_f32(x)
+    assert (got == want).all() and got.tolist() == [0x7F, 0xFF]
+    assert np.isnan(oracle.e4m3_to_f64(got)).all()
 
 
 def test_e4m3_saturates_beyond_448():

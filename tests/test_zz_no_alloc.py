@@ -5,7 +5,9 @@ it through the C ABI and compare it with msa_index_select (decode mode, caller w
 the same inputs, for two different problems in a row and then the first one again, so that
 state left in the shared array by one call cannot leak into the next.
 
-This file is collected last on purpose (its name sorts after the other test files).
+This file is collected last on purpose (its name sorts after the other test files). The
+check that problems larger than the fixed scratch are rejected before any launch needs no GPU
+and lives with the host-only tests of the C ABI.
 """
 import ctypes
 
@@ -59,16 +61,3 @@ def test_no_alloc_select_matches_workspace_select(cuda_ok):
         assert torch.equal(got, ref)
         assert (got[..., 0] >= 0).all()
 
-
-def test_no_alloc_rejects_problems_beyond_its_scratch(cuda_ok):
-    shape = Shape.make(64, 512, 64)
-    sel = torch.zeros(64, 64, 16, dtype=torch.int32, device="cuda")
-    fake = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
-    q_pos = torch.zeros(64, dtype=torch.int32, device="cuda")
-    pooled = torch.zeros(16, device="cuda")
-    L = msa.load()
-    max_pos = 4_000_000
-    st = L.msa_index_select_decode_noalloc(ctypes.byref(shape), fake.data_ptr(), q_pos.data_ptr(), max_pos,
-                                           pooled.data_ptr(), max_pos // 128 + 1, sel.data_ptr(),
-                                           torch.cuda.current_stream().cuda_stream)
-    assert st == 3      # MSA_ERR_WORKSPACE: the fixed scratch is too small; nothing was launched
