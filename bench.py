@@ -109,6 +109,19 @@ def decode_step_bytes(w) -> dict:
     return {"kv": kv, "pooled": pooled, "small": small, "total": kv + pooled + small}
 
 
+def decode_step_bytes_fp8(w) -> dict:
+    """Algorithmic HBM bytes of one decode step over the FP8 cache: as decode_step_bytes, but
+    the selected closed blocks are read as one e4m3 byte per value plus a key and a value scale;
+    the query's own block is read in bf16."""
+    base = decode_step_bytes(w)
+    kv = 0
+    for L in w.ctx:
+        c = L // w.Bk
+        nfull = min(c, w.topk - 1)
+        kv += w.G * (nfull * (w.Bk * w.d * 2 + 2 * 4) + ((L % w.Bk) + 1) * w.d * 2 * 2)
+    return dict(base, kv=kv, total=kv + base["pooled"] + base["small"])
+
+
 def _per_block_counts(N: int, Bk: int, k: int):
     """(tokens, fully-past blocks kept per token) for every query block of an N-token prefill."""
     for c in range((N + Bk - 1) // Bk):
@@ -483,15 +496,25 @@ def time_prefill(torch, w, dev, steps, warmup, flush_l2):
     return t_index, t_main, launches
 
 
-def time_decode(torch, w, dev, steps, warmup, flush_l2):
-    """Decode step of workload w replayed from a CUDA graph: per-step device seconds."""
+def time_decode(torch, w, dev, steps, warmup, flush_l2, fp8=False):
+    """Decode step of workload w replayed from a CUDA graph: per-step device seconds. With fp8,
+    the closed blocks are read from an e4m3 cache quantised from the bf16 one beforehand."""
     from block_sparse_gqa_branch_b200 import msa_get_device_status, pipeline
     ds = build_decode_state(w, dev)
     bufs = pipeline.decode_buffers(w.B, w.Hq, w.G, max(w.ctx), dev)
+    f8 = None
+    if fp8:
+        f8 = pipeline.fp8_cache(ds["k_cache"], ds["v_cache"], ds["pooled"].shape[2])
+        for b in range(w.B):
+            pipeline.fp8_quantize_sequence(ds["k_cache"], ds["v_cache"], f8, b, w.ctx[b], w.Hq)
 
     def call():
-        pipeline.decode_step(ds["q"], ds["q_idx"], ds["k_idx_new"], ds["k_new"], ds["v_new"], ds["ctx"],
-                             ds["k_cache"], ds["v_cache"], ds["tail"], ds["pooled"], bufs)
+        if fp8:
+            pipeline.decode_step_fp8(ds["q"], ds["q_idx"], ds["k_idx_new"], ds["k_new"], ds["v_new"], ds["ctx"],
+                                     ds["k_cache"], ds["v_cache"], ds["tail"], ds["pooled"], f8, bufs)
+        else:
+            pipeline.decode_step(ds["q"], ds["q_idx"], ds["k_idx_new"], ds["k_new"], ds["v_new"], ds["ctx"],
+                                 ds["k_cache"], ds["v_cache"], ds["tail"], ds["pooled"], bufs)
     call()
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
@@ -513,7 +536,7 @@ def time_decode(torch, w, dev, steps, warmup, flush_l2):
         if st_ != 0:
             raise SystemExit(f"device status {st_} in {w.name} {key}: {info}")
     del graph
-    return [a.elapsed_time(b) * 1e-3 for a, b in ts], 3 * steps
+    return [a.elapsed_time(b) * 1e-3 for a, b in ts], (4 if fp8 else 3) * steps
 
 
 def prefill_report(w, t_index, t_main, peaks, peak_src, world, launches, traffic_name=None, scale=1.0):
@@ -549,25 +572,27 @@ def prefill_report(w, t_index, t_main, peaks, peak_src, world, launches, traffic
     }
 
 
-def decode_report(w, t_dec, peaks, peak_src, launches, traffic_name=None, scale=1.0):
+def decode_report(w, t_dec, peaks, peak_src, launches, traffic_name=None, scale=1.0, fp8=False):
     tdec = statistics.mean(t_dec)
-    dbytes = decode_step_bytes(w)
+    dbytes = decode_step_bytes_fp8(w) if fp8 else decode_step_bytes(w)
     gbs = dbytes["total"] / tdec / 1e9
     traffic, tnote = captured_traffic(traffic_name, scale) if traffic_name else (None, "not captured")
     return {
         "workload": w.name, "decode_step_us": tdec * 1e6, "gpu_launches": int(launches),
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, "traffic_note": tnote,
-                     "kernel": "decode step (append + select + attention, one graph replay)",
+                     "kernel": ("decode step over the FP8 cache (append + close + select + attention, one graph replay)"
+                                if fp8 else "decode step (append + select + attention, one graph replay)"),
                      "algorithmic": f"{dbytes['total']} B per step", "peak_source": f"{peak_src} copy"},
     }
 
 
-def topk_report(torch, dev, steps, warmup, peaks, peak_src, with_torch=True):
+def topk_report(torch, dev, steps, warmup, peaks, peak_src, with_torch=True, rows=8 * 131072):
     """Exp-free top-k (msa_topk_rows) on the block scores of 8 groups at 131,072 tokens:
-    [1,048,576, 1024] fp32 seeded normal values on the device, k = 15; 4.3 GB exceed L2."""
+    [1,048,576, 1024] fp32 seeded normal values on the device, k = 15; 4.3 GB exceed L2.
+    (`rows` smaller only for profiler captures.)"""
     import block_sparse_gqa_branch_b200 as msa
-    rows, n, k = 8 * 131072, 1024, 15
+    n, k = 1024, 15
     s = torch.randn(rows, n, device=dev, generator=torch.Generator(device=dev).manual_seed(0x4D5341))
     idx = torch.empty(rows, k, dtype=torch.int32, device=dev)
 
@@ -594,7 +619,7 @@ def topk_report(torch, dev, steps, warmup, peaks, peak_src, with_torch=True):
     traffic, tnote = captured_traffic("topk_rows", rows / CAPTURES["topk_rows"]["rows"]) \
         if "topk_rows" in CAPTURES else (None, "no capture recorded")
     del s
-    return {"workload": "topk_rows_1048576x1024_k15", "metric": "exp-free top-k rows/s (k = 15 of 1,024 fp32)",
+    return {"workload": f"topk_rows_{rows}x1024_k15", "metric": "exp-free top-k rows/s (k = 15 of 1,024 fp32)",
             "value": rows / t, "unit": "rows/s", "ms": t * 1e3, "gpu_launches": int(launches),
             "torch_topk_ms": None if t_ref is None else t_ref * 1e3,
             "speedup_vs_torch_topk": None if t_ref is None else t_ref / t,
@@ -819,6 +844,11 @@ def run_ours(args):
             scale=(decode_step_bytes(DECODE_1M)["total"] / CAPTURES["decode_step"]["algorithmic_bytes"]
                    if "decode_step" in CAPTURES else 1.0))
         torch.cuda.empty_cache()
+        td8, l8 = time_decode(torch, DECODE, dev, n_x, w_x, flush_l2, fp8=True)
+        r8 = decode_report(DECODE, [max_over_ranks(statistics.mean(td8))], peaks, peak_src, l8, fp8=True)
+        r8["workload"] = DECODE.name + "_fp8kv"
+        extra[r8["workload"]] = r8
+        torch.cuda.empty_cache()
         tk = topk_report(torch, dev, n_x, w_x, peaks, peak_src)
         tk["ms"] = max_over_ranks(tk["ms"])
         tk["value"] = 8 * 131072 * world / (tk["ms"] * 1e-3)
@@ -892,11 +922,11 @@ def run_topk(args):
     msa.load()
     peaks, peak_src = load_peaks()
     with ClockSampler(local) as clk:
-        r = topk_report(torch, dev, args.steps, args.warmup, peaks, peak_src)
+        r = topk_report(torch, dev, args.steps, args.warmup, peaks, peak_src, rows=args.topk_rows)
     line = {"metric": r["metric"], "value": r["value"], "unit": r["unit"], "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded normal scores generated on the device)",
-            "config": {"workload": r["workload"], "rows": 8 * 131072, "n": 1024, "k": 15,
+            "config": {"workload": r["workload"], "rows": args.topk_rows, "n": 1024, "k": 15,
                        "l2": "inputs (4.3 GB) larger than L2, no flush"},
             "roofline": r["roofline"], "torch_topk_ms": r["torch_topk_ms"],
             "speedup_vs_torch_topk": r["speedup_vs_torch_topk"], "clocks": clk.summary(),
@@ -920,6 +950,7 @@ def main():
                     help="run one half of the step (profiler captures; not a benchmark value)")
     ap.add_argument("--prefill-tokens", type=int, default=0, help="smaller prefill for profiler captures")
     ap.add_argument("--decode-batch", type=int, default=0, help="smaller decode batch for profiler captures")
+    ap.add_argument("--topk-rows", type=int, default=8 * 131072, help="rows of the top-k benchmark (captures)")
     ap.add_argument("--topk", action="store_true",
                     help="the exp-free top-k micro-benchmark against torch.topk instead of the step")
     args = ap.parse_args()

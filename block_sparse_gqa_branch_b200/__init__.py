@@ -21,7 +21,9 @@ __all__ = [
     "msa_pool_index_keys", "msa_index_select", "msa_sparse_attn_prefill",
     "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_get_device_status",
     "msa_index_select_decode_noalloc", "msa_selftest_wait_timeout", "msa_kernel_launches",
-    "msa_topk_rows",
+    "msa_topk_rows", "msa_fp8_quantize_blocks", "msa_fp8_close_blocks", "msa_sparse_attn_decode_fp8",
+    "msa_pool_index_keys_chunk", "msa_index_select_chunk", "msa_sparse_attn_prefill_chunk",
+    "msa_prefill_chunk_workspace_size",
     "OP_INDEX_SELECT_PREFILL", "OP_INDEX_SELECT_DECODE", "OP_ATTN_PREFILL", "OP_ATTN_DECODE",
     "EXPORTED_SYMBOLS",
 ]
@@ -42,6 +44,9 @@ EXPORTED_SYMBOLS = [
     "msa_pool_index_keys", "msa_index_select", "msa_sparse_attn_prefill",
     "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_get_device_status",
     "msa_index_select_decode_noalloc", "msa_selftest_wait_timeout", "msa_topk_rows",
+    "msa_fp8_quantize_blocks", "msa_fp8_close_blocks", "msa_sparse_attn_decode_fp8",
+    "msa_pool_index_keys_chunk", "msa_index_select_chunk", "msa_sparse_attn_prefill_chunk",
+    "msa_prefill_chunk_workspace_size",
 ]
 
 
@@ -87,6 +92,8 @@ def load():
         L.msa_kernel_launches.restype = ctypes.c_uint64
         L.msa_workspace_size.restype = SZ
         L.msa_workspace_size.argtypes = [SP, I32, I64]
+        L.msa_prefill_chunk_workspace_size.restype = SZ
+        L.msa_prefill_chunk_workspace_size.argtypes = [SP, I64, I64]
         for name, args in {
             "msa_pool_index_keys": [SP, P, I64, P, I64, P, P],
             "msa_index_select": [SP, P, I64, P, I64, P, I64, P, P, SZ, P],
@@ -97,6 +104,12 @@ def load():
             "msa_index_select_decode_noalloc": [SP, P, P, I64, P, I64, P, P],
             "msa_selftest_wait_timeout": [P, SZ, P],
             "msa_topk_rows": [P, I64, I64, I32, P, P, P],
+            "msa_fp8_quantize_blocks": [SP, P, P, I64, I64, P, P, P, P, I64, P],
+            "msa_fp8_close_blocks": [SP, P, P, P, I64, P, P, P, P, I64, P, SZ, P],
+            "msa_sparse_attn_decode_fp8": [SP, P, P, P, P, P, I64, P, P, I64, P, I64, P, P, P, P, SZ, P],
+            "msa_pool_index_keys_chunk": [SP, P, I64, I64, P, I64, P, P],
+            "msa_index_select_chunk": [SP, P, I64, I64, P, I64, P, P, SZ, P],
+            "msa_sparse_attn_prefill_chunk": [SP, P, P, P, I64, I64, I64, P, P, P, P, SZ, P],
         }.items():
             f = getattr(L, name)
             f.restype = ctypes.c_int
@@ -224,3 +237,59 @@ def msa_topk_rows(scores, k: int, idx, val=None, stream=None):
     rows, n = scores.shape
     _check(load().msa_topk_rows(_ptr(scores), rows, n, k, _ptr(idx), _ptr(val), _stream(stream)),
            "msa_topk_rows")
+
+
+def msa_fp8_quantize_blocks(shape: Shape, k_cache, v_cache, l_cap: int, n_tokens: int, k_codes, v_codes, k_scale,
+                            v_scale, nb_cap: int, stream=None):
+    """e4m3 codes and per-block scales of blocks j < n_tokens / 128 of the bf16 caches."""
+    _check(load().msa_fp8_quantize_blocks(ctypes.byref(shape), _ptr(k_cache), _ptr(v_cache), l_cap, n_tokens,
+                                          _ptr(k_codes), _ptr(v_codes), _ptr(k_scale), _ptr(v_scale), nb_cap,
+                                          _stream(stream)),
+           "msa_fp8_quantize_blocks")
+
+
+def msa_fp8_close_blocks(shape: Shape, ctx_len, k_cache, v_cache, l_cap: int, k_codes, v_codes, k_scale, v_scale,
+                         nb_cap: int, workspace, stream=None):
+    """Quantise the blocks that this decode step's new tokens complete (after the append)."""
+    _check(load().msa_fp8_close_blocks(ctypes.byref(shape), _ptr(ctx_len), _ptr(k_cache), _ptr(v_cache), l_cap,
+                                       _ptr(k_codes), _ptr(v_codes), _ptr(k_scale), _ptr(v_scale), nb_cap,
+                                       _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "msa_fp8_close_blocks")
+
+
+def msa_sparse_attn_decode_fp8(shape: Shape, q, k_codes, v_codes, k_scale, v_scale, nb_cap: int, k_cache, v_cache,
+                               l_cap: int, q_pos, max_pos: int, sel, out, lse, workspace, stream=None):
+    """Decode attention over the FP8 cache (closed blocks) and the bf16 cache (own block)."""
+    _check(load().msa_sparse_attn_decode_fp8(ctypes.byref(shape), _ptr(q), _ptr(k_codes), _ptr(v_codes),
+                                             _ptr(k_scale), _ptr(v_scale), nb_cap, _ptr(k_cache), _ptr(v_cache),
+                                             l_cap, _ptr(q_pos), max_pos, _ptr(sel), _ptr(out), _ptr(lse),
+                                             _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "msa_sparse_attn_decode_fp8")
+
+
+def msa_prefill_chunk_workspace_size(shape: Shape, q_start: int, n_queries: int) -> int:
+    return load().msa_prefill_chunk_workspace_size(ctypes.byref(shape), q_start, n_queries)
+
+
+def msa_pool_index_keys_chunk(shape: Shape, k_idx, q_start: int, n: int, pooled, nb_cap: int, tail_sum, stream=None):
+    """Pool the blocks a chunk of index keys completes; keep the open block's running sum."""
+    _check(load().msa_pool_index_keys_chunk(ctypes.byref(shape), _ptr(k_idx), q_start, n, _ptr(pooled), nb_cap,
+                                            _ptr(tail_sum), _stream(stream)),
+           "msa_pool_index_keys_chunk")
+
+
+def msa_index_select_chunk(shape: Shape, q_idx, q_start: int, n: int, pooled, nb_cap: int, sel, workspace,
+                           stream=None):
+    """Selection for the chunk's queries at positions q_start .. q_start + n - 1."""
+    _check(load().msa_index_select_chunk(ctypes.byref(shape), _ptr(q_idx), q_start, n, _ptr(pooled), nb_cap,
+                                         _ptr(sel), _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "msa_index_select_chunk")
+
+
+def msa_sparse_attn_prefill_chunk(shape: Shape, q, k_cache, v_cache, l_cap: int, q_start: int, n: int, sel, out, lse,
+                                  workspace, stream=None):
+    """Main Branch for the chunk's queries against the caches (positions 0 .. q_start + n - 1)."""
+    _check(load().msa_sparse_attn_prefill_chunk(ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), l_cap,
+                                                q_start, n, _ptr(sel), _ptr(out), _ptr(lse), _ptr(workspace),
+                                                _nbytes(workspace), _stream(stream)),
+           "msa_sparse_attn_prefill_chunk")

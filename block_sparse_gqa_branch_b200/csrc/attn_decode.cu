@@ -48,6 +48,7 @@ __device__ __forceinline__ uint32_t kv_off(int row, int col) {
 
 struct DecMaps {
     CUtensorMap k128, v128, k32, v32;   // boxes of 64 columns x 128 rows (full blocks) / 32 rows (diagonal)
+    CUtensorMap k8, v8;                 // FP8 variant: e4m3 codes, boxes of 128 bytes x 128 rows (full blocks)
 };
 
 struct __align__(1024) DecSmem {
@@ -60,7 +61,8 @@ struct __align__(1024) DecSmem {
     uint64_t full_k[kDecStages], full_v[kDecStages], empty[kDecStages];
     uint64_t parked[kDecStages];                // 8 warp states parked (queue of group ends)
     int meta_bg[kDecStages], meta_ntok[kDecStages], meta_fin[kDecStages], meta_nfrag[kDecStages],
-        meta_frag[kDecStages];
+        meta_frag[kDecStages], meta_fp8[kDecStages];
+    float meta_ks[kDecStages], meta_vs[kDecStages];   // FP8 variant: the block's key / value scales
     int park_stage[kDecStages];                 // stage holding the parked states (-1 = end)
     int row_sel[kRowCache][kTopK];              // loader: selection rows and positions
     int row_pos[kRowCache];
@@ -79,7 +81,40 @@ struct DecArgs {
     WsHeader* hdr;
     float scale_log2;
     double inv_grid, inv_items;                 // 1 / gridDim.x, 1 / (B G 16)
+    const float* k_scale;                       // FP8 variant: [B, G, nb_cap] per-block scales
+    const float* v_scale;
+    int64_t nb_cap;
 };
+
+// FP8 variant: widen this warp's 16 rows (kbase..kbase+15) of an e4m3 block, which TMA left as
+// [128 rows][128 B] (128B swizzle) at the start of `buf`, in place into the bf16 tile layout of
+// the full blocks ([d half][128 rows][128 B], 128B swizzle). The source bytes of a row lie
+// inside the row's half-0 destination, which only this warp writes, so every lane reads its
+// codes before any lane writes.
+__device__ __forceinline__ void widen_fp8_rows(uint8_t* buf, int kbase, int lane) {
+    const int row = kbase + (lane >> 1), h = lane & 1;      // lane pair per row, one d half each
+    uint4 c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int ch = 4 * h + i;                           // 16 codes: d = 16 ch .. 16 ch + 15
+        c[i] = *reinterpret_cast<const uint4*>(buf + row * 128 + ((ch ^ (row & 7)) << 4));
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t w[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
+        uint32_t o[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            o[2 * e] = bf16x2_from_e4m3x2(uint16_t(w[e] & 0xFFFFu));
+            o[2 * e + 1] = bf16x2_from_e4m3x2(uint16_t(w[e] >> 16));
+        }
+        // codes d = 64 h + 16 i .. +15 -> chunks (2 i) and (2 i + 1) of d half h
+        *reinterpret_cast<uint4*>(buf + h * 16384 + sw128(row, 2 * i)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(buf + h * 16384 + sw128(row, 2 * i + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+    __syncwarp();
+}
 
 // first item of CTA c when n items are cut into `grid` contiguous ranges: floor(c * n / grid)
 __device__ __forceinline__ int range_begin(int c, int n, int grid, double inv_grid) {
@@ -188,6 +223,7 @@ __device__ __forceinline__ void clear_state(WarpState& st) {
     st.l0 = st.l1 = 0.f;
 }
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __grid_constant__ DecMaps maps,
                                                                     const DecArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -281,13 +317,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
                 }
                 ntok = j < 0 ? 0 : (j == c ? pos - c * kBlock + 1 : kBlock);
                 const bool full = ntok == kBlock;
+                const bool f8 = kFp8 && j >= 0 && j < c;          // a closed block: e4m3 codes
                 const int nload = full ? kBlock : (ntok + kDecDiagRows - 1) / kDecDiagRows * kDecDiagRows;
-                mbar_expect_tx(&sm.full_k[stage], uint32_t(nload) * 256u + uint32_t(Hg) * qrow);
-                mbar_expect_tx(&sm.full_v[stage], uint32_t(nload) * 256u);
+                const uint32_t row_bytes = f8 ? 128u : 256u;
+                mbar_expect_tx(&sm.full_k[stage], uint32_t(nload) * row_bytes + uint32_t(Hg) * qrow);
+                mbar_expect_tx(&sm.full_v[stage], uint32_t(nload) * row_bytes);
                 const int row0 = int(int64_t(bg) * a.l_cap + int64_t(j < 0 ? 0 : j) * kBlock);
                 uint8_t* ks = sm.kv[stage][0];
                 uint8_t* vs = sm.kv[stage][1];
-                if (full) {
+                sm.meta_fp8[stage] = f8 ? 1 : 0;
+                if (f8) {
+                    tma_load_2d_hint(ks, &maps.k8, 0, row0, &sm.full_k[stage], pol);
+                } else if (full) {
                     for (int h = 0; h < 2; ++h)
                         tma_load_2d_hint(ks + h * 16384, &maps.k128, h * 64, row0, &sm.full_k[stage], pol);
                 } else {
@@ -297,7 +338,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
                 }
                 const uint16_t* qg = a.q + size_t(bg) * Hg * kHeadDim;
                 for (int h = 0; h < Hg; ++h) bulk_load(sm.q[stage][h], qg + h * kHeadDim, qrow, &sm.full_k[stage]);
-                if (full) {
+                if (f8) {
+                    tma_load_2d_hint(vs, &maps.v8, 0, row0, &sm.full_v[stage], pol);
+                    const size_t si = size_t(bg) * a.nb_cap + j;
+                    sm.meta_ks[stage] = __ldg(a.k_scale + si);
+                    sm.meta_vs[stage] = __ldg(a.v_scale + si);
+                } else if (full) {
                     for (int h = 0; h < 2; ++h)
                         tma_load_2d_hint(vs + h * 16384, &maps.v128, h * 64, row0, &sm.full_v[stage], pol);
                 } else {
@@ -526,7 +572,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
         }
         const int ntok = sm.meta_ntok[stage], fin = sm.meta_fin[stage];
         const bool active = kbase < ntok;
+        const bool f8 = kFp8 && sm.meta_fp8[stage] != 0;   // e4m3 codes: scores and P take the scales
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        if (f8) widen_fp8_rows(sm.kv[stage][0], kbase, lane);
         if (active) {
             const uint8_t* Ks = sm.kv[stage][0];
             const uint16_t* q0 = sm.q[stage][gq];       // query rows gq, gq + 8 (A fragments)
@@ -550,13 +598,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
         }
         // ---- online softmax of this warp's 16 keys (rows gq, gq + 8 of the accumulators)
         float mx0 = -INFINITY, mx1 = -INFINITY;
+        const float s_scale = f8 ? sm.meta_ks[stage] * a.scale_log2 : a.scale_log2;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const bool v = kbase + nt * 8 + 2 * tq + e < ntok;
-                s[nt][e] = v ? s[nt][e] * a.scale_log2 : -INFINITY;
-                s[nt][2 + e] = v ? s[nt][2 + e] * a.scale_log2 : -INFINITY;
+                s[nt][e] = v ? s[nt][e] * s_scale : -INFINITY;
+                s[nt][2 + e] = v ? s[nt][2 + e] * s_scale : -INFINITY;
                 mx0 = fmaxf(mx0, s[nt][e]);
                 mx1 = fmaxf(mx1, s[nt][2 + e]);
             }
@@ -592,6 +641,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
         if (active) {
             if (!warp_wait_all(&sm.full_v[stage], ph, a.hdr)) break;
             uint8_t* Vs = sm.kv[stage][1];
+            if (f8) widen_fp8_rows(Vs, kbase, lane);
             if (ntok < kbase + 16) {                    // rows past the query must be finite: zero them
                 const int r0 = ntok - kbase;             // 1 .. 15
                 for (int i = lane; i < (16 - r0) * 16; i += 32) {
@@ -600,8 +650,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
                 }
                 __syncwarp();
             }
-            const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]), pa1 = pack_bf16x2(p[0][2], p[0][3]);
-            const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]), pa3 = pack_bf16x2(p[1][2], p[1][3]);
+            // FP8: the values are code x scale, so P is weighted by the block's value scale
+            const float vsc = f8 ? sm.meta_vs[stage] : 1.f;
+            const uint32_t pa0 = pack_bf16x2(p[0][0] * vsc, p[0][1] * vsc), pa1 = pack_bf16x2(p[0][2] * vsc, p[0][3] * vsc);
+            const uint32_t pa2 = pack_bf16x2(p[1][0] * vsc, p[1][1] * vsc), pa3 = pack_bf16x2(p[1][2] * vsc, p[1][3] * vsc);
             const uint32_t vrow = smem_u32(Vs);
             const int row = kbase + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
@@ -613,7 +665,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
             }
         }
         if (!fin) {
-            if (active && ntok < kbase + 16) fence_proxy_async();   // zeroed rows before the next TMA fill
+            if (f8 || (active && ntok < kbase + 16)) fence_proxy_async();   // rewritten rows before the next TMA fill
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);   // this warp is done with the stage
             continue;
@@ -654,13 +706,22 @@ int num_sms();
 
 msa_status_t launch_attn_decode(const void* k_cache, const void* v_cache, const void* q, int64_t l_cap,
                                 const int32_t* q_pos, int64_t max_pos, const int32_t* sel, int B, int G, int Hg,
-                                void* out, float* lse, void* ws, cudaStream_t st) {
+                                void* out, float* lse, void* ws, cudaStream_t st, const void* k8, const void* v8,
+                                const float* k_scale, const float* v_scale, int64_t nb_cap) {
+    const bool fp8 = k8 != nullptr;
     DecMaps maps;
     const uint64_t rows = uint64_t(B) * G * uint64_t(l_cap);
     msa_status_t e = make_tmap_bf16(&maps.k128, k_cache, rows, kHeadDim, 64, 128);
     if (e == MSA_OK) e = make_tmap_bf16(&maps.v128, v_cache, rows, kHeadDim, 64, 128);
     if (e == MSA_OK) e = make_tmap_bf16(&maps.k32, k_cache, rows, kHeadDim, 64, kDecDiagRows);
     if (e == MSA_OK) e = make_tmap_bf16(&maps.v32, v_cache, rows, kHeadDim, 64, kDecDiagRows);
+    if (fp8) {
+        if (e == MSA_OK) e = make_tmap_u8(&maps.k8, k8, rows, kHeadDim, 128, 128);
+        if (e == MSA_OK) e = make_tmap_u8(&maps.v8, v8, rows, kHeadDim, 128, 128);
+    } else {
+        maps.k8 = maps.k128;                         // unused by the bf16 variant
+        maps.v8 = maps.v128;
+    }
     if (e != MSA_OK) return e;
     const size_t nbg = size_t(B) * G;
     char* p = static_cast<char*>(ws);
@@ -673,13 +734,15 @@ msa_status_t launch_attn_decode(const void* k_cache, const void* v_cache, const 
     a.ctr = reinterpret_cast<unsigned int*>(p + sizeof(WsHeader));
     a.part = reinterpret_cast<float*>(p + sizeof(WsHeader) + (nbg * sizeof(unsigned int) + 255) / 256 * 256);
     a.scale_log2 = 1.4426950408889634f / sqrtf(float(kHeadDim));
+    a.k_scale = k_scale; a.v_scale = v_scale; a.nb_cap = nb_cap;
     const int smem = int(sizeof(DecSmem)) + 1024;
-    static std::atomic<bool> attr_set[64];          // per device; setting it twice is harmless
+    auto kern = fp8 ? attn_decode_kernel<true> : attn_decode_kernel<false>;
+    static std::atomic<bool> attr_set[2][64];       // per variant and device; setting it twice is harmless
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
-        cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        attr_set[dev].store(true, std::memory_order_relaxed);
+    if (dev >= 0 && dev < 64 && !attr_set[fp8][dev].load(std::memory_order_relaxed)) {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        attr_set[fp8][dev].store(true, std::memory_order_relaxed);
     }
     const int64_t n_items = int64_t(B) * G * kTopK;
     const int grid = int(n_items < num_sms() ? n_items : num_sms());   // persistent: one CTA per SM
@@ -696,7 +759,7 @@ msa_status_t launch_attn_decode(const void* k_cache, const void* v_cache, const 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     count_launch();
-    cudaLaunchKernelEx(&cfg, attn_decode_kernel, maps, a);
+    cudaLaunchKernelEx(&cfg, kern, maps, a);
     return cuda_status();
 }
 

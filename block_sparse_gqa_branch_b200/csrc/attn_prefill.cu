@@ -36,8 +36,11 @@ constexpr int kKvThreads = 352;         // warps 0-7 softmax/epilogue, 8 Q loads
 static_assert(kRange % kCountChunk == 0 && kRange % kBlock == 0, "range must hold whole chunks and blocks");
 
 // ------------------------------------------------------------------ workspace layout
+// Queries are the n tokens at positions P .. P + n - 1 of each sequence (P = 0 for a whole
+// prefill; P > 0 for a chunk against a cache that holds positions 0 .. P + n - 1). Token
+// indices inside the kernels are chunk-relative (i = t - P); block ids are absolute.
 struct PrefillLayout {
-    int nb, nR, nbins_seg, tpt;
+    int nb, nR, nbins_seg, tpt;     // nb: key blocks that can be selected (ceil((P + n) / Bk))
     size_t nbins, max_items, max_entries;
     size_t off_counts, off_offsets, off_nitems, off_items, off_list, off_lse, off_o, total;
 };
@@ -45,16 +48,19 @@ struct PrefillLayout {
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 __host__ __device__ inline int64_t imin64(int64_t x, int64_t y) { return x < y ? x : y; }
 
-PrefillLayout prefill_layout(int B, int64_t N, int G, int Hg) {
+PrefillLayout prefill_layout(int B, int64_t N, int G, int Hg, int64_t P) {
     PrefillLayout L{};
-    L.nb = int((N + kBlock - 1) / kBlock);
+    L.nb = int((P + N + kBlock - 1) / kBlock);
     L.nR = int((N + kRange - 1) / kRange);
     L.nbins_seg = L.nb + 1;                                   // blocks + one bin for the diagonal items
     L.tpt = kBlock / Hg;
     L.nbins = size_t(B) * G * L.nR * L.nbins_seg;
     L.max_entries = size_t(B) * N * G * (kTopK - 1);
+    // list items: at most one per started run of kMaxTilesPerItem tiles plus one per bin;
+    // diagonal items: one per (range, query block) overlap, at most (query blocks + ranges)
+    const size_t nqb = size_t((P + N - 1) / kBlock - P / kBlock + 1);
     L.max_items = L.max_entries / (size_t(L.tpt) * kMaxTilesPerItem) + 1 + size_t(B) * G * L.nR * L.nb +
-                  size_t(B) * G * L.nb;
+                  size_t(B) * G * (nqb + L.nR);
     size_t o = sizeof(WsHeader);
     L.off_counts = o;   o = align_up(o + L.nbins * 4, 256);
     L.off_offsets = o;  o = align_up(o + L.nbins * 4, 256);
@@ -67,12 +73,14 @@ PrefillLayout prefill_layout(int B, int64_t N, int G, int Hg) {
     return L;
 }
 
-size_t prefill_attn_ws_bytes(int B, int64_t N, int G, int Hg) { return prefill_layout(B, N, G, Hg).total; }
+size_t prefill_attn_ws_bytes(int B, int64_t N, int G, int Hg, int64_t P) {
+    return prefill_layout(B, N, G, Hg, P).total;
+}
 
 // ------------------------------------------------------------------ CSR: count
-// grid (ceil(N / 1024), G, B), 256 threads, dynamic smem nb ints.
-__global__ void __launch_bounds__(256) csr_count_kernel(const int32_t* __restrict__ sel, int64_t N, int G, int nb,
-                                                        int nR, int* __restrict__ counts, WsHeader* hdr) {
+// grid (ceil(N / 1024), G, B), 256 threads, dynamic smem nb ints. N queries from position P.
+__global__ void __launch_bounds__(256) csr_count_kernel(const int32_t* __restrict__ sel, int64_t N, int64_t P, int G,
+                                                        int nb, int nR, int* __restrict__ counts, WsHeader* hdr) {
     extern __shared__ int hist[];
     const int g = blockIdx.y, b = blockIdx.z;
     const int64_t t0 = int64_t(blockIdx.x) * kCountChunk;
@@ -82,7 +90,7 @@ __global__ void __launch_bounds__(256) csr_count_kernel(const int32_t* __restric
     __syncthreads();
     for (int64_t t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
         const int4* row = reinterpret_cast<const int4*>(sel + ((size_t(b) * N + t) * G + g) * kTopK);
-        const int c = int(t / kBlock);
+        const int c = int((P + t) / kBlock);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const int4 v = row[q];
@@ -107,15 +115,17 @@ __global__ void __launch_bounds__(256) csr_count_kernel(const int32_t* __restric
 // work items in bin order: {b*G+g, j (| kDiagFlag), first entry (or first token), count}.
 __global__ void __launch_bounds__(1024) csr_scan_kernel(int* __restrict__ counts, int* __restrict__ offsets,
                                                         int4* __restrict__ items, int* __restrict__ n_items,
-                                                        int64_t nbins, int nb, int nR, int64_t N, int tpt) {
+                                                        int64_t nbins, int nb, int nR, int64_t N, int64_t P, int tpt) {
     __shared__ long long s_e[1024], s_i[1024];
     const int nbs = nb + 1;
     const int64_t per = (nbins + 1023) / 1024;
     const int64_t lo = imin64(nbins, int64_t(threadIdx.x) * per), hi = imin64(nbins, lo + per);
     const int items_per_max = kMaxTilesPerItem * tpt;
+    // query blocks [c0, c1) that hold positions of range R (queries R kRange .. (R + 1) kRange - 1)
     auto diag_blocks = [&](int R, int& c0, int& c1) {
-        c0 = R * (kRange / kBlock);
-        c1 = min(nb, (R + 1) * (kRange / kBlock));
+        const int64_t a = P + int64_t(R) * kRange, z = P + imin64(N, int64_t(R + 1) * kRange);
+        c0 = int(a / kBlock);
+        c1 = int((z - 1) / kBlock) + 1;
     };
     long long se = 0, si = 0;
     for (int64_t bin = lo; bin < hi; ++bin) {
@@ -155,10 +165,15 @@ __global__ void __launch_bounds__(1024) csr_scan_kernel(int* __restrict__ counts
                 items[ioff++] = make_int4(bg, j, int(eoff + k0), min(items_per_max, cnt - k0));
             eoff += cnt;
         } else {
+            // diagonal items: the range's queries inside block c, as (first query index, count)
             int c0, c1;
             diag_blocks(R, c0, c1);
-            for (int c = c0; c < c1; ++c)
-                items[ioff++] = make_int4(bg, c | kDiagFlag, c * kBlock, int(imin64(kBlock, N - int64_t(c) * kBlock)));
+            const int64_t qa = int64_t(R) * kRange, qz = imin64(N, int64_t(R + 1) * kRange);
+            for (int c = c0; c < c1; ++c) {
+                const int64_t f = int64_t(c) * kBlock - P > qa ? int64_t(c) * kBlock - P : qa;
+                const int64_t e = imin64(qz, int64_t(c + 1) * kBlock - P);
+                items[ioff++] = make_int4(bg, c | kDiagFlag, int(f), int(e - f));
+            }
         }
     }
     if (threadIdx.x == 1023) {
@@ -169,16 +184,16 @@ __global__ void __launch_bounds__(1024) csr_scan_kernel(int* __restrict__ counts
 
 // ------------------------------------------------------------------ CSR: fill
 // one thread per (b, t, g): appends (t, slot) to the list of every fully-past selected block
-__global__ void __launch_bounds__(256) csr_fill_kernel(const int32_t* __restrict__ sel, int64_t N, int G, int nb,
-                                                       int nR, const int* __restrict__ offsets,
+__global__ void __launch_bounds__(256) csr_fill_kernel(const int32_t* __restrict__ sel, int64_t N, int64_t P, int G,
+                                                       int nb, int nR, const int* __restrict__ offsets,
                                                        int* __restrict__ cursors, int* __restrict__ list,
                                                        int64_t total) {
     const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= total) return;
     const int g = int(idx % G);
-    const int64_t t = (idx / G) % N;
+    const int64_t t = (idx / G) % N;                  // query index (position P + t)
     const int b = int(idx / (int64_t(G) * N));
-    const int c = int(t / kBlock);
+    const int c = int((P + t) / kBlock);
     const int R = int(t / kRange);
     const int4* row = reinterpret_cast<const int4*>(sel + size_t(idx) * kTopK);
     const size_t seg = (size_t(b * G + g) * nR + R) * (nb + 1);
@@ -216,7 +231,8 @@ struct __align__(1024) KvSmem {
 };
 
 struct PrefillArgs {
-    int64_t N;
+    int64_t N;                     // queries per sequence (positions P .. P + N - 1)
+    int64_t P;                     // position of the first query
     int G, Hg, Hq, tpt;
     int* n_items;                  // [0] = number of work items, [1] = next item to hand out
     const int4* items;
@@ -500,16 +516,17 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
                     const uint64_t hi = (uint64_t(reinterpret_cast<uintptr_t>(a.list + item.first + item.n)) + 15) & ~uint64_t(15);
                     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(lo), "r"(uint32_t(hi - lo)) : "memory");
                 }
-                const int row0 = int(int64_t(item.bg) * a.N + int64_t(item.j) * kBlock);
+                // block j of (sequence, group) bg: rows past the last query position are zeros
+                const int row0 = item.j * kBlock;
                 const int kb = ic & 1;
                 if (!mbar_wait(&sm.k_empty[kb], ((ic >> 1) & 1) ^ 1, a.hdr, KID_ATTN_PREFILL)) { sm.abort_flag = 1; break; }
                 mbar_arrive_expect_tx(&sm.k_full[kb], 32768);
-                tma_load_2d_hint(sm.k[kb], &tmK, 0, row0, &sm.k_full[kb], stream);
-                tma_load_2d_hint(sm.k[kb] + 16384, &tmK, 64, row0, &sm.k_full[kb], stream);
+                tma_load_3d_hint(sm.k[kb], &tmK, 0, row0, item.bg, &sm.k_full[kb], stream);
+                tma_load_3d_hint(sm.k[kb] + 16384, &tmK, 64, row0, item.bg, &sm.k_full[kb], stream);
                 if (!mbar_wait(&sm.v_empty, (ic & 1) ^ 1, a.hdr, KID_ATTN_PREFILL)) { sm.abort_flag = 1; break; }
                 mbar_arrive_expect_tx(&sm.v_full, 32768);
-                tma_load_2d_hint(sm.v, &tmV, 0, row0, &sm.v_full, stream);
-                tma_load_2d_hint(sm.v + 16384, &tmV, 64, row0, &sm.v_full, stream);
+                tma_load_3d_hint(sm.v, &tmV, 0, row0, item.bg, &sm.v_full, stream);
+                tma_load_3d_hint(sm.v + 16384, &tmV, 64, row0, item.bg, &sm.v_full, stream);
             }
         }
         __syncwarp();
@@ -590,8 +607,9 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
                     if (item.diag) t = item.first + e;
                     else { const int v = __ldg(a.list + item.first + e); t = v / kSlots; slot = v % kSlots; }
                 }
-                // columns past lim are masked (causal mask of the diagonal block)
-                const int lim = item.diag ? t - item.j * kBlock : kBlock - 1;
+                // columns past lim are masked (causal mask of the diagonal block; t is the
+                // query index, P + t its position)
+                const int lim = item.diag ? int(a.P + t - int64_t(item.j) * kBlock) : kBlock - 1;
                 if (!warp_wait(&sm.s_full[w], use & 1, a.hdr)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t va[32], vb[32];
@@ -755,9 +773,9 @@ int num_sms() {
 }
 
 msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, const CUtensorMap& tmK, const CUtensorMap& tmV, int64_t N,
-                            int B, int G, int Hg, const int32_t* sel, void* out, float* lse, void* ws,
-                            cudaStream_t st) {
-    const PrefillLayout L = prefill_layout(B, N, G, Hg);
+                            int64_t P, int64_t l_cap, int B, int G, int Hg, const int32_t* sel, void* out, float* lse,
+                            void* ws, cudaStream_t st) {
+    const PrefillLayout L = prefill_layout(B, N, G, Hg, P);
     char* base = static_cast<char*>(ws);
     WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
     int* counts = reinterpret_cast<int*>(base + L.off_counts);
@@ -776,19 +794,19 @@ msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, cons
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(csr_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         count_launch();
-        csr_count_kernel<<<grid, 256, smem, st>>>(sel, N, G, L.nb, L.nR, counts, hdr);
+        csr_count_kernel<<<grid, 256, smem, st>>>(sel, N, P, G, L.nb, L.nR, counts, hdr);
     }
     count_launch();
-    csr_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, items, nitems, int64_t(L.nbins), L.nb, L.nR, N, L.tpt);
+    csr_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, items, nitems, int64_t(L.nbins), L.nb, L.nR, N, P, L.tpt);
     {
         const int64_t total = int64_t(B) * N * G;
         count_launch();
-        csr_fill_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(sel, N, G, L.nb, L.nR, offsets,
+        csr_fill_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(sel, N, P, G, L.nb, L.nR, offsets,
                                                                                    counts, list, total);
     }
     {
         PrefillArgs a;
-        a.N = N; a.G = G; a.Hg = Hg; a.Hq = G * Hg; a.tpt = L.tpt;
+        a.N = N; a.P = P; a.G = G; a.Hg = Hg; a.Hq = G * Hg; a.tpt = L.tpt;
         a.n_items = nitems; a.items = items; a.list = list; a.part_lse = part_lse; a.part_o = part_o;
         a.q = static_cast<const uint16_t*>(q);
         a.hdr = hdr;

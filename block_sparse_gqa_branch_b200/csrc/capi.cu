@@ -14,16 +14,22 @@ namespace msa {
 void launch_pool(const void*, int, int, int64_t, float*, int64_t, float*, cudaStream_t);
 void launch_append(const void*, const void*, const void*, const int32_t*, int, int, void*, void*, int64_t,
                    float*, float*, int64_t, void*, cudaStream_t);
-void launch_select_prefill_mma(const void*, int, int, int64_t, const float*, int64_t, int32_t*, cudaStream_t);
+void launch_select_prefill_mma(const void*, int, int, int64_t, int64_t, const float*, int64_t, int32_t*, cudaStream_t);
+void launch_pool_chunk(const void*, int, int, int64_t, int64_t, float*, int64_t, float*, cudaStream_t);
 void launch_select_decode(const void*, const int32_t*, int64_t, int, int, const float*, int64_t, int32_t*,
                           void*, cudaStream_t);
 size_t decode_select_ws_bytes(int, int, int64_t);
 msa_status_t launch_attn_decode(const void*, const void*, const void*, int64_t, const int32_t*, int64_t, const int32_t*,
-                                int, int, int, void*, float*, void*, cudaStream_t);
+                                int, int, int, void*, float*, void*, cudaStream_t, const void*, const void*,
+                                const float*, const float*, int64_t);
+void launch_fp8_quantize(const void*, const void*, int64_t, int64_t, int, int, void*, void*, float*, float*, int64_t,
+                         cudaStream_t);
+void launch_fp8_close(const void*, const void*, int64_t, const int32_t*, int, int, void*, void*, float*, float*, int64_t,
+                      void*, cudaStream_t);
 size_t decode_attn_ws_bytes(int, int, int);
-size_t prefill_attn_ws_bytes(int, int64_t, int, int);
-msa_status_t launch_attn_prefill_tc(const void*, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, int64_t, int,
-                                    int, int, const int32_t*, void*, float*, void*, cudaStream_t);
+size_t prefill_attn_ws_bytes(int, int64_t, int, int, int64_t);
+msa_status_t launch_attn_prefill_tc(const void*, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, int64_t,
+                                    int64_t, int64_t, int, int, int, const int32_t*, void*, float*, void*, cudaStream_t);
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
@@ -86,6 +92,42 @@ msa_status_t make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uin
     }
     return MSA_OK;
 }
+msa_status_t make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                          uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return MSA_ERR_CUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error = int(r);
+        return MSA_ERR_CUDA;
+    }
+    return MSA_OK;
+}
+// Key / value rows of every (sequence, group) as a 3-D bf16 tensor (64-column halves, rows,
+// sequence x group) whose row extent is `rows_valid` of the `l_cap` rows each (sequence, group)
+// holds: a 128-row box that reaches past the valid rows is zero-filled there by the copy.
+msa_status_t make_tmap_kv3d(CUtensorMap* m, const void* base, uint64_t rows_valid, uint64_t l_cap, uint64_t nbg) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return MSA_ERR_CUDA;
+    cuuint64_t dims[3] = {uint64_t(kHeadDim), rows_valid, nbg};
+    cuuint64_t strides[2] = {uint64_t(kHeadDim) * 2, l_cap * kHeadDim * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error = int(r);
+        return MSA_ERR_CUDA;
+    }
+    return MSA_OK;
+}
 msa_status_t make_tmap_q_rows(CUtensorMap* m, const void* base, uint64_t rows) {
     auto fn = encode_fn();
     if (fn == nullptr) return MSA_ERR_CUDA;
@@ -133,7 +175,7 @@ size_t ws_size(const msa_shape_t* s, int32_t op, int64_t n) {
             return decode_select_ws_bytes(s->batch, s->n_kv_groups, n);
         case MSA_OP_ATTN_PREFILL:
             if (n < 1) return 0;
-            return prefill_attn_ws_bytes(s->batch, n, s->n_kv_groups, hg);
+            return prefill_attn_ws_bytes(s->batch, n, s->n_kv_groups, hg, 0);
         case MSA_OP_ATTN_DECODE: return decode_attn_ws_bytes(s->batch, s->n_kv_groups, hg);
         default: return 0;
     }
@@ -192,7 +234,7 @@ msa_status_t msa_index_select(const msa_shape_t* shape, const void* q_idx, int64
         MSA_REQ(nb_cap >= (n_queries - 1) / kBlock, MSA_ERR_INVALID_ARGUMENT);
         const size_t need = ws_size(shape, MSA_OP_INDEX_SELECT_PREFILL, n_queries);
         MSA_REQ(workspace != nullptr && workspace_bytes >= need, MSA_ERR_WORKSPACE);
-        launch_select_prefill_mma(q_idx, B, G, n_queries, pooled, nb_cap, sel, st);
+        launch_select_prefill_mma(q_idx, B, G, n_queries, 0, pooled, nb_cap, sel, st);
     } else {                                       // decode: one query per sequence at q_pos[b]
         MSA_REQ(n_queries == 1, MSA_ERR_INVALID_ARGUMENT);
         MSA_REQ(max_pos <= kMaxPos, MSA_ERR_UNSUPPORTED);
@@ -204,11 +246,16 @@ msa_status_t msa_index_select(const msa_shape_t* shape, const void* q_idx, int64
     return cuda_status();
 }
 
-msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const void* q, const void* k, const void* v,
-                                     int64_t n_tokens, const int32_t* sel, void* out, float* lse, void* workspace,
-                                     size_t workspace_bytes, msa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// Main Branch prefill for the n queries at positions P .. P + n - 1 against k, v [B, G, l_cap, d]
+// (P = 0, l_cap = n: a whole prefill).
+msa_status_t attn_prefill_impl(const msa_shape_t* shape, const void* q, const void* k, const void* v, int64_t l_cap,
+                               int64_t P, int64_t n_tokens, const int32_t* sel, void* out, float* lse,
+                               void* workspace, size_t workspace_bytes, msa_stream_t stream) {
     MSA_TRY(check_shape(shape));
-    MSA_REQ(n_tokens >= 1 && n_tokens < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(n_tokens >= 1 && n_tokens < (int64_t(1) << 31) && P >= 0 && P + n_tokens <= l_cap, MSA_ERR_INVALID_ARGUMENT);
     MSA_REQ(q && k && v && sel && out && aligned16(q) && aligned16(k) && aligned16(v) && aligned16(sel) &&
                 aligned16(out) && (lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u) == 0),
             MSA_ERR_INVALID_ARGUMENT);
@@ -218,17 +265,70 @@ msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const void* q, co
     // shared memory
     MSA_REQ(int64_t(B) * n_tokens * G * (kTopK - 1) < (int64_t(1) << 31) &&
                 int64_t(B) * n_tokens * Hq * kTopK < (int64_t(1) << 31) &&
-                int64_t(B) * G * n_tokens + kBlock < (int64_t(1) << 31) && (n_tokens + kBlock - 1) / kBlock <= 48 * 1024,
+                int64_t(B) * G * l_cap + kBlock < (int64_t(1) << 31) &&
+                (P + n_tokens + kBlock - 1) / kBlock <= 48 * 1024,
             MSA_ERR_UNSUPPORTED);
-    const size_t need = ws_size(shape, MSA_OP_ATTN_PREFILL, n_tokens);
+    const size_t need = prefill_attn_ws_bytes(B, n_tokens, G, hg, P);
     MSA_REQ(workspace != nullptr && aligned16(workspace) && need > 0 && workspace_bytes >= need, MSA_ERR_WORKSPACE);
     CUtensorMap tmQ, tmK, tmV;
     MSA_TRY(make_tmap_bf16(&tmQ, q, uint64_t(B) * n_tokens * Hq, kHeadDim, 64, uint32_t(hg)));
-    MSA_TRY(make_tmap_bf16(&tmK, k, uint64_t(B) * G * n_tokens, kHeadDim, 64, 128));
-    MSA_TRY(make_tmap_bf16(&tmV, v, uint64_t(B) * G * n_tokens, kHeadDim, 64, 128));
-    MSA_TRY(launch_attn_prefill_tc(q, tmQ, tmK, tmV, n_tokens, B, G, hg, sel, out, lse, workspace,
+    // rows past P + n_tokens (the chunk's last position) read as zeros
+    MSA_TRY(make_tmap_kv3d(&tmK, k, uint64_t(P + n_tokens), uint64_t(l_cap), uint64_t(B) * G));
+    MSA_TRY(make_tmap_kv3d(&tmV, v, uint64_t(P + n_tokens), uint64_t(l_cap), uint64_t(B) * G));
+    MSA_TRY(launch_attn_prefill_tc(q, tmQ, tmK, tmV, n_tokens, P, l_cap, B, G, hg, sel, out, lse, workspace,
                                    reinterpret_cast<cudaStream_t>(stream)));
     return cuda_status();
+}
+}  // namespace
+
+extern "C" {
+
+msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const void* q, const void* k, const void* v,
+                                     int64_t n_tokens, const int32_t* sel, void* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, msa_stream_t stream) {
+    return attn_prefill_impl(shape, q, k, v, n_tokens, 0, n_tokens, sel, out, lse, workspace, workspace_bytes,
+                             stream);
+}
+
+size_t msa_prefill_chunk_workspace_size(const msa_shape_t* shape, int64_t q_start, int64_t n_queries) {
+    if (check_shape(shape) != MSA_OK || q_start < 0 || n_queries < 1) return 0;
+    return prefill_attn_ws_bytes(shape->batch, n_queries, shape->n_kv_groups, shape->n_q_heads / shape->n_kv_groups,
+                                 q_start);
+}
+
+msa_status_t msa_pool_index_keys_chunk(const msa_shape_t* shape, const void* k_idx, int64_t q_start, int64_t n,
+                                       float* pooled, int64_t nb_cap, float* tail_sum, msa_stream_t stream) {
+    MSA_TRY(check_shape(shape));
+    MSA_REQ(n >= 1 && q_start >= 0 && q_start + n < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(k_idx && aligned16(k_idx) && tail_sum && aligned16(tail_sum), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(nb_cap >= (q_start + n) / kBlock && (q_start + n < kBlock * (q_start / kBlock + 1) ||
+                                                 (pooled != nullptr && aligned16(pooled))),
+            MSA_ERR_INVALID_ARGUMENT);
+    launch_pool_chunk(k_idx, shape->batch, shape->n_kv_groups, n, q_start, pooled, nb_cap, tail_sum,
+                      reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status();
+}
+
+msa_status_t msa_index_select_chunk(const msa_shape_t* shape, const void* q_idx, int64_t q_start, int64_t n,
+                                    const float* pooled, int64_t nb_cap, int32_t* sel, void* workspace,
+                                    size_t workspace_bytes, msa_stream_t stream) {
+    MSA_TRY(check_shape(shape));
+    MSA_REQ(q_idx && aligned16(q_idx) && sel && aligned16(sel), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(n >= 1 && q_start >= 0 && q_start + n < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(nb_cap >= (q_start + n - 1) / kBlock, MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(pooled == nullptr ? q_start + n - 1 < kBlock : aligned16(pooled), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(workspace != nullptr && workspace_bytes >= header_only(), MSA_ERR_WORKSPACE);
+    launch_select_prefill_mma(q_idx, shape->batch, shape->n_kv_groups, n, q_start, pooled, nb_cap, sel,
+                              reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status();
+}
+
+msa_status_t msa_sparse_attn_prefill_chunk(const msa_shape_t* shape, const void* q, const void* k_cache,
+                                           const void* v_cache, int64_t l_cap, int64_t q_start, int64_t n,
+                                           const int32_t* sel, void* out, float* lse, void* workspace,
+                                           size_t workspace_bytes, msa_stream_t stream) {
+    return attn_prefill_impl(shape, q, k_cache, v_cache, l_cap, q_start, n, sel, out, lse, workspace,
+                             workspace_bytes, stream);
 }
 
 msa_status_t msa_pooled_keys_append(const msa_shape_t* shape, const void* k_idx_new, const void* k_new,
@@ -267,7 +367,64 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const void* q, con
     const size_t need = ws_size(shape, MSA_OP_ATTN_DECODE, max_pos);
     MSA_REQ(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need, MSA_ERR_WORKSPACE);
     MSA_TRY(launch_attn_decode(k_cache, v_cache, q, l_cap, q_pos, max_pos, sel, B, G, shape->n_q_heads / G, out, lse,
-                               workspace, reinterpret_cast<cudaStream_t>(stream)));
+                               workspace, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr, nullptr,
+                               0));
+    return cuda_status();
+}
+
+msa_status_t msa_fp8_quantize_blocks(const msa_shape_t* shape, const void* k_cache, const void* v_cache, int64_t l_cap,
+                                     int64_t n_tokens, void* k_codes, void* v_codes, float* k_scale, float* v_scale,
+                                     int64_t nb_cap, msa_stream_t stream) {
+    MSA_TRY(check_shape(shape));
+    MSA_REQ(n_tokens >= 0 && l_cap >= n_tokens && l_cap >= 1, MSA_ERR_INVALID_ARGUMENT);
+    const int64_t nblk = n_tokens / kBlock;
+    MSA_REQ(nb_cap >= nblk && nblk <= 65535, MSA_ERR_INVALID_ARGUMENT);
+    if (nblk == 0) return MSA_OK;
+    MSA_REQ(k_cache && v_cache && k_codes && v_codes && k_scale && v_scale && aligned16(k_cache) &&
+                aligned16(v_cache) && aligned16(k_codes) && aligned16(v_codes) &&
+                (reinterpret_cast<uintptr_t>(k_scale) & 3u) == 0 && (reinterpret_cast<uintptr_t>(v_scale) & 3u) == 0,
+            MSA_ERR_INVALID_ARGUMENT);
+    launch_fp8_quantize(k_cache, v_cache, l_cap, nblk, shape->batch, shape->n_kv_groups, k_codes, v_codes, k_scale,
+                        v_scale, nb_cap, reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status();
+}
+
+msa_status_t msa_fp8_close_blocks(const msa_shape_t* shape, const int32_t* ctx_len, const void* k_cache,
+                                  const void* v_cache, int64_t l_cap, void* k_codes, void* v_codes, float* k_scale,
+                                  float* v_scale, int64_t nb_cap, void* workspace, size_t workspace_bytes,
+                                  msa_stream_t stream) {
+    MSA_TRY(check_shape(shape));
+    MSA_REQ(ctx_len && k_cache && v_cache && k_codes && v_codes && k_scale && v_scale && aligned16(k_cache) &&
+                aligned16(v_cache) && aligned16(k_codes) && aligned16(v_codes) &&
+                (reinterpret_cast<uintptr_t>(k_scale) & 3u) == 0 && (reinterpret_cast<uintptr_t>(v_scale) & 3u) == 0,
+            MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(l_cap >= kBlock && nb_cap >= 1, MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(workspace != nullptr && workspace_bytes >= header_only(), MSA_ERR_WORKSPACE);
+    launch_fp8_close(k_cache, v_cache, l_cap, ctx_len, shape->batch, shape->n_kv_groups, k_codes, v_codes, k_scale,
+                     v_scale, nb_cap, workspace, reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status();
+}
+
+msa_status_t msa_sparse_attn_decode_fp8(const msa_shape_t* shape, const void* q, const void* k_codes,
+                                        const void* v_codes, const float* k_scale, const float* v_scale,
+                                        int64_t nb_cap, const void* k_cache, const void* v_cache, int64_t l_cap,
+                                        const int32_t* q_pos, int64_t max_pos, const int32_t* sel, void* out,
+                                        float* lse, void* workspace, size_t workspace_bytes, msa_stream_t stream) {
+    MSA_TRY(check_shape(shape));
+    MSA_REQ(q && k_codes && v_codes && k_scale && v_scale && k_cache && v_cache && q_pos && sel && out &&
+                aligned16(q) && aligned16(k_codes) && aligned16(v_codes) && aligned16(k_cache) &&
+                aligned16(v_cache) && aligned16(sel) && aligned16(out) &&
+                (reinterpret_cast<uintptr_t>(k_scale) & 3u) == 0 && (reinterpret_cast<uintptr_t>(v_scale) & 3u) == 0 &&
+                (lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u) == 0),
+            MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(l_cap >= 1 && max_pos >= 0 && max_pos < l_cap && nb_cap >= max_pos / kBlock, MSA_ERR_INVALID_ARGUMENT);
+    const int B = shape->batch, G = shape->n_kv_groups;
+    MSA_REQ(int64_t(B) * G * l_cap + kBlock < (int64_t(1) << 31), MSA_ERR_UNSUPPORTED);
+    const size_t need = ws_size(shape, MSA_OP_ATTN_DECODE, max_pos);
+    MSA_REQ(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need, MSA_ERR_WORKSPACE);
+    MSA_TRY(launch_attn_decode(k_cache, v_cache, q, l_cap, q_pos, max_pos, sel, B, G, shape->n_q_heads / G, out, lse,
+                               workspace, reinterpret_cast<cudaStream_t>(stream), k_codes, v_codes, k_scale, v_scale,
+                               nb_cap));
     return cuda_status();
 }
 

@@ -23,6 +23,13 @@ msa_status_t cuda_status();                       // MSA_ERR_CUDA if the last la
 // 2-D bf16 TMA descriptor (rows x cols, row stride = cols), box box_cols x box_rows, 128B swizzle
 msa_status_t make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                             uint32_t box_rows);
+// 2-D uint8 TMA descriptor (rows x cols bytes, row stride = cols), box box_cols x box_rows, 128B swizzle
+msa_status_t make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                          uint32_t box_rows);
+// Key / value cache rows as a 3-D bf16 tensor {128 columns, rows_valid rows, nbg} with row stride
+// 256 B and (sequence, group) stride l_cap rows; box {64, 128, 1}, 128B swizzle; rows at or past
+// rows_valid are zero-filled by the copy.
+msa_status_t make_tmap_kv3d(CUtensorMap* m, const void* base, uint64_t rows_valid, uint64_t l_cap, uint64_t nbg);
 // Rows of 128 bf16 viewed as (64 columns, row, d half): box {64, 8, 2} lands 8 rows with both
 // halves as [half][8 rows][128 B] (128B swizzle)
 msa_status_t make_tmap_q_rows(CUtensorMap* m, const void* base, uint64_t rows);
@@ -48,7 +55,7 @@ static_assert(sizeof(WsHeader) == 256, "workspace header must be 256 bytes");
 
 enum KernelId : int {
     KID_POOL = 1, KID_SELECT_PREFILL = 2, KID_SELECT_DECODE = 3, KID_APPEND = 4,
-    KID_ATTN_DECODE = 5, KID_ATTN_PREFILL = 6, KID_CSR = 7, KID_COMBINE = 8, KID_SELFTEST = 9
+    KID_ATTN_DECODE = 5, KID_ATTN_PREFILL = 6, KID_CSR = 7, KID_COMBINE = 8, KID_SELFTEST = 9, KID_FP8 = 10
 };
 
 __device__ __forceinline__ void record_error(WsHeader* h, unsigned code, int kid, int blk,
@@ -270,6 +277,17 @@ __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t saddr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(saddr));
+}
+
+// Two e4m3 codes (lo in the low byte) -> two bf16 values, exactly (every e4m3 value is a bf16
+// value): e4m3 -> f16 by the hardware conversion, then f16 -> f32 -> bf16 (no rounding occurs).
+__device__ __forceinline__ uint32_t bf16x2_from_e4m3x2(uint16_t codes) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(codes));
+    float lo, hi;
+    asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"(uint16_t(h & 0xFFFFu)));
+    asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"(uint16_t(h >> 16)));
+    return pack_bf16x2(lo, hi);
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {

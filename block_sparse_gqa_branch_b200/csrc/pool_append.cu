@@ -79,6 +79,79 @@ void launch_pool(const void* k_idx, int B, int G, int64_t n_tokens, float* poole
                                           nb_cap, tail_sum);
 }
 
+// ---------------------------------------------------------------- chunk pooling
+// Pooling for a chunk of n index-key rows at positions P .. P + n - 1 (k_idx [B, n, G, dI])
+// appended to a sequence whose first P positions are already pooled: tail_sum holds the plain
+// sum over the open block's cached positions Bk floor(P / Bk) .. P - 1. Two launches, in
+// stream order: every block the chunk completes (the first one adds the cached running sum),
+// then the new running sum of the trailing open block, which overwrites tail_sum only after
+// the first launch has read it.
+// grid (blocks, B), 256 threads; block j = j_first + blockIdx.x, positions max(Bk j, P) ..
+// min(Bk (j + 1), P + n) - 1.
+__global__ void __launch_bounds__(256) pool_chunk_kernel(const uint16_t* __restrict__ k_idx, int64_t n, int64_t P,
+                                                         int G, float* __restrict__ pooled, int64_t nb_cap,
+                                                         float* __restrict__ tail_sum, int64_t j_first,
+                                                         int trailing) {
+    extern __shared__ float red[];                      // [nparts][G*dI]
+    const int b = blockIdx.y;
+    const int64_t j = j_first + blockIdx.x;
+    const int ncol = G * kIndexDim;
+    const int nchunk = ncol / 8;
+    const int nparts = nchunk >= 256 ? 1 : 256 / nchunk;
+    const int64_t p0 = j * kBlock > P ? j * kBlock : P;
+    const int64_t p1 = (j + 1) * kBlock < P + n ? (j + 1) * kBlock : P + n;
+    const int ntok = int(p1 - p0);                      // >= 0
+    const uint4* base = reinterpret_cast<const uint4*>(k_idx + (size_t(b) * n + (p0 - P)) * ncol);
+    for (int c0 = 0; c0 < nchunk; c0 += 256 / nparts) {
+        const int chunk = c0 + (threadIdx.x % (256 / nparts));
+        const int part = threadIdx.x / (256 / nparts);
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (chunk < nchunk && part < nparts) {
+#pragma unroll 4
+            for (int t = part; t < ntok; t += nparts) {
+                uint4 v = __ldg(base + size_t(t) * nchunk + chunk);
+                acc[0] += bf16_lo(v.x); acc[1] += bf16_hi(v.x);
+                acc[2] += bf16_lo(v.y); acc[3] += bf16_hi(v.y);
+                acc[4] += bf16_lo(v.z); acc[5] += bf16_hi(v.z);
+                acc[6] += bf16_lo(v.w); acc[7] += bf16_hi(v.w);
+            }
+            float* r = red + (size_t(part) * nchunk + chunk) * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) r[e] = acc[e];
+        }
+    }
+    __syncthreads();
+    // the block's positions before P are the cached running sum (only the block holding P)
+    const bool with_cached = P % kBlock != 0 && j == P / kBlock;
+    for (int col = threadIdx.x; col < ncol; col += 256) {
+        float s = 0.f;
+        for (int q = 0; q < nparts; ++q) s += red[size_t(q) * ncol + col];
+        const int g = col / kIndexDim, i = col % kIndexDim;
+        float* ts = tail_sum + (size_t(b) * G + g) * kIndexDim + i;
+        if (with_cached) s = *ts + s;
+        if (trailing) *ts = s;
+        else pooled[((size_t(b) * G + g) * nb_cap + j) * kIndexDim + i] = s * (1.0f / kBlock);
+    }
+}
+
+void launch_pool_chunk(const void* k_idx, int B, int G, int64_t n, int64_t P, float* pooled, int64_t nb_cap,
+                       float* tail_sum, cudaStream_t st) {
+    const int nchunk = G * kIndexDim / 8;
+    const int nparts = nchunk >= 256 ? 1 : 256 / nchunk;
+    const size_t smem = size_t(nparts) * G * kIndexDim * sizeof(float);
+    if (smem > 48 * 1024)
+        cudaFuncSetAttribute(pool_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    const int64_t j0 = P / kBlock, jt = (P + n) / kBlock;      // blocks j0 .. jt - 1 complete in the chunk
+    if (jt > j0) {
+        count_launch();
+        pool_chunk_kernel<<<dim3(unsigned(jt - j0), unsigned(B)), 256, smem, st>>>(
+            static_cast<const uint16_t*>(k_idx), n, P, G, pooled, nb_cap, tail_sum, j0, 0);
+    }
+    count_launch();                                              // the trailing open block (maybe empty)
+    pool_chunk_kernel<<<dim3(1u, unsigned(B)), 256, smem, st>>>(static_cast<const uint16_t*>(k_idx), n, P, G, pooled,
+                                                              nb_cap, tail_sum, jt, 1);
+}
+
 // ---------------------------------------------------------------- decode append
 // grid B, block 256. Writes the new token's K/V rows into the caches at position L_b and
 // folds its index keys into the open block's running sum; closes the block into `pooled`

@@ -64,30 +64,34 @@ __device__ __forceinline__ uint32_t split3_pack(float x0, float x1, int part) {
     return pack_bf16x2(r0 - m0, r1 - m1);
 }
 
+// Queries are the N tokens at positions P .. P + N - 1 (P = 0 for a whole prefill, P > 0 for a
+// chunk against cached blocks); query row i of q_idx and sel is position P + i. One CTA per
+// 128-token query block c that holds any of them.
 __global__ void __launch_bounds__(128, 2) select_prefill_mma_kernel(const uint16_t* __restrict__ q_idx, int64_t N,
-                                                                 int G, const float* __restrict__ pooled,
+                                                                 int64_t P, int G, const float* __restrict__ pooled,
                                                                  int64_t nb_cap, int32_t* __restrict__ sel) {
     __shared__ __align__(16) uint16_t kst[3][kSelPass][kKRow];
     __shared__ float scs[128][kSRow];
-    const int c = int(gridDim.x) - 1 - int(blockIdx.x), g = blockIdx.y, b = blockIdx.z;
+    const int c = int(P / kBlock) + int(gridDim.x) - 1 - int(blockIdx.x), g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gq = lane >> 2, tq = lane & 3;
-    const int64_t t = int64_t(c) * kBlock + tid;
-    const bool live = t < N;
-    int32_t* out = sel + ((size_t(b) * N + t) * G + g) * kTopK;
+    const int64_t t = int64_t(c) * kBlock + tid;       // position
+    const bool live = t >= P && t < P + N;
+    int32_t* out = sel + ((size_t(b) * N + (live ? t - P : 0)) * G + g) * kTopK;
     if (c + 1 <= kTopK) {
         if (live) write_all_blocks(out, c);
         return;
     }
-    // A fragments of this warp's 32 query rows (m-tile m: rows 16 m + gq and + 8)
+    // A fragments of this warp's 32 query rows (m-tile m: rows 16 m + gq and + 8); rows outside
+    // the queries read a valid query row and are never written
     uint32_t qa[2][4][4];
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
         int64_t ra = int64_t(c) * kBlock + warp * 32 + m * 16 + gq, rb = ra + 8;
-        ra = ra < N ? ra : N - 1;
-        rb = rb < N ? rb : N - 1;
-        const uint16_t* pa = q_idx + ((size_t(b) * N + ra) * G + g) * kIndexDim;
-        const uint16_t* pb = q_idx + ((size_t(b) * N + rb) * G + g) * kIndexDim;
+        ra = ra < P ? P : (ra < P + N ? ra : P + N - 1);
+        rb = rb < P ? P : (rb < P + N ? rb : P + N - 1);
+        const uint16_t* pa = q_idx + ((size_t(b) * N + (ra - P)) * G + g) * kIndexDim;
+        const uint16_t* pb = q_idx + ((size_t(b) * N + (rb - P)) * G + g) * kIndexDim;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
             qa[m][ks][0] = __ldg(reinterpret_cast<const uint32_t*>(pa + ks * 16 + 2 * tq));
@@ -186,11 +190,12 @@ __global__ void __launch_bounds__(128, 2) select_prefill_mma_kernel(const uint16
     for (int q4 = 0; q4 < 4; ++q4) o[q4] = make_int4(ids[4 * q4], ids[4 * q4 + 1], ids[4 * q4 + 2], ids[4 * q4 + 3]);
 }
 
-void launch_select_prefill_mma(const void* q_idx, int B, int G, int64_t N, const float* pooled,
+void launch_select_prefill_mma(const void* q_idx, int B, int G, int64_t N, int64_t P, const float* pooled,
                                int64_t nb_cap, int32_t* sel, cudaStream_t st) {
-    dim3 grid(static_cast<unsigned>((N + kBlock - 1) / kBlock), static_cast<unsigned>(G), static_cast<unsigned>(B));
+    const int64_t nqb = (P + N - 1) / kBlock - P / kBlock + 1;    // query blocks holding positions P .. P + N - 1
+    dim3 grid(static_cast<unsigned>(nqb), static_cast<unsigned>(G), static_cast<unsigned>(B));
     count_launch();
-    select_prefill_mma_kernel<<<grid, 128, 0, st>>>(static_cast<const uint16_t*>(q_idx), N, G, pooled, nb_cap, sel);
+    select_prefill_mma_kernel<<<grid, 128, 0, st>>>(static_cast<const uint16_t*>(q_idx), N, P, G, pooled, nb_cap, sel);
 }
 
 

@@ -9,8 +9,10 @@ from __future__ import annotations
 import torch
 
 from . import (BLOCK, INDEX_DIM, TOPK, OP_ATTN_DECODE, OP_ATTN_PREFILL, OP_INDEX_SELECT_DECODE,
-               OP_INDEX_SELECT_PREFILL, Shape, msa_index_select, msa_pool_index_keys,
-               msa_pooled_keys_append, msa_sparse_attn_decode, msa_sparse_attn_prefill,
+               OP_INDEX_SELECT_PREFILL, Shape, msa_fp8_close_blocks, msa_fp8_quantize_blocks,
+               msa_index_select, msa_index_select_chunk, msa_pool_index_keys, msa_pool_index_keys_chunk,
+               msa_pooled_keys_append, msa_prefill_chunk_workspace_size, msa_sparse_attn_decode,
+               msa_sparse_attn_decode_fp8, msa_sparse_attn_prefill, msa_sparse_attn_prefill_chunk,
                msa_workspace_size)
 
 
@@ -86,3 +88,66 @@ def decode_step(q, q_idx, k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, ta
     msa_sparse_attn_decode(s, q, k_cache, v_cache, l_cap, ctx_len, mp, bufs["sel"], bufs["out"], bufs["lse"],
                            bufs["ws_attn"], stream)
     return bufs["out"], bufs["lse"], bufs["sel"]
+
+
+def fp8_cache(k_cache, v_cache, n_blocks_cap: int):
+    """Empty FP8 cache matching bf16 caches [B, G, l_cap, 128]: codes (uint8, same layout) and
+    per-block scales [B, G, n_blocks_cap] (fp32)."""
+    B, G, l_cap, d = k_cache.shape
+    dev = k_cache.device
+    return {"k_codes": torch.zeros(B, G, l_cap, d, dtype=torch.uint8, device=dev),
+            "v_codes": torch.zeros(B, G, l_cap, d, dtype=torch.uint8, device=dev),
+            "k_scale": torch.ones(B, G, n_blocks_cap, dtype=torch.float32, device=dev),
+            "v_scale": torch.ones(B, G, n_blocks_cap, dtype=torch.float32, device=dev),
+            "nb_cap": n_blocks_cap}
+
+
+def fp8_quantize_sequence(k_cache, v_cache, f8: dict, b: int, n_tokens: int, n_q_heads: int, stream=None):
+    """Quantise the closed blocks of sequence b's first n_tokens positions (all groups)."""
+    G, l_cap = k_cache.shape[1], k_cache.shape[2]
+    msa_fp8_quantize_blocks(Shape.make(1, n_q_heads, G), k_cache[b], v_cache[b], l_cap, n_tokens,
+                            f8["k_codes"][b], f8["v_codes"][b], f8["k_scale"][b], f8["v_scale"][b], f8["nb_cap"],
+                            stream)
+
+
+def decode_step_fp8(q, q_idx, k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, tail_sum, pooled, f8: dict,
+                    bufs: dict, stream=None):
+    """One decode step over the FP8 cache: append the new token (bf16 cache + pooled keys),
+    quantise the blocks it closes, select, attend (closed blocks from the e4m3 codes, the own
+    block from bf16). Returns (out, lse, sel)."""
+    s, mp = bufs["shape"], bufs["max_pos"]
+    l_cap = k_cache.shape[2]
+    nb_cap = pooled.shape[2]
+    msa_pooled_keys_append(s, k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, l_cap, tail_sum, pooled,
+                           nb_cap, bufs["ws_append"], stream)
+    msa_fp8_close_blocks(s, ctx_len, k_cache, v_cache, l_cap, f8["k_codes"], f8["v_codes"], f8["k_scale"],
+                         f8["v_scale"], f8["nb_cap"], bufs["ws_append"], stream)
+    msa_index_select(s, q_idx, 1, ctx_len, mp, pooled, nb_cap, bufs["sel"], bufs["ws_select"], stream)
+    msa_sparse_attn_decode_fp8(s, q, f8["k_codes"], f8["v_codes"], f8["k_scale"], f8["v_scale"], f8["nb_cap"],
+                               k_cache, v_cache, l_cap, ctx_len, mp, bufs["sel"], bufs["out"], bufs["lse"],
+                               bufs["ws_attn"], stream)
+    return bufs["out"], bufs["lse"], bufs["sel"]
+
+
+def prefill_chunk(q, q_idx, k_idx, k_cache, v_cache, q_start: int, pooled, tail_sum, n_q_heads: int, stream=None,
+                  with_lse: bool = True):
+    """One chunk of a chunked prefill: the n tokens at positions q_start .. q_start + n - 1.
+    q [B,n,Hq,128], q_idx/k_idx [B,n,G,64]; k_cache/v_cache [B,G,l_cap,128] must already hold the
+    chunk's K and V rows; pooled [B,G,nb_cap,64] and tail_sum [B,G,64] hold the pooled state of
+    positions 0 .. q_start - 1 and are advanced past the chunk. A convenience for tests and
+    examples: it allocates the chunk's outputs and workspaces on every call (a serving loop
+    would size them once). Returns (out, lse, sel, workspaces)."""
+    B, n, G = q_idx.shape[0], q_idx.shape[1], q_idx.shape[2]
+    dev = q.device
+    shape = Shape.make(B, n_q_heads, G)
+    nb_cap = pooled.shape[2]
+    l_cap = k_cache.shape[2]
+    sel = torch.empty(B, n, G, TOPK, dtype=torch.int32, device=dev)
+    out = torch.empty(B, n, n_q_heads, 128, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, n, n_q_heads, dtype=torch.float32, device=dev) if with_lse else None
+    ws_sel = torch.zeros(256, dtype=torch.uint8, device=dev)
+    ws = torch.zeros(msa_prefill_chunk_workspace_size(shape, q_start, n), dtype=torch.uint8, device=dev)
+    msa_pool_index_keys_chunk(shape, k_idx, q_start, n, pooled, nb_cap, tail_sum, stream)
+    msa_index_select_chunk(shape, q_idx, q_start, n, pooled, nb_cap, sel, ws_sel, stream)
+    msa_sparse_attn_prefill_chunk(shape, q, k_cache, v_cache, l_cap, q_start, n, sel, out, lse, ws, stream)
+    return out, lse, sel, {"ws_select": ws_sel, "ws_attn": ws}

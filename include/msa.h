@@ -185,6 +185,47 @@ msa_status_t msa_sparse_attn_prefill(const msa_shape_t *shape, const void *q, co
                                      size_t workspace_bytes, msa_stream_t stream);
 
 /*
+ * Chunked prefill: a chunk of n new tokens at positions P .. P + n - 1 (P = q_start) of every
+ * sequence, against caches that already hold positions 0 .. P - 1. Source: youmind article
+ * "MiniMax M3 sparse attention agents", bullet "Predictable cost at every length" (every query
+ * reads the same fixed budget of 16 blocks = 2,048 key-value tokens, whatever the length); the
+ * chunk is this library's reading of the step between a prefill and decode. Every query of the
+ * chunk selects among all fully-past blocks -- cached ones and those the chunk itself completes
+ * -- exactly as in a whole prefill, so the chunked results equal rows P .. P + n - 1 of a
+ * prefill of the whole sequence (up to the order of the fp32 sums in the pooled keys).
+ * Order of a chunk: msa_pool_index_keys_chunk, msa_index_select_chunk, then (once the chunk's
+ * K and V rows are in the caches) msa_sparse_attn_prefill_chunk.
+ */
+
+/* Pool the chunk's index keys k_idx [B, n, G, d_I] (positions P .. P + n - 1) into pooled
+ * [B, G, nb_cap, d_I] for every block the chunk completes, and keep tail_sum [B, G, d_I] -- the
+ * plain sum of the open block's positions, which must hold positions Bk floor(P / Bk) .. P - 1
+ * on entry (zeros when P is a multiple of Bk) -- current. pooled may be NULL when no block
+ * completes. (P + n) / Bk <= nb_cap. */
+msa_status_t msa_pool_index_keys_chunk(const msa_shape_t *shape, const void *k_idx, int64_t q_start, int64_t n,
+                                       float *pooled, int64_t nb_cap, float *tail_sum, msa_stream_t stream);
+
+/* Block scores and exp-free top-k selection for the chunk's index queries q_idx [B, n, G, d_I]
+ * (row i at position P + i); sel [B, n, G, k] as msa_index_select. pooled must hold every full
+ * block below P + n (after msa_pool_index_keys_chunk). Workspace: >= 256 bytes. */
+msa_status_t msa_index_select_chunk(const msa_shape_t *shape, const void *q_idx, int64_t q_start, int64_t n,
+                                    const float *pooled, int64_t nb_cap, int32_t *sel, void *workspace,
+                                    size_t workspace_bytes, msa_stream_t stream);
+
+/* Main Branch for the chunk: q [B, n, Hq, d] (row i at position P + i), k_cache, v_cache
+ * [B, G, l_cap, d] holding positions 0 .. P + n - 1 (P + n <= l_cap), sel from
+ * msa_index_select_chunk; out [B, n, Hq, d], lse [B, n, Hq] or NULL. Workspace of
+ * msa_prefill_chunk_workspace_size(shape, P, n) bytes. Size limits as msa_sparse_attn_prefill
+ * with N = n, plus B*G*l_cap + Bk < 2^31 and (P + n) / Bk <= 49152. */
+msa_status_t msa_sparse_attn_prefill_chunk(const msa_shape_t *shape, const void *q, const void *k_cache,
+                                           const void *v_cache, int64_t l_cap, int64_t q_start, int64_t n,
+                                           const int32_t *sel, void *out, float *lse, void *workspace,
+                                           size_t workspace_bytes, msa_stream_t stream);
+
+/* Workspace bytes of msa_sparse_attn_prefill_chunk (0 for an invalid shape, P < 0 or n < 1). */
+size_t msa_prefill_chunk_workspace_size(const msa_shape_t *shape, int64_t q_start, int64_t n_queries);
+
+/*
  * Decode: append the new token to the caches and keep the pooled keys current (the pages
  * fix only the block size; the incremental update is this library's reading of it).
  *   ctx_len   device int32 [B]: tokens already cached (L_b); the new token goes to position L_b
@@ -217,6 +258,52 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t *shape, const void *q, con
                                     int64_t max_pos, const int32_t *sel, void *out, float *lse,
                                     void *workspace, size_t workspace_bytes,
                                     msa_stream_t stream);
+
+/*
+ * FP8 (e4m3) key-value cache of the decode step. Source: KuCoin flash "MiniMax launches MSA
+ * sparse attention method and MiniMax-M3 model", "ME AI News" paragraph (the SM100 attention
+ * kernel also takes FP8 inputs); the pages give no format, so this library's reading is:
+ *  - every CLOSED 128-token block of a group's keys, and of its values, is stored as e4m3
+ *    codes ("E4M3FN": 4 exponent bits, bias 7, 3 mantissa bits, largest finite 448) with one
+ *    fp32 scale per (sequence, group, block): scale = amax / 448 (1 for an all-zero block),
+ *    code = e4m3(x / scale), the division in fp32, nearest with ties to the even mantissa,
+ *    saturating at +-448; a stored value is code x scale;
+ *  - the open block -- always the newest query's own block -- stays in the bf16 cache until it
+ *    fills (a per-block scale would otherwise change with every append).
+ *   k_codes, v_codes  uint8 [B, G, l_cap, d]   the bf16 cache's layout with one byte per value
+ *   k_scale, v_scale  fp32 [B, G, nb_cap]      one scale per block
+ * These entry points validate and launch like the others; codes and scales of blocks that are
+ * not (yet) closed are not read.
+ */
+
+/* Quantise blocks j < n_tokens / Bk of every sequence and group from the bf16 caches
+ * k_cache, v_cache [B, G, l_cap, d] (after a prefill of n_tokens tokens; n_tokens <= l_cap,
+ * n_tokens / Bk <= nb_cap). */
+msa_status_t msa_fp8_quantize_blocks(const msa_shape_t *shape, const void *k_cache, const void *v_cache,
+                                     int64_t l_cap, int64_t n_tokens, void *k_codes, void *v_codes,
+                                     float *k_scale, float *v_scale, int64_t nb_cap, msa_stream_t stream);
+
+/* Decode step, after msa_pooled_keys_append: for every sequence whose new token (at position
+ * ctx_len[b], device int32 [B]) completes block j = ctx_len[b] / Bk, quantise that block from
+ * the bf16 caches. A position outside [0, l_cap) or a block j >= nb_cap is a device bounds
+ * error recorded in `workspace` (>= 256 bytes, zeroed before first use). */
+msa_status_t msa_fp8_close_blocks(const msa_shape_t *shape, const int32_t *ctx_len, const void *k_cache,
+                                  const void *v_cache, int64_t l_cap, void *k_codes, void *v_codes,
+                                  float *k_scale, float *v_scale, int64_t nb_cap, void *workspace,
+                                  size_t workspace_bytes, msa_stream_t stream);
+
+/* Main Branch, decode, over the FP8 cache: as msa_sparse_attn_decode, but every selected
+ * block below the query's own one is read as e4m3 codes and scales (half the bytes of bf16);
+ * the query's own block is read from the bf16 caches k_cache, v_cache. Scores are
+ * scale_k * (q . code) and the values code x scale_v, accumulated in fp32.
+ *   nb_cap  blocks per (sequence, group) in k_scale / v_scale; must be >= max_pos / Bk
+ *   workspace of msa_workspace_size(MSA_OP_ATTN_DECODE, max_pos) */
+msa_status_t msa_sparse_attn_decode_fp8(const msa_shape_t *shape, const void *q, const void *k_codes,
+                                        const void *v_codes, const float *k_scale, const float *v_scale,
+                                        int64_t nb_cap, const void *k_cache, const void *v_cache,
+                                        int64_t l_cap, const int32_t *q_pos, int64_t max_pos,
+                                        const int32_t *sel, void *out, float *lse, void *workspace,
+                                        size_t workspace_bytes, msa_stream_t stream);
 
 /*
  * Synchronises `stream`, returns the status recorded in the workspace's error word by the

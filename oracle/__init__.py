@@ -283,6 +283,33 @@ def prefill(x: dict, Hq: int, G: int, Bk: int = 128, topk: int = 16, sel: Option
     return res
 
 
+def prefill_chunk(q: np.ndarray, q_idx: np.ndarray, k_idx: np.ndarray, K: np.ndarray, V: np.ndarray, P: int,
+                  Hq: int, G: int, Bk: int = 128, topk: int = 16, sel: Optional[np.ndarray] = None,
+                  nthreads: Optional[int] = None):
+    """A chunk of a chunked prefill for one sequence: the n queries at positions P .. P + n - 1
+    against everything up to P + n - 1 (youmind article "MiniMax M3 sparse attention agents",
+    bullet "Predictable cost at every length": the same 16-block budget at every length).
+    Steps 1-4 exactly as in a whole prefill, at those positions: pooled keys of every full block
+    below P + n, selection among the fully-past blocks, attention over the selected keys u <= t.
+    q [n, Hq, d], q_idx [n, G, dI] (the chunk's rows); k_idx [>= P + n, G, dI], K, V [G, >= P + n, d]
+    (the sequence so far, the chunk included). If ``sel`` [n, G, topk] is given, attention runs on
+    it. Returns dict(sel [n,G,topk], kth [n,G], pooled [G,nb,dI], out [n,Hq,d], lse [n,Hq])."""
+    n = q.shape[0]
+    Hg = Hq // G
+    t = np.arange(P, P + n, dtype=np.int64)
+    pooled, _ = pool(k_idx[:P + n], Bk)
+    res = {"sel": np.zeros((n, G, topk), np.int32), "kth": np.zeros((n, G), np.float64), "pooled": pooled,
+           "out": np.zeros((n, Hq, q.shape[-1]), np.float64), "lse": np.zeros((n, Hq), np.float64)}
+    for g in range(G):
+        s_, kth, _ = select_rows(t, q_idx[:, g, :], pooled[g], Bk, topk, nthreads)
+        res["sel"][:, g], res["kth"][:, g] = s_, kth
+        use = s_ if sel is None else sel[:, g]
+        o, lse, _ = attend_rows(t, q[:, g * Hg:(g + 1) * Hg, :], K[g], V[g], use, Bk, topk, False, nthreads)
+        res["out"][:, g * Hg:(g + 1) * Hg] = o
+        res["lse"][:, g * Hg:(g + 1) * Hg] = lse
+    return res
+
+
 def dense_gqa(x: dict, Hq: int, G: int, nthreads: Optional[int] = None):
     """Dense causal GQA attention (every key u <= t) with the same layouts; the comparator
     the pages measure MSA against. Returns (out [B,N,Hq,d], lse [B,N,Hq])."""

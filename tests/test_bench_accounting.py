@@ -87,3 +87,12 @@ def test_recorded_captures_are_close_to_their_models():
         assert 1.0 <= c["decode_step"]["bytes"] / c["decode_step"]["algorithmic_bytes"] < 1.05
     if "prefill_main" in c:
         assert 0.9 <= c["prefill_main"]["bytes"] / c["prefill_main"]["model_bytes"] < 1.2
+
+
+def test_fp8_decode_step_bytes_closed_form():
+    w = bench.DECODE
+    d8, d = bench.decode_step_bytes_fp8(w), bench.decode_step_bytes(w)
+    per_bg_kv = 15 * (128 * 128 * 1 * 2 + 2 * 4) + 1 * 128 * 2 * 2   # e4m3 K and V + scales, own block bf16
+    assert d8["kv"] == 128 * per_bg_kv
+    assert d8["pooled"] == d["pooled"] and d8["small"] == d["small"]
+    assert d8["total"] == 97311744

@@ -146,3 +146,47 @@ def test_no_alloc_select_rejects_problems_beyond_its_scratch(L):
     # invalid arguments come first
     assert L.msa_index_select_decode_noalloc(shape, None, FAKE2, 100, FAKE, 1, FAKE, None) == 1
     assert L.msa_index_select_decode_noalloc(shape, FAKE, FAKE2, 1 << 25, FAKE, 1 << 18, FAKE, None) == 2
+
+
+def test_fp8_entry_points_validate_before_launch(L):
+    s = ctypes.byref(_shape())
+    # quantise: n_tokens beyond the cache, nb_cap too small, misaligned codes; zero blocks = nothing to do
+    assert L.msa_fp8_quantize_blocks(s, FAKE, FAKE, 100, 200, FAKE, FAKE, FAKE, FAKE, 4, None) == 1
+    assert L.msa_fp8_quantize_blocks(s, FAKE, FAKE, 1024, 1024, FAKE, FAKE, FAKE, FAKE, 7, None) == 1
+    assert L.msa_fp8_quantize_blocks(s, FAKE, FAKE, 1024, 1024, FAKE + 8, FAKE, FAKE, FAKE, 8, None) == 1
+    assert L.msa_fp8_quantize_blocks(s, FAKE, FAKE, 1024, 100, FAKE, FAKE, FAKE, FAKE, 8, None) == 0
+    assert L.msa_fp8_quantize_blocks(ctypes.byref(_shape(head_dim=64)), FAKE, FAKE, 1024, 1024, FAKE, FAKE, FAKE,
+                                     FAKE, 8, None) == 2
+    # close: missing workspace, misaligned scale
+    assert L.msa_fp8_close_blocks(s, FAKE, FAKE, FAKE, 1024, FAKE, FAKE, FAKE, FAKE, 8, None, 0, None) == 3
+    assert L.msa_fp8_close_blocks(s, FAKE, FAKE, FAKE, 1024, FAKE, FAKE, FAKE + 2, FAKE, 8, FAKE, 256, None) == 1
+    # decode attention: nb_cap below max_pos / 128, position beyond the cache, workspace
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 8, FAKE, FAKE, 1024, FAKE, 1000, FAKE, FAKE, None, FAKE, 1 << 20, None]
+    assert L.msa_sparse_attn_decode_fp8(s, *args[:5], 6, *args[6:]) == 1
+    assert L.msa_sparse_attn_decode_fp8(s, *args[:10], 1024, *args[11:]) == 1
+    assert L.msa_sparse_attn_decode_fp8(s, *args[:15], 64, None) == 3
+    assert L.msa_sparse_attn_decode_fp8(s, None, *args[1:]) == 1
+
+
+def test_chunk_entry_points_validate_before_launch(L):
+    s = ctypes.byref(_shape(n_q_heads=16, n_kv_groups=2))
+    big = msa.msa_prefill_chunk_workspace_size(Shape.make(1, 16, 2), 1000, 500)
+    assert big > msa.msa_prefill_chunk_workspace_size(Shape.make(1, 16, 2), 0, 500) > 256
+    assert msa.msa_prefill_chunk_workspace_size(Shape.make(1, 16, 2), -1, 500) == 0
+    assert msa.msa_prefill_chunk_workspace_size(Shape.make(1, 16, 2), 0, 0) == 0
+    # a whole prefill is the chunk at P = 0 against a cache of exactly n rows
+    assert msa.msa_prefill_chunk_workspace_size(Shape.make(1, 16, 2), 0, 777) == \
+        msa.msa_workspace_size(Shape.make(1, 16, 2), msa.OP_ATTN_PREFILL, 777)
+    # pooling: no tail buffer, nb_cap too small, completed blocks without pooled
+    assert L.msa_pool_index_keys_chunk(s, FAKE, 100, 50, FAKE, 4, None, None) == 1
+    assert L.msa_pool_index_keys_chunk(s, FAKE, 100, 600, FAKE, 4, FAKE, None) == 1
+    assert L.msa_pool_index_keys_chunk(s, FAKE, 100, 200, None, 4, FAKE, None) == 1
+    assert L.msa_pool_index_keys_chunk(s, FAKE, 100, 0, FAKE, 4, FAKE, None) == 1
+    # selection: workspace, nb_cap
+    assert L.msa_index_select_chunk(s, FAKE, 1000, 500, FAKE, 11, FAKE2, None, 0, None) == 3
+    assert L.msa_index_select_chunk(s, FAKE, 1000, 500, FAKE, 10, FAKE2, FAKE, 256, None) == 1
+    # attention: the chunk must fit in the cache; the workspace depends on P
+    assert L.msa_sparse_attn_prefill_chunk(s, FAKE, FAKE, FAKE, 1400, 1000, 500, FAKE, FAKE, None, FAKE, big,
+                                           None) == 1
+    assert L.msa_sparse_attn_prefill_chunk(s, FAKE, FAKE, FAKE, 1500, 1000, 500, FAKE, FAKE, None, FAKE, big - 16,
+                                           None) == 3

@@ -457,3 +457,34 @@ def test_attention_grad_identities():
     assert not g0Q.any() and not g0K.any()
     np.testing.assert_array_equal(g0V[0], dO[0].sum(axis=0))
     assert not g0V[1:].any()
+
+
+# ----------------------------------------------------------------------------- chunked prefill
+@pytest.mark.parametrize("P,n", [(0, 300), (1000, 700), (1700, 1), (128 * 20, 128 * 3 + 5)])
+def test_chunk_rows_equal_whole_prefill_rows(P, n):
+    # a chunk at positions P .. P + n - 1 against the sequence so far is rows P .. P + n - 1 of a
+    # prefill of the whole sequence (the definition is per query position)
+    w, x = make(N=P + n, Hq=4, G=2, seed=P + n)
+    full = oracle.prefill(x, w.Hq, w.G)
+    r = oracle.prefill_chunk(x["q"][0, P:], x["q_idx"][0, P:], x["k_idx"][0], x["k"][0], x["v"][0], P, w.Hq, w.G)
+    assert (r["sel"] == full["sel"][0, P:]).all()
+    np.testing.assert_array_equal(r["kth"], full["kth"][0, P:])
+    np.testing.assert_array_equal(r["out"], full["out"][0, P:])
+    np.testing.assert_array_equal(r["lse"], full["lse"][0, P:])
+
+
+def test_chunk_reduces_to_dense_causal_attention_when_every_block_fits():
+    # P + n <= 2048: every query takes every block, so a chunk is dense causal GQA attention over
+    # positions 0 .. t (torch fp64 SDPA with an explicit mask on the chunk's rows)
+    P, n = 900, 400
+    w, x = make(N=P + n, Hq=4, G=2, seed=5)
+    r = oracle.prefill_chunk(x["q"][0, P:], x["q_idx"][0, P:], x["k_idx"][0], x["k"][0], x["v"][0], P, w.Hq, w.G)
+    q = torch.from_numpy(f32(x["q"][0, P:]))                   # [n, Hq, d]
+    Hg = w.Hq // w.G
+    t = torch.arange(P, P + n)[:, None]
+    mask = torch.arange(P + n)[None, :] <= t                 # [n, P + n]
+    for h in range(w.Hq):
+        kf = torch.from_numpy(f32(x["k"][0, h // Hg]))
+        vf = torch.from_numpy(f32(x["v"][0, h // Hg]))
+        ref = _sdpa_masked(q[:, h][None], kf, vf, mask)[0]
+        np.testing.assert_allclose(r["out"][:, h], ref.numpy(), rtol=0, atol=1e-12)
