@@ -86,11 +86,12 @@ struct DecArgs {
     int64_t nb_cap;
 };
 
-// FP8 variant: widen this warp's 16 rows (kbase..kbase+15) of an e4m3 block, which TMA left as
-// [128 rows][128 B] (128B swizzle) at the start of `buf`, in place into the bf16 tile layout of
-// the full blocks ([d half][128 rows][128 B], 128B swizzle). The source bytes of a row lie
-// inside the row's half-0 destination, which only this warp writes, so every lane reads its
-// codes before any lane writes.
+// FP8 variant: widen this warp's 16 rows (kbase..kbase+15) of an e4m3 value block, which TMA
+// left as [128 rows][128 B] (128B swizzle) at the start of `buf`, in place into f16 in the
+// 16-bit tile layout of the full blocks ([d half][128 rows][128 B], 128B swizzle), so that the
+// P V step reads it like a bf16 block. The source bytes of a row lie inside the row's half-0
+// destination, which only this warp writes, so every lane reads its codes before any lane
+// writes.
 __device__ __forceinline__ void widen_fp8_rows(uint8_t* buf, int kbase, int lane) {
     const int row = kbase + (lane >> 1), h = lane & 1;      // lane pair per row, one d half each
     uint4 c[4];
@@ -106,8 +107,8 @@ __device__ __forceinline__ void widen_fp8_rows(uint8_t* buf, int kbase, int lane
         uint32_t o[8];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            o[2 * e] = bf16x2_from_e4m3x2(uint16_t(w[e] & 0xFFFFu));
-            o[2 * e + 1] = bf16x2_from_e4m3x2(uint16_t(w[e] >> 16));
+            o[2 * e] = f16x2_from_e4m3x2(uint16_t(w[e] & 0xFFFFu));
+            o[2 * e + 1] = f16x2_from_e4m3x2(uint16_t(w[e] >> 16));
         }
         // codes d = 64 h + 16 i .. +15 -> chunks (2 i) and (2 i + 1) of d half h
         *reinterpret_cast<uint4*>(buf + h * 16384 + sw128(row, 2 * i)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -574,8 +575,30 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
         const bool active = kbase < ntok;
         const bool f8 = kFp8 && sm.meta_fp8[stage] != 0;   // e4m3 codes: scores and P take the scales
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        if (f8) widen_fp8_rows(sm.kv[stage][0], kbase, lane);
-        if (active) {
+        if (f8) {
+            // FP8 block: f16 MMAs (every e4m3 code is exact in f16); the query rows go to f16 (exact
+            // in f16's normal range) and the key codes straight from the e4m3 tile
+            // ([128 rows][128 B], 128B swizzle) into B fragments
+            const uint8_t* K8 = sm.kv[stage][0];
+            const uint16_t* q0 = sm.q[stage][gq];
+            const uint16_t* q1 = sm.q[stage][gq + 8];
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const int d0 = ks * 16 + 2 * tq;
+                const uint32_t a0 = f16x2_from_bf16x2(*reinterpret_cast<const uint32_t*>(q0 + d0));
+                const uint32_t a1 = f16x2_from_bf16x2(*reinterpret_cast<const uint32_t*>(q1 + d0));
+                const uint32_t a2 = f16x2_from_bf16x2(*reinterpret_cast<const uint32_t*>(q0 + d0 + 8));
+                const uint32_t a3 = f16x2_from_bf16x2(*reinterpret_cast<const uint32_t*>(q1 + d0 + 8));
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int key = kbase + nt * 8 + gq;
+                    const uint8_t* kr = K8 + key * 128 + ((ks ^ (key & 7)) << 4) + 2 * tq;
+                    const uint32_t b0 = f16x2_from_e4m3x2(*reinterpret_cast<const uint16_t*>(kr));
+                    const uint32_t b1 = f16x2_from_e4m3x2(*reinterpret_cast<const uint16_t*>(kr + 8));
+                    mma_f16_16816(s[nt], a0, a1, a2, a3, b0, b1);
+                }
+            }
+        } else if (active) {
             const uint8_t* Ks = sm.kv[stage][0];
             const uint16_t* q0 = sm.q[stage][gq];       // query rows gq, gq + 8 (A fragments)
             const uint16_t* q1 = sm.q[stage][gq + 8];
@@ -650,18 +673,30 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
                 }
                 __syncwarp();
             }
-            // FP8: the values are code x scale, so P is weighted by the block's value scale
-            const float vsc = f8 ? sm.meta_vs[stage] : 1.f;
-            const uint32_t pa0 = pack_bf16x2(p[0][0] * vsc, p[0][1] * vsc), pa1 = pack_bf16x2(p[0][2] * vsc, p[0][3] * vsc);
-            const uint32_t pa2 = pack_bf16x2(p[1][0] * vsc, p[1][1] * vsc), pa3 = pack_bf16x2(p[1][2] * vsc, p[1][3] * vsc);
             const uint32_t vrow = smem_u32(Vs);
             const int row = kbase + (lane & 7) + ((lane >> 3) & 1) * 8;
+            if (f8) {
+                // the values are code x scale: P is weighted by the block's value scale, in f16
+                const float vsc = sm.meta_vs[stage];
+                const uint32_t pa0 = pack_f16x2(p[0][0] * vsc, p[0][1] * vsc), pa1 = pack_f16x2(p[0][2] * vsc, p[0][3] * vsc);
+                const uint32_t pa2 = pack_f16x2(p[1][0] * vsc, p[1][1] * vsc), pa3 = pack_f16x2(p[1][2] * vsc, p[1][3] * vsc);
 #pragma unroll
-            for (int dn = 0; dn < 8; ++dn) {
-                uint32_t v0, v1, v2, v3;
-                ldsm_x4_trans(vrow + kv_off(row, dn * 16 + (lane >> 4) * 8), v0, v1, v2, v3);
-                mma_bf16_16816(st.o[2 * dn], pa0, pa1, pa2, pa3, v0, v1);
-                mma_bf16_16816(st.o[2 * dn + 1], pa0, pa1, pa2, pa3, v2, v3);
+                for (int dn = 0; dn < 8; ++dn) {
+                    uint32_t v0, v1, v2, v3;
+                    ldsm_x4_trans(vrow + kv_off(row, dn * 16 + (lane >> 4) * 8), v0, v1, v2, v3);
+                    mma_f16_16816(st.o[2 * dn], pa0, pa1, pa2, pa3, v0, v1);
+                    mma_f16_16816(st.o[2 * dn + 1], pa0, pa1, pa2, pa3, v2, v3);
+                }
+            } else {
+                const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]), pa1 = pack_bf16x2(p[0][2], p[0][3]);
+                const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]), pa3 = pack_bf16x2(p[1][2], p[1][3]);
+#pragma unroll
+                for (int dn = 0; dn < 8; ++dn) {
+                    uint32_t v0, v1, v2, v3;
+                    ldsm_x4_trans(vrow + kv_off(row, dn * 16 + (lane >> 4) * 8), v0, v1, v2, v3);
+                    mma_bf16_16816(st.o[2 * dn], pa0, pa1, pa2, pa3, v0, v1);
+                    mma_bf16_16816(st.o[2 * dn + 1], pa0, pa1, pa2, pa3, v2, v3);
+                }
             }
         }
         if (!fin) {

@@ -15,6 +15,8 @@ void launch_pool(const void*, int, int, int64_t, float*, int64_t, float*, cudaSt
 void launch_append(const void*, const void*, const void*, const int32_t*, int, int, void*, void*, int64_t,
                    float*, float*, int64_t, void*, cudaStream_t);
 void launch_select_prefill_mma(const void*, int, int, int64_t, int64_t, const float*, int64_t, int32_t*, cudaStream_t);
+msa_status_t launch_select_prefill_tc(const void*, int, int, int64_t, int64_t, const float*, int64_t, int32_t*, void*,
+                                      cudaStream_t);
 void launch_pool_chunk(const void*, int, int, int64_t, int64_t, float*, int64_t, float*, cudaStream_t);
 void launch_select_decode(const void*, const int32_t*, int64_t, int, int, const float*, int64_t, int32_t*,
                           void*, cudaStream_t);
@@ -118,6 +120,22 @@ msa_status_t make_tmap_kv3d(CUtensorMap* m, const void* base, uint64_t rows_vali
     cuuint64_t dims[3] = {uint64_t(kHeadDim), rows_valid, nbg};
     cuuint64_t strides[2] = {uint64_t(kHeadDim) * 2, l_cap * kHeadDim * 2};
     cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error = int(r);
+        return MSA_ERR_CUDA;
+    }
+    return MSA_OK;
+}
+msa_status_t make_tmap_qidx(CUtensorMap* m, const void* base, int G, uint64_t rows) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return MSA_ERR_CUDA;
+    cuuint64_t dims[3] = {uint64_t(kIndexDim), uint64_t(G), rows};
+    cuuint64_t strides[2] = {uint64_t(kIndexDim) * 2, uint64_t(G) * kIndexDim * 2};
+    cuuint32_t box[3] = {64, 1, 128};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -234,7 +252,7 @@ msa_status_t msa_index_select(const msa_shape_t* shape, const void* q_idx, int64
         MSA_REQ(nb_cap >= (n_queries - 1) / kBlock, MSA_ERR_INVALID_ARGUMENT);
         const size_t need = ws_size(shape, MSA_OP_INDEX_SELECT_PREFILL, n_queries);
         MSA_REQ(workspace != nullptr && workspace_bytes >= need, MSA_ERR_WORKSPACE);
-        launch_select_prefill_mma(q_idx, B, G, n_queries, 0, pooled, nb_cap, sel, st);
+        MSA_TRY(launch_select_prefill_tc(q_idx, B, G, n_queries, 0, pooled, nb_cap, sel, workspace, st));
     } else {                                       // decode: one query per sequence at q_pos[b]
         MSA_REQ(n_queries == 1, MSA_ERR_INVALID_ARGUMENT);
         MSA_REQ(max_pos <= kMaxPos, MSA_ERR_UNSUPPORTED);
@@ -318,8 +336,8 @@ msa_status_t msa_index_select_chunk(const msa_shape_t* shape, const void* q_idx,
     MSA_REQ(nb_cap >= (q_start + n - 1) / kBlock, MSA_ERR_INVALID_ARGUMENT);
     MSA_REQ(pooled == nullptr ? q_start + n - 1 < kBlock : aligned16(pooled), MSA_ERR_INVALID_ARGUMENT);
     MSA_REQ(workspace != nullptr && workspace_bytes >= header_only(), MSA_ERR_WORKSPACE);
-    launch_select_prefill_mma(q_idx, shape->batch, shape->n_kv_groups, n, q_start, pooled, nb_cap, sel,
-                              reinterpret_cast<cudaStream_t>(stream));
+    MSA_TRY(launch_select_prefill_tc(q_idx, shape->batch, shape->n_kv_groups, n, q_start, pooled, nb_cap, sel,
+                                     workspace, reinterpret_cast<cudaStream_t>(stream)));
     return cuda_status();
 }
 

@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(256) fp8_quantize_kernel(const Fp8Args a) {
 // grid (1, 2 G, B): the block that the token at position ctx_len[b] completes, if it does
 __global__ void __launch_bounds__(256) fp8_close_kernel(const Fp8Args a, const int32_t* __restrict__ ctx_len,
                                                         WsHeader* hdr) {
+    grid_dep_launch();                     // the selection may start: it reads no code or scale
     grid_dep_wait();                       // the append that wrote the token has completed
     const int g = blockIdx.y >> 1, which = blockIdx.y & 1, b = blockIdx.z;
     const int pos = ctx_len[b];

@@ -30,6 +30,9 @@ msa_status_t make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint6
 // 256 B and (sequence, group) stride l_cap rows; box {64, 128, 1}, 128B swizzle; rows at or past
 // rows_valid are zero-filled by the copy.
 msa_status_t make_tmap_kv3d(CUtensorMap* m, const void* base, uint64_t rows_valid, uint64_t l_cap, uint64_t nbg);
+// Index queries q_idx [rows, G, 64] bf16 as a 3-D tensor {64, G, rows}; box {64, 1, 128}: 128
+// rows of one group, [128 rows][128 B] with the 128B swizzle
+msa_status_t make_tmap_qidx(CUtensorMap* m, const void* base, int G, uint64_t rows);
 // Rows of 128 bf16 viewed as (64 columns, row, d half): box {64, 8, 2} lands 8 rows with both
 // halves as [half][8 rows][128 B] (128B swizzle)
 msa_status_t make_tmap_q_rows(CUtensorMap* m, const void* base, uint64_t rows);
@@ -279,15 +282,31 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t saddr, uint32_t& r0, uint
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(saddr));
 }
 
-// Two e4m3 codes (lo in the low byte) -> two bf16 values, exactly (every e4m3 value is a bf16
-// value): e4m3 -> f16 by the hardware conversion, then f16 -> f32 -> bf16 (no rounding occurs).
-__device__ __forceinline__ uint32_t bf16x2_from_e4m3x2(uint16_t codes) {
+// Two e4m3 codes (lo in the low byte) -> two f16 values, exactly (every e4m3 value is a normal
+// f16 value or zero), by the hardware conversion.
+__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint16_t codes) {
     uint32_t h;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(codes));
-    float lo, hi;
-    asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"(uint16_t(h & 0xFFFFu)));
-    asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"(uint16_t(h >> 16)));
-    return pack_bf16x2(lo, hi);
+    return h;
+}
+// two floats -> packed f16x2 (round to nearest even), lo in the low half
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(hi), "f"(lo));
+    return h;
+}
+// packed bf16x2 -> packed f16x2 (exact for values in the normal f16 range)
+__device__ __forceinline__ uint32_t f16x2_from_bf16x2(uint32_t w) {
+    return pack_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+// warp MMA m16n8k16 with f16 operands and fp32 accumulators
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {

@@ -1,0 +1,250 @@
+// select_tc.cu -- Index Branch for prefill on the 5th-generation tensor cores: block scores as
+// one dense contraction per 128-query tile, and the exp-free top-15 per query.
+//
+// Sources: youmind article "MiniMax M3 sparse attention agents", paragraph "The mechanism that
+// changes this" (score the context in blocks, keep the most relevant per query and GQA group)
+// and bullet "Predictable cost at every length" (k = 16 blocks of 128 tokens); KuCoin flash
+// "MiniMax launches MSA sparse attention method and MiniMax-M3 model", summary (exp-free top-k).
+//
+// One CTA of 128 threads per (128-token query block c, group g, sequence b), heaviest blocks
+// first. The tile's index queries Q_I (128 x 64 bf16) arrive by TMA. The fully-past candidates
+// j < c go 64 per chunk: the threads stage the chunk's pooled keys (fp32), each split exactly
+// into three bf16 terms (hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid): 24
+// significant bits), as three K-major shared-memory operands; one thread issues the 12
+// tcgen05.mma (3 terms x 4 k-steps of 16) that accumulate S = Q_I x Kbar^T (128 x 64, fp32)
+// into tensor memory. Scores are fp32-accurate (a single bf16 term would move selections
+// beyond the near-tie rule). Two S buffers let chunk k + 1's MMAs run while chunk k is ranked;
+// 64-candidate chunks keep the CTA at 65 KB of shared memory, three CTAs per SM.
+// Thread i owns query row i (tensor-memory lane i): it reads its row's 64 scores with
+// tcgen05.ld, marks without branches the candidates that beat its current 15th best, and
+// inserts only those, in id order, into its running best 15 -- compares only, so equal scores
+// keep the lower block id. The 1/sqrt(d_I) factor is an exact power of two and cannot change
+// the order, so it is not applied.
+#include <atomic>
+
+#include "msa_common.cuh"
+
+namespace msa {
+
+constexpr int kTcRows = 128;       // queries per tile (MMA M)
+constexpr int kTcCand = 64;        // candidates per chunk (MMA N)
+constexpr int kTcKeep = kTopK - 1;
+
+struct __align__(1024) SelTcSmem {
+    uint8_t q[kTcRows * 128];               // Q_I tile [128 rows][64 bf16], 128B swizzle
+    uint8_t kb[2][3][kTcCand * 128];        // split pooled keys [buf][hi, mid, lo][64 cand][64 bf16], 128B swizzle
+    uint64_t q_full, mma_done[2];
+    uint32_t tmem_base;
+};
+
+__device__ __forceinline__ void split3(float x, float& h, float& m, float& l) {
+    h = __bfloat162float(__float2bfloat16_rn(x));
+    const float r = x - h;
+    m = __bfloat162float(__float2bfloat16_rn(r));
+    l = r - m;
+}
+
+__device__ __forceinline__ void sort16_ids(int (&x)[16]) {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+#pragma unroll
+        for (int i = (r & 1); i + 1 < 16; i += 2) {
+            const int a = min(x[i], x[i + 1]), bb = max(x[i], x[i + 1]);
+            x[i] = a; x[i + 1] = bb;
+        }
+    }
+}
+
+// Queries are the N tokens at positions P .. P + N - 1 (P = 0 for a whole prefill); query row i
+// of q_idx and sel is position P + i.
+__global__ void __launch_bounds__(128) select_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                                int64_t N, int64_t P, int G,
+                                                                const float* __restrict__ pooled, int64_t nb_cap,
+                                                                int32_t* __restrict__ sel, WsHeader* hdr) {
+    extern __shared__ uint8_t smem_raw[];
+    SelTcSmem& sm = *reinterpret_cast<SelTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int c = int((P + N - 1) / kBlock) - int(blockIdx.x), g = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t t = int64_t(c) * kBlock + tid;            // this thread's query position
+    const bool live = t >= P && t < P + N;
+    int32_t* out = sel + ((size_t(b) * N + (live ? t - P : 0)) * G + g) * kTopK;
+    if (c + 1 <= kTopK) {                                    // every block 0..c is taken
+        if (live) {
+            int4* o = reinterpret_cast<int4*>(out);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                o[q] = make_int4(4 * q <= c ? 4 * q : -1, 4 * q + 1 <= c ? 4 * q + 1 : -1,
+                                 4 * q + 2 <= c ? 4 * q + 2 : -1, 4 * q + 3 <= c ? 4 * q + 3 : -1);
+        }
+        return;
+    }
+    if (tid == 0) {
+        mbar_init(&sm.q_full, 1);
+        mbar_init(&sm.mma_done[0], 1);
+        mbar_init(&sm.mma_done[1], 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&tmQ);
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 2 * kTcCand);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    if (tid == 0) {
+        // rows 128 c - P .. + 127 of this sequence's queries (rows outside the queries are read
+        // as zeros or as a neighbour's rows and never written)
+        mbar_arrive_expect_tx(&sm.q_full, kTcRows * 128);
+        tma_load_3d(sm.q, &tmQ, 0, g, int(int64_t(b) * N + int64_t(c) * kBlock - P), &sm.q_full);
+    }
+    const int nchunks = (c + kTcCand - 1) / kTcCand;
+    const float4* prow = reinterpret_cast<const float4*>(pooled + (size_t(b) * G + g) * nb_cap * kIndexDim);
+    const uint32_t idesc = idesc_bf16_f32(kTcRows, kTcCand, 0, 0);   // both operands K-major
+
+    // threads 2 i and 2 i + 1 stage candidate j0 + i of a chunk, 32 dims each: three 128-byte
+    // rows (one per term)
+    auto stage = [&](int k) {
+        const int r = tid >> 1, j = k * kTcCand + r;
+        uint8_t* dst = sm.kb[k & 1][0];
+#pragma unroll
+        for (int ch = 4 * (tid & 1); ch < 4 * (tid & 1) + 4; ++ch) {   // 8 dims per 16-byte chunk
+            float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+            if (j < c) {
+                v0 = __ldg(prow + size_t(j) * (kIndexDim / 4) + 2 * ch);
+                v1 = __ldg(prow + size_t(j) * (kIndexDim / 4) + 2 * ch + 1);
+            }
+            const float xs[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            float hs[8], ms[8], ls[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) split3(xs[e], hs[e], ms[e], ls[e]);
+            const uint32_t off = sw128(uint32_t(r), uint32_t(ch));
+            *reinterpret_cast<uint4*>(dst + off) = make_uint4(pack_bf16x2(hs[0], hs[1]), pack_bf16x2(hs[2], hs[3]),
+                                                              pack_bf16x2(hs[4], hs[5]), pack_bf16x2(hs[6], hs[7]));
+            *reinterpret_cast<uint4*>(dst + kTcCand * 128 + off) =
+                make_uint4(pack_bf16x2(ms[0], ms[1]), pack_bf16x2(ms[2], ms[3]), pack_bf16x2(ms[4], ms[5]),
+                           pack_bf16x2(ms[6], ms[7]));
+            *reinterpret_cast<uint4*>(dst + 2 * kTcCand * 128 + off) =
+                make_uint4(pack_bf16x2(ls[0], ls[1]), pack_bf16x2(ls[2], ls[3]), pack_bf16x2(ls[4], ls[5]),
+                           pack_bf16x2(ls[6], ls[7]));
+        }
+        fence_proxy_async();                                 // visible to the tensor cores
+    };
+    // one thread: S[buf] = sum over the three terms of Q_I x term^T
+    auto issue = [&](int k) {
+        const int buf = k & 1;
+        const uint32_t qb = smem_u32(sm.q), kbase = smem_u32(sm.kb[buf][0]);
+#pragma unroll
+        for (int part = 0; part < 3; ++part)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc_mma_ss(tmem + buf * kTcCand, sdesc_sw128(qb + ks * 32, 16, 1024),
+                          sdesc_sw128(kbase + part * kTcCand * 128 + ks * 32, 16, 1024), idesc,
+                          (part | ks) != 0);
+        tc_commit(&sm.mma_done[buf]);
+    };
+
+    float best[kTcKeep];
+    int bid[kTcKeep];
+#pragma unroll
+    for (int i = 0; i < kTcKeep; ++i) { best[i] = -INFINITY; bid[i] = 0x7fffffff; }
+    // Every wait is bounded. A wait that gives up makes its warp stop ranking; the whole CTA then
+    // leaves the loop at the next barrier, and thread 0 waits (bounded) for the MMAs it issued
+    // before the tensor memory is freed.
+    bool ok = true;
+    int issued = 0, waited = 0;                              // chunks whose MMAs were issued / waited for
+    stage(0);
+    __syncthreads();
+    if (tid == 0) {
+        ok = mbar_wait(&sm.q_full, 0, hdr, KID_SELECT_PREFILL);
+        if (ok) {
+            tc_fence_after();
+            issue(0);
+            issued = 1;
+        }
+    }
+    ok = __syncthreads_and(ok);
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    for (int k = 0; ok && k < nchunks; ++k) {
+        if (k + 1 < nchunks) stage(k + 1);                   // its buffer's MMAs (chunk k - 1) are done
+        tc_fence_before();
+        if (!__syncthreads_and(ok)) { ok = false; break; }   // staged; chunk k - 1's scores all read
+        tc_fence_after();
+        if (tid == 0 && k + 1 < nchunks) { issue(k + 1); issued = k + 2; }
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.mma_done[k & 1], (k >> 1) & 1, hdr, KID_SELECT_PREFILL));
+        if (!ok) continue;                                   // the loop ends at the next barrier
+        waited = k + 1;
+        tc_fence_after();
+        const int j0 = k * kTcCand;
+#pragma unroll 1
+        for (int q32 = 0; q32 < kTcCand / 32; ++q32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + (k & 1) * kTcCand + q32 * 32, v);
+            tmem_wait_ld();
+            // mark the candidates that beat the current 15th score (no branches), then insert
+            // only those, in id order: the warp runs as many rounds as its busiest lane
+            unsigned msk = 0u;
+            const float thr = best[kTcKeep - 1];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                msk |= (j0 + q32 * 32 + i < c && __uint_as_float(v[i]) > thr) ? (1u << i) : 0u;
+            while (msk != 0u) {
+                const int i = __ffs(msk) - 1;
+                msk &= msk - 1u;
+                float sc = 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) sc = e == i ? __uint_as_float(v[e]) : sc;
+                if (sc > best[kTcKeep - 1]) {
+                    best[kTcKeep - 1] = sc; bid[kTcKeep - 1] = j0 + q32 * 32 + i;
+#pragma unroll
+                    for (int r = kTcKeep - 1; r > 0; --r) {
+                        if (best[r] > best[r - 1]) {
+                            float tv = best[r]; best[r] = best[r - 1]; best[r - 1] = tv;
+                            int ti = bid[r]; bid[r] = bid[r - 1]; bid[r - 1] = ti;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    if (tid == 0)                                            // MMAs issued but not waited for (failure path)
+        for (int kk = waited; kk < issued; ++kk) mbar_wait(&sm.mma_done[kk & 1], (kk >> 1) & 1, hdr, KID_SELECT_PREFILL);
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 2 * kTcCand);
+    }
+    if (!ok || !live) return;
+    int ids[16];
+#pragma unroll
+    for (int i = 0; i < kTcKeep; ++i) ids[i] = bid[i];
+    ids[15] = c;
+    sort16_ids(ids);
+    int4* o = reinterpret_cast<int4*>(out);
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) o[q4] = make_int4(ids[4 * q4], ids[4 * q4 + 1], ids[4 * q4 + 2], ids[4 * q4 + 3]);
+}
+
+msa_status_t launch_select_prefill_tc(const void* q_idx, int B, int G, int64_t N, int64_t P, const float* pooled,
+                                      int64_t nb_cap, int32_t* sel, void* ws, cudaStream_t st) {
+    CUtensorMap tmQ;
+    msa_status_t e = make_tmap_qidx(&tmQ, q_idx, G, uint64_t(B) * N);
+    if (e != MSA_OK) return e;
+    const int64_t nqb = (P + N - 1) / kBlock - P / kBlock + 1;   // query blocks holding positions P .. P + N - 1
+    const int smem = int(sizeof(SelTcSmem)) + 1024;
+    static std::atomic<bool> attr_set[64];      // per device; setting it twice is harmless
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
+        cudaFuncSetAttribute(select_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        attr_set[dev].store(true, std::memory_order_relaxed);
+    }
+    dim3 grid(static_cast<unsigned>(nqb), static_cast<unsigned>(G), static_cast<unsigned>(B));
+    count_launch();
+    select_prefill_tc_kernel<<<grid, 128, smem, st>>>(tmQ, N, P, G, pooled, nb_cap, sel, static_cast<WsHeader*>(ws));
+    return MSA_OK;
+}
+
+}  // namespace msa

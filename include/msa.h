@@ -295,7 +295,9 @@ msa_status_t msa_fp8_close_blocks(const msa_shape_t *shape, const int32_t *ctx_l
 /* Main Branch, decode, over the FP8 cache: as msa_sparse_attn_decode, but every selected
  * block below the query's own one is read as e4m3 codes and scales (half the bytes of bf16);
  * the query's own block is read from the bf16 caches k_cache, v_cache. Scores are
- * scale_k * (q . code) and the values code x scale_v, accumulated in fp32.
+ * scale_k * (q . code) and the values code x scale_v, accumulated in fp32; on the e4m3 blocks
+ * the products run in f16, which holds every code exactly and every bf16 query value in its
+ * normal range, so query values must stay below 65504 in magnitude.
  *   nb_cap  blocks per (sequence, group) in k_scale / v_scale; must be >= max_pos / Bk
  *   workspace of msa_workspace_size(MSA_OP_ATTN_DECODE, max_pos) */
 msa_status_t msa_sparse_attn_decode_fp8(const msa_shape_t *shape, const void *q, const void *k_codes,
