@@ -23,8 +23,8 @@ __all__ = [
     "msa_index_select_decode_noalloc", "msa_selftest_wait_timeout", "msa_kernel_launches",
     "msa_topk_rows", "msa_fp8_quantize_blocks", "msa_fp8_close_blocks", "msa_sparse_attn_decode_fp8",
     "msa_pool_index_keys_chunk", "msa_index_select_chunk", "msa_sparse_attn_prefill_chunk",
-    "msa_prefill_chunk_workspace_size",
-    "OP_INDEX_SELECT_PREFILL", "OP_INDEX_SELECT_DECODE", "OP_ATTN_PREFILL", "OP_ATTN_DECODE",
+    "msa_prefill_chunk_workspace_size", "msa_sparse_attn_prefill_backward",
+    "OP_INDEX_SELECT_PREFILL", "OP_ATTN_PREFILL_BACKWARD", "OP_INDEX_SELECT_DECODE", "OP_ATTN_PREFILL", "OP_ATTN_DECODE",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -32,6 +32,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libmsa.so")
 
 OP_INDEX_SELECT_PREFILL, OP_INDEX_SELECT_DECODE, OP_ATTN_PREFILL, OP_ATTN_DECODE = 0, 1, 2, 3
+OP_ATTN_PREFILL_BACKWARD = 4
 HEAD_DIM, INDEX_DIM, BLOCK, TOPK = 128, 64, 128, 16
 
 STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARGUMENT", 2: "MSA_ERR_UNSUPPORTED",
@@ -46,7 +47,7 @@ EXPORTED_SYMBOLS = [
     "msa_index_select_decode_noalloc", "msa_selftest_wait_timeout", "msa_topk_rows",
     "msa_fp8_quantize_blocks", "msa_fp8_close_blocks", "msa_sparse_attn_decode_fp8",
     "msa_pool_index_keys_chunk", "msa_index_select_chunk", "msa_sparse_attn_prefill_chunk",
-    "msa_prefill_chunk_workspace_size",
+    "msa_prefill_chunk_workspace_size", "msa_sparse_attn_prefill_backward",
 ]
 
 
@@ -110,6 +111,7 @@ def load():
             "msa_pool_index_keys_chunk": [SP, P, I64, I64, P, I64, P, P],
             "msa_index_select_chunk": [SP, P, I64, I64, P, I64, P, P, SZ, P],
             "msa_sparse_attn_prefill_chunk": [SP, P, P, P, I64, I64, I64, P, P, P, P, SZ, P],
+            "msa_sparse_attn_prefill_backward": [SP, P, P, P, I64, P, P, P, P, P, P, P, P, SZ, P],
         }.items():
             f = getattr(L, name)
             f.restype = ctypes.c_int
@@ -293,3 +295,14 @@ def msa_sparse_attn_prefill_chunk(shape: Shape, q, k_cache, v_cache, l_cap: int,
                                                 q_start, n, _ptr(sel), _ptr(out), _ptr(lse), _ptr(workspace),
                                                 _nbytes(workspace), _stream(stream)),
            "msa_sparse_attn_prefill_chunk")
+
+
+def msa_sparse_attn_prefill_backward(shape: Shape, q, k, v, n_tokens: int, sel, out, lse, d_out, dq, dk, dv,
+                                     workspace, stream=None):
+    """Gradients dq [B,N,Hq,128], dk, dv [B,G,N,128] (fp32) of the prefill's main branch for the
+    upstream gradient d_out, the selection held fixed."""
+    _check(load().msa_sparse_attn_prefill_backward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), n_tokens,
+                                                   _ptr(sel), _ptr(out), _ptr(lse), _ptr(d_out), _ptr(dq),
+                                                   _ptr(dk), _ptr(dv), _ptr(workspace), _nbytes(workspace),
+                                                   _stream(stream)),
+           "msa_sparse_attn_prefill_backward")

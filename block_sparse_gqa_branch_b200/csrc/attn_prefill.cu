@@ -772,9 +772,18 @@ int num_sms() {
     return v > 0 ? v : 148;
 }
 
-msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, const CUtensorMap& tmK, const CUtensorMap& tmV, int64_t N,
-                            int64_t P, int64_t l_cap, int B, int G, int Hg, const int32_t* sel, void* out, float* lse,
-                            void* ws, cudaStream_t st) {
+// Bytes of the workspace's inverted index (header, counts, offsets, item list, entries): the
+// part the backward pass shares with the forward; and where its parts start.
+size_t inverted_index_bytes(int B, int64_t N, int G, int Hg) { return prefill_layout(B, N, G, Hg, 0).off_lse; }
+IndexOffsets inverted_index_offsets(int B, int64_t N, int G, int Hg) {
+    const PrefillLayout L = prefill_layout(B, N, G, Hg, 0);
+    return IndexOffsets{L.off_nitems, L.off_items, L.off_list};
+}
+
+// The inverted index of a selection in `ws` (memset + count + scan + fill): work items
+// {b G + g, block j (| kDiagFlag), first entry (or first query), count} in (b, g, range, j)
+// order, their number in nitems[0] and a zeroed hand-out counter in nitems[1].
+void launch_inverted_index(const int32_t* sel, int64_t N, int64_t P, int B, int G, int Hg, void* ws, cudaStream_t st) {
     const PrefillLayout L = prefill_layout(B, N, G, Hg, P);
     char* base = static_cast<char*>(ws);
     WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
@@ -783,9 +792,6 @@ msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, cons
     int* nitems = reinterpret_cast<int*>(base + L.off_nitems);
     int4* items = reinterpret_cast<int4*>(base + L.off_items);
     int* list = reinterpret_cast<int*>(base + L.off_list);
-    float* part_lse = reinterpret_cast<float*>(base + L.off_lse);
-    uint16_t* part_o = reinterpret_cast<uint16_t*>(base + L.off_o);
-
     cudaMemsetAsync(counts, 0, L.nbins * sizeof(int), st);
     {
         dim3 grid(static_cast<unsigned>((N + kCountChunk - 1) / kCountChunk), static_cast<unsigned>(G),
@@ -804,6 +810,20 @@ msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, cons
         csr_fill_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(sel, N, P, G, L.nb, L.nR, offsets,
                                                                                    counts, list, total);
     }
+}
+
+msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, const CUtensorMap& tmK, const CUtensorMap& tmV, int64_t N,
+                            int64_t P, int B, int G, int Hg, const int32_t* sel, void* out, float* lse,
+                            void* ws, cudaStream_t st) {
+    const PrefillLayout L = prefill_layout(B, N, G, Hg, P);
+    char* base = static_cast<char*>(ws);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
+    int* nitems = reinterpret_cast<int*>(base + L.off_nitems);
+    int4* items = reinterpret_cast<int4*>(base + L.off_items);
+    int* list = reinterpret_cast<int*>(base + L.off_list);
+    float* part_lse = reinterpret_cast<float*>(base + L.off_lse);
+    uint16_t* part_o = reinterpret_cast<uint16_t*>(base + L.off_o);
+    launch_inverted_index(sel, N, P, B, G, Hg, ws, st);
     {
         PrefillArgs a;
         a.N = N; a.P = P; a.G = G; a.Hg = Hg; a.Hq = G * Hg; a.tpt = L.tpt;

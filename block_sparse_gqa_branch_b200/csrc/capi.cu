@@ -30,8 +30,11 @@ void launch_fp8_close(const void*, const void*, int64_t, const int32_t*, int, in
                       void*, cudaStream_t);
 size_t decode_attn_ws_bytes(int, int, int);
 size_t prefill_attn_ws_bytes(int, int64_t, int, int, int64_t);
+size_t backward_ws_bytes(int, int64_t, int, int);
+msa_status_t launch_attn_backward(const void*, const void*, const void*, int64_t, int, int, int, const int32_t*,
+                                  const void*, const float*, const void*, float*, float*, float*, void*, cudaStream_t);
 msa_status_t launch_attn_prefill_tc(const void*, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, int64_t,
-                                    int64_t, int64_t, int, int, int, const int32_t*, void*, float*, void*, cudaStream_t);
+                                    int64_t, int, int, int, const int32_t*, void*, float*, void*, cudaStream_t);
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
@@ -195,6 +198,9 @@ size_t ws_size(const msa_shape_t* s, int32_t op, int64_t n) {
             if (n < 1) return 0;
             return prefill_attn_ws_bytes(s->batch, n, s->n_kv_groups, hg, 0);
         case MSA_OP_ATTN_DECODE: return decode_attn_ws_bytes(s->batch, s->n_kv_groups, hg);
+        case MSA_OP_ATTN_PREFILL_BACKWARD:
+            if (n < 1) return 0;
+            return backward_ws_bytes(s->batch, n, s->n_kv_groups, hg);
         default: return 0;
     }
 }
@@ -293,7 +299,7 @@ msa_status_t attn_prefill_impl(const msa_shape_t* shape, const void* q, const vo
     // rows past P + n_tokens (the chunk's last position) read as zeros
     MSA_TRY(make_tmap_kv3d(&tmK, k, uint64_t(P + n_tokens), uint64_t(l_cap), uint64_t(B) * G));
     MSA_TRY(make_tmap_kv3d(&tmV, v, uint64_t(P + n_tokens), uint64_t(l_cap), uint64_t(B) * G));
-    MSA_TRY(launch_attn_prefill_tc(q, tmQ, tmK, tmV, n_tokens, P, l_cap, B, G, hg, sel, out, lse, workspace,
+    MSA_TRY(launch_attn_prefill_tc(q, tmQ, tmK, tmV, n_tokens, P, B, G, hg, sel, out, lse, workspace,
                                    reinterpret_cast<cudaStream_t>(stream)));
     return cuda_status();
 }
@@ -306,6 +312,28 @@ msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const void* q, co
                                      size_t workspace_bytes, msa_stream_t stream) {
     return attn_prefill_impl(shape, q, k, v, n_tokens, 0, n_tokens, sel, out, lse, workspace, workspace_bytes,
                              stream);
+}
+
+msa_status_t msa_sparse_attn_prefill_backward(const msa_shape_t* shape, const void* q, const void* k, const void* v,
+                                              int64_t n_tokens, const int32_t* sel, const void* out, const float* lse,
+                                              const void* d_out, float* dq, float* dk, float* dv, void* workspace,
+                                              size_t workspace_bytes, msa_stream_t stream) {
+    MSA_TRY(check_shape(shape));
+    MSA_REQ(n_tokens >= 1 && n_tokens < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(q && k && v && sel && out && lse && d_out && dq && dk && dv && aligned16(q) && aligned16(k) &&
+                aligned16(v) && aligned16(sel) && aligned16(out) && aligned16(d_out) && aligned16(dq) &&
+                aligned16(dk) && aligned16(dv) && (reinterpret_cast<uintptr_t>(lse) & 3u) == 0,
+            MSA_ERR_INVALID_ARGUMENT);
+    const int B = shape->batch, G = shape->n_kv_groups, Hq = shape->n_q_heads, hg = Hq / G;
+    MSA_REQ(int64_t(B) * n_tokens * G * (kTopK - 1) < (int64_t(1) << 31) &&
+                int64_t(B) * n_tokens * Hq * kTopK < (int64_t(1) << 31) &&
+                (n_tokens + kBlock - 1) / kBlock <= 48 * 1024,
+            MSA_ERR_UNSUPPORTED);
+    const size_t need = backward_ws_bytes(B, n_tokens, G, hg);
+    MSA_REQ(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need, MSA_ERR_WORKSPACE);
+    MSA_TRY(launch_attn_backward(q, k, v, n_tokens, B, G, hg, sel, out, lse, d_out, dq, dk, dv, workspace,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status();
 }
 
 size_t msa_prefill_chunk_workspace_size(const msa_shape_t* shape, int64_t q_start, int64_t n_queries) {

@@ -37,6 +37,9 @@ msa_status_t make_tmap_qidx(CUtensorMap* m, const void* base, int G, uint64_t ro
 // halves as [half][8 rows][128 B] (128B swizzle)
 msa_status_t make_tmap_q_rows(CUtensorMap* m, const void* base, uint64_t rows);
 
+// byte offsets, inside a prefill workspace, of the inverted index's item count, items and entries
+struct IndexOffsets { size_t nitems, items, list; };
+
 // largest query position the decode path supports (bounds its workspaces and row indices)
 constexpr int64_t kMaxDecodePos = (int64_t(1) << 24) - 1;
 

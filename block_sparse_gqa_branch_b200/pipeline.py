@@ -8,7 +8,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (BLOCK, INDEX_DIM, TOPK, OP_ATTN_DECODE, OP_ATTN_PREFILL, OP_INDEX_SELECT_DECODE,
+from . import (BLOCK, INDEX_DIM, TOPK, OP_ATTN_DECODE, OP_ATTN_PREFILL, OP_ATTN_PREFILL_BACKWARD,
+               OP_INDEX_SELECT_DECODE, msa_sparse_attn_prefill_backward,
                OP_INDEX_SELECT_PREFILL, Shape, msa_fp8_close_blocks, msa_fp8_quantize_blocks,
                msa_index_select, msa_index_select_chunk, msa_pool_index_keys, msa_pool_index_keys_chunk,
                msa_pooled_keys_append, msa_prefill_chunk_workspace_size, msa_sparse_attn_decode,
@@ -151,3 +152,21 @@ def prefill_chunk(q, q_idx, k_idx, k_cache, v_cache, q_start: int, pooled, tail_
     msa_index_select_chunk(shape, q_idx, q_start, n, pooled, nb_cap, sel, ws_sel, stream)
     msa_sparse_attn_prefill_chunk(shape, q, k_cache, v_cache, l_cap, q_start, n, sel, out, lse, ws, stream)
     return out, lse, sel, {"ws_select": ws_sel, "ws_attn": ws}
+
+
+def backward_buffers(B: int, N: int, Hq: int, G: int, device) -> dict:
+    """Gradient outputs (fp32) and the zeroed workspace of the main branch's backward pass."""
+    shape = Shape.make(B, Hq, G)
+    return {"shape": shape, "N": N,
+            "dq": torch.empty(B, N, Hq, 128, dtype=torch.float32, device=device),
+            "dk": torch.empty(B, G, N, 128, dtype=torch.float32, device=device),
+            "dv": torch.empty(B, G, N, 128, dtype=torch.float32, device=device),
+            "ws": _ws(shape, OP_ATTN_PREFILL_BACKWARD, N, device)}
+
+
+def prefill_backward(q, k, v, d_out, fwd: dict, bwd: dict, stream=None):
+    """Backward pass of the main branch after a prefill whose buffers are `fwd` (sel, out, lse).
+    Returns (dq, dk, dv)."""
+    msa_sparse_attn_prefill_backward(bwd["shape"], q, k, v, bwd["N"], fwd["sel"], fwd["out"], fwd["lse"], d_out,
+                                     bwd["dq"], bwd["dk"], bwd["dv"], bwd["ws"], stream)
+    return bwd["dq"], bwd["dk"], bwd["dv"]

@@ -77,7 +77,8 @@ enum {
     MSA_OP_INDEX_SELECT_PREFILL = 0,
     MSA_OP_INDEX_SELECT_DECODE = 1,
     MSA_OP_ATTN_PREFILL = 2,
-    MSA_OP_ATTN_DECODE = 3
+    MSA_OP_ATTN_DECODE = 3,
+    MSA_OP_ATTN_PREFILL_BACKWARD = 4
 };
 
 /* Version of this ABI (bumped on any incompatible change). */
@@ -99,6 +100,7 @@ uint64_t msa_kernel_launches(void);
  *  op = MSA_OP_INDEX_SELECT_DECODE:  n = max_pos (largest query position)
  *  op = MSA_OP_ATTN_PREFILL:         n = number of tokens per sequence
  *  op = MSA_OP_ATTN_DECODE:          n = max_pos
+ *  op = MSA_OP_ATTN_PREFILL_BACKWARD: n = number of tokens per sequence
  * Returns 0 for an invalid shape or op.
  */
 size_t msa_workspace_size(const msa_shape_t *shape, int32_t op, int64_t n);
@@ -224,6 +226,29 @@ msa_status_t msa_sparse_attn_prefill_chunk(const msa_shape_t *shape, const void 
 
 /* Workspace bytes of msa_sparse_attn_prefill_chunk (0 for an invalid shape, P < 0 or n < 1). */
 size_t msa_prefill_chunk_workspace_size(const msa_shape_t *shape, int64_t q_start, int64_t n_queries);
+
+/*
+ * Main Branch, backward pass of a prefill: the gradient of the outputs with respect to q, k and
+ * v, the selection held fixed (a discrete choice). Sources: youmind article "MiniMax M3 sparse
+ * attention agents", bullet on MSA-CPT, and KuCoin MSA launch flash, "ME AI News" (MSA-PT):
+ * the model is trained through the sparse attention. With z_u = q . k_u / sqrt(d) over the
+ * keys u of the forward (selected blocks, u <= t), p = softmax(z), o = sum p_u v_u and the
+ * upstream gradient dO of o: dV_u += p_u dO, dS_u = p_u (dO . v_u - dO . o),
+ * dQ = sum_u dS_u k_u / sqrt(d), dK_u += dS_u q / sqrt(d) (summed over heads and queries).
+ *   q, k, v, sel      as msa_sparse_attn_prefill (N = n_tokens)
+ *   out, lse          the forward's outputs (bf16 [B, N, Hq, d], fp32 [B, N, Hq]; lse required)
+ *   d_out             bf16 [B, N, Hq, d]  upstream gradient of out
+ *   dq                fp32 [B, N, Hq, d]  out
+ *   dk, dv            fp32 [B, G, N, d]   out (every row written; rows no query attends are 0)
+ *   workspace of msa_workspace_size(MSA_OP_ATTN_PREFILL_BACKWARD, N)
+ * Sums over blocks and queries run in fp32 with atomic adds, so the low bits of the results
+ * may differ between runs. Size limits as msa_sparse_attn_prefill.
+ */
+msa_status_t msa_sparse_attn_prefill_backward(const msa_shape_t *shape, const void *q, const void *k,
+                                              const void *v, int64_t n_tokens, const int32_t *sel,
+                                              const void *out, const float *lse, const void *d_out,
+                                              float *dq, float *dk, float *dv, void *workspace,
+                                              size_t workspace_bytes, msa_stream_t stream);
 
 /*
  * Decode: append the new token to the caches and keep the pooled keys current (the pages

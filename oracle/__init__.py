@@ -130,27 +130,46 @@ def topk_rows(scores: np.ndarray, k: int) -> np.ndarray:
 
 
 def attend_grad(t: np.ndarray, q_rows: np.ndarray, K: np.ndarray, V: np.ndarray, sel: Optional[np.ndarray],
-                dO: np.ndarray, Bk: int = 128):
+                dO: np.ndarray, Bk: int = 128, nthreads: Optional[int] = None):
     """Gradient of step 4 for queries of one (sequence, group), the selection held fixed.
     q_rows [n, Hg, d] (bf16 bits), K, V [L, d] (bf16 bits), sel [n, k] or None (every key u <= t),
     dO [n, Hg, d] (float64). Returns (dQ [n, Hg, d], dK [L, d], dV [L, d]) in float64, dK and dV
-    summed over every row and head."""
+    summed over every row and head. Rows are split over threads, each with its own key-gradient
+    sums, added in row order at the end."""
     t = _c(t, np.int64)
     q = _c(q_rows, np.uint16)
     K, V = _c(K, np.uint16), _c(V, np.uint16)
     g = _c(dO, np.float64)
     n, Hg, d = q.shape
     dQ = np.zeros((n, Hg, d), np.float64)
+
+    def rows(lo, hi):
+        # each worker sums its rows' key gradients into its own arrays
+        dK = np.zeros(K.shape, np.float64)
+        dV = np.zeros(V.shape, np.float64)
+        for r in range(lo, hi):
+            s = None if sel is None else _c(sel[r], np.int32)
+            ns = 0 if s is None else int((s >= 0).sum())
+            for h in range(Hg):
+                out = np.zeros(d, np.float64)
+                lib().oracle_attend_row_grad(_p(np.ascontiguousarray(q[r, h])), _p(K), _p(V), d, int(t[r]), _p(s), ns,
+                                             Bk, _p(np.ascontiguousarray(g[r, h])), _p(out), _p(dK), _p(dV))
+                dQ[r, h] = out
+        return dK, dV
+
+    nth = max(1, min(nthreads or default_threads(), n))
+    bounds = [(i * n // nth, (i + 1) * n // nth) for i in range(nth)]
+    if nth == 1:
+        parts = [rows(0, n)]
+    else:
+        import concurrent.futures
+        with concurrent.futures.ThreadPoolExecutor(max_workers=nth) as ex:
+            parts = list(ex.map(lambda b: rows(*b), bounds))
     dK = np.zeros(K.shape, np.float64)
     dV = np.zeros(V.shape, np.float64)
-    for r in range(n):
-        s = None if sel is None else _c(sel[r], np.int32)
-        ns = 0 if s is None else int((s >= 0).sum())
-        for h in range(Hg):
-            out = np.zeros(d, np.float64)
-            lib().oracle_attend_row_grad(_p(np.ascontiguousarray(q[r, h])), _p(K), _p(V), d, int(t[r]), _p(s), ns,
-                                         Bk, _p(np.ascontiguousarray(g[r, h])), _p(out), _p(dK), _p(dV))
-            dQ[r, h] = out
+    for pk, pv in parts:                # in row order, so the result does not depend on threads
+        dK += pk
+        dV += pv
     return dQ, dK, dV
 
 

@@ -22,6 +22,16 @@ CANCEL_RATIO = 0.1
 MAX_ABS_TOL = 2e-2
 MEAN_ABS_TOL = 2e-3
 
+# Gradients of the main branch (dQ, dK, dV), relative to the reference's own magnitude (they are
+# not O(1) like the outputs). Every gradient element is a sum of terms in which the kernel rounds
+# one factor to bf16 (p for dV, dS = p (dP - D) for dQ and dK, whose D is formed from the
+# forward's bf16 output): at most three roundings of 2^-9 relative each, accumulated in fp32.
+# Random rounding errors of a sum stay near eps = 3 * 2^-9 of its typical magnitude, so the
+# mean |err| is held to eps of the mean |ref| and the max |err| to 4 eps of the max |ref|.
+GRAD_EPS = 3 * 2.0 ** -9
+GRAD_REL_MEAN = GRAD_EPS
+GRAD_REL_MAX = 4 * GRAD_EPS
+
 # workload label -> counters (rows checked, rows differing, near-ties, cancellation near-ties)
 TIE_LOG: dict = {}
 
@@ -93,3 +103,16 @@ def assert_close_attention(gpu, ref, what=""):
     assert mx <= MAX_ABS_TOL, f"{what}: max abs err {mx:.3e} > {MAX_ABS_TOL}"
     assert mn <= MEAN_ABS_TOL, f"{what}: mean abs err {mn:.3e} > {MEAN_ABS_TOL}"
     return mx, mn
+
+
+def assert_close_gradient(gpu, ref, what=""):
+    """A gradient against the fp64 reference: mean |err| <= GRAD_REL_MEAN * mean |ref| and
+    max |err| <= GRAD_REL_MAX * max |ref|."""
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert np.isfinite(gpu).all(), f"{what}: non-finite gradient"
+    e = np.abs(gpu - ref)
+    mean_ref, max_ref = float(np.abs(ref).mean()), float(np.abs(ref).max())
+    assert e.mean() <= GRAD_REL_MEAN * mean_ref, f"{what}: mean |err| {e.mean():.3e} > {GRAD_REL_MEAN:.2e} x {mean_ref:.3e}"
+    assert e.max() <= GRAD_REL_MAX * max_ref, f"{what}: max |err| {e.max():.3e} > {GRAD_REL_MAX:.2e} x {max_ref:.3e}"
+    return float(e.mean() / max(mean_ref, 1e-300)), float(e.max() / max(max_ref, 1e-300))
