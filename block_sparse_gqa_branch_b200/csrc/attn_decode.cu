@@ -189,30 +189,35 @@ __device__ __forceinline__ float4* park_addr(DecSmem& sm, int s, int w, int g, i
 }
 
 // Fold the partial of another CTA (max, sum, o of rows gq, gq + 8) into st.
+// Every load of the partial goes out before any value is used (rows gq, gq + 8 past Hg read
+// row 0 and are ignored).
 __device__ __forceinline__ void merge_partial(WarpState& st, const float* pf, int Hg, int ooff, int gq, int tq) {
+    const int r0 = gq < Hg ? gq : 0, r1 = gq + 8 < Hg ? gq + 8 : 0;
+    const float2 ml0 = ld_cg_f2pair(pf + r0, pf + Hg + r0), ml1 = ld_cg_f2pair(pf + r1, pf + Hg + r1);
+    const float m0 = ml0.x, l0 = ml0.y, m1 = ml1.x, l1 = ml1.y;
+    float2 x0[16], x1[16];
+    ld_cg_f2x16_s32(pf + ooff + r0 * kHeadDim + 2 * tq, x0);
+    ld_cg_f2x16_s32(pf + ooff + r1 * kHeadDim + 2 * tq, x1);
     float wa0 = 1.f, wb0 = 0.f, wa1 = 1.f, wb1 = 0.f, mn;
     if (gq < Hg) {
-        lse_weights(st.m0, __ldcg(pf + gq), mn, wa0, wb0);
-        st.l0 = st.l0 * wa0 + __ldcg(pf + Hg + gq) * wb0;
+        lse_weights(st.m0, m0, mn, wa0, wb0);
+        st.l0 = st.l0 * wa0 + l0 * wb0;
         st.m0 = mn;
     }
     if (gq + 8 < Hg) {
-        lse_weights(st.m1, __ldcg(pf + gq + 8), mn, wa1, wb1);
-        st.l1 = st.l1 * wa1 + __ldcg(pf + Hg + gq + 8) * wb1;
+        lse_weights(st.m1, m1, mn, wa1, wb1);
+        st.l1 = st.l1 * wa1 + l1 * wb1;
         st.m1 = mn;
     }
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) {
-        const int col = nt * 8 + 2 * tq;
         if (gq < Hg) {
-            const float2 x = __ldcg(reinterpret_cast<const float2*>(pf + ooff + gq * kHeadDim + col));
-            st.o[nt][0] = st.o[nt][0] * wa0 + x.x * wb0;
-            st.o[nt][1] = st.o[nt][1] * wa0 + x.y * wb0;
+            st.o[nt][0] = st.o[nt][0] * wa0 + x0[nt].x * wb0;
+            st.o[nt][1] = st.o[nt][1] * wa0 + x0[nt].y * wb0;
         }
         if (gq + 8 < Hg) {
-            const float2 x = __ldcg(reinterpret_cast<const float2*>(pf + ooff + (gq + 8) * kHeadDim + col));
-            st.o[nt][2] = st.o[nt][2] * wa1 + x.x * wb1;
-            st.o[nt][3] = st.o[nt][3] * wa1 + x.y * wb1;
+            st.o[nt][2] = st.o[nt][2] * wa1 + x1[nt].x * wb1;
+            st.o[nt][3] = st.o[nt][3] * wa1 + x1[nt].y * wb1;
         }
     }
 }

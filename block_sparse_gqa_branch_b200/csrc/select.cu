@@ -296,11 +296,17 @@ __global__ void __launch_bounds__(kSelThreads) select_decode_kernel(
     unsigned long long best = 0ull;                      // lanes 0-15: this warp's best 16
     for (int base = lo; base < hi; base += kSelThreads) {
         const int r0 = base + wid * 32;                  // this warp's 32 rows
+        // all 16 loads of the lane go out before any is used; in the span's last pass rows past
+        // the span read its last row and are ignored
         float4 v[16];
+        if (base + kSelThreads <= hi) {
+            ld_nc_f4x16_s512(rows + size_t(r0 + half) * (kIndexDim / 4) + part, v);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int r = r0 + 2 * i + half;
-            v[i] = r < hi ? __ldg(rows + size_t(r) * (kIndexDim / 4) + part) : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < 16; ++i) {
+                const int r = r0 + 2 * i + half;
+                v[i] = ld_nc_f4(rows + size_t(r < hi ? r : hi - 1) * (kIndexDim / 4) + part);
+            }
         }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
