@@ -539,6 +539,84 @@ def time_decode(torch, w, dev, steps, warmup, flush_l2, fp8=False):
     return [a.elapsed_time(b) * 1e-3 for a, b in ts], (4 if fp8 else 3) * steps
 
 
+def time_backward(torch, w, dev, steps, warmup, flush_l2):
+    """Backward pass of the main branch after a prefill of workload w (its selection, output and
+    lse; upstream gradient seeded like q): per-step device seconds of msa_sparse_attn_prefill_backward."""
+    from block_sparse_gqa_branch_b200 import msa_get_device_status, pipeline
+    x = synth.prefill_inputs_torch(w, dev)
+    fwd = pipeline.prefill_buffers(w.B, w.N, w.Hq, w.G, dev)
+    pipeline.prefill(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], fwd)
+    del fwd["ws_attn"], fwd["ws_select"]
+    torch.cuda.empty_cache()
+    d_out = synth.normal_bf16_torch(w.seed + 99, synth.STREAM_Q, w.B * w.N * w.Hq * w.d, dev).view(w.B, w.N, w.Hq, w.d)
+    bwd = pipeline.backward_buffers(w.B, w.N, w.Hq, w.G, dev)
+    stream = torch.cuda.current_stream()
+    ts = []
+    for s in range(warmup + steps):
+        flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pipeline.prefill_backward(x["q"], x["k"], x["v"], d_out, fwd, bwd)
+        e1.record(stream)
+        if s >= warmup:
+            ts.append((e0, e1))
+    torch.cuda.synchronize()
+    st_, info = msa_get_device_status(bwd["ws"])
+    if st_ != 0:
+        raise SystemExit(f"device status {st_} in the backward pass: {info}")
+    return [a.elapsed_time(b) * 1e-3 for a, b in ts]
+
+
+def time_prefill_chunked(torch, w, dev, chunk, steps, warmup, flush_l2):
+    """A prefill of workload w in chunks of `chunk` tokens against a cache (pool, select and
+    attention per chunk, caches filled with the chunk's K/V beforehand): per-step seconds of
+    all chunks."""
+    from block_sparse_gqa_branch_b200 import (Shape, msa_get_device_status, msa_index_select_chunk,
+                                              msa_pool_index_keys_chunk, msa_prefill_chunk_workspace_size,
+                                              msa_sparse_attn_prefill_chunk)
+    x = synth.prefill_inputs_torch(w, dev)
+    B, N, G, Hq = w.B, w.N, w.G, w.Hq
+    shape = Shape.make(B, Hq, G)
+    nb_cap = (N + 127) // 128
+    pooled = torch.zeros(B, G, nb_cap, 64, device=dev)
+    tail = torch.zeros(B, G, 64, device=dev)
+    starts = list(range(0, N, chunk))
+    qs = [x["q"][:, p:p + chunk].contiguous() for p in starts]
+    qis = [x["q_idx"][:, p:p + chunk].contiguous() for p in starts]
+    kis = [x["k_idx"][:, p:p + chunk].contiguous() for p in starts]
+    del x["q"]
+    sel = [torch.empty(B, min(chunk, N - p), G, 16, dtype=torch.int32, device=dev) for p in starts]
+    out = [torch.empty(B, min(chunk, N - p), Hq, 128, dtype=torch.bfloat16, device=dev) for p in starts]
+    lse = [torch.empty(B, min(chunk, N - p), Hq, dtype=torch.float32, device=dev) for p in starts]
+    ws_sel = torch.zeros(256, dtype=torch.uint8, device=dev)
+    ws = torch.zeros(max(msa_prefill_chunk_workspace_size(shape, p, min(chunk, N - p)) for p in starts),
+                     dtype=torch.uint8, device=dev)
+
+    def run():
+        tail.zero_()
+        for i, p in enumerate(starts):
+            n = min(chunk, N - p)
+            msa_pool_index_keys_chunk(shape, kis[i], p, n, pooled, nb_cap, tail)
+            msa_index_select_chunk(shape, qis[i], p, n, pooled, nb_cap, sel[i], ws_sel)
+            msa_sparse_attn_prefill_chunk(shape, qs[i], x["k"], x["v"], N, p, n, sel[i], out[i], lse[i], ws)
+    stream = torch.cuda.current_stream()
+    ts = []
+    for s in range(warmup + steps):
+        flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        if s >= warmup:
+            ts.append((e0, e1))
+    torch.cuda.synchronize()
+    for buf in (ws_sel, ws):
+        st_, info = msa_get_device_status(buf)
+        if st_ != 0:
+            raise SystemExit(f"device status {st_} in the chunked prefill: {info}")
+    return [a.elapsed_time(b) * 1e-3 for a, b in ts], len(starts)
+
+
 def prefill_report(w, t_index, t_main, peaks, peak_src, world, launches, traffic_name=None, scale=1.0):
     tidx, tmain = statistics.mean(t_index), statistics.mean(t_main)
     flops = prefill_main_flops(w)
@@ -848,6 +926,28 @@ def run_ours(args):
         r8 = decode_report(DECODE, [max_over_ranks(statistics.mean(td8))], peaks, peak_src, l8, fp8=True)
         r8["workload"] = DECODE.name + "_fp8kv"
         extra[r8["workload"]] = r8
+        torch.cuda.empty_cache()
+        tb = max_over_ranks(statistics.mean(time_backward(torch, PREFILL_32K, dev, n_x, w_x, flush_l2)))
+        bflops = 2.5 * prefill_main_flops(PREFILL_32K)          # S, dP, dV, dK, dQ: five products
+        extra[PREFILL_32K.name + "_backward"] = {
+            "workload": PREFILL_32K.name + "_backward", "backward_ms": tb * 1e3,
+            "value": PREFILL_32K.N * PREFILL_32K.B * world / tb, "unit": "tok/s",
+            "roofline": {"bound": "tensor", "achieved": bflops / tb / 1e12, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": bflops / tb / 1e12 / peaks["bf16_tflops"], "traffic": None,
+                         "kernel": "main-branch backward (msa_sparse_attn_prefill_backward: inverted index, D, dQ/dK/dV)",
+                         "algorithmic": f"{bflops:.4e} FLOP per launch (10 x 128 per attended head-key pair)",
+                         "peak_source": f"{peak_src} burst bf16"}}
+        torch.cuda.empty_cache()
+        tc, nchunks = time_prefill_chunked(torch, PREFILL, dev, 16384, n_x, w_x, flush_l2)
+        tc = max_over_ranks(statistics.mean(tc))
+        cflops = prefill_main_flops(PREFILL)
+        extra[PREFILL.name + "_chunked16k"] = {
+            "workload": PREFILL.name + f" in {nchunks} chunks of 16,384 tokens", "prefill_ms": tc * 1e3,
+            "value": PREFILL.N * PREFILL.B * world / tc, "unit": "tok/s",
+            "roofline": {"bound": "tensor", "achieved": cflops / tc / 1e12, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": cflops / tc / 1e12 / peaks["bf16_tflops"], "traffic": None,
+                         "kernel": "chunked prefill, all chunks (pooling, selection and main branch per chunk)",
+                         "algorithmic": f"{cflops:.4e} main-branch FLOP per pass", "peak_source": f"{peak_src} burst bf16"}}
         torch.cuda.empty_cache()
         tk = topk_report(torch, dev, n_x, w_x, peaks, peak_src)
         tk["ms"] = max_over_ranks(tk["ms"])

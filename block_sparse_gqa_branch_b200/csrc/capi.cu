@@ -14,7 +14,6 @@ namespace msa {
 void launch_pool(const void*, int, int, int64_t, float*, int64_t, float*, cudaStream_t);
 void launch_append(const void*, const void*, const void*, const int32_t*, int, int, void*, void*, int64_t,
                    float*, float*, int64_t, void*, cudaStream_t);
-void launch_select_prefill_mma(const void*, int, int, int64_t, int64_t, const float*, int64_t, int32_t*, cudaStream_t);
 msa_status_t launch_select_prefill_tc(const void*, int, int, int64_t, int64_t, const float*, int64_t, int32_t*, void*,
                                       cudaStream_t);
 void launch_pool_chunk(const void*, int, int, int64_t, int64_t, float*, int64_t, float*, cudaStream_t);

@@ -5,10 +5,11 @@
 // GQA group) and bullet "Predictable cost at every length" (k = 16); KuCoin flash "MiniMax
 // launches MSA sparse attention method and MiniMax-M3 model", summary (exp-free top-k).
 //
-// Every score is s_j = q_I . kbar_j in fp32 (the 1/sqrt(d_I) factor is an exact power of two
-// and cannot change the order, so it is not applied). Ranking uses only compares: the
-// running top-15 keeps the earlier (lower) block on equal scores, which is the order
-// (score desc, id asc). The query's own block is added and the ids are written ascending.
+// Decode: one query per (sequence, group). Every score is s_j = q_I . kbar_j in fp32 (the
+// 1/sqrt(d_I) factor is an exact power of two and cannot change the order, so it is not
+// applied). Ranking uses only compares of order-preserving keys (score, then the inverted block
+// id, so equal scores rank the lower block first). The query's own block is added and the ids
+// are written ascending. (The prefill selection is in select_tc.cu.)
 #include <cooperative_groups.h>
 
 #include "msa_common.cuh"
@@ -16,18 +17,6 @@
 namespace msa {
 
 constexpr int kKeep = kTopK - 1;   // best fully-past blocks kept besides the diagonal one
-
-// Sort 16 ids ascending in registers (odd-even transposition network).
-__device__ __forceinline__ void sort16(int (&x)[16]) {
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-#pragma unroll
-        for (int i = (r & 1); i + 1 < 16; i += 2) {
-            const int a = min(x[i], x[i + 1]), bb = max(x[i], x[i + 1]);
-            x[i] = a; x[i + 1] = bb;
-        }
-    }
-}
 
 __device__ __forceinline__ void write_all_blocks(int32_t* out, int c) {
     int4* o = reinterpret_cast<int4*>(out);
@@ -41,163 +30,6 @@ __device__ __forceinline__ void write_all_blocks(int32_t* out, int c) {
         o[q] = v;
     }
 }
-
-// ------------------------------------------------------------------ prefill, warp MMAs
-// The same selection with the scores of a 128-token query block as one dense contraction
-// S = Q_I (128 x 64, bf16) x Kbar^T (64 x c) on the tensor cores (mma.sync m16n8k16, fp32
-// accumulation). Kbar is fp32; each value is split exactly into three bf16 terms
-// (hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid): 24 significant bits), so the
-// contraction keeps fp32 accuracy. Candidates go 32 per pass: the CTA stages the pass's split
-// keys in shared memory, each warp computes the scores of its 32 queries, writes them to
-// shared memory, and thread i ranks query i's 32 new scores into its running best 15 (only
-// compares). Query blocks are taken heaviest first (block c = gridDim.x - 1 - blockIdx.x).
-constexpr int kSelPass = 32;            // candidates per pass
-constexpr int kKRow = 72;               // bf16 per staged candidate row (64 + 8: no bank conflicts)
-constexpr int kSRow = kSelPass + 1;     // floats per staged score row (odd: conflict-free row reads)
-
-__device__ __forceinline__ uint32_t split3_pack(float x0, float x1, int part) {
-    const float h0 = __bfloat162float(__float2bfloat16_rn(x0)), h1 = __bfloat162float(__float2bfloat16_rn(x1));
-    if (part == 0) return pack_bf16x2(h0, h1);
-    const float r0 = x0 - h0, r1 = x1 - h1;
-    const float m0 = __bfloat162float(__float2bfloat16_rn(r0)), m1 = __bfloat162float(__float2bfloat16_rn(r1));
-    if (part == 1) return pack_bf16x2(m0, m1);
-    return pack_bf16x2(r0 - m0, r1 - m1);
-}
-
-// Queries are the N tokens at positions P .. P + N - 1 (P = 0 for a whole prefill, P > 0 for a
-// chunk against cached blocks); query row i of q_idx and sel is position P + i. One CTA per
-// 128-token query block c that holds any of them.
-__global__ void __launch_bounds__(128, 2) select_prefill_mma_kernel(const uint16_t* __restrict__ q_idx, int64_t N,
-                                                                 int64_t P, int G, const float* __restrict__ pooled,
-                                                                 int64_t nb_cap, int32_t* __restrict__ sel) {
-    __shared__ __align__(16) uint16_t kst[3][kSelPass][kKRow];
-    __shared__ float scs[128][kSRow];
-    const int c = int(P / kBlock) + int(gridDim.x) - 1 - int(blockIdx.x), g = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gq = lane >> 2, tq = lane & 3;
-    const int64_t t = int64_t(c) * kBlock + tid;       // position
-    const bool live = t >= P && t < P + N;
-    int32_t* out = sel + ((size_t(b) * N + (live ? t - P : 0)) * G + g) * kTopK;
-    if (c + 1 <= kTopK) {
-        if (live) write_all_blocks(out, c);
-        return;
-    }
-    // A fragments of this warp's 32 query rows (m-tile m: rows 16 m + gq and + 8); rows outside
-    // the queries read a valid query row and are never written
-    uint32_t qa[2][4][4];
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-        int64_t ra = int64_t(c) * kBlock + warp * 32 + m * 16 + gq, rb = ra + 8;
-        ra = ra < P ? P : (ra < P + N ? ra : P + N - 1);
-        rb = rb < P ? P : (rb < P + N ? rb : P + N - 1);
-        const uint16_t* pa = q_idx + ((size_t(b) * N + (ra - P)) * G + g) * kIndexDim;
-        const uint16_t* pb = q_idx + ((size_t(b) * N + (rb - P)) * G + g) * kIndexDim;
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            qa[m][ks][0] = __ldg(reinterpret_cast<const uint32_t*>(pa + ks * 16 + 2 * tq));
-            qa[m][ks][1] = __ldg(reinterpret_cast<const uint32_t*>(pb + ks * 16 + 2 * tq));
-            qa[m][ks][2] = __ldg(reinterpret_cast<const uint32_t*>(pa + ks * 16 + 8 + 2 * tq));
-            qa[m][ks][3] = __ldg(reinterpret_cast<const uint32_t*>(pb + ks * 16 + 8 + 2 * tq));
-        }
-    }
-    float best[kKeep];
-    int bid[kKeep];
-#pragma unroll
-    for (int k = 0; k < kKeep; ++k) { best[k] = -INFINITY; bid[k] = 0x7fffffff; }
-
-    const float4* pk = reinterpret_cast<const float4*>(pooled + (size_t(b) * G + g) * nb_cap * kIndexDim);
-    for (int j0 = 0; j0 < c; j0 += kSelPass) {
-        const int nj = min(kSelPass, c - j0);
-        __syncthreads();                                 // the previous pass's keys have been read
-#pragma unroll
-        for (int r = 0; r < kSelPass * 16 / 128; ++r) {  // 32 candidates x 16 float4, 4 per thread
-            const int i = tid + 128 * r, cand = i >> 4, f4 = i & 15;
-            const float4 v = cand < nj ? __ldg(pk + size_t(j0 + cand) * (kIndexDim / 4) + f4) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int part = 0; part < 3; ++part) {
-                uint2 w;
-                w.x = split3_pack(v.x, v.y, part);
-                w.y = split3_pack(v.z, v.w, part);
-                *reinterpret_cast<uint2*>(&kst[part][cand][f4 * 4]) = w;
-            }
-        }
-        __syncthreads();
-        float acc[2][4][4];
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-            for (int n = 0; n < 4; ++n) acc[m][n][0] = acc[m][n][1] = acc[m][n][2] = acc[m][n][3] = 0.f;
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-#pragma unroll
-            for (int part = 0; part < 3; ++part) {
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint16_t* kr = &kst[part][n * 8 + gq][ks * 16 + 2 * tq];
-                    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr);
-                    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + 8);
-#pragma unroll
-                    for (int m = 0; m < 2; ++m)
-                        mma_bf16_16816(acc[m][n], qa[m][ks][0], qa[m][ks][1], qa[m][ks][2], qa[m][ks][3], b0, b1);
-                }
-            }
-        }
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-            for (int n = 0; n < 4; ++n) {
-                const int r = warp * 32 + m * 16 + gq, col = n * 8 + 2 * tq;
-                scs[r][col] = acc[m][n][0];
-                scs[r][col + 1] = acc[m][n][1];
-                scs[r + 8][col] = acc[m][n][2];
-                scs[r + 8][col + 1] = acc[m][n][3];
-            }
-        __syncwarp();                                    // a warp's rows are its own lanes' queries
-        // Mark the pass's candidates above the current 15th score (no branches), then insert
-        // only those, in id order: the warp runs as many insertion rounds as its busiest lane.
-        unsigned msk = 0u;
-        {
-            const float thr = best[kKeep - 1];
-#pragma unroll
-            for (int jj = 0; jj < kSelPass; ++jj)
-                msk |= (jj < nj && scs[tid][jj] > thr) ? (1u << jj) : 0u;
-        }
-        while (msk != 0u) {
-            const int jj = __ffs(msk) - 1;
-            msk &= msk - 1u;
-            const float sc = scs[tid][jj];
-            if (sc > best[kKeep - 1]) {
-                best[kKeep - 1] = sc; bid[kKeep - 1] = j0 + jj;
-#pragma unroll
-                for (int k = kKeep - 1; k > 0; --k) {
-                    if (best[k] > best[k - 1]) {
-                        float tv = best[k]; best[k] = best[k - 1]; best[k - 1] = tv;
-                        int ti = bid[k]; bid[k] = bid[k - 1]; bid[k - 1] = ti;
-                    }
-                }
-            }
-        }
-        __syncwarp();
-    }
-    if (!live) return;
-    int ids[16];
-#pragma unroll
-    for (int k = 0; k < kKeep; ++k) ids[k] = bid[k];
-    ids[15] = c;
-    sort16(ids);
-    int4* o = reinterpret_cast<int4*>(out);
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) o[q4] = make_int4(ids[4 * q4], ids[4 * q4 + 1], ids[4 * q4 + 2], ids[4 * q4 + 3]);
-}
-
-void launch_select_prefill_mma(const void* q_idx, int B, int G, int64_t N, int64_t P, const float* pooled,
-                               int64_t nb_cap, int32_t* sel, cudaStream_t st) {
-    const int64_t nqb = (P + N - 1) / kBlock - P / kBlock + 1;    // query blocks holding positions P .. P + N - 1
-    dim3 grid(static_cast<unsigned>(nqb), static_cast<unsigned>(G), static_cast<unsigned>(B));
-    count_launch();
-    select_prefill_mma_kernel<<<grid, 128, 0, st>>>(static_cast<const uint16_t*>(q_idx), N, P, G, pooled, nb_cap, sel);
-}
-
 
 // ------------------------------------------------------------------ decode, split + merge
 // One query per (sequence, group); its candidates [0, c) are split over 8 k CTAs that form k

@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(128) select_prefill_tc_kernel(const __grid_con
     ok = __syncthreads_and(ok);
     const uint32_t lane_off = uint32_t(warp * 32) << 16;
     for (int k = 0; ok && k < nchunks; ++k) {
+        __syncthreads();                                     // chunk k - 1's stashed scores all read
         if (k + 1 < nchunks) stage(k + 1);                   // its buffer's MMAs (chunk k - 1) are done
         tc_fence_before();
         if (!__syncthreads_and(ok)) { ok = false; break; }   // staged; chunk k - 1's scores all read
@@ -177,6 +178,10 @@ __global__ void __launch_bounds__(128) select_prefill_tc_kernel(const __grid_con
         waited = k + 1;
         tc_fence_after();
         const int j0 = k * kTcCand;
+        // the chunk's operand buffer is free once its MMAs are done: it stashes each thread's
+        // 32 scores of a pass (row stride 33 floats: conflict-free), so that an insertion reads
+        // its score with one shared-memory load
+        float* stash = reinterpret_cast<float*>(sm.kb[k & 1][0]) + tid * 33;
 #pragma unroll 1
         for (int q32 = 0; q32 < kTcCand / 32; ++q32) {
             uint32_t v[32];
@@ -189,12 +194,14 @@ __global__ void __launch_bounds__(128) select_prefill_tc_kernel(const __grid_con
 #pragma unroll
             for (int i = 0; i < 32; ++i)
                 msk |= (j0 + q32 * 32 + i < c && __uint_as_float(v[i]) > thr) ? (1u << i) : 0u;
+            if (__any_sync(0xffffffffu, msk != 0u)) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) stash[i] = __uint_as_float(v[i]);
+            }
             while (msk != 0u) {
                 const int i = __ffs(msk) - 1;
                 msk &= msk - 1u;
-                float sc = 0.f;
-#pragma unroll
-                for (int e = 0; e < 32; ++e) sc = e == i ? __uint_as_float(v[e]) : sc;
+                const float sc = stash[i];
                 if (sc > best[kTcKeep - 1]) {
                     best[kTcKeep - 1] = sc; bid[kTcKeep - 1] = j0 + q32 * 32 + i;
 #pragma unroll
