@@ -784,8 +784,14 @@ msa_status_t launch_attn_decode(const void* k_cache, const void* v_cache, const 
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         attr_set[fp8][dev].store(true, std::memory_order_relaxed);
     }
+    // Persistent CTAs over the (sequence, group, block) items, cut into even contiguous ranges.
+    // When the groups fill at least half the SMs, one CTA per group: no group is split, so no
+    // partial state crosses CTAs (merging split groups costs a few microseconds of tail);
+    // otherwise one CTA per SM, splitting groups to spread the bytes.
     const int64_t n_items = int64_t(B) * G * kTopK;
-    const int grid = int(n_items < num_sms() ? n_items : num_sms());   // persistent: one CTA per SM
+    const int64_t n_groups = int64_t(B) * G;
+    const int sms = num_sms();
+    const int grid = int(2 * n_groups >= sms ? (n_groups < sms ? n_groups : sms) : (n_items < sms ? n_items : sms));
     a.inv_grid = 1.0 / double(grid);
     a.inv_items = 1.0 / double(n_items);
     cudaLaunchConfig_t cfg = {};
