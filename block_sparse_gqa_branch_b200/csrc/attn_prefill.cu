@@ -220,8 +220,50 @@ __global__ void __launch_bounds__(256) csr_fill_kernel(const int32_t* __restrict
 }
 
 // ------------------------------------------------------------------ combine
-// One thread per (b, t, g, head, 32-column quarter): log-sum-exp merge of the query's
-// partials (fully-past slots 0..n-2 and the diagonal slot 15).
+// 16 floats at p[0..15] (one address each), issued back to back, streaming
+__device__ __forceinline__ void ld_cs_f1x16(const float* const (&p)[kSlots], float (&v)[kSlots]) {
+    asm volatile(
+        "ld.global.cs.f32 %0, [%16];\n\tld.global.cs.f32 %1, [%17];\n\tld.global.cs.f32 %2, [%18];\n\t"
+        "ld.global.cs.f32 %3, [%19];\n\tld.global.cs.f32 %4, [%20];\n\tld.global.cs.f32 %5, [%21];\n\t"
+        "ld.global.cs.f32 %6, [%22];\n\tld.global.cs.f32 %7, [%23];\n\tld.global.cs.f32 %8, [%24];\n\t"
+        "ld.global.cs.f32 %9, [%25];\n\tld.global.cs.f32 %10, [%26];\n\tld.global.cs.f32 %11, [%27];\n\t"
+        "ld.global.cs.f32 %12, [%28];\n\tld.global.cs.f32 %13, [%29];\n\tld.global.cs.f32 %14, [%30];\n\t"
+        "ld.global.cs.f32 %15, [%31];"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]), "=f"(v[8]),
+          "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+        : "l"(p[0]), "l"(p[1]), "l"(p[2]), "l"(p[3]), "l"(p[4]), "l"(p[5]), "l"(p[6]), "l"(p[7]), "l"(p[8]),
+          "l"(p[9]), "l"(p[10]), "l"(p[11]), "l"(p[12]), "l"(p[13]), "l"(p[14]), "l"(p[15]));
+}
+// 64 contiguous bytes at each of four addresses, issued back to back, streaming
+__device__ __forceinline__ void ld_cs_64Bx4(const uint16_t* const (&p)[4], uint4 (&v)[4][4]) {
+    asm volatile(
+        "ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%64];\n\tld.global.cs.v4.u32 {%4, %5, %6, %7}, [%64+16];\n\t"
+        "ld.global.cs.v4.u32 {%8, %9, %10, %11}, [%64+32];\n\tld.global.cs.v4.u32 {%12, %13, %14, %15}, [%64+48];\n\t"
+        "ld.global.cs.v4.u32 {%16, %17, %18, %19}, [%65];\n\tld.global.cs.v4.u32 {%20, %21, %22, %23}, [%65+16];\n\t"
+        "ld.global.cs.v4.u32 {%24, %25, %26, %27}, [%65+32];\n\tld.global.cs.v4.u32 {%28, %29, %30, %31}, [%65+48];\n\t"
+        "ld.global.cs.v4.u32 {%32, %33, %34, %35}, [%66];\n\tld.global.cs.v4.u32 {%36, %37, %38, %39}, [%66+16];\n\t"
+        "ld.global.cs.v4.u32 {%40, %41, %42, %43}, [%66+32];\n\tld.global.cs.v4.u32 {%44, %45, %46, %47}, [%66+48];\n\t"
+        "ld.global.cs.v4.u32 {%48, %49, %50, %51}, [%67];\n\tld.global.cs.v4.u32 {%52, %53, %54, %55}, [%67+16];\n\t"
+        "ld.global.cs.v4.u32 {%56, %57, %58, %59}, [%67+32];\n\tld.global.cs.v4.u32 {%60, %61, %62, %63}, [%67+48];"
+        : "=r"(v[0][0].x), "=r"(v[0][0].y), "=r"(v[0][0].z), "=r"(v[0][0].w), "=r"(v[0][1].x), "=r"(v[0][1].y),
+          "=r"(v[0][1].z), "=r"(v[0][1].w), "=r"(v[0][2].x), "=r"(v[0][2].y), "=r"(v[0][2].z), "=r"(v[0][2].w),
+          "=r"(v[0][3].x), "=r"(v[0][3].y), "=r"(v[0][3].z), "=r"(v[0][3].w), "=r"(v[1][0].x), "=r"(v[1][0].y),
+          "=r"(v[1][0].z), "=r"(v[1][0].w), "=r"(v[1][1].x), "=r"(v[1][1].y), "=r"(v[1][1].z), "=r"(v[1][1].w),
+          "=r"(v[1][2].x), "=r"(v[1][2].y), "=r"(v[1][2].z), "=r"(v[1][2].w), "=r"(v[1][3].x), "=r"(v[1][3].y),
+          "=r"(v[1][3].z), "=r"(v[1][3].w), "=r"(v[2][0].x), "=r"(v[2][0].y), "=r"(v[2][0].z), "=r"(v[2][0].w),
+          "=r"(v[2][1].x), "=r"(v[2][1].y), "=r"(v[2][1].z), "=r"(v[2][1].w), "=r"(v[2][2].x), "=r"(v[2][2].y),
+          "=r"(v[2][2].z), "=r"(v[2][2].w), "=r"(v[2][3].x), "=r"(v[2][3].y), "=r"(v[2][3].z), "=r"(v[2][3].w),
+          "=r"(v[3][0].x), "=r"(v[3][0].y), "=r"(v[3][0].z), "=r"(v[3][0].w), "=r"(v[3][1].x), "=r"(v[3][1].y),
+          "=r"(v[3][1].z), "=r"(v[3][1].w), "=r"(v[3][2].x), "=r"(v[3][2].y), "=r"(v[3][2].z), "=r"(v[3][2].w),
+          "=r"(v[3][3].x), "=r"(v[3][3].y), "=r"(v[3][3].z), "=r"(v[3][3].w)
+        : "l"(p[0]), "l"(p[1]), "l"(p[2]), "l"(p[3]));
+}
+
+// One thread per (b, t, g, head, 32-column quarter): log-sum-exp merge of the query's partials
+// (fully-past slots 0..n-2 and the diagonal slot 15). Every slot's log-sum-exp and 64 bytes of
+// o are requested before any is used (1 KB in flight per thread: the merge runs on a few SMs
+// beside the attention and needs deep memory pipelines there); the slots a query does not use
+// are read but weighed out with zero.
 __device__ __forceinline__ void combine_one(const int32_t* __restrict__ sel, const float* __restrict__ part_lse,
                                             const uint16_t* __restrict__ part_o, int64_t N, int G, int Hg,
                                             uint16_t* __restrict__ out, float* __restrict__ lse, int64_t gid) {
@@ -230,6 +272,20 @@ __device__ __forceinline__ void combine_one(const int32_t* __restrict__ sel, con
     const int64_t btg = (gid >> 2) / Hg;                   // (b * N + t) * G + g
     const int g = int(btg % G);
     const int64_t bt = btg / G;
+    const size_t pbase = size_t(btg) * kSlots;
+    const float* lp[kSlots];
+#pragma unroll
+    for (int s = 0; s < kSlots; ++s) lp[s] = part_lse + (pbase + s) * Hg + h;
+    float lse_s[kSlots];
+    ld_cs_f1x16(lp, lse_s);
+    uint4 x[kSlots][4];
+#pragma unroll
+    for (int s4 = 0; s4 < kSlots; s4 += 4) {
+        const uint16_t* op[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) op[i] = part_o + ((pbase + s4 + i) * Hg + h) * kHeadDim + q4 * 32;
+        ld_cs_64Bx4(op, *reinterpret_cast<uint4(*)[4][4]>(&x[s4][0]));
+    }
     const int4* srow = reinterpret_cast<const int4*>(sel + size_t(btg) * kTopK);
     int nsel = 0;
 #pragma unroll
@@ -237,28 +293,25 @@ __device__ __forceinline__ void combine_one(const int32_t* __restrict__ sel, con
         const int4 v = __ldg(srow + q);
         nsel += (v.x >= 0) + (v.y >= 0) + (v.z >= 0) + (v.w >= 0);
     }
-    const size_t pbase = size_t(btg) * kSlots;
-    float lse_s[kSlots];
     float M = -INFINITY;
 #pragma unroll
     for (int s = 0; s < kSlots; ++s) {
         const bool use = (s == kDiagSlot) || (s < nsel - 1);
-        lse_s[s] = use ? __ldcs(part_lse + (pbase + s) * Hg + h) : -INFINITY;
+        lse_s[s] = use ? lse_s[s] : -INFINITY;
         M = fmaxf(M, lse_s[s]);
     }
     float acc[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc[i] = 0.f;
     float L = 0.f;
-#pragma unroll 4
+#pragma unroll
     for (int s = 0; s < kSlots; ++s) {
-        if (lse_s[s] == -INFINITY) continue;
-        const float wgt = fast_exp2(lse_s[s] - M);
+        const bool use = lse_s[s] != -INFINITY;
+        const float wgt = use ? fast_exp2(lse_s[s] - M) : 0.f;
         L += wgt;
-        const uint4* src = reinterpret_cast<const uint4*>(part_o + ((pbase + s) * Hg + h) * kHeadDim + q4 * 32);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const uint4 u = __ldcs(src + q);
+            const uint4 u = use ? x[s][q] : make_uint4(0u, 0u, 0u, 0u);   // unused slots may hold anything
             acc[8 * q + 0] = fmaf(wgt, bf16_lo(u.x), acc[8 * q + 0]);
             acc[8 * q + 1] = fmaf(wgt, bf16_hi(u.x), acc[8 * q + 1]);
             acc[8 * q + 2] = fmaf(wgt, bf16_lo(u.y), acc[8 * q + 2]);

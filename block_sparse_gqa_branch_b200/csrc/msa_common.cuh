@@ -132,34 +132,21 @@ __device__ __forceinline__ float4 ld_nc_f4(const float4* p) {
     asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
     return v;
 }
-// 16 float4 at p, p + 32, p + 64, ... (a stride of 512 bytes)
-__device__ __forceinline__ void ld_nc_f4x16_s512(const float4* p, float4 (&v)[16]) {
+// 8 float4 at p, p + 32, ..., p + 224 (a stride of 512 bytes)
+__device__ __forceinline__ void ld_nc_f4x8_s512(const float4* p, float4 (&v)[8]) {
     asm volatile(
-        "ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%64];\n\t"
-        "ld.global.nc.v4.f32 {%4, %5, %6, %7}, [%64+512];\n\t"
-        "ld.global.nc.v4.f32 {%8, %9, %10, %11}, [%64+1024];\n\t"
-        "ld.global.nc.v4.f32 {%12, %13, %14, %15}, [%64+1536];\n\t"
-        "ld.global.nc.v4.f32 {%16, %17, %18, %19}, [%64+2048];\n\t"
-        "ld.global.nc.v4.f32 {%20, %21, %22, %23}, [%64+2560];\n\t"
-        "ld.global.nc.v4.f32 {%24, %25, %26, %27}, [%64+3072];\n\t"
-        "ld.global.nc.v4.f32 {%28, %29, %30, %31}, [%64+3584];\n\t"
-        "ld.global.nc.v4.f32 {%32, %33, %34, %35}, [%64+4096];\n\t"
-        "ld.global.nc.v4.f32 {%36, %37, %38, %39}, [%64+4608];\n\t"
-        "ld.global.nc.v4.f32 {%40, %41, %42, %43}, [%64+5120];\n\t"
-        "ld.global.nc.v4.f32 {%44, %45, %46, %47}, [%64+5632];\n\t"
-        "ld.global.nc.v4.f32 {%48, %49, %50, %51}, [%64+6144];\n\t"
-        "ld.global.nc.v4.f32 {%52, %53, %54, %55}, [%64+6656];\n\t"
-        "ld.global.nc.v4.f32 {%56, %57, %58, %59}, [%64+7168];\n\t"
-        "ld.global.nc.v4.f32 {%60, %61, %62, %63}, [%64+7680];"
+        "ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%32];\n\t"
+        "ld.global.nc.v4.f32 {%4, %5, %6, %7}, [%32+512];\n\t"
+        "ld.global.nc.v4.f32 {%8, %9, %10, %11}, [%32+1024];\n\t"
+        "ld.global.nc.v4.f32 {%12, %13, %14, %15}, [%32+1536];\n\t"
+        "ld.global.nc.v4.f32 {%16, %17, %18, %19}, [%32+2048];\n\t"
+        "ld.global.nc.v4.f32 {%20, %21, %22, %23}, [%32+2560];\n\t"
+        "ld.global.nc.v4.f32 {%24, %25, %26, %27}, [%32+3072];\n\t"
+        "ld.global.nc.v4.f32 {%28, %29, %30, %31}, [%32+3584];"
         : "=f"(v[0].x), "=f"(v[0].y), "=f"(v[0].z), "=f"(v[0].w), "=f"(v[1].x), "=f"(v[1].y), "=f"(v[1].z), "=f"(v[1].w),
           "=f"(v[2].x), "=f"(v[2].y), "=f"(v[2].z), "=f"(v[2].w), "=f"(v[3].x), "=f"(v[3].y), "=f"(v[3].z), "=f"(v[3].w),
           "=f"(v[4].x), "=f"(v[4].y), "=f"(v[4].z), "=f"(v[4].w), "=f"(v[5].x), "=f"(v[5].y), "=f"(v[5].z), "=f"(v[5].w),
-          "=f"(v[6].x), "=f"(v[6].y), "=f"(v[6].z), "=f"(v[6].w), "=f"(v[7].x), "=f"(v[7].y), "=f"(v[7].z), "=f"(v[7].w),
-          "=f"(v[8].x), "=f"(v[8].y), "=f"(v[8].z), "=f"(v[8].w), "=f"(v[9].x), "=f"(v[9].y), "=f"(v[9].z), "=f"(v[9].w),
-          "=f"(v[10].x), "=f"(v[10].y), "=f"(v[10].z), "=f"(v[10].w), "=f"(v[11].x), "=f"(v[11].y), "=f"(v[11].z),
-          "=f"(v[11].w), "=f"(v[12].x), "=f"(v[12].y), "=f"(v[12].z), "=f"(v[12].w), "=f"(v[13].x), "=f"(v[13].y),
-          "=f"(v[13].z), "=f"(v[13].w), "=f"(v[14].x), "=f"(v[14].y), "=f"(v[14].z), "=f"(v[14].w), "=f"(v[15].x),
-          "=f"(v[15].y), "=f"(v[15].z), "=f"(v[15].w)
+          "=f"(v[6].x), "=f"(v[6].y), "=f"(v[6].z), "=f"(v[6].w), "=f"(v[7].x), "=f"(v[7].y), "=f"(v[7].z), "=f"(v[7].w)
         : "l"(p));
 }
 // 16 float2 at p, p + 4, p + 8, ... (a stride of 32 bytes), from L2

@@ -83,7 +83,7 @@ __device__ __forceinline__ void merge8(unsigned long long (*l)[16], int n) {
     }
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_decode_kernel(
+__global__ void __launch_bounds__(kSelThreads, 8) select_decode_kernel(
     const uint16_t* __restrict__ q_idx, const int32_t* __restrict__ q_pos, int64_t max_pos, int G,
     const float* __restrict__ pooled, int64_t nb_cap, int32_t* __restrict__ sel,
     unsigned long long* __restrict__ cand, unsigned int* __restrict__ ctr, WsHeader* hdr) {
@@ -128,28 +128,33 @@ __global__ void __launch_bounds__(kSelThreads) select_decode_kernel(
     unsigned long long best = 0ull;                      // lanes 0-15: this warp's best 16
     for (int base = lo; base < hi; base += kSelThreads) {
         const int r0 = base + wid * 32;                  // this warp's 32 rows
-        // all 16 loads of the lane go out before any is used; in the span's last pass rows past
-        // the span read its last row and are ignored
-        float4 v[16];
-        if (base + kSelThreads <= hi) {
-            ld_nc_f4x16_s512(rows + size_t(r0 + half) * (kIndexDim / 4) + part, v);
-        } else {
+        // the lane's 16 rows in two halves of 8: each half's loads go out back to back and are
+        // scored before the next half is loaded (64 registers, so that eight CTAs fit on an SM
+        // and a whole decode batch runs in one wave); in the span's last pass rows past the span
+        // read its last row and are ignored
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = r0 + 2 * i + half;
-                v[i] = ld_nc_f4(rows + size_t(r < hi ? r : hi - 1) * (kIndexDim / 4) + part);
+        for (int hb = 0; hb < 2; ++hb) {
+            float4 v[8];
+            if (base + kSelThreads <= hi) {
+                ld_nc_f4x8_s512(rows + size_t(r0 + 16 * hb + half) * (kIndexDim / 4) + part, v);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = r0 + 16 * hb + 2 * i + half;
+                    v[i] = ld_nc_f4(rows + size_t(r < hi ? r : hi - 1) * (kIndexDim / 4) + part);
+                }
             }
-        }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            // fixed order: x, y, z, w, then a butterfly over the 16 lanes of this half-warp
-            float d = fmaf(qv.x, v[i].x, 0.f);
-            d = fmaf(qv.y, v[i].y, d);
-            d = fmaf(qv.z, v[i].z, d);
-            d = fmaf(qv.w, v[i].w, d);
+            for (int i = 0; i < 8; ++i) {
+                // fixed order: x, y, z, w, then a butterfly over the 16 lanes of this half-warp
+                float d = fmaf(qv.x, v[i].x, 0.f);
+                d = fmaf(qv.y, v[i].y, d);
+                d = fmaf(qv.z, v[i].z, d);
+                d = fmaf(qv.w, v[i].w, d);
 #pragma unroll
-            for (int off = 8; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-            if (part == 0) sc[wid * 32 + 2 * i + half] = d;
+                for (int off = 8; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+                if (part == 0) sc[wid * 32 + 16 * hb + 2 * i + half] = d;
+            }
         }
         __syncwarp();
         const int j = r0 + lane;
