@@ -231,6 +231,7 @@ size_t msa_workspace_size(const msa_shape_t* shape, int32_t op, int64_t n) { ret
 
 msa_status_t msa_pool_index_keys(const msa_shape_t* shape, const void* k_idx, int64_t n_tokens, float* pooled,
                                  int64_t nb_cap, float* tail_sum, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
     MSA_REQ(n_tokens >= 0 && n_tokens < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
     MSA_REQ(n_tokens == 0 || (k_idx != nullptr && aligned16(k_idx)), MSA_ERR_INVALID_ARGUMENT);
@@ -245,6 +246,7 @@ msa_status_t msa_pool_index_keys(const msa_shape_t* shape, const void* k_idx, in
 msa_status_t msa_index_select(const msa_shape_t* shape, const void* q_idx, int64_t n_queries, const int32_t* q_pos,
                               int64_t max_pos, const float* pooled, int64_t nb_cap, int32_t* sel, void* workspace,
                               size_t workspace_bytes, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
     MSA_REQ(q_idx != nullptr && aligned16(q_idx) && sel != nullptr && aligned16(sel), MSA_ERR_INVALID_ARGUMENT);
     MSA_REQ(pooled == nullptr ? max_pos < kBlock : aligned16(pooled), MSA_ERR_INVALID_ARGUMENT);
@@ -309,6 +311,7 @@ extern "C" {
 msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const void* q, const void* k, const void* v,
                                      int64_t n_tokens, const int32_t* sel, void* out, float* lse, void* workspace,
                                      size_t workspace_bytes, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     return attn_prefill_impl(shape, q, k, v, n_tokens, 0, n_tokens, sel, out, lse, workspace, workspace_bytes,
                              stream);
 }
@@ -317,6 +320,7 @@ msa_status_t msa_sparse_attn_prefill_backward(const msa_shape_t* shape, const vo
                                               int64_t n_tokens, const int32_t* sel, const void* out, const float* lse,
                                               const void* d_out, float* dq, float* dk, float* dv, void* workspace,
                                               size_t workspace_bytes, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
     MSA_REQ(n_tokens >= 1 && n_tokens < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
     MSA_REQ(q && k && v && sel && out && lse && d_out && dq && dk && dv && aligned16(q) && aligned16(k) &&
@@ -343,6 +347,7 @@ size_t msa_prefill_chunk_workspace_size(const msa_shape_t* shape, int64_t q_star
 
 msa_status_t msa_pool_index_keys_chunk(const msa_shape_t* shape, const void* k_idx, int64_t q_start, int64_t n,
                                        float* pooled, int64_t nb_cap, float* tail_sum, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
     MSA_REQ(n >= 1 && q_start >= 0 && q_start + n < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
     MSA_REQ(k_idx && aligned16(k_idx) && tail_sum && aligned16(tail_sum), MSA_ERR_INVALID_ARGUMENT);
@@ -357,6 +362,7 @@ msa_status_t msa_pool_index_keys_chunk(const msa_shape_t* shape, const void* k_i
 msa_status_t msa_index_select_chunk(const msa_shape_t* shape, const void* q_idx, int64_t q_start, int64_t n,
                                     const float* pooled, int64_t nb_cap, int32_t* sel, void* workspace,
                                     size_t workspace_bytes, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
     MSA_REQ(q_idx && aligned16(q_idx) && sel && aligned16(sel), MSA_ERR_INVALID_ARGUMENT);
     MSA_REQ(n >= 1 && q_start >= 0 && q_start + n < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
@@ -372,6 +378,7 @@ msa_status_t msa_sparse_attn_prefill_chunk(const msa_shape_t* shape, const void*
                                            const void* v_cache, int64_t l_cap, int64_t q_start, int64_t n,
                                            const int32_t* sel, void* out, float* lse, void* workspace,
                                            size_t workspace_bytes, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     return attn_prefill_impl(shape, q, k_cache, v_cache, l_cap, q_start, n, sel, out, lse, workspace,
                              workspace_bytes, stream);
 }
@@ -380,6 +387,7 @@ msa_status_t msa_pooled_keys_append(const msa_shape_t* shape, const void* k_idx_
                                     const void* v_new, const int32_t* ctx_len, void* k_cache, void* v_cache,
                                     int64_t l_cap, float* tail_sum, float* pooled, int64_t nb_cap, void* workspace,
                                     size_t workspace_bytes, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
     MSA_REQ(k_idx_new && aligned16(k_idx_new) && ctx_len && tail_sum && aligned16(tail_sum) && pooled &&
                 aligned16(pooled),
@@ -401,6 +409,7 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const void* q, con
                                     const void* v_cache, int64_t l_cap, const int32_t* q_pos, int64_t max_pos,
                                     const int32_t* sel, void* out, float* lse, void* workspace,
                                     size_t workspace_bytes, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
     MSA_REQ(q && k_cache && v_cache && q_pos && sel && out && aligned16(q) && aligned16(k_cache) &&
                 aligned16(v_cache) && aligned16(sel) && aligned16(out) &&
@@ -420,6 +429,7 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const void* q, con
 msa_status_t msa_fp8_quantize_blocks(const msa_shape_t* shape, const void* k_cache, const void* v_cache, int64_t l_cap,
                                      int64_t n_tokens, void* k_codes, void* v_codes, float* k_scale, float* v_scale,
                                      int64_t nb_cap, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
     MSA_REQ(n_tokens >= 0 && l_cap >= n_tokens && l_cap >= 1, MSA_ERR_INVALID_ARGUMENT);
     const int64_t nblk = n_tokens / kBlock;
@@ -438,6 +448,7 @@ msa_status_t msa_fp8_close_blocks(const msa_shape_t* shape, const int32_t* ctx_l
                                   const void* v_cache, int64_t l_cap, void* k_codes, void* v_codes, float* k_scale,
                                   float* v_scale, int64_t nb_cap, void* workspace, size_t workspace_bytes,
                                   msa_stream_t stream) {
+    MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
     MSA_REQ(ctx_len && k_cache && v_cache && k_codes && v_codes && k_scale && v_scale && aligned16(k_cache) &&
                 aligned16(v_cache) && aligned16(k_codes) && aligned16(v_codes) &&
@@ -455,6 +466,7 @@ msa_status_t msa_sparse_attn_decode_fp8(const msa_shape_t* shape, const void* q,
                                         int64_t nb_cap, const void* k_cache, const void* v_cache, int64_t l_cap,
                                         const int32_t* q_pos, int64_t max_pos, const int32_t* sel, void* out,
                                         float* lse, void* workspace, size_t workspace_bytes, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
     MSA_REQ(q && k_codes && v_codes && k_scale && v_scale && k_cache && v_cache && q_pos && sel && out &&
                 aligned16(q) && aligned16(k_codes) && aligned16(v_codes) && aligned16(k_cache) &&

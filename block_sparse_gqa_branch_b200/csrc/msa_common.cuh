@@ -8,9 +8,21 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "msa.h"
 
 namespace msa {
+
+// One NVTX range per C-ABI call, named for the entry point: a profiler attached to the process
+// shows each call's kernels under it; without one, push and pop return at once.
+struct CallRange {
+    explicit CallRange(const char* name) { nvtxRangePushA(name); }
+    ~CallRange() { nvtxRangePop(); }
+    CallRange(const CallRange&) = delete;
+    CallRange& operator=(const CallRange&) = delete;
+};
+#define MSA_CALL_RANGE() ::msa::CallRange msa_call_range_(__func__)
 
 // host-side count of kernels enqueued by libmsa (see msa_kernel_launches)
 void count_launch(unsigned n = 1);

@@ -312,6 +312,7 @@ extern "C" msa_status_t msa_index_select_decode_noalloc(const msa_shape_t* shape
                                                         const int32_t* q_pos, int64_t max_pos,
                                                         const float* pooled, int64_t nb_cap, int32_t* sel,
                                                         msa_stream_t stream) {
+    MSA_CALL_RANGE();
     using namespace msa;
     msa_status_t s = check_shape(shape);
     if (s != MSA_OK) return s;

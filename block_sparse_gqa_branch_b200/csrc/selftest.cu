@@ -18,6 +18,7 @@ __global__ void __launch_bounds__(32) selftest_timeout_kernel(WsHeader* hdr) {
 }  // namespace msa
 
 extern "C" msa_status_t msa_selftest_wait_timeout(void* workspace, size_t workspace_bytes, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     using namespace msa;
     if (workspace == nullptr || workspace_bytes < sizeof(WsHeader) || !aligned16(workspace)) return MSA_ERR_WORKSPACE;
     count_launch();

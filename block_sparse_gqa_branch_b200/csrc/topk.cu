@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const float* __
 
 extern "C" msa_status_t msa_topk_rows(const float* scores, int64_t rows, int64_t n, int32_t k, int32_t* idx,
                                       float* val, msa_stream_t stream) {
+    MSA_CALL_RANGE();
     using namespace msa;
     if (rows < 0 || k < 1 || k > kTopkMax || n < k || n > kTopkMaxCols) return MSA_ERR_INVALID_ARGUMENT;
     if (rows == 0) return MSA_OK;
