@@ -32,8 +32,6 @@ constexpr int kSlots = 16;              // partial slots per (token, group); slo
 constexpr int kDiagSlot = 15;
 constexpr int kDiagFlag = int(0x40000000);
 constexpr int kKvThreads = 352;         // warps 0-7 softmax/epilogue, 8 Q loads, 9 MMA, 10 K/V loads
-constexpr int kMaxSegs = 8;             // launches the (sequence, group) pairs are split into
-constexpr int kMergeCtas = 20;          // CTAs of a launch that merge the previous segment's partials
 
 static_assert(kRange % kCountChunk == 0 && kRange % kBlock == 0, "range must hold whole chunks and blocks");
 
@@ -44,7 +42,7 @@ static_assert(kRange % kCountChunk == 0 && kRange % kBlock == 0, "range must hol
 struct PrefillLayout {
     int nb, nR, nbins_seg, tpt;     // nb: key blocks that can be selected (ceil((P + n) / Bk))
     size_t nbins, max_items, max_entries;
-    size_t off_counts, off_offsets, off_nitems, off_pairs, off_items, off_list, off_lse, off_o, total;
+    size_t off_counts, off_offsets, off_nitems, off_items, off_list, off_lse, off_o, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -66,8 +64,7 @@ PrefillLayout prefill_layout(int B, int64_t N, int G, int Hg, int64_t P) {
     size_t o = sizeof(WsHeader);
     L.off_counts = o;   o = align_up(o + L.nbins * 4, 256);
     L.off_offsets = o;  o = align_up(o + L.nbins * 4, 256);
-    L.off_nitems = o;   o = align_up(o + 4 * (2 + kMaxSegs), 256);
-    L.off_pairs = o;    o = align_up(o + 4 * (size_t(B) * G + 1), 256);
+    L.off_nitems = o;   o = align_up(o + 16, 256);
     L.off_items = o;    o = align_up(o + L.max_items * 16, 256);
     L.off_list = o;     o = align_up(o + L.max_entries * 4, 256);
     L.off_lse = o;      o = align_up(o + size_t(B) * N * G * kSlots * Hg * 4, 256);
@@ -118,8 +115,7 @@ __global__ void __launch_bounds__(256) csr_count_kernel(const int32_t* __restric
 // work items in bin order: {b*G+g, j (| kDiagFlag), first entry (or first token), count}.
 __global__ void __launch_bounds__(1024) csr_scan_kernel(int* __restrict__ counts, int* __restrict__ offsets,
                                                         int4* __restrict__ items, int* __restrict__ n_items,
-                                                        int* __restrict__ pair_start, int64_t nbins, int nb, int nR,
-                                                        int64_t N, int64_t P, int tpt) {
+                                                        int64_t nbins, int nb, int nR, int64_t N, int64_t P, int tpt) {
     __shared__ long long s_e[1024], s_i[1024];
     const int nbs = nb + 1;
     const int64_t per = (nbins + 1023) / 1024;
@@ -161,7 +157,6 @@ __global__ void __launch_bounds__(1024) csr_scan_kernel(int* __restrict__ counts
         const int64_t seg = bin / nbs;
         const int R = int(seg % nR);
         const int bg = int(seg / nR);
-        if (j == 0 && R == 0) pair_start[bg] = int(ioff);     // first item of (sequence, group) bg
         if (j < nb) {
             const int cnt = counts[bin];
             offsets[bin] = int(eoff);
@@ -183,9 +178,7 @@ __global__ void __launch_bounds__(1024) csr_scan_kernel(int* __restrict__ counts
     }
     if (threadIdx.x == 1023) {
         n_items[0] = int(ioff);
-        n_items[1] = 0;                                   // work-item counter of a single pass over all items
-        for (int s = 0; s < kMaxSegs; ++s) n_items[2 + s] = 0;   // counters of the segmented passes
-        pair_start[nbins / (int64_t(nR) * nbs)] = int(ioff);
+        n_items[1] = 0;                                   // work-item counter of the tensor-core kernel
     }
 }
 
@@ -219,124 +212,6 @@ __global__ void __launch_bounds__(256) csr_fill_kernel(const int32_t* __restrict
     }
 }
 
-// ------------------------------------------------------------------ combine
-// 16 floats at p[0..15] (one address each), issued back to back, streaming
-__device__ __forceinline__ void ld_cs_f1x16(const float* const (&p)[kSlots], float (&v)[kSlots]) {
-    asm volatile(
-        "ld.global.cs.f32 %0, [%16];\n\tld.global.cs.f32 %1, [%17];\n\tld.global.cs.f32 %2, [%18];\n\t"
-        "ld.global.cs.f32 %3, [%19];\n\tld.global.cs.f32 %4, [%20];\n\tld.global.cs.f32 %5, [%21];\n\t"
-        "ld.global.cs.f32 %6, [%22];\n\tld.global.cs.f32 %7, [%23];\n\tld.global.cs.f32 %8, [%24];\n\t"
-        "ld.global.cs.f32 %9, [%25];\n\tld.global.cs.f32 %10, [%26];\n\tld.global.cs.f32 %11, [%27];\n\t"
-        "ld.global.cs.f32 %12, [%28];\n\tld.global.cs.f32 %13, [%29];\n\tld.global.cs.f32 %14, [%30];\n\t"
-        "ld.global.cs.f32 %15, [%31];"
-        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]), "=f"(v[8]),
-          "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
-        : "l"(p[0]), "l"(p[1]), "l"(p[2]), "l"(p[3]), "l"(p[4]), "l"(p[5]), "l"(p[6]), "l"(p[7]), "l"(p[8]),
-          "l"(p[9]), "l"(p[10]), "l"(p[11]), "l"(p[12]), "l"(p[13]), "l"(p[14]), "l"(p[15]));
-}
-// 64 contiguous bytes at each of four addresses, issued back to back, streaming
-__device__ __forceinline__ void ld_cs_64Bx4(const uint16_t* const (&p)[4], uint4 (&v)[4][4]) {
-    asm volatile(
-        "ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%64];\n\tld.global.cs.v4.u32 {%4, %5, %6, %7}, [%64+16];\n\t"
-        "ld.global.cs.v4.u32 {%8, %9, %10, %11}, [%64+32];\n\tld.global.cs.v4.u32 {%12, %13, %14, %15}, [%64+48];\n\t"
-        "ld.global.cs.v4.u32 {%16, %17, %18, %19}, [%65];\n\tld.global.cs.v4.u32 {%20, %21, %22, %23}, [%65+16];\n\t"
-        "ld.global.cs.v4.u32 {%24, %25, %26, %27}, [%65+32];\n\tld.global.cs.v4.u32 {%28, %29, %30, %31}, [%65+48];\n\t"
-        "ld.global.cs.v4.u32 {%32, %33, %34, %35}, [%66];\n\tld.global.cs.v4.u32 {%36, %37, %38, %39}, [%66+16];\n\t"
-        "ld.global.cs.v4.u32 {%40, %41, %42, %43}, [%66+32];\n\tld.global.cs.v4.u32 {%44, %45, %46, %47}, [%66+48];\n\t"
-        "ld.global.cs.v4.u32 {%48, %49, %50, %51}, [%67];\n\tld.global.cs.v4.u32 {%52, %53, %54, %55}, [%67+16];\n\t"
-        "ld.global.cs.v4.u32 {%56, %57, %58, %59}, [%67+32];\n\tld.global.cs.v4.u32 {%60, %61, %62, %63}, [%67+48];"
-        : "=r"(v[0][0].x), "=r"(v[0][0].y), "=r"(v[0][0].z), "=r"(v[0][0].w), "=r"(v[0][1].x), "=r"(v[0][1].y),
-          "=r"(v[0][1].z), "=r"(v[0][1].w), "=r"(v[0][2].x), "=r"(v[0][2].y), "=r"(v[0][2].z), "=r"(v[0][2].w),
-          "=r"(v[0][3].x), "=r"(v[0][3].y), "=r"(v[0][3].z), "=r"(v[0][3].w), "=r"(v[1][0].x), "=r"(v[1][0].y),
-          "=r"(v[1][0].z), "=r"(v[1][0].w), "=r"(v[1][1].x), "=r"(v[1][1].y), "=r"(v[1][1].z), "=r"(v[1][1].w),
-          "=r"(v[1][2].x), "=r"(v[1][2].y), "=r"(v[1][2].z), "=r"(v[1][2].w), "=r"(v[1][3].x), "=r"(v[1][3].y),
-          "=r"(v[1][3].z), "=r"(v[1][3].w), "=r"(v[2][0].x), "=r"(v[2][0].y), "=r"(v[2][0].z), "=r"(v[2][0].w),
-          "=r"(v[2][1].x), "=r"(v[2][1].y), "=r"(v[2][1].z), "=r"(v[2][1].w), "=r"(v[2][2].x), "=r"(v[2][2].y),
-          "=r"(v[2][2].z), "=r"(v[2][2].w), "=r"(v[2][3].x), "=r"(v[2][3].y), "=r"(v[2][3].z), "=r"(v[2][3].w),
-          "=r"(v[3][0].x), "=r"(v[3][0].y), "=r"(v[3][0].z), "=r"(v[3][0].w), "=r"(v[3][1].x), "=r"(v[3][1].y),
-          "=r"(v[3][1].z), "=r"(v[3][1].w), "=r"(v[3][2].x), "=r"(v[3][2].y), "=r"(v[3][2].z), "=r"(v[3][2].w),
-          "=r"(v[3][3].x), "=r"(v[3][3].y), "=r"(v[3][3].z), "=r"(v[3][3].w)
-        : "l"(p[0]), "l"(p[1]), "l"(p[2]), "l"(p[3]));
-}
-
-// One thread per (b, t, g, head, 32-column quarter): log-sum-exp merge of the query's partials
-// (fully-past slots 0..n-2 and the diagonal slot 15). Every slot's log-sum-exp and 64 bytes of
-// o are requested before any is used (1 KB in flight per thread: the merge runs on a few SMs
-// beside the attention and needs deep memory pipelines there); the slots a query does not use
-// are read but weighed out with zero.
-__device__ __forceinline__ void combine_one(const int32_t* __restrict__ sel, const float* __restrict__ part_lse,
-                                            const uint16_t* __restrict__ part_o, int64_t N, int G, int Hg,
-                                            uint16_t* __restrict__ out, float* __restrict__ lse, int64_t gid) {
-    const int q4 = int(gid & 3);
-    const int h = int((gid >> 2) % Hg);
-    const int64_t btg = (gid >> 2) / Hg;                   // (b * N + t) * G + g
-    const int g = int(btg % G);
-    const int64_t bt = btg / G;
-    const size_t pbase = size_t(btg) * kSlots;
-    const float* lp[kSlots];
-#pragma unroll
-    for (int s = 0; s < kSlots; ++s) lp[s] = part_lse + (pbase + s) * Hg + h;
-    float lse_s[kSlots];
-    ld_cs_f1x16(lp, lse_s);
-    uint4 x[kSlots][4];
-#pragma unroll
-    for (int s4 = 0; s4 < kSlots; s4 += 4) {
-        const uint16_t* op[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) op[i] = part_o + ((pbase + s4 + i) * Hg + h) * kHeadDim + q4 * 32;
-        ld_cs_64Bx4(op, *reinterpret_cast<uint4(*)[4][4]>(&x[s4][0]));
-    }
-    const int4* srow = reinterpret_cast<const int4*>(sel + size_t(btg) * kTopK);
-    int nsel = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int4 v = __ldg(srow + q);
-        nsel += (v.x >= 0) + (v.y >= 0) + (v.z >= 0) + (v.w >= 0);
-    }
-    float M = -INFINITY;
-#pragma unroll
-    for (int s = 0; s < kSlots; ++s) {
-        const bool use = (s == kDiagSlot) || (s < nsel - 1);
-        lse_s[s] = use ? lse_s[s] : -INFINITY;
-        M = fmaxf(M, lse_s[s]);
-    }
-    float acc[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-    float L = 0.f;
-#pragma unroll
-    for (int s = 0; s < kSlots; ++s) {
-        const bool use = lse_s[s] != -INFINITY;
-        const float wgt = use ? fast_exp2(lse_s[s] - M) : 0.f;
-        L += wgt;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint4 u = use ? x[s][q] : make_uint4(0u, 0u, 0u, 0u);   // unused slots may hold anything
-            acc[8 * q + 0] = fmaf(wgt, bf16_lo(u.x), acc[8 * q + 0]);
-            acc[8 * q + 1] = fmaf(wgt, bf16_hi(u.x), acc[8 * q + 1]);
-            acc[8 * q + 2] = fmaf(wgt, bf16_lo(u.y), acc[8 * q + 2]);
-            acc[8 * q + 3] = fmaf(wgt, bf16_hi(u.y), acc[8 * q + 3]);
-            acc[8 * q + 4] = fmaf(wgt, bf16_lo(u.z), acc[8 * q + 4]);
-            acc[8 * q + 5] = fmaf(wgt, bf16_hi(u.z), acc[8 * q + 5]);
-            acc[8 * q + 6] = fmaf(wgt, bf16_lo(u.w), acc[8 * q + 6]);
-            acc[8 * q + 7] = fmaf(wgt, bf16_hi(u.w), acc[8 * q + 7]);
-        }
-    }
-    const float inv = 1.f / L;
-    const int Hq = G * Hg;
-    uint4* dst = reinterpret_cast<uint4*>(out + ((size_t(bt) * Hq + size_t(g) * Hg + h) * kHeadDim) + q4 * 32);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint4 o;
-        o.x = pack_bf16x2(acc[8 * q + 0] * inv, acc[8 * q + 1] * inv);
-        o.y = pack_bf16x2(acc[8 * q + 2] * inv, acc[8 * q + 3] * inv);
-        o.z = pack_bf16x2(acc[8 * q + 4] * inv, acc[8 * q + 5] * inv);
-        o.w = pack_bf16x2(acc[8 * q + 6] * inv, acc[8 * q + 7] * inv);
-        dst[q] = o;
-    }
-    if (lse != nullptr && q4 == 0) lse[size_t(bt) * Hq + size_t(g) * Hg + h] = (M + __log2f(L)) * 0.69314718055994530942f;
-}
-
 // ------------------------------------------------------------------ the tensor-core kernel
 constexpr int kQStages = 3;
 constexpr int kRing = 8;           // work items handed from the scheduler to the other roles
@@ -359,14 +234,7 @@ struct PrefillArgs {
     int64_t N;                     // queries per sequence (positions P .. P + N - 1)
     int64_t P;                     // position of the first query
     int G, Hg, Hq, tpt;
-    int* n_items;                  // [0] = number of work items, [2 + s] = next item of segment s
-    const int* pair_start;         // first item of every (sequence, group) pair; [B G] = number of items
-    int n_pairs, n_segs;           // B G pairs, split into n_segs contiguous segments
-    int seg_attn, seg_merge;       // this launch: attention of segment seg_attn, merge of seg_merge (-1: none)
-    int n_attn_ctas;               // CTAs [0, n_attn_ctas) attend, the others merge
-    const int32_t* sel;            // merge: selection rows, output and lse
-    uint16_t* out;
-    float* lse;
+    int* n_items;                  // [0] = number of work items, [1] = next item to hand out
     const int4* items;
     const int* list;
     float* part_lse;
@@ -539,28 +407,9 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
                                                                      const __grid_constant__ CUtensorMap tmO,
                                                                      const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    if (int(blockIdx.x) >= a.n_attn_ctas) {
-        // merge CTAs: the partials of segment seg_merge, whose attention finished in the previous
-        // launch on this stream
-        const int p0 = a.seg_merge * a.n_pairs / a.n_segs, p1 = (a.seg_merge + 1) * a.n_pairs / a.n_segs;
-        const int64_t per_pair = a.N * a.Hg * 4;
-        const int64_t total = int64_t(p1 - p0) * per_pair;
-        const int64_t stride = int64_t(gridDim.x - a.n_attn_ctas) * blockDim.x;
-        for (int64_t i = int64_t(blockIdx.x - a.n_attn_ctas) * blockDim.x + threadIdx.x; i < total; i += stride) {
-            const int bg = p0 + int(i / per_pair);
-            const int64_t r = i % per_pair;             // (t, h, quarter) within the pair
-            const int64_t t = r / (a.Hg * 4);
-            const int b = bg / a.G, g = bg % a.G;
-            const int64_t gid = (((int64_t(b) * a.N + t) * a.G + g) * a.Hg + (r / 4) % a.Hg) * 4 + (r & 3);
-            combine_one(a.sel, a.part_lse, a.part_o, a.N, a.G, a.Hg, a.out, a.lse, gid);
-        }
-        return;
-    }
     KvSmem& sm = *reinterpret_cast<KvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // this launch's items: those of the pairs of segment seg_attn
-    const int item_lo = a.pair_start[a.seg_attn * a.n_pairs / a.n_segs];
-    const int item_hi = a.pair_start[(a.seg_attn + 1) * a.n_pairs / a.n_segs];
+    const int n_items = *a.n_items;
     const int tpt = a.tpt, Hg = a.Hg;
 
     if (threadIdx.x == 0) {
@@ -656,8 +505,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
                     sm.abort_flag = 1;
                     break;
                 }
-                int k = item_lo + atomicAdd(a.n_items + 2 + a.seg_attn, 1);
-                if (k >= item_hi) k = -1;
+                int k = atomicAdd(a.n_items + 1, 1);
+                if (k >= n_items) k = -1;
                 sm.item_ring[slot] = k;
                 mbar_arrive(&sm.item_full[slot]);
                 if (k < 0) break;
@@ -842,6 +691,75 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
     }
 }
 
+// ------------------------------------------------------------------ combine
+// One thread per (b, t, g, head, 32-column quarter): log-sum-exp merge of the query's
+// partials (fully-past slots 0..n-2 and the diagonal slot 15).
+__global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict__ sel,
+                                                      const float* __restrict__ part_lse,
+                                                      const uint16_t* __restrict__ part_o, int64_t N, int G,
+                                                      int Hg, uint16_t* __restrict__ out, float* __restrict__ lse,
+                                                      int64_t total) {
+    const int64_t gid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (gid >= total) return;
+    const int q4 = int(gid & 3);
+    const int h = int((gid >> 2) % Hg);
+    const int64_t btg = (gid >> 2) / Hg;                   // (b * N + t) * G + g
+    const int g = int(btg % G);
+    const int64_t bt = btg / G;
+    const int4* srow = reinterpret_cast<const int4*>(sel + size_t(btg) * kTopK);
+    int nsel = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int4 v = __ldg(srow + q);
+        nsel += (v.x >= 0) + (v.y >= 0) + (v.z >= 0) + (v.w >= 0);
+    }
+    const size_t pbase = size_t(btg) * kSlots;
+    float lse_s[kSlots];
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kSlots; ++s) {
+        const bool use = (s == kDiagSlot) || (s < nsel - 1);
+        lse_s[s] = use ? __ldcs(part_lse + (pbase + s) * Hg + h) : -INFINITY;
+        M = fmaxf(M, lse_s[s]);
+    }
+    float acc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+    float L = 0.f;
+#pragma unroll 4
+    for (int s = 0; s < kSlots; ++s) {
+        if (lse_s[s] == -INFINITY) continue;
+        const float wgt = fast_exp2(lse_s[s] - M);
+        L += wgt;
+        const uint4* src = reinterpret_cast<const uint4*>(part_o + ((pbase + s) * Hg + h) * kHeadDim + q4 * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 u = __ldcs(src + q);
+            acc[8 * q + 0] = fmaf(wgt, bf16_lo(u.x), acc[8 * q + 0]);
+            acc[8 * q + 1] = fmaf(wgt, bf16_hi(u.x), acc[8 * q + 1]);
+            acc[8 * q + 2] = fmaf(wgt, bf16_lo(u.y), acc[8 * q + 2]);
+            acc[8 * q + 3] = fmaf(wgt, bf16_hi(u.y), acc[8 * q + 3]);
+            acc[8 * q + 4] = fmaf(wgt, bf16_lo(u.z), acc[8 * q + 4]);
+            acc[8 * q + 5] = fmaf(wgt, bf16_hi(u.z), acc[8 * q + 5]);
+            acc[8 * q + 6] = fmaf(wgt, bf16_lo(u.w), acc[8 * q + 6]);
+            acc[8 * q + 7] = fmaf(wgt, bf16_hi(u.w), acc[8 * q + 7]);
+        }
+    }
+    const float inv = 1.f / L;
+    const int Hq = G * Hg;
+    uint4* dst = reinterpret_cast<uint4*>(out + ((size_t(bt) * Hq + size_t(g) * Hg + h) * kHeadDim) + q4 * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 o;
+        o.x = pack_bf16x2(acc[8 * q + 0] * inv, acc[8 * q + 1] * inv);
+        o.y = pack_bf16x2(acc[8 * q + 2] * inv, acc[8 * q + 3] * inv);
+        o.z = pack_bf16x2(acc[8 * q + 4] * inv, acc[8 * q + 5] * inv);
+        o.w = pack_bf16x2(acc[8 * q + 6] * inv, acc[8 * q + 7] * inv);
+        dst[q] = o;
+    }
+    if (lse != nullptr && q4 == 0) lse[size_t(bt) * Hq + size_t(g) * Hg + h] = (M + __log2f(L)) * 0.69314718055994530942f;
+}
+
 // ------------------------------------------------------------------ host launcher
 int num_sms() {
     static std::atomic<int> n[64];                  // per device, filled on first use
@@ -885,9 +803,7 @@ void launch_inverted_index(const int32_t* sel, int64_t N, int64_t P, int B, int 
         csr_count_kernel<<<grid, 256, smem, st>>>(sel, N, P, G, L.nb, L.nR, counts, hdr);
     }
     count_launch();
-    int* pair_start = reinterpret_cast<int*>(base + L.off_pairs);
-    csr_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, items, nitems, pair_start, int64_t(L.nbins), L.nb, L.nR, N, P,
-                                        L.tpt);
+    csr_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, items, nitems, int64_t(L.nbins), L.nb, L.nR, N, P, L.tpt);
     {
         const int64_t total = int64_t(B) * N * G;
         count_launch();
@@ -903,7 +819,6 @@ msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, cons
     char* base = static_cast<char*>(ws);
     WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
     int* nitems = reinterpret_cast<int*>(base + L.off_nitems);
-    const int* pair_start = reinterpret_cast<const int*>(base + L.off_pairs);
     int4* items = reinterpret_cast<int4*>(base + L.off_items);
     int* list = reinterpret_cast<int*>(base + L.off_list);
     float* part_lse = reinterpret_cast<float*>(base + L.off_lse);
@@ -929,30 +844,15 @@ msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, cons
         if (st_map == MSA_OK && Hg >= 8) st_map = make_tmap_q_rows(&tmQ3, q, uint64_t(B) * N * G * Hg);
         if (st_map != MSA_OK) return st_map;
         const CUtensorMap& tmQ = Hg >= 8 ? tmQ3 : tmQ2;
-        // The (sequence, group) pairs are split into n_segs contiguous segments. Launch s attends
-        // segment s on most SMs while kMergeCtas CTAs merge the partials of segment s - 1 (done in
-        // the previous launch on this stream); a last launch merges the last segment on every SM.
-        // The attention is latency-bound and the merge HBM-bound, so the merge runs in its shadow.
-        const int sms = num_sms();
-        const int n_pairs = B * G;
-        const int n_segs = n_pairs < kMaxSegs ? n_pairs : kMaxSegs;
-        a.pair_start = pair_start;
-        a.n_pairs = n_pairs;
-        a.n_segs = n_segs;
-        a.sel = sel;
-        a.out = static_cast<uint16_t*>(out);
-        a.lse = lse;
-        const int n_merge_mid = kMergeCtas < sms / 4 ? kMergeCtas : (sms / 4 > 0 ? sms / 4 : 1);
-        for (int seg = 0; seg <= n_segs; ++seg) {
-            const bool attend = seg < n_segs, merge = seg > 0;
-            const int n_merge = merge ? (attend ? n_merge_mid : sms) : 0;
-            const int n_attn = attend ? sms - n_merge : 0;
-            a.seg_attn = attend ? seg : 0;
-            a.seg_merge = merge ? seg - 1 : -1;
-            a.n_attn_ctas = n_attn;
-            count_launch();
-            attn_kvmajor_kernel<<<n_attn + n_merge, kKvThreads, smem, st>>>(tmQ, tmK, tmV, tmO, a);
-        }
+        count_launch();
+        attn_kvmajor_kernel<<<num_sms(), kKvThreads, smem, st>>>(tmQ, tmK, tmV, tmO, a);
+    }
+    {
+        const int64_t total = int64_t(B) * N * G * Hg * 4;
+        count_launch();
+        combine_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(sel, part_lse, part_o, N, G, Hg,
+                                                                                  static_cast<uint16_t*>(out), lse,
+                                                                                  total);
     }
     return MSA_OK;
 }

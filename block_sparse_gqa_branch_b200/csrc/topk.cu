@@ -51,21 +51,7 @@ __device__ __forceinline__ uint32_t warp_sort_desc32(uint32_t x, int lane) {
     return x;
 }
 
-// A lane's share of the chunk at `base` of row r (n % 4 == 0) copied asynchronously into the
-// warp's staging buffer, [step][lane] float4: columns past n copy the row's first four values
-// and are masked by the reader.
-__device__ __forceinline__ void stage_chunk4(float4* buf, const float* r, int base, int n, int lane) {
-#pragma unroll
-    for (int i = 0; i < kTopkSteps; ++i) {
-        const int c0 = base + (i * 32 + lane) * 4;
-        cp_async16(smem_u32(buf + i * 32 + lane), r + (c0 < n ? c0 : 0));
-    }
-    cp_async_commit();
-}
-
-// VEC = 4: rows start 16-byte aligned (n % 4 == 0) and are read as float4; the first chunk of
-// the warp's next row is copied into shared memory (cp.async) while the current row is ranked.
-// VEC = 1 otherwise.
+// VEC = 4: rows start 16-byte aligned (n % 4 == 0) and are read as float4; VEC = 1 otherwise.
 template <int VEC>
 __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const float* __restrict__ scores, int64_t rows,
                                                                   int n, int k, int32_t* __restrict__ idx,
@@ -74,12 +60,6 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const float* __
     constexpr int kChunk = 32 * kPer;
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = int64_t(gridDim.x) * kTopkWarps;
-    __shared__ float4 staged[VEC == 4 ? kTopkWarps * kTopkSteps * 32 : 1];
-    float4* mine = staged + (VEC == 4 ? (threadIdx.x >> 5) * kTopkSteps * 32 : 0);
-    if constexpr (VEC == 4) {
-        const int64_t row0 = int64_t(blockIdx.x) * kTopkWarps + (threadIdx.x >> 5);
-        if (row0 < rows) stage_chunk4(mine, scores + row0 * n, 0, n, lane);
-    }
     for (int64_t row = int64_t(blockIdx.x) * kTopkWarps + (threadIdx.x >> 5); row < rows; row += nwarps) {
         const float* r = scores + row * n;
         unsigned long long best = 0ull;       // lanes 0-15: the best 16 keys so far, descending
@@ -87,23 +67,15 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const float* __
         for (int base = 0; base < n; base += kChunk) {
             uint32_t code[kPer];
             uint32_t valid = 0u;              // bit p: this lane's value p is a column < n
-            float4 xs[kTopkSteps];
-            if constexpr (VEC == 4) {
-                if (base != 0) stage_chunk4(mine, r, base, n, lane);   // later chunks of a long row
-                cp_async_wait<0>();
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < kTopkSteps; ++i) xs[i] = mine[i * 32 + lane];
-                __syncwarp();                 // every lane has read the buffer
-                const int64_t nxt = row + nwarps;
-                if (base + kChunk >= n && nxt < rows) stage_chunk4(mine, scores + nxt * n, 0, n, lane);
-            }
 #pragma unroll
             for (int i = 0; i < kTopkSteps; ++i) {
                 const int c0 = base + (i * 32 + lane) * VEC;
                 if constexpr (VEC == 4) {
-                    const float4 x = xs[i];
-                    if (c0 < n) valid |= 0xfu << (4 * i);
+                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (c0 < n) {
+                        x = __ldcs(reinterpret_cast<const float4*>(r + c0));
+                        valid |= 0xfu << (4 * i);
+                    }
                     code[4 * i + 0] = score_code(x.x);
                     code[4 * i + 1] = score_code(x.y);
                     code[4 * i + 2] = score_code(x.z);
