@@ -16,12 +16,14 @@
 //     Hg heads with warp MMAs, turns them into probabilities in registers (the accumulator
 //     layout of S is the A-operand layout of P) and accumulates all 128 output columns with
 //     its own online softmax, so the warps never wait for one another. At the last item of a
-//     group in this CTA each warp parks its state in its own 16 rows of the stage;
-//   * epilogue (warp 9): folds the 8 parked states by log-sum-exp, releases the stage, and
-//     either writes the output (the group lies in this CTA) or deals with the other CTAs that
-//     hold parts of the group: if all of them are in it merges their partials (max, sum, o)
-//     into its registers, otherwise it leaves its own partial for the last one to arrive.
-//     None of this global-memory traffic stalls the compute warps.
+//     group in this CTA each warp parks its state in its own 16 rows of the stage. When the
+//     whole group ran in this CTA the 8 warps then fold the parked states together (warp w
+//     the output columns 16w..16w+15) and write the output;
+//   * epilogue (warp 9), for a group split across CTAs: folds the 8 parked states by
+//     log-sum-exp, releases the stage, and deals with the other CTAs that hold parts of the
+//     group: if all of them are in it merges their partials (max, sum, o) into its registers,
+//     otherwise it leaves its own partial for the last one to arrive. None of this
+//     global-memory traffic stalls the compute warps.
 #include <atomic>
 
 #include "msa_common.cuh"
@@ -60,6 +62,7 @@ struct __align__(1024) DecSmem {
     float om[kMaxHg], ol[kMaxHg];
     uint64_t full_k[kDecStages], full_v[kDecStages], empty[kDecStages];
     uint64_t parked[kDecStages];                // 8 warp states parked (queue of group ends)
+    uint64_t fold;                              // 8 warp states parked for a fold by the compute warps
     int meta_bg[kDecStages], meta_ntok[kDecStages], meta_fin[kDecStages], meta_nfrag[kDecStages],
         meta_frag[kDecStages], meta_fp8[kDecStages];
     float meta_ks[kDecStages], meta_vs[kDecStages];   // FP8 variant: the block's key / value scales
@@ -222,6 +225,42 @@ __device__ __forceinline__ void merge_partial(WarpState& st, const float* pf, in
     }
 }
 
+// A group whose items all ran in this CTA is finished by the 8 compute warps together: once all
+// have parked their states in the stage, warp w folds column group w (columns 16 w .. 16 w + 15;
+// group w + 8 for rows gq + 8 when Hg > 8) of the 8 states by log-sum-exp and writes those
+// output columns, so the fold runs 8 warps wide instead of on the epilogue warp alone.
+__device__ __forceinline__ void fold_write_columns(DecSmem& sm, int stage, int warp, int lane, int Hg,
+                                                   size_t orow, uint16_t* __restrict__ out, float* __restrict__ lse) {
+    const int gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int row = gq + 8 * half;
+        if (row >= Hg) continue;
+        const int g = warp + 8 * half;
+        float mw[kDecWarps];
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) {
+            mw[w] = sm.pm[stage][w][row];
+            M = fmaxf(M, mw[w]);
+        }
+        float L = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) {
+            const float wt = mw[w] == -INFINITY ? 0.f : fast_exp2(mw[w] - M);
+            L += sm.pl[stage][w][row] * wt;
+            const float4 x = *park_addr(sm, stage, w, g, lane);
+            acc.x += x.x * wt; acc.y += x.y * wt; acc.z += x.z * wt; acc.w += x.w * wt;
+        }
+        const float inv = 1.f / L;
+        uint16_t* o = out + (orow + row) * kHeadDim + 16 * warp + 2 * tq;
+        *reinterpret_cast<uint32_t*>(o) = pack_bf16x2(acc.x * inv, acc.y * inv);
+        *reinterpret_cast<uint32_t*>(o + 8) = pack_bf16x2(acc.z * inv, acc.w * inv);
+        if (lse != nullptr && warp == 0 && tq == 0) lse[orow + row] = (M + log2f(L)) * 0.69314718055994530942f;
+    }
+}
+
 __device__ __forceinline__ void clear_state(WarpState& st) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) st.o[i][0] = st.o[i][1] = st.o[i][2] = st.o[i][3] = 0.f;
@@ -246,6 +285,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
             mbar_init(&sm.empty[s], kDecWarps);
             mbar_init(&sm.parked[s], kDecWarps);
         }
+        mbar_init(&sm.fold, kDecWarps);
         fence_barrier_init();
     }
     for (int i = tid; i < kDecStages * kMaxHg * kQRow; i += kDecThreads) (&sm.q[0][0][0])[i] = 0;   // rows >= Hg stay 0
@@ -564,6 +604,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
     WarpState st;
     clear_state(st);
     int nfin = 0;                                       // group ends parked so far
+    int nfold = 0;                                      // groups folded by the compute warps so far
     for (int n = 0;; ++n) {
         const int stage = n % kDecStages;
         const uint32_t ph = (n / kDecStages) & 1;
@@ -727,6 +768,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
             sm.pl[stage][warp][gq + 8] = st.l1;
         }
         fence_proxy_async();                            // smem writes before the stage's next TMA fill
+        if (sm.meta_nfrag[stage] == 1) {
+            // the whole group ran in this CTA: fold it here, 8 warps wide
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.fold);
+            if (!warp_wait_all(&sm.fold, uint32_t(nfold & 1), a.hdr)) break;
+            ++nfold;
+            const size_t orow = size_t(bg / G) * G * Hg + size_t(bg % G) * Hg;
+            fold_write_columns(sm, stage, warp, lane, Hg, orow, a.out, a.lse);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[stage]);   // this warp has read the parked states
+            clear_state(st);
+            continue;
+        }
         const int qs = nfin % kDecStages;
         if (warp == 0 && lane == 0) sm.park_stage[qs] = stage;
         __syncwarp();

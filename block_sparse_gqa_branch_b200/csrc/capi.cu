@@ -16,6 +16,7 @@ void launch_append(const void*, const void*, const void*, const int32_t*, int, i
                    float*, float*, int64_t, void*, cudaStream_t);
 msa_status_t launch_select_prefill_tc(const void*, int, int, int64_t, int64_t, const float*, int64_t, int32_t*, void*,
                                       cudaStream_t);
+size_t select_prefill_ws_bytes(int, int, int64_t);
 void launch_pool_chunk(const void*, int, int, int64_t, int64_t, float*, int64_t, float*, cudaStream_t);
 void launch_select_decode(const void*, const int32_t*, int64_t, int, int, const float*, int64_t, int32_t*,
                           void*, cudaStream_t);
@@ -189,7 +190,9 @@ size_t ws_size(const msa_shape_t* s, int32_t op, int64_t n) {
     if (check_shape(s) != MSA_OK || n < 0) return 0;
     const int hg = s->n_q_heads / s->n_kv_groups;
     switch (op) {
-        case MSA_OP_INDEX_SELECT_PREFILL: return header_only();
+        case MSA_OP_INDEX_SELECT_PREFILL:
+            if (n < 1) return 0;
+            return select_prefill_ws_bytes(s->batch, s->n_kv_groups, n);
         case MSA_OP_INDEX_SELECT_DECODE:
             if (n > kMaxPos) return 0;
             return decode_select_ws_bytes(s->batch, s->n_kv_groups, n);
@@ -258,7 +261,7 @@ msa_status_t msa_index_select(const msa_shape_t* shape, const void* q_idx, int64
         MSA_REQ(max_pos >= n_queries - 1, MSA_ERR_INVALID_ARGUMENT);
         MSA_REQ(nb_cap >= (n_queries - 1) / kBlock, MSA_ERR_INVALID_ARGUMENT);
         const size_t need = ws_size(shape, MSA_OP_INDEX_SELECT_PREFILL, n_queries);
-        MSA_REQ(workspace != nullptr && workspace_bytes >= need, MSA_ERR_WORKSPACE);
+        MSA_REQ(workspace != nullptr && aligned16(workspace) && need > 0 && workspace_bytes >= need, MSA_ERR_WORKSPACE);
         MSA_TRY(launch_select_prefill_tc(q_idx, B, G, n_queries, 0, pooled, nb_cap, sel, workspace, st));
     } else {                                       // decode: one query per sequence at q_pos[b]
         MSA_REQ(n_queries == 1, MSA_ERR_INVALID_ARGUMENT);
@@ -368,7 +371,8 @@ msa_status_t msa_index_select_chunk(const msa_shape_t* shape, const void* q_idx,
     MSA_REQ(n >= 1 && q_start >= 0 && q_start + n < (int64_t(1) << 31), MSA_ERR_INVALID_ARGUMENT);
     MSA_REQ(nb_cap >= (q_start + n - 1) / kBlock, MSA_ERR_INVALID_ARGUMENT);
     MSA_REQ(pooled == nullptr ? q_start + n - 1 < kBlock : aligned16(pooled), MSA_ERR_INVALID_ARGUMENT);
-    MSA_REQ(workspace != nullptr && workspace_bytes >= header_only(), MSA_ERR_WORKSPACE);
+    const size_t need = ws_size(shape, MSA_OP_INDEX_SELECT_PREFILL, q_start + n);
+    MSA_REQ(workspace != nullptr && aligned16(workspace) && need > 0 && workspace_bytes >= need, MSA_ERR_WORKSPACE);
     MSA_TRY(launch_select_prefill_tc(q_idx, shape->batch, shape->n_kv_groups, n, q_start, pooled, nb_cap, sel,
                                      workspace, reinterpret_cast<cudaStream_t>(stream)));
     return cuda_status();

@@ -167,6 +167,25 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t* __restrict_
                                                      WsHeader* hdr) {
     grid_dep_launch();                 // the selection may start: it does not read what this writes
     const int b = blockIdx.x;
+    // Every load goes out before the first use (one memory round trip: the selection streams
+    // HBM at the same time, so each dependent round trip here would stretch the step).
+    const int nvec = G * kHeadDim / 8;                     // 16-byte vectors per token and tensor
+    const int nidx = G * kIndexDim;
+    uint4 kv[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+    float xi[2] = {0.f, 0.f}, ts[2] = {0.f, 0.f};
+    const int i0 = threadIdx.x;
+    if (k_new != nullptr && i0 < nvec) {
+        kv[0] = __ldg(reinterpret_cast<const uint4*>(k_new) + size_t(b) * nvec + i0);
+        kv[1] = __ldg(reinterpret_cast<const uint4*>(v_new) + size_t(b) * nvec + i0);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int i = i0 + r * 256;
+        if (i < nidx) {
+            xi[r] = bf16_to_f32(__ldg(k_idx_new + size_t(b) * nidx + i));
+            ts[r] = tail_sum[size_t(b) * nidx + i];
+        }
+    }
     const int pos = ctx_len[b];
     const int64_t j = pos / kBlock;
     const bool close = ((pos + 1) % kBlock) == 0;
@@ -175,23 +194,25 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t* __restrict_
         return;
     }
     if (k_new != nullptr) {
-        const int nvec = G * kHeadDim / 8;                 // 16-byte vectors per token
-        for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+        for (int i = i0; i < nvec; i += 256) {
             const int g = i / (kHeadDim / 8), c = i % (kHeadDim / 8);
-            const size_t src = (size_t(b) * G + g) * (kHeadDim / 8) + c;
+            const uint4 kx = i == i0 ? kv[0] : __ldg(reinterpret_cast<const uint4*>(k_new) + size_t(b) * nvec + i);
+            const uint4 vx = i == i0 ? kv[1] : __ldg(reinterpret_cast<const uint4*>(v_new) + size_t(b) * nvec + i);
             const size_t dst = ((size_t(b) * G + g) * l_cap + pos) * (kHeadDim / 8) + c;
-            reinterpret_cast<uint4*>(k_cache)[dst] = reinterpret_cast<const uint4*>(k_new)[src];
-            reinterpret_cast<uint4*>(v_cache)[dst] = reinterpret_cast<const uint4*>(v_new)[src];
+            reinterpret_cast<uint4*>(k_cache)[dst] = kx;
+            reinterpret_cast<uint4*>(v_cache)[dst] = vx;
         }
     }
     const bool fresh = (pos % kBlock) == 0;
-    for (int i = threadIdx.x; i < G * kIndexDim; i += blockDim.x) {
+    for (int i = i0; i < nidx; i += 256) {
         const int g = i / kIndexDim, e = i % kIndexDim;
         const size_t o = (size_t(b) * G + g) * kIndexDim + e;
-        const float x = bf16_to_f32(k_idx_new[o]);
-        const float s = fresh ? x : tail_sum[o] + x;
-        tail_sum[o] = s;
-        if (close) pooled[((size_t(b) * G + g) * nb_cap + j) * kIndexDim + e] = s * (1.0f / kBlock);
+        const int r = (i - i0) / 256;
+        const float x = r < 2 ? xi[r] : bf16_to_f32(k_idx_new[o]);
+        const float t = r < 2 ? ts[r] : tail_sum[o];
+        const float sum = fresh ? x : t + x;
+        tail_sum[o] = sum;
+        if (close) pooled[((size_t(b) * G + g) * nb_cap + j) * kIndexDim + e] = sum * (1.0f / kBlock);
     }
 }
 

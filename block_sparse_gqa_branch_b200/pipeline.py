@@ -146,7 +146,7 @@ def prefill_chunk(q, q_idx, k_idx, k_cache, v_cache, q_start: int, pooled, tail_
     sel = torch.empty(B, n, G, TOPK, dtype=torch.int32, device=dev)
     out = torch.empty(B, n, n_q_heads, 128, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(B, n, n_q_heads, dtype=torch.float32, device=dev) if with_lse else None
-    ws_sel = torch.zeros(256, dtype=torch.uint8, device=dev)
+    ws_sel = torch.zeros(msa_workspace_size(shape, OP_INDEX_SELECT_PREFILL, q_start + n), dtype=torch.uint8, device=dev)
     ws = torch.zeros(msa_prefill_chunk_workspace_size(shape, q_start, n), dtype=torch.uint8, device=dev)
     msa_pool_index_keys_chunk(shape, k_idx, q_start, n, pooled, nb_cap, tail_sum, stream)
     msa_index_select_chunk(shape, q_idx, q_start, n, pooled, nb_cap, sel, ws_sel, stream)

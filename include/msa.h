@@ -96,7 +96,10 @@ uint64_t msa_kernel_launches(void);
 
 /*
  * Workspace bytes needed by one operation.
- *  op = MSA_OP_INDEX_SELECT_PREFILL: n = number of query tokens per sequence
+ *  op = MSA_OP_INDEX_SELECT_PREFILL: n = one past the last query position (the number of query
+ *                                    tokens per sequence for a whole prefill, P + n for a chunk);
+ *                                    the workspace holds the pooled keys of the fully-past
+ *                                    blocks split into three bf16 terms (384 B per block and group)
  *  op = MSA_OP_INDEX_SELECT_DECODE:  n = max_pos (largest query position)
  *  op = MSA_OP_ATTN_PREFILL:         n = number of tokens per sequence
  *  op = MSA_OP_ATTN_DECODE:          n = max_pos
@@ -209,7 +212,8 @@ msa_status_t msa_pool_index_keys_chunk(const msa_shape_t *shape, const void *k_i
 
 /* Block scores and exp-free top-k selection for the chunk's index queries q_idx [B, n, G, d_I]
  * (row i at position P + i); sel [B, n, G, k] as msa_index_select. pooled must hold every full
- * block below P + n (after msa_pool_index_keys_chunk). Workspace: >= 256 bytes. */
+ * block below P + n (after msa_pool_index_keys_chunk). Workspace (16-byte aligned) of
+ * msa_workspace_size(MSA_OP_INDEX_SELECT_PREFILL, P + n). */
 msa_status_t msa_index_select_chunk(const msa_shape_t *shape, const void *q_idx, int64_t q_start, int64_t n,
                                     const float *pooled, int64_t nb_cap, int32_t *sel, void *workspace,
                                     size_t workspace_bytes, msa_stream_t stream);

@@ -48,7 +48,11 @@ def test_workspace_sizes(L):
     s = Shape.make(16, 64, 8)
     assert msa.msa_workspace_size(s, msa.OP_ATTN_DECODE, 131072) >= 256 + 16 * 8 * 16 * 8 * 130 * 4
     assert msa.msa_workspace_size(s, msa.OP_INDEX_SELECT_DECODE, 131072) > 256
-    assert msa.msa_workspace_size(s, msa.OP_INDEX_SELECT_PREFILL, 4096) >= 256
+    # prefill selection: the header, then the fully-past blocks' pooled keys split into three bf16
+    # terms (3 x 64 x 2 B per block and group), in whole 64-block chunks
+    for n, nbp in ((1, 64), (128, 64), (129, 64), (4096, 64), (8193, 64), (8321, 128), (131072, 1024)):
+        assert msa.msa_workspace_size(s, msa.OP_INDEX_SELECT_PREFILL, n) == 256 + 16 * 8 * 3 * nbp * 128, n
+    assert msa.msa_workspace_size(s, msa.OP_INDEX_SELECT_PREFILL, 0) == 0
     assert msa.msa_workspace_size(s, 17, 10) == 0
     assert msa.msa_workspace_size(Shape.make(1, 6, 4), msa.OP_ATTN_DECODE, 10) == 0      # Hq % G
     assert msa.msa_workspace_size(Shape.make(1, 24, 1), msa.OP_ATTN_DECODE, 10) == 0     # Hg = 24
@@ -185,6 +189,11 @@ def test_chunk_entry_points_validate_before_launch(L):
     # selection: workspace, nb_cap
     assert L.msa_index_select_chunk(s, FAKE, 1000, 500, FAKE, 11, FAKE2, None, 0, None) == 3
     assert L.msa_index_select_chunk(s, FAKE, 1000, 500, FAKE, 10, FAKE2, FAKE, 256, None) == 1
+    # the workspace covers the split keys of every block below P + n
+    need = msa.msa_workspace_size(_shape(n_q_heads=16, n_kv_groups=2), msa.OP_INDEX_SELECT_PREFILL, 1500)
+    assert need > 256
+    assert L.msa_index_select_chunk(s, FAKE, 1000, 500, FAKE, 11, FAKE2, FAKE, need - 16, None) == 3
+    assert L.msa_index_select_chunk(s, FAKE, 1000, 500, FAKE, 11, FAKE2, FAKE + 8, need, None) == 3
     # attention: the chunk must fit in the cache; the workspace depends on P
     assert L.msa_sparse_attn_prefill_chunk(s, FAKE, FAKE, FAKE, 1400, 1000, 500, FAKE, FAKE, None, FAKE, big,
                                            None) == 1
