@@ -24,6 +24,7 @@ __all__ = [
     "msa_topk_rows", "msa_fp8_quantize_blocks", "msa_fp8_close_blocks", "msa_sparse_attn_decode_fp8",
     "msa_pool_index_keys_chunk", "msa_index_select_chunk", "msa_sparse_attn_prefill_chunk",
     "msa_prefill_chunk_workspace_size", "msa_sparse_attn_prefill_backward",
+    "msa_kernel_timing_enable", "msa_kernel_timing_read", "KERNEL_NAMES",
     "OP_INDEX_SELECT_PREFILL", "OP_ATTN_PREFILL_BACKWARD", "OP_INDEX_SELECT_DECODE", "OP_ATTN_PREFILL", "OP_ATTN_DECODE",
     "EXPORTED_SYMBOLS",
 ]
@@ -48,7 +49,13 @@ EXPORTED_SYMBOLS = [
     "msa_fp8_quantize_blocks", "msa_fp8_close_blocks", "msa_sparse_attn_decode_fp8",
     "msa_pool_index_keys_chunk", "msa_index_select_chunk", "msa_sparse_attn_prefill_chunk",
     "msa_prefill_chunk_workspace_size", "msa_sparse_attn_prefill_backward",
+    "msa_kernel_timing_enable", "msa_kernel_timing_read",
 ]
+
+# MSA_KERNEL_* ids of include/msa.h
+KERNEL_NAMES = {1: "pool", 2: "select_prefill", 3: "select_decode", 4: "append", 5: "attn_decode",
+                6: "attn_prefill", 7: "inverted_index", 8: "combine", 9: "selftest", 10: "fp8_quantize",
+                11: "split_keys", 12: "attn_backward", 13: "backward_dot", 14: "topk"}
 
 
 class Shape(ctypes.Structure):
@@ -91,6 +98,10 @@ def load():
         L.msa_status_string.argtypes = [ctypes.c_int]
         L.msa_last_cuda_error.restype = I32
         L.msa_kernel_launches.restype = ctypes.c_uint64
+        L.msa_kernel_timing_enable.restype = I32
+        L.msa_kernel_timing_enable.argtypes = [I32]
+        L.msa_kernel_timing_read.restype = I32
+        L.msa_kernel_timing_read.argtypes = [P, P, I32]
         L.msa_workspace_size.restype = SZ
         L.msa_workspace_size.argtypes = [SP, I32, I64]
         L.msa_prefill_chunk_workspace_size.restype = SZ
@@ -161,6 +172,21 @@ def msa_status_string(status: int) -> str:
 
 def msa_kernel_launches() -> int:
     return load().msa_kernel_launches()
+
+
+def msa_kernel_timing_enable(on: bool) -> bool:
+    """Switch per-kernel event timing on or off; returns the previous setting."""
+    return bool(load().msa_kernel_timing_enable(1 if on else 0))
+
+
+def msa_kernel_timing_read(cap: int = 1 << 16) -> list:
+    """The timed launches since the last read, in launch order: [(kernel name, ms), ...]."""
+    kid = (ctypes.c_int32 * cap)()
+    ms = (ctypes.c_float * cap)()
+    n = load().msa_kernel_timing_read(ctypes.cast(kid, ctypes.c_void_p), ctypes.cast(ms, ctypes.c_void_p), cap)
+    if n < 0:
+        raise MSAError(4, "msa_kernel_timing_read")
+    return [(KERNEL_NAMES.get(int(kid[i]), str(int(kid[i]))), float(ms[i])) for i in range(n)]
 
 
 def msa_workspace_size(shape: Shape, op: int, n: int) -> int:

@@ -303,7 +303,7 @@ msa_status_t launch_attn_backward(const void* q, const void* k, const void* v, i
     cudaMemsetAsync(dv, 0, size_t(B) * G * N * kHeadDim * sizeof(float), st);
     {
         const int64_t rows = int64_t(B) * N * Hq;
-        count_launch();
+        const KernelTimer kt(KID_BWD_DOT, st);
         bwd_dot_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(
             static_cast<const uint16_t*>(d_out), static_cast<const uint16_t*>(out), dd, rows);
     }
@@ -330,7 +330,7 @@ msa_status_t launch_attn_backward(const void* q, const void* k, const void* v, i
         cudaFuncSetAttribute(attn_backward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         attr_set[dev].store(true, std::memory_order_relaxed);
     }
-    count_launch();
+    const KernelTimer kt(KID_ATTN_BACKWARD, st);
     attn_backward_kernel<<<num_sms(), kBwdThreads, smem, st>>>(a);
     return MSA_OK;
 }

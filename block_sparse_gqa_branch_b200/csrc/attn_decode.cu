@@ -858,7 +858,7 @@ msa_status_t launch_attn_decode(const void* k_cache, const void* v_cache, const 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    count_launch();
+    const KernelTimer kt(KID_ATTN_DECODE, st);
     cudaLaunchKernelEx(&cfg, kern, maps, a);
     return cuda_status();
 }

@@ -799,14 +799,16 @@ void launch_inverted_index(const int32_t* sel, int64_t N, int64_t P, int B, int 
         const size_t smem = size_t(L.nb) * sizeof(int);
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(csr_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        count_launch();
+        const KernelTimer kt(KID_CSR, st);
         csr_count_kernel<<<grid, 256, smem, st>>>(sel, N, P, G, L.nb, L.nR, counts, hdr);
     }
-    count_launch();
-    csr_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, items, nitems, int64_t(L.nbins), L.nb, L.nR, N, P, L.tpt);
+    {
+        const KernelTimer kt(KID_CSR, st);
+        csr_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, items, nitems, int64_t(L.nbins), L.nb, L.nR, N, P, L.tpt);
+    }
     {
         const int64_t total = int64_t(B) * N * G;
-        count_launch();
+        const KernelTimer kt(KID_CSR, st);
         csr_fill_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(sel, N, P, G, L.nb, L.nR, offsets,
                                                                                    counts, list, total);
     }
@@ -844,12 +846,12 @@ msa_status_t launch_attn_prefill_tc(const void* q, const CUtensorMap& tmQ2, cons
         if (st_map == MSA_OK && Hg >= 8) st_map = make_tmap_q_rows(&tmQ3, q, uint64_t(B) * N * G * Hg);
         if (st_map != MSA_OK) return st_map;
         const CUtensorMap& tmQ = Hg >= 8 ? tmQ3 : tmQ2;
-        count_launch();
+        const KernelTimer kt(KID_ATTN_PREFILL, st);
         attn_kvmajor_kernel<<<num_sms(), kKvThreads, smem, st>>>(tmQ, tmK, tmV, tmO, a);
     }
     {
         const int64_t total = int64_t(B) * N * G * Hg * 4;
-        count_launch();
+        const KernelTimer kt(KID_COMBINE, st);
         combine_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(sel, part_lse, part_o, N, G, Hg,
                                                                                   static_cast<uint16_t*>(out), lse,
                                                                                   total);

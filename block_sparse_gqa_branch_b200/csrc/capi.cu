@@ -6,6 +6,8 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "msa_common.cuh"
 
@@ -38,6 +40,39 @@ msa_status_t launch_attn_prefill_tc(const void*, const CUtensorMap&, const CUten
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// kernel timing records: (kernel id, start event, end event) in launch order
+struct TimingRec {
+    int kid;
+    cudaEvent_t a, b;
+};
+static std::atomic<bool> g_timing{false};
+static std::mutex g_timing_mu;
+static std::vector<TimingRec> g_timing_recs;
+
+KernelTimer::KernelTimer(int kid, cudaStream_t st) : kid_(kid), st_(st) {
+    count_launch();
+    if (!g_timing.load(std::memory_order_relaxed)) return;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
+    if (cudaEventCreate(&a_) != cudaSuccess) {
+        a_ = nullptr;
+        return;
+    }
+    if (cudaEventCreate(&b_) != cudaSuccess) {
+        cudaEventDestroy(a_);
+        a_ = nullptr;
+        return;
+    }
+    cudaEventRecord(a_, st);
+}
+
+KernelTimer::~KernelTimer() {
+    if (a_ == nullptr) return;
+    cudaEventRecord(b_, st_);
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    g_timing_recs.push_back(TimingRec{kid_, a_, b_});
+}
 
 thread_local int g_last_cuda_error = 0;
 
@@ -229,6 +264,30 @@ const char* msa_status_string(msa_status_t s) {
 int32_t msa_last_cuda_error(void) { return g_last_cuda_error; }
 
 uint64_t msa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int32_t msa_kernel_timing_enable(int32_t on) { return g_timing.exchange(on != 0) ? 1 : 0; }
+
+int32_t msa_kernel_timing_read(int32_t* kernel, float* ms, int32_t cap) {
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    int32_t n = 0;
+    bool failed = false;
+    for (const TimingRec& r : g_timing_recs) {
+        if (!failed && n < cap && kernel != nullptr && ms != nullptr) {
+            float t = 0.f;
+            if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
+                failed = true;
+            } else {
+                kernel[n] = r.kid;
+                ms[n] = t;
+                ++n;
+            }
+        }
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    g_timing_recs.clear();
+    return failed ? -1 : n;
+}
 
 size_t msa_workspace_size(const msa_shape_t* shape, int32_t op, int64_t n) { return ws_size(shape, op, n); }
 

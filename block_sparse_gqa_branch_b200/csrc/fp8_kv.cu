@@ -114,7 +114,7 @@ void launch_fp8_quantize(const void* k, const void* v, int64_t l_cap, int64_t n_
     if (n_blocks <= 0) return;
     Fp8Args a{static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v), static_cast<uint8_t*>(k8),
               static_cast<uint8_t*>(v8), ks, vs, l_cap, nb_cap, G};
-    count_launch();
+    const KernelTimer kt(KID_FP8, st);
     fp8_quantize_kernel<<<dim3(unsigned(n_blocks), unsigned(2 * G), unsigned(B)), 256, 0, st>>>(a);
 }
 
@@ -131,7 +131,7 @@ void launch_fp8_close(const void* k, const void* v, int64_t l_cap, const int32_t
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    count_launch();
+    const KernelTimer kt(KID_FP8, st);
     cudaLaunchKernelEx(&cfg, fp8_close_kernel, a, ctx_len, static_cast<WsHeader*>(ws));
 }
 

@@ -71,9 +71,30 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header must be 256 bytes");
 
+// kernel ids: the MSA_KERNEL_* values of msa.h (workspace error info[0], timing records)
 enum KernelId : int {
-    KID_POOL = 1, KID_SELECT_PREFILL = 2, KID_SELECT_DECODE = 3, KID_APPEND = 4,
-    KID_ATTN_DECODE = 5, KID_ATTN_PREFILL = 6, KID_CSR = 7, KID_COMBINE = 8, KID_SELFTEST = 9, KID_FP8 = 10
+    KID_POOL = MSA_KERNEL_POOL, KID_SELECT_PREFILL = MSA_KERNEL_SELECT_PREFILL,
+    KID_SELECT_DECODE = MSA_KERNEL_SELECT_DECODE, KID_APPEND = MSA_KERNEL_APPEND,
+    KID_ATTN_DECODE = MSA_KERNEL_ATTN_DECODE, KID_ATTN_PREFILL = MSA_KERNEL_ATTN_PREFILL,
+    KID_CSR = MSA_KERNEL_INVERTED_INDEX, KID_COMBINE = MSA_KERNEL_COMBINE, KID_SELFTEST = MSA_KERNEL_SELFTEST,
+    KID_FP8 = MSA_KERNEL_FP8, KID_SPLIT = MSA_KERNEL_SPLIT_KEYS, KID_ATTN_BACKWARD = MSA_KERNEL_ATTN_BACKWARD,
+    KID_BWD_DOT = MSA_KERNEL_BACKWARD_DOT, KID_TOPK = MSA_KERNEL_TOPK
+};
+
+// Counts a launch (msa_kernel_launches) and, while kernel timing is on and the stream is not
+// being captured, brackets it with two events on the stream (msa_kernel_timing_read). Declared
+// in the scope that ends right after the launch.
+class KernelTimer {
+  public:
+    KernelTimer(int kid, cudaStream_t st);
+    ~KernelTimer();
+    KernelTimer(const KernelTimer&) = delete;
+    KernelTimer& operator=(const KernelTimer&) = delete;
+
+  private:
+    int kid_;
+    cudaStream_t st_;
+    cudaEvent_t a_ = nullptr, b_ = nullptr;
 };
 
 __device__ __forceinline__ void record_error(WsHeader* h, unsigned code, int kid, int blk,

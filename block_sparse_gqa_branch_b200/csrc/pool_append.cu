@@ -65,7 +65,7 @@ void launch_pool(const void* k_idx, int B, int G, int64_t n_tokens, float* poole
                  float* tail_sum, cudaStream_t st) {
     if (tail_sum && n_tokens % kBlock == 0) {
         int64_t n = int64_t(B) * G * kIndexDim;
-        count_launch();
+        const KernelTimer kt(KID_POOL, st);
         zero_kernel<<<int((n + 255) / 256), 256, 0, st>>>(tail_sum, n);
     }
     if (n_tokens == 0) return;
@@ -74,7 +74,7 @@ void launch_pool(const void* k_idx, int B, int G, int64_t n_tokens, float* poole
     size_t smem = size_t(nparts) * G * kIndexDim * sizeof(float);
     if (smem > 48 * 1024) cudaFuncSetAttribute(pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     dim3 grid(unsigned((n_tokens + kBlock - 1) / kBlock), unsigned(B));
-    count_launch();
+    const KernelTimer kt(KID_POOL, st);
     pool_kernel<<<grid, 256, smem, st>>>(static_cast<const uint16_t*>(k_idx), n_tokens, G, pooled,
                                           nb_cap, tail_sum);
 }
@@ -143,11 +143,11 @@ void launch_pool_chunk(const void* k_idx, int B, int G, int64_t n, int64_t P, fl
         cudaFuncSetAttribute(pool_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     const int64_t j0 = P / kBlock, jt = (P + n) / kBlock;      // blocks j0 .. jt - 1 complete in the chunk
     if (jt > j0) {
-        count_launch();
+        const KernelTimer kt(KID_POOL, st);
         pool_chunk_kernel<<<dim3(unsigned(jt - j0), unsigned(B)), 256, smem, st>>>(
             static_cast<const uint16_t*>(k_idx), n, P, G, pooled, nb_cap, tail_sum, j0, 0);
     }
-    count_launch();                                              // the trailing open block (maybe empty)
+    const KernelTimer kt(KID_POOL, st);                          // the trailing open block (maybe empty)
     pool_chunk_kernel<<<dim3(1u, unsigned(B)), 256, smem, st>>>(static_cast<const uint16_t*>(k_idx), n, P, G, pooled,
                                                               nb_cap, tail_sum, jt, 1);
 }
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t* __restrict_
 void launch_append(const void* k_idx_new, const void* k_new, const void* v_new, const int32_t* ctx_len,
                    int B, int G, void* k_cache, void* v_cache, int64_t l_cap, float* tail_sum,
                    float* pooled, int64_t nb_cap, void* ws, cudaStream_t st) {
-    count_launch();
+    const KernelTimer kt(KID_APPEND, st);
     append_kernel<<<B, 256, 0, st>>>(static_cast<const uint16_t*>(k_idx_new),
                                      static_cast<const uint16_t*>(k_new),
                                      static_cast<const uint16_t*>(v_new), ctx_len, G,

@@ -260,7 +260,7 @@ void launch_select_decode(const void* q_idx, const int32_t* q_pos, int64_t max_p
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    count_launch();
+    const KernelTimer kt(KID_SELECT_DECODE, st);
     cudaLaunchKernelEx(&cfg, select_decode_kernel, static_cast<const uint16_t*>(q_idx), q_pos, max_pos, G, pooled,
                        nb_cap, sel, cand, ctr, hdr);
 }

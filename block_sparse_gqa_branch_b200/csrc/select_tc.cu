@@ -303,7 +303,7 @@ msa_status_t launch_select_prefill_tc(const void* q_idx, int B, int G, int64_t N
     uint16_t* split = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + select_split_offset());
     {
         const int64_t threads = nbp * 8;
-        count_launch();
+        const KernelTimer kt(KID_SPLIT, st);
         split_pooled_kernel<<<dim3(unsigned((threads + 255) / 256), unsigned(B * G)), 256, 0, st>>>(pooled, nb_cap, ncand,
                                                                                               nbp, split);
     }
@@ -317,7 +317,7 @@ msa_status_t launch_select_prefill_tc(const void* q_idx, int B, int G, int64_t N
         attr_set[dev].store(true, std::memory_order_relaxed);
     }
     dim3 grid(static_cast<unsigned>(nqb), static_cast<unsigned>(G), static_cast<unsigned>(B));
-    count_launch();
+    const KernelTimer kt(KID_SELECT_PREFILL, st);
     select_prefill_tc_kernel<<<grid, 128, smem, st>>>(tmQ, N, P, G, split, nbp, sel, static_cast<WsHeader*>(ws));
     return MSA_OK;
 }

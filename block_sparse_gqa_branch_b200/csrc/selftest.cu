@@ -21,7 +21,7 @@ extern "C" msa_status_t msa_selftest_wait_timeout(void* workspace, size_t worksp
     MSA_CALL_RANGE();
     using namespace msa;
     if (workspace == nullptr || workspace_bytes < sizeof(WsHeader) || !aligned16(workspace)) return MSA_ERR_WORKSPACE;
-    count_launch();
+    const KernelTimer kt(KID_SELFTEST, reinterpret_cast<cudaStream_t>(stream));
     selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<WsHeader*>(workspace));
     return cuda_status();
 }

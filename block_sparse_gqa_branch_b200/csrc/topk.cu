@@ -139,7 +139,7 @@ extern "C" msa_status_t msa_topk_rows(const float* scores, int64_t rows, int64_t
     const int64_t want = (rows + kTopkWarps - 1) / kTopkWarps;
     const int blocks = int(want < int64_t(num_sms()) * 16 ? want : int64_t(num_sms()) * 16);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    count_launch();
+    const KernelTimer kt(KID_TOPK, st);
     if (n % 4 == 0)
         topk_rows_kernel<4><<<blocks, kTopkThreads, 0, st>>>(scores, rows, int(n), k, idx, val);
     else

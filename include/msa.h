@@ -94,6 +94,39 @@ int32_t msa_last_cuda_error(void);
  * once, at capture; graph replays are not counted. */
 uint64_t msa_kernel_launches(void);
 
+/* Kernel ids: workspace error records (info[0] of msa_get_device_status) and timing records. */
+enum {
+    MSA_KERNEL_POOL = 1,             /* pooling (and its chunked form), running-sum reset */
+    MSA_KERNEL_SELECT_PREFILL = 2,   /* prefill block scores + exp-free top-k (tensor cores) */
+    MSA_KERNEL_SELECT_DECODE = 3,    /* decode block scores + exp-free top-k */
+    MSA_KERNEL_APPEND = 4,           /* decode append and pooled-key update */
+    MSA_KERNEL_ATTN_DECODE = 5,      /* decode main branch (bf16 or FP8 cache) */
+    MSA_KERNEL_ATTN_PREFILL = 6,     /* prefill main branch, key-value-major attention */
+    MSA_KERNEL_INVERTED_INDEX = 7,   /* prefill / backward: inverted index of the selection */
+    MSA_KERNEL_COMBINE = 8,          /* prefill: log-sum-exp merge of the partials */
+    MSA_KERNEL_SELFTEST = 9,
+    MSA_KERNEL_FP8 = 10,             /* FP8 cache: block quantisation */
+    MSA_KERNEL_SPLIT_KEYS = 11,      /* prefill selection: pooled keys split into bf16 terms */
+    MSA_KERNEL_ATTN_BACKWARD = 12,   /* main-branch backward: dQ, dK, dV */
+    MSA_KERNEL_BACKWARD_DOT = 13,    /* main-branch backward: D = dO . o per row */
+    MSA_KERNEL_TOPK = 14             /* msa_topk_rows */
+};
+
+/*
+ * Per-kernel device time, for benchmarks and profiling. While timing is on, every kernel this
+ * library enqueues on a stream that is not being captured is bracketed by two CUDA events on
+ * that stream (kernels enqueued during a stream capture, and graph replays, are not timed).
+ * The records are kept, in launch order, until read.
+ *   msa_kernel_timing_enable(on): on != 0 switches timing on, 0 off; returns the previous state.
+ *   msa_kernel_timing_read(kernel, ms, cap): waits for the recorded events, writes up to cap
+ *     records -- kernel[i] an MSA_KERNEL_* id, ms[i] that launch's device time in milliseconds
+ *     -- then drops every record and its events; returns the number written, or -1 after a
+ *     CUDA error (the records are dropped all the same). Host arrays; NULL with cap 0 only
+ *     drops the records.
+ */
+int32_t msa_kernel_timing_enable(int32_t on);
+int32_t msa_kernel_timing_read(int32_t *kernel, float *ms, int32_t cap);
+
 /*
  * Workspace bytes needed by one operation.
  *  op = MSA_OP_INDEX_SELECT_PREFILL: n = one past the last query position (the number of query

@@ -96,3 +96,13 @@ def test_fp8_decode_step_bytes_closed_form():
     assert d8["kv"] == 128 * per_bg_kv
     assert d8["pooled"] == d["pooled"] and d8["small"] == d["small"]
     assert d8["total"] == 97311744
+
+
+def test_kernel_means_per_step():
+    recs = [("split_keys", 0.01), ("select_prefill", 1.0), ("attn_prefill", 14.0), ("combine", 6.0),
+            ("split_keys", 0.03), ("select_prefill", 1.2), ("attn_prefill", 16.0), ("combine", 6.0),
+            ("inverted_index", 0.1), ("inverted_index", 0.3)]
+    k = bench.kernel_means(recs, 2)
+    assert k["attn_prefill"] == {"ms": 15.0, "launches": 1.0}
+    assert abs(k["split_keys"]["ms"] - 0.02) < 1e-12 and k["inverted_index"]["launches"] == 1.0
+    assert set(k) == {"split_keys", "select_prefill", "attn_prefill", "combine", "inverted_index"}

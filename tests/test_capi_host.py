@@ -199,3 +199,13 @@ def test_chunk_entry_points_validate_before_launch(L):
                                            None) == 1
     assert L.msa_sparse_attn_prefill_chunk(s, FAKE, FAKE, FAKE, 1500, 1000, 500, FAKE, FAKE, None, FAKE, big - 16,
                                            None) == 3
+
+
+def test_kernel_timing_switch_and_empty_read(L):
+    # no kernel is enqueued here: switching timing on and off and reading no records needs no GPU
+    assert L.msa_kernel_timing_enable(1) == 0
+    assert L.msa_kernel_timing_enable(1) == 1
+    assert L.msa_kernel_timing_enable(0) == 1
+    assert L.msa_kernel_timing_read(None, None, 0) == 0
+    assert msa.msa_kernel_timing_read() == []
+    assert set(msa.KERNEL_NAMES) == set(range(1, 15))
