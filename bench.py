@@ -829,9 +829,13 @@ def run_ours(args):
         return reduce_max(x, world, dev)
 
     wp, wd = workloads(args)
-    do_prefill, do_decode = args.only in (None, "prefill"), args.only in (None, "decode")
-    x = synth.prefill_inputs_torch(wp, dev)
-    pbufs = pipeline.prefill_buffers(wp.B, wp.N, wp.Hq, wp.G, dev)
+    do_prefill, do_decode = args.only in (None, "prefill", "index"), args.only in (None, "decode")
+    do_main = args.only in (None, "prefill")
+    x = synth.prefill_inputs_torch(wp, dev) if do_prefill else None
+    if do_prefill and not do_main:                 # index branch alone: its inputs only
+        x = {"q_idx": x["q_idx"], "k_idx": x["k_idx"]}
+        torch.cuda.empty_cache()
+    pbufs = pipeline.prefill_buffers(wp.B, wp.N, wp.Hq, wp.G, dev, with_main=do_main) if do_prefill else None
     ds = build_decode_state(wd, dev) if do_decode else None
     dbufs = pipeline.decode_buffers(wd.B, wd.Hq, wd.G, max(wd.ctx), dev) if do_decode else None
     flush_l2 = make_flusher(torch, dev)
@@ -844,7 +848,9 @@ def run_ours(args):
     # eager warm-up (sets kernel attributes), then capture the decode step in a CUDA graph
     graph = None
     if do_prefill:
-        pipeline.prefill(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], pbufs)
+        pipeline.prefill_index(x["q_idx"], x["k_idx"], pbufs)
+    if do_main:
+        pipeline.prefill_main(x["q"], x["k"], x["v"], pbufs)
     if do_decode:
         decode_call()
         torch.cuda.synchronize()
@@ -863,7 +869,7 @@ def run_ours(args):
         if do_prefill:
             pipeline.prefill_index(x["q_idx"], x["k_idx"], pbufs)
         e1.record(stream)
-        if do_prefill:
+        if do_main:
             pipeline.prefill_main(x["q"], x["k"], x["v"], pbufs)
         e2.record(stream)
         flush_l2()
@@ -898,7 +904,7 @@ def run_ours(args):
     gpu_launches = launches_eager + decode_graph_kernels * args.steps
 
     # check the device error words after the timed region
-    for key in ("ws_select", "ws_attn"):
+    for key in (("ws_select", "ws_attn") if do_main else ("ws_select",) if do_prefill else ()):
         st_, info = msa.msa_get_device_status(pbufs[key])
         if st_ != 0:
             raise SystemExit(f"device status {st_} in prefill {key}: {info}")
@@ -912,10 +918,12 @@ def run_ours(args):
     tidx = max_over_ranks(statistics.mean(t_index))
     tdec = max_over_ranks(statistics.mean(t_dec))
     peaks, peak_src = load_peaks()
-    pre = prefill_report(wp, [tidx], [tmain], peaks, peak_src, world, launches_eager, kernels,
-                         traffic_name="prefill_main",
-                         scale=(prefill_main_bytes(wp)["model"] / CAPTURES["prefill_main"]["model_bytes"]
-                                if "prefill_main" in CAPTURES else 1.0))
+    pre = None
+    if do_main:
+        pre = prefill_report(wp, [tidx], [tmain], peaks, peak_src, world, launches_eager, kernels,
+                             traffic_name="prefill_main",
+                             scale=(prefill_main_bytes(wp)["model"] / CAPTURES["prefill_main"]["model_bytes"]
+                                    if "prefill_main" in CAPTURES else 1.0))
     dec = decode_report(wd, [tdec], peaks, peak_src, decode_graph_kernels * args.steps,
                         traffic_name="decode_step",
                         scale=(decode_step_bytes(wd)["total"] / CAPTURES["decode_step"]["algorithmic_bytes"]
@@ -1025,11 +1033,11 @@ def run_ours(args):
         "prefill_index_ms": tidx * 1e3,
         "prefill_main_ms": tmain * 1e3,
         "decode_step_us": tdec * 1e6,
-        "roofline": pre["roofline"] if do_prefill else None,
-        "roofline_call": pre["roofline_call"] if do_prefill else None,
-        "prefill_kernels_ms": pre["kernels_ms"] if do_prefill else None,
-        "prefill_hbm": pre["hbm"] if do_prefill else None,
-        "roofline_index": pre["roofline_index"] if do_prefill else None,
+        "roofline": pre["roofline"] if pre is not None else None,
+        "roofline_call": pre["roofline_call"] if pre is not None else None,
+        "prefill_kernels_ms": pre["kernels_ms"] if pre is not None else None,
+        "prefill_hbm": pre["hbm"] if pre is not None else None,
+        "roofline_index": pre["roofline_index"] if pre is not None else None,
         "roofline_decode": dec["roofline"] if do_decode else None,
         "clocks": clocks,
         "gpu_launches": int(gpu_launches),
@@ -1080,7 +1088,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the other workloads (32K planted prefill, 1M ragged decode, top-k)")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time")
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "index", "decode"], default=None,
                     help="run one half of the step (profiler captures; not a benchmark value)")
     ap.add_argument("--prefill-tokens", type=int, default=0, help="smaller prefill for profiler captures")
     ap.add_argument("--decode-batch", type=int, default=0, help="smaller decode batch for profiler captures")

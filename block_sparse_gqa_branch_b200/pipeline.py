@@ -24,7 +24,9 @@ def _ws(shape: Shape, op: int, n: int, device) -> torch.Tensor:
     return torch.zeros(size, dtype=torch.uint8, device=device)
 
 
-def prefill_buffers(B: int, N: int, Hq: int, G: int, device, with_lse: bool = True) -> dict:
+def prefill_buffers(B: int, N: int, Hq: int, G: int, device, with_lse: bool = True, with_main: bool = True) -> dict:
+    """Buffers of a prefill of N tokens; with_main=False leaves out the main branch's output and
+    workspace (an index-branch-only run)."""
     shape = Shape.make(B, Hq, G)
     nb = max(1, N // BLOCK)
     return {
@@ -32,10 +34,10 @@ def prefill_buffers(B: int, N: int, Hq: int, G: int, device, with_lse: bool = Tr
         "pooled": torch.zeros(B, G, nb, INDEX_DIM, dtype=torch.float32, device=device),
         "tail_sum": torch.zeros(B, G, INDEX_DIM, dtype=torch.float32, device=device),
         "sel": torch.empty(B, N, G, TOPK, dtype=torch.int32, device=device),
-        "out": torch.empty(B, N, Hq, 128, dtype=torch.bfloat16, device=device),
-        "lse": torch.empty(B, N, Hq, dtype=torch.float32, device=device) if with_lse else None,
+        "out": torch.empty(B, N, Hq, 128, dtype=torch.bfloat16, device=device) if with_main else None,
+        "lse": torch.empty(B, N, Hq, dtype=torch.float32, device=device) if with_lse and with_main else None,
         "ws_select": _ws(shape, OP_INDEX_SELECT_PREFILL, N, device),
-        "ws_attn": _ws(shape, OP_ATTN_PREFILL, N, device),
+        "ws_attn": _ws(shape, OP_ATTN_PREFILL, N, device) if with_main else None,
     }
 
 
