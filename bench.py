@@ -587,9 +587,10 @@ def time_prefill_chunked(torch, w, dev, chunk, steps, warmup, flush_l2):
     """A prefill of workload w in chunks of `chunk` tokens against a cache (pool, select and
     attention per chunk, caches filled with the chunk's K/V beforehand): per-step seconds of
     all chunks."""
-    from block_sparse_gqa_branch_b200 import (Shape, msa_get_device_status, msa_index_select_chunk,
-                                              msa_pool_index_keys_chunk, msa_prefill_chunk_workspace_size,
-                                              msa_sparse_attn_prefill_chunk)
+    from block_sparse_gqa_branch_b200 import (OP_INDEX_SELECT_PREFILL, Shape, msa_get_device_status,
+                                              msa_index_select_chunk, msa_pool_index_keys_chunk,
+                                              msa_prefill_chunk_workspace_size, msa_sparse_attn_prefill_chunk,
+                                              msa_workspace_size)
     x = synth.prefill_inputs_torch(w, dev)
     B, N, G, Hq = w.B, w.N, w.G, w.Hq
     shape = Shape.make(B, Hq, G)
@@ -604,7 +605,7 @@ def time_prefill_chunked(torch, w, dev, chunk, steps, warmup, flush_l2):
     sel = [torch.empty(B, min(chunk, N - p), G, 16, dtype=torch.int32, device=dev) for p in starts]
     out = [torch.empty(B, min(chunk, N - p), Hq, 128, dtype=torch.bfloat16, device=dev) for p in starts]
     lse = [torch.empty(B, min(chunk, N - p), Hq, dtype=torch.float32, device=dev) for p in starts]
-    ws_sel = torch.zeros(256, dtype=torch.uint8, device=dev)
+    ws_sel = torch.zeros(msa_workspace_size(shape, OP_INDEX_SELECT_PREFILL, N), dtype=torch.uint8, device=dev)
     ws = torch.zeros(max(msa_prefill_chunk_workspace_size(shape, p, min(chunk, N - p)) for p in starts),
                      dtype=torch.uint8, device=dev)
 
