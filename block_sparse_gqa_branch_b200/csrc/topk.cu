@@ -51,69 +51,141 @@ __device__ __forceinline__ uint32_t warp_sort_desc32(uint32_t x, int lane) {
     return x;
 }
 
+// the float at the bottom of the values whose code is >= c (c a code of a non-NaN value, or 0)
+__device__ __forceinline__ float code_floor(uint32_t c) {
+    if (c == 0u) return -INFINITY;                                   // below every real code
+    return __uint_as_float((c & 0x80000000u) ? (c ^ 0x80000000u) : ~c);
+}
+
+constexpr int kStash = 36;                    // floats per lane in the staging rows (16-byte aligned, few conflicts)
+constexpr int kList = 128;                    // passing values one chunk may hand to the merge rounds
+
+// One round per value a lane still holds: the exact merge of the values in `pass` (codes in
+// code[]) into the running best 16. Used for chunks the fast path does not take.
+template <int VEC, int kPer>
+__device__ __forceinline__ void merge_lanes(unsigned long long& best, uint32_t pass, const uint32_t (&code)[kPer],
+                                            int base, int lane) {
+    while (__any_sync(0xffffffffu, pass != 0u)) {
+        unsigned long long key = 0ull;                  // below every real key
+        if (pass != 0u) {
+            const int p = __ffs(int(pass)) - 1;
+            pass &= pass - 1u;
+            uint32_t cp = 0u;
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) cp = (q == p) ? code[q] : cp;
+            const int col = base + ((p / VEC) * 32 + lane) * VEC + (p % VEC);
+            key = (static_cast<unsigned long long>(cp) << 32) | uint32_t(~col);
+        }
+        key = warp_sort_desc(key, lane);
+        const unsigned long long top16 = __shfl_sync(0xffffffffu, key, 31 - lane);   // lanes 16-31: ascending
+        best = warp_merge_desc(lane < 16 ? best : top16, lane);
+    }
+}
+
 // VEC = 4: rows start 16-byte aligned (n % 4 == 0) and are read as float4; VEC = 1 otherwise.
+// Fast path of a chunk (no NaN in it, at most kList values passing): the lane maxima and the
+// pass test are float compares against the bound's floor value (the same set as the codes'
+// test: the code order is the float order once NaN is out, with -0 equal to +0); the passing
+// values are compacted into the warp's list in shared memory, so that one 32-wide round of
+// sort and merge takes 32 of them whatever lanes they came from.
 template <int VEC>
-__global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const float* __restrict__ scores, int64_t rows,
+__global__ void __launch_bounds__(kTopkThreads, 3) topk_rows_kernel(const float* __restrict__ scores, int64_t rows,
                                                                   int n, int k, int32_t* __restrict__ idx,
                                                                   float* __restrict__ val) {
     constexpr int kPer = kTopkSteps * VEC;    // values per lane and chunk
     constexpr int kChunk = 32 * kPer;
-    const int lane = threadIdx.x & 31;
+    __shared__ __align__(16) float stash[kTopkWarps][32 * kStash];
+    __shared__ unsigned long long list[kTopkWarps][kList];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    float* my = &stash[wid][lane * kStash];
+    unsigned long long* wl = list[wid];
     const int64_t nwarps = int64_t(gridDim.x) * kTopkWarps;
-    for (int64_t row = int64_t(blockIdx.x) * kTopkWarps + (threadIdx.x >> 5); row < rows; row += nwarps) {
+    for (int64_t row = int64_t(blockIdx.x) * kTopkWarps + wid; row < rows; row += nwarps) {
         const float* r = scores + row * n;
         unsigned long long best = 0ull;       // lanes 0-15: the best 16 keys so far, descending
         uint32_t floor_code = 0u;             // code of the running k-th best
         for (int base = 0; base < n; base += kChunk) {
-            uint32_t code[kPer];
+            float v[kPer];
             uint32_t valid = 0u;              // bit p: this lane's value p is a column < n
 #pragma unroll
             for (int i = 0; i < kTopkSteps; ++i) {
                 const int c0 = base + (i * 32 + lane) * VEC;
                 if constexpr (VEC == 4) {
-                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                    float4 x = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
                     if (c0 < n) {
                         x = __ldcs(reinterpret_cast<const float4*>(r + c0));
                         valid |= 0xfu << (4 * i);
                     }
-                    code[4 * i + 0] = score_code(x.x);
-                    code[4 * i + 1] = score_code(x.y);
-                    code[4 * i + 2] = score_code(x.z);
-                    code[4 * i + 3] = score_code(x.w);
+                    v[4 * i + 0] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
                 } else {
-                    float x = 0.f;
+                    float x = -INFINITY;
                     if (c0 < n) {
                         x = __ldcs(r + c0);
                         valid |= 1u << i;
                     }
-                    code[i] = score_code(x);
+                    v[i] = x;
                 }
             }
-            uint32_t lmax = 0u;
+            // lane maximum (a NaN is caught by the sums: it or inf - inf sends the chunk down the
+            // exact path)
+            float lm = -INFINITY, s0 = 0.f, s1 = 0.f;
 #pragma unroll
             for (int p = 0; p < kPer; ++p) {
-                code[p] = ((valid >> p) & 1u) ? code[p] : 0u;      // 0: below every real code
-                lmax = max(lmax, code[p]);
+                lm = fmaxf(lm, v[p]);                    // invalid values are -inf
+                if (p & 1) s1 += ((valid >> p) & 1u) ? v[p] : 0.f;
+                else s0 += ((valid >> p) & 1u) ? v[p] : 0.f;
             }
-            const uint32_t kth_lane_max = __shfl_sync(0xffffffffu, warp_sort_desc32(lmax, lane), k - 1);
+            const bool nan_here = (s0 + s1) != (s0 + s1);
+            const uint32_t lcode = valid != 0u ? score_code(lm) : 0u;
+            const uint32_t kth_lane_max = __shfl_sync(0xffffffffu, warp_sort_desc32(lcode, lane), k - 1);
             const uint32_t bound = max(kth_lane_max, floor_code);
+            const float bf = code_floor(bound);
             uint32_t pass = 0u;
 #pragma unroll
-            for (int p = 0; p < kPer; ++p) pass |= (((valid >> p) & 1u) != 0u && code[p] >= bound) ? (1u << p) : 0u;
-            while (__any_sync(0xffffffffu, pass != 0u)) {
-                unsigned long long key = 0ull;                  // below every real key
-                if (pass != 0u) {
+            for (int p = 0; p < kPer; ++p) pass |= (((valid >> p) & 1u) != 0u && v[p] >= bf) ? (1u << p) : 0u;
+            const int cnt = __popc(pass);
+            int incl = cnt;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += y;
+            }
+            const int total = __shfl_sync(0xffffffffu, incl, 31);
+            if (__any_sync(0xffffffffu, nan_here) || total > kList) {
+                // exact path: codes of every value, one round per value a lane holds
+                uint32_t code[kPer];
+                uint32_t pass_c = 0u;
+#pragma unroll
+                for (int p = 0; p < kPer; ++p) {
+                    code[p] = ((valid >> p) & 1u) ? score_code(v[p]) : 0u;     // 0: below every real code
+                    pass_c |= (((valid >> p) & 1u) != 0u && code[p] >= bound) ? (1u << p) : 0u;
+                }
+                merge_lanes<VEC, kPer>(best, pass_c, code, base, lane);
+            } else if (total > 0) {
+                if constexpr (VEC == 4) {
+#pragma unroll
+                    for (int i = 0; i < kTopkSteps; ++i)
+                        *reinterpret_cast<float4*>(my + 4 * i) = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kPer; ++i) my[i] = v[i];
+                }
+                __syncwarp();
+                int o = incl - cnt;                      // this lane's first list slot; o + cnt <= total <= kList
+                while (pass != 0u) {
                     const int p = __ffs(int(pass)) - 1;
                     pass &= pass - 1u;
-                    uint32_t cp = 0u;
-#pragma unroll
-                    for (int q = 0; q < kPer; ++q) cp = (q == p) ? code[q] : cp;
                     const int col = base + ((p / VEC) * 32 + lane) * VEC + (p % VEC);
-                    key = (static_cast<unsigned long long>(cp) << 32) | uint32_t(~col);
+                    wl[o++] = (static_cast<unsigned long long>(score_code(my[p])) << 32) | uint32_t(~col);
                 }
-                key = warp_sort_desc(key, lane);
-                const unsigned long long top16 = __shfl_sync(0xffffffffu, key, 31 - lane);   // lanes 16-31: ascending
-                best = warp_merge_desc(lane < 16 ? best : top16, lane);
+                __syncwarp();
+                for (int r0 = 0; r0 < total; r0 += 32) {
+                    unsigned long long key = r0 + lane < total ? wl[r0 + lane] : 0ull;
+                    key = warp_sort_desc(key, lane);
+                    const unsigned long long top16 = __shfl_sync(0xffffffffu, key, 31 - lane);
+                    best = warp_merge_desc(lane < 16 ? best : top16, lane);
+                }
+                __syncwarp();                            // the list and the staging rows are free again
             }
             floor_code = uint32_t(__shfl_sync(0xffffffffu, best, k - 1) >> 32);
         }
