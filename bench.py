@@ -47,7 +47,35 @@ CSRC = os.path.join(ROOT, "block_sparse_gqa_branch_b200", "csrc")
 # (source_sha16 of the listed files). A capture stands only while those sources are unchanged:
 # when any of them changes, the bench reports traffic null until the capture is taken again.
 # Each entry says which workload was captured and how it is scaled to the bench's workload.
-CAPTURES = {}
+CAPTURES = {
+    "decode_step": {
+        # attn_decode_kernel 32,133,120 B read + 17,408 B written; select_decode_kernel 8,428,800 B read
+        "bytes": 32133120 + 17408 + 8428800,
+        "algorithmic_bytes": 40052736,          # decode_step_bytes of the batch-4 workload
+        "sources": ["attn_decode.cu", "select.cu"], "sha16": "1891545d555978a2",
+        "note": "attention + selection DRAM bytes at decode_128k_b4_h64g8 (ncu --set full, one launch each), "
+                "scaled to the bench's batch by the algorithmic bytes (both kernels' work is per (sequence, group))",
+        "profile": "profiles/attn_decode_kernel_decode128k_b4.md, profiles/select_decode_kernel_decode128k_b4.md"},
+    "attn_prefill": {
+        # attn_kvmajor_kernel at a prefill of 8,192 tokens: 251,435,776 B read + 1.873639e9 B written
+        "bytes": 251435776 + 1873639000, "model_bytes": 2130214912,   # prefill_main_bytes(...)["attn_model"] at 8K
+        "sources": ["attn_prefill.cu"], "sha16": "0938664ab0d8cdfa",
+        "note": "DRAM bytes of attn_kvmajor_kernel at prefill_8192_h64g8 (ncu --set full, one launch), scaled to "
+                "the bench's prefill by this build's byte model of the kernel (partial writes are 88% of it)",
+        "profile": "profiles/attn_kvmajor_kernel_prefill8k.md"},
+    "prefill_main": {
+        # attention (above) + combine_kernel 1,931,644,000 B read + 90,566,656 B written, same run and size
+        "bytes": 251435776 + 1873639000 + 1931644000 + 90566656, "model_bytes": 4208001024,
+        "sources": ["attn_prefill.cu"], "sha16": "0938664ab0d8cdfa",
+        "note": "DRAM bytes of the attention and combine kernels at prefill_8192_h64g8 (the inverted index's three "
+                "small kernels not captured), scaled by the main-branch call's byte model",
+        "profile": "profiles/attn_kvmajor_kernel_prefill8k.md, profiles/combine_kernel_prefill8k.md"},
+    "topk_rows": {
+        "bytes": 536922112 + 7836928, "rows": 131072,
+        "sources": ["topk.cu"], "sha16": "a5bb54c67fd9d582",
+        "note": "DRAM bytes of topk_rows_kernel at 131,072 x 1,024 (ncu --set full, one launch), scaled by rows",
+        "profile": "profiles/topk_rows_kernel_131072x1024.md"},
+}
 
 
 def source_sha16(files) -> str:
@@ -151,7 +179,8 @@ def prefill_main_bytes(w, range_tokens: int = 16384) -> dict:
     kv_model = B * G * kv_tiles * Bk * d * 2 * 2
     partials = rows * (d * 2 + 4)
     model = 3 * sel + 2 * entries * 4 + q + kv_model + 2 * partials + out
-    return {"algorithmic": q + sel + kv_once + out, "model": model, "partial_rows": rows,
+    attn_model = q + kv_model + partials + entries * 4       # the attention kernel alone
+    return {"algorithmic": q + sel + kv_once + out, "model": model, "attn_model": attn_model, "partial_rows": rows,
             "partials": partials}
 
 
@@ -634,7 +663,7 @@ def time_prefill_chunked(torch, w, dev, chunk, steps, warmup, flush_l2):
     return [a.elapsed_time(b) * 1e-3 for a, b in ts], len(starts)
 
 
-def prefill_report(w, t_index, t_main, peaks, peak_src, world, launches, kernels, traffic_name=None, scale=1.0):
+def prefill_report(w, t_index, t_main, peaks, peak_src, world, launches, kernels):
     """kernels: per-kernel device ms per step timed live in the same steps (kernel_means); the
     roofline is that of the dominant kernel, attn_kvmajor_kernel, over its own launch time."""
     tidx, tmain = statistics.mean(t_index), statistics.mean(t_main)
@@ -643,7 +672,12 @@ def prefill_report(w, t_index, t_main, peaks, peak_src, world, launches, kernels
     t_attn = kernels["attn_prefill"]["ms"] * 1e-3
     ach_k = flops / t_attn / 1e12
     mb = prefill_main_bytes(w)
-    traffic, tnote = captured_traffic(traffic_name, scale) if traffic_name else (None, "not captured")
+    # captured DRAM bytes of a smaller prefill, scaled by this build's byte model (partial writes dominate)
+    cap_a, cap_m = CAPTURES.get("attn_prefill"), CAPTURES.get("prefill_main")
+    traffic, tnote = (captured_traffic("attn_prefill", mb["attn_model"] / cap_a["model_bytes"]) if cap_a
+                      else (None, "no capture recorded"))
+    call_traffic, cnote = (captured_traffic("prefill_main", mb["model"] / cap_m["model_bytes"]) if cap_m
+                           else (None, "no capture recorded"))
     idx_flops = prefill_index_flops(w)
     idx_bytes = prefill_index_bytes(w)
     return {
@@ -662,6 +696,7 @@ def prefill_report(w, t_index, t_main, peaks, peak_src, world, launches, kernels
                           "algorithmic": f"{flops:.4e} FLOP per call", "peak_source": f"{peak_src} burst bf16"},
         "kernels_ms": {k: round(v["ms"], 4) for k, v in kernels.items()},
         "hbm": {"algorithmic_bytes": mb["algorithmic"], "model_bytes": mb["model"],
+                "traffic": call_traffic, "traffic_note": cnote,
                 "achieved_gbs": mb["algorithmic"] / tmain / 1e9,
                 "frac": mb["algorithmic"] / tmain / 1e9 / peaks["hbm_gbs"],
                 "model_frac": mb["model"] / tmain / 1e9 / peaks["hbm_gbs"],
@@ -921,10 +956,7 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     pre = None
     if do_main:
-        pre = prefill_report(wp, [tidx], [tmain], peaks, peak_src, world, launches_eager, kernels,
-                             traffic_name="prefill_main",
-                             scale=(prefill_main_bytes(wp)["model"] / CAPTURES["prefill_main"]["model_bytes"]
-                                    if "prefill_main" in CAPTURES else 1.0))
+        pre = prefill_report(wp, [tidx], [tmain], peaks, peak_src, world, launches_eager, kernels)
     dec = decode_report(wd, [tdec], peaks, peak_src, decode_graph_kernels * args.steps,
                         traffic_name="decode_step",
                         scale=(decode_step_bytes(wd)["total"] / CAPTURES["decode_step"]["algorithmic_bytes"]
@@ -952,9 +984,7 @@ def run_ours(args):
         ti2, tm2, l2, k2 = time_prefill(torch, PREFILL_32K, dev, n_x, w_x, flush_l2)
         k2 = {k: {"ms": max_over_ranks(k2[k]["ms"]), "launches": k2[k]["launches"]} for k in sorted(k2)}
         r = prefill_report(PREFILL_32K, [max_over_ranks(statistics.mean(ti2))], [max_over_ranks(statistics.mean(tm2))],
-                           peaks, peak_src, world, l2, k2, traffic_name="prefill_main",
-                           scale=(prefill_main_bytes(PREFILL_32K)["model"] / CAPTURES["prefill_main"]["model_bytes"]
-                                  if "prefill_main" in CAPTURES else 1.0))
+                           peaks, peak_src, world, l2, k2)
         extra[PREFILL_32K.name] = r
         torch.cuda.empty_cache()
         td5, l5 = time_decode(torch, DECODE_1M, dev, n_x, w_x, flush_l2)

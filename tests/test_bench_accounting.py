@@ -87,6 +87,19 @@ def test_recorded_captures_are_close_to_their_models():
         assert 1.0 <= c["decode_step"]["bytes"] / c["decode_step"]["algorithmic_bytes"] < 1.05
     if "prefill_main" in c:
         assert 0.9 <= c["prefill_main"]["bytes"] / c["prefill_main"]["model_bytes"] < 1.2
+    if "attn_prefill" in c:
+        assert 0.9 <= c["attn_prefill"]["bytes"] / c["attn_prefill"]["model_bytes"] < 1.2
+    if "topk_rows" in c:
+        rows = c["topk_rows"]["rows"]
+        assert 1.0 <= c["topk_rows"]["bytes"] / (rows * 1024 * 4 + rows * 15 * 4) < 1.02
+
+
+def test_attention_byte_model_is_part_of_the_call_model():
+    m = bench.prefill_main_bytes(bench.PREFILL)
+    # the call = attention + inverted index + combine: attention writes the partials once, the
+    # combine reads them back
+    assert m["partials"] < m["attn_model"] < m["model"] - m["partials"]
+    assert m["partial_rows"] == 133234688
 
 
 def test_fp8_decode_step_bytes_closed_form():
