@@ -49,10 +49,10 @@ CSRC = os.path.join(ROOT, "block_sparse_gqa_branch_b200", "csrc")
 # Each entry says which workload was captured and how it is scaled to the bench's workload.
 CAPTURES = {
     "decode_step": {
-        # attn_decode_kernel 32,133,120 B read + 17,408 B written; select_decode_kernel 8,428,800 B read
-        "bytes": 32133120 + 17408 + 8428800,
+        # attn_decode_kernel 32,132,608 B read + 6,144 B written; select_decode_kernel 8,428,800 B read
+        "bytes": 32132608 + 6144 + 8428800,
         "algorithmic_bytes": 40052736,          # decode_step_bytes of the batch-4 workload
-        "sources": ["attn_decode.cu", "select.cu"], "sha16": "1891545d555978a2",
+        "sources": ["attn_decode.cu", "select.cu"], "sha16": "10befc6ca47e5ecb",
         "note": "attention + selection DRAM bytes at decode_128k_b4_h64g8 (ncu --set full, one launch each), "
                 "scaled to the bench's batch by the algorithmic bytes (both kernels' work is per (sequence, group))",
         "profile": "profiles/attn_decode_kernel_decode128k_b4.md, profiles/select_decode_kernel_decode128k_b4.md"},

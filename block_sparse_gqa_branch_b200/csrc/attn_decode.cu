@@ -302,6 +302,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
         const uint32_t qrow = kHeadDim * 2u;
         int cache0 = 0, cachen = 0;                           // groups [cache0, cache0 + cachen) fetched
         int cur_bg = -1, pos = 0, nsel = 0, nfrag = 1, frag = 0;
+        float ks_l = 1.f, vs_l = 1.f;                        // FP8: scales of the group's slot `lane`
         bool need_frag = false;
         int n = 0;
         bool ok = true;
@@ -340,6 +341,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
                     nsel = 0;
                 }
                 need_frag = nsel > 0;
+                if constexpr (kFp8) {
+                    // the scales of all the group's closed blocks in one round trip (lane i: slot i),
+                    // instead of one dependent load per item on the issuing lane
+                    ks_l = vs_l = 1.f;
+                    const int jl = lane < kTopK ? sm.row_sel[r][lane] : -1;
+                    if (nsel > 0 && jl >= 0 && jl < pos / kBlock) {
+                        const size_t si = size_t(bg) * a.nb_cap + jl;
+                        ks_l = __ldg(a.k_scale + si);
+                        vs_l = __ldg(a.v_scale + si);
+                    }
+                }
             }
             if (slot >= nsel) continue;                       // the row's tail is empty
             const int stage = n % kDecStages;
@@ -353,6 +365,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
             }
             // The copies go out first; the item's description and the arrivals that complete the
             // stage follow (the phase cannot complete before those arrivals).
+            float ksv = 1.f, vsv = 1.f;
+            if constexpr (kFp8) {
+                ksv = __shfl_sync(0xffffffffu, ks_l, slot);
+                vsv = __shfl_sync(0xffffffffu, vs_l, slot);
+            }
             int ntok = 0;
             if (lane == 0) {
                 const int c = pos / kBlock;
@@ -386,9 +403,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
                 for (int h = 0; h < Hg; ++h) bulk_load(sm.q[stage][h], qg + h * kHeadDim, qrow, &sm.full_k[stage]);
                 if (f8) {
                     tma_load_2d_hint(vs, &maps.v8, 0, row0, &sm.full_v[stage], pol);
-                    const size_t si = size_t(bg) * a.nb_cap + j;
-                    sm.meta_ks[stage] = __ldg(a.k_scale + si);
-                    sm.meta_vs[stage] = __ldg(a.v_scale + si);
+                    sm.meta_ks[stage] = ksv;
+                    sm.meta_vs[stage] = vsv;
                 } else if (full) {
                     for (int h = 0; h < 2; ++h)
                         tma_load_2d_hint(vs + h * 16384, &maps.v128, h * 64, row0, &sm.full_v[stage], pol);
