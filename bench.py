@@ -38,6 +38,7 @@ METRIC = "MSA prefill tok/s & decode step µs at 128K ctx; % of HBM/tensor roofl
 PREFILL = synth.WORKLOADS["prefill_128k_h64g8"]
 DECODE = synth.WORKLOADS["decode_128k_b16_h64g8"]
 PREFILL_32K = synth.WORKLOADS["prefill_32k_h64g8_planted"]
+PREFILL_4K = synth.WORKLOADS["prefill_4k_h4g1"]
 DECODE_1M = synth.WORKLOADS["decode_1m_ragged_b4_h64g8"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CSRC = os.path.join(ROOT, "block_sparse_gqa_branch_b200", "csrc")
@@ -986,6 +987,12 @@ def run_ours(args):
         r = prefill_report(PREFILL_32K, [max_over_ranks(statistics.mean(ti2))], [max_over_ranks(statistics.mean(tm2))],
                            peaks, peak_src, world, l2, k2)
         extra[PREFILL_32K.name] = r
+        torch.cuda.empty_cache()
+        # the small prefill (4,096 tokens, 4 query heads / 1 group): launch-bound, L2-resident
+        ti4, tm4, l4, k4 = time_prefill(torch, PREFILL_4K, dev, n_x, w_x, flush_l2)
+        k4 = {k: {"ms": max_over_ranks(k4[k]["ms"]), "launches": k4[k]["launches"]} for k in sorted(k4)}
+        extra[PREFILL_4K.name] = prefill_report(PREFILL_4K, [max_over_ranks(statistics.mean(ti4))],
+                                                [max_over_ranks(statistics.mean(tm4))], peaks, peak_src, world, l4, k4)
         torch.cuda.empty_cache()
         td5, l5 = time_decode(torch, DECODE_1M, dev, n_x, w_x, flush_l2)
         extra[DECODE_1M.name] = decode_report(
