@@ -299,7 +299,7 @@ __device__ __forceinline__ bool issue_o(KvSmem& sm, const PrefillArgs a, uint32_
     const uint32_t tS = tmem + buf * 128, tO = tmem + 256 + buf * 128;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks)
-        tc_mma_ts(tO, tS + ks * 8, sdesc_sw128(vbase + ks * 2048, 16384, 1024), idesc_o, ks > 0);
+        tc_mma_ts(tO, tS + 64 + ks * 8, sdesc_sw128(vbase + ks * 2048, 16384, 1024), idesc_o, ks > 0);
     tc_commit(&sm.o_full[buf]);
     if (p.last) tc_commit(&sm.v_empty);
     return true;
@@ -637,11 +637,17 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
                 const float ms = (mx == -INFINITY) ? 0.f : mx * sl2;
                 const float2 nm = make_float2(-ms, -ms);
                 float2 l2 = make_float2(0.f, 0.f);
+                // p = 2^(s*scale - m) -> TMEM as bf16, into columns 64..127 of the S buffer (the
+                // second half's S, already read): the second half first, from the registers the
+                // max pass left it in, then the first half, read again
 #pragma unroll
-                for (int p = 0; p < 2; ++p) {                       // p = 2^(s*scale - m), P -> TMEM as bf16
-                    tmem_ld32(tS + p * 64, va);
-                    tmem_ld32(tS + p * 64 + 32, vb);
-                    tmem_wait_ld();
+                for (int pp = 0; pp < 2; ++pp) {
+                    const int p = 1 - pp;
+                    if (p == 0) {
+                        tmem_ld32(tS, va);
+                        tmem_ld32(tS + 32, vb);
+                        tmem_wait_ld();
+                    }
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
                         uint32_t pk[16];
@@ -659,7 +665,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
                             l2 = fadd2(l2, pv);
                             pk[i] = pack_bf16x2(pv.x, pv.y);
                         }
-                        tmem_st16(tS + p * 32 + q * 16, pk);
+                        tmem_st16(tS + 64 + p * 32 + q * 16, pk);
                     }
                 }
                 tmem_wait_st();
