@@ -621,10 +621,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) attn_kvmajor_kernel(const __gri
                     tmem_wait_ld();
                     if (!item.diag) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(va[i]));
-                            m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(vb[i]));
-                        }
+                        for (int i = 0; i < 32; ++i)
+                            m4[i & 3] = fmax3(m4[i & 3], __uint_as_float(va[i]), __uint_as_float(vb[i]));
                     } else {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
