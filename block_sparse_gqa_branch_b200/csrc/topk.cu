@@ -18,6 +18,8 @@
 // about 20 of a chunk's 1,024 values pass, so a chunk costs its loads, a few integer
 // instructions per value and two or three rounds. No exponential and no float arithmetic
 // is used: only integer compares of the codes.
+#include <type_traits>
+
 #include "msa_common.cuh"
 
 namespace msa {
@@ -104,24 +106,26 @@ __global__ void __launch_bounds__(kTopkThreads, 3) topk_rows_kernel(const float*
         const float* r = scores + row * n;
         unsigned long long best = 0ull;       // lanes 0-15: the best 16 keys so far, descending
         uint32_t floor_code = 0u;             // code of the running k-th best
-        for (int base = 0; base < n; base += kChunk) {
+        // one chunk; kFull: every column of the chunk is < n (no per-value validity tests)
+        auto chunk = [&](int base, auto full_tag) {
+            constexpr bool kFull = decltype(full_tag)::value;
             float v[kPer];
-            uint32_t valid = 0u;              // bit p: this lane's value p is a column < n
+            uint32_t valid = kFull ? 0xffffffffu : 0u;   // bit p: this lane's value p is a column < n
 #pragma unroll
             for (int i = 0; i < kTopkSteps; ++i) {
                 const int c0 = base + (i * 32 + lane) * VEC;
                 if constexpr (VEC == 4) {
                     float4 x = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-                    if (c0 < n) {
+                    if (kFull || c0 < n) {
                         x = __ldcs(reinterpret_cast<const float4*>(r + c0));
-                        valid |= 0xfu << (4 * i);
+                        if (!kFull) valid |= 0xfu << (4 * i);
                     }
                     v[4 * i + 0] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
                 } else {
                     float x = -INFINITY;
-                    if (c0 < n) {
+                    if (kFull || c0 < n) {
                         x = __ldcs(r + c0);
-                        valid |= 1u << i;
+                        if (!kFull) valid |= 1u << i;
                     }
                     v[i] = x;
                 }
@@ -130,19 +134,23 @@ __global__ void __launch_bounds__(kTopkThreads, 3) topk_rows_kernel(const float*
             // exact path)
             float lm = -INFINITY, s0 = 0.f, s1 = 0.f;
 #pragma unroll
+            for (int p = 0; p + 1 < kPer; p += 2) lm = fmax3(lm, v[p], v[p + 1]);   // invalid values are -inf
+            if constexpr (kPer % 2 == 1) lm = fmaxf(lm, v[kPer - 1]);
+#pragma unroll
             for (int p = 0; p < kPer; ++p) {
-                lm = fmaxf(lm, v[p]);                    // invalid values are -inf
-                if (p & 1) s1 += ((valid >> p) & 1u) ? v[p] : 0.f;
-                else s0 += ((valid >> p) & 1u) ? v[p] : 0.f;
+                const float x = (kFull || ((valid >> p) & 1u)) ? v[p] : 0.f;
+                if (p & 1) s1 += x;
+                else s0 += x;
             }
             const bool nan_here = (s0 + s1) != (s0 + s1);
-            const uint32_t lcode = valid != 0u ? score_code(lm) : 0u;
+            const uint32_t lcode = (kFull || valid != 0u) ? score_code(lm) : 0u;
             const uint32_t kth_lane_max = __shfl_sync(0xffffffffu, warp_sort_desc32(lcode, lane), k - 1);
             const uint32_t bound = max(kth_lane_max, floor_code);
             const float bf = code_floor(bound);
             uint32_t pass = 0u;
 #pragma unroll
-            for (int p = 0; p < kPer; ++p) pass |= (((valid >> p) & 1u) != 0u && v[p] >= bf) ? (1u << p) : 0u;
+            for (int p = 0; p < kPer; ++p)
+                pass |= ((kFull || ((valid >> p) & 1u) != 0u) && v[p] >= bf) ? (1u << p) : 0u;
             const int cnt = __popc(pass);
             int incl = cnt;
 #pragma unroll
@@ -187,6 +195,10 @@ __global__ void __launch_bounds__(kTopkThreads, 3) topk_rows_kernel(const float*
                 }
                 __syncwarp();                            // the list and the staging rows are free again
             }
+        };
+        for (int base = 0; base < n; base += kChunk) {
+            if (base + kChunk <= n) chunk(base, std::true_type{});
+            else chunk(base, std::false_type{});
             floor_code = uint32_t(__shfl_sync(0xffffffffu, best, k - 1) >> 32);
         }
         if (lane < k) {                       // n >= k: the first chunk alone passes k values
