@@ -4,8 +4,8 @@
 One step = one pass of the whole hot path on synthetic inputs already resident in HBM:
   * prefill of 131,072 tokens, batch 1, 64 query heads / 8 KV groups (pooling, block scoring +
     exp-free top-16 selection, main-branch sparse attention), and
-  * one decode step of a batch of 16 sequences at 131,072 cached tokens (append + pooled-key
-    update, selection, attention split over the selected blocks), replayed from a CUDA graph.
+  * one decode step of a batch of 16 sequences at 131,072 cached tokens (selection, append +
+    pooled-key update, attention split over the selected blocks), replayed from a CUDA graph.
 L2 is flushed (256 MiB write, then 256 MiB read) before every timed step, outside the events.
 
 Printed value: prefill tokens/s over all ranks (131,072 x N / slowest rank's prefill time).
@@ -722,8 +722,8 @@ def decode_report(w, t_dec, peaks, peak_src, launches, traffic_name=None, scale=
         "workload": w.name, "decode_step_us": tdec * 1e6, "gpu_launches": int(launches),
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, "traffic_note": tnote,
-                     "kernel": ("decode step over the FP8 cache (append + close + select + attention, one graph replay)"
-                                if fp8 else "decode step (append + select + attention, one graph replay)"),
+                     "kernel": ("decode step over the FP8 cache (select + append + close + attention, one graph replay)"
+                                if fp8 else "decode step (select + append + attention, one graph replay)"),
                      "algorithmic": f"{dbytes['total']} B per step", "peak_source": f"{peak_src} copy"},
     }
 

@@ -155,7 +155,10 @@ void launch_pool_chunk(const void* k_idx, int B, int G, int64_t n, int64_t P, fl
 // ---------------------------------------------------------------- decode append
 // grid B, block 256. Writes the new token's K/V rows into the caches at position L_b and
 // folds its index keys into the open block's running sum; closes the block into `pooled`
-// when it becomes full.
+// when it becomes full. Launched with programmatic dependent launch: it may run during the
+// tail of the kernel before it in the stream (a decode step's selection, which reads only the
+// pooled keys of blocks below the open one), and it completes only after that kernel has, so
+// that a kernel waiting for this one also sees the one before.
 __global__ void __launch_bounds__(256) append_kernel(const uint16_t* __restrict__ k_idx_new,
                                                      const uint16_t* __restrict__ k_new,
                                                      const uint16_t* __restrict__ v_new,
@@ -165,7 +168,7 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t* __restrict_
                                                      float* __restrict__ tail_sum,
                                                      float* __restrict__ pooled, int64_t nb_cap,
                                                      WsHeader* hdr) {
-    grid_dep_launch();                 // the selection may start: it does not read what this writes
+    grid_dep_launch();                 // the next kernel may start its prologue
     const int b = blockIdx.x;
     // Every load goes out before the first use (one memory round trip: the selection streams
     // HBM at the same time, so each dependent round trip here would stretch the step).
@@ -191,6 +194,7 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t* __restrict_
     const bool close = ((pos + 1) % kBlock) == 0;
     if (pos < 0 || pos >= l_cap || (close && j >= nb_cap)) {
         if (threadIdx.x == 0) record_error(hdr, MSA_ERR_DEVICE_BOUNDS, KID_APPEND, b, 0, pos);
+        grid_dep_wait();
         return;
     }
     if (k_new != nullptr) {
@@ -214,17 +218,26 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t* __restrict_
         tail_sum[o] = sum;
         if (close) pooled[((size_t(b) * G + g) * nb_cap + j) * kIndexDim + e] = sum * (1.0f / kBlock);
     }
+    grid_dep_wait();                   // complete only after the kernel before this one
 }
 
 void launch_append(const void* k_idx_new, const void* k_new, const void* v_new, const int32_t* ctx_len,
                    int B, int G, void* k_cache, void* v_cache, int64_t l_cap, float* tail_sum,
                    float* pooled, int64_t nb_cap, void* ws, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(B));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     const KernelTimer kt(KID_APPEND, st);
-    append_kernel<<<B, 256, 0, st>>>(static_cast<const uint16_t*>(k_idx_new),
-                                     static_cast<const uint16_t*>(k_new),
-                                     static_cast<const uint16_t*>(v_new), ctx_len, G,
-                                     static_cast<uint16_t*>(k_cache), static_cast<uint16_t*>(v_cache),
-                                     l_cap, tail_sum, pooled, nb_cap, static_cast<WsHeader*>(ws));
+    cudaLaunchKernelEx(&cfg, append_kernel, static_cast<const uint16_t*>(k_idx_new),
+                       static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new), ctx_len, G,
+                       static_cast<uint16_t*>(k_cache), static_cast<uint16_t*>(v_cache), l_cap, tail_sum, pooled,
+                       nb_cap, static_cast<WsHeader*>(ws));
 }
 
 }  // namespace msa

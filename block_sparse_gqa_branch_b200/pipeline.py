@@ -78,16 +78,19 @@ def decode_buffers(B: int, Hq: int, G: int, max_pos: int, device, with_lse: bool
 
 def decode_step(q, q_idx, k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, tail_sum, pooled,
                 bufs: dict, stream=None):
-    """One decode step: append the new token (KV + pooled keys), select, attend.
+    """One decode step: select, append the new token (KV + pooled keys), attend.
     ctx_len [B] int32 on the device = tokens cached before the step (the new token's position).
     Caches: k_cache/v_cache [B,G,l_cap,128] bf16, pooled [B,G,nb_cap,64] fp32, tail_sum [B,G,64].
+    The selection comes first: it scores only blocks below the new token's own, which the append
+    does not change, so the append runs in its shadow (programmatic dependent launch) and the
+    attention, which needs both, waits for the append's completion (after the selection's).
     Returns (out [B,Hq,128], lse [B,Hq], sel [B,G,16])."""
     s, mp = bufs["shape"], bufs["max_pos"]
     l_cap = k_cache.shape[2]
     nb_cap = pooled.shape[2]
+    msa_index_select(s, q_idx, 1, ctx_len, mp, pooled, nb_cap, bufs["sel"], bufs["ws_select"], stream)
     msa_pooled_keys_append(s, k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, l_cap, tail_sum, pooled,
                            nb_cap, bufs["ws_append"], stream)
-    msa_index_select(s, q_idx, 1, ctx_len, mp, pooled, nb_cap, bufs["sel"], bufs["ws_select"], stream)
     msa_sparse_attn_decode(s, q, k_cache, v_cache, l_cap, ctx_len, mp, bufs["sel"], bufs["out"], bufs["lse"],
                            bufs["ws_attn"], stream)
     return bufs["out"], bufs["lse"], bufs["sel"]
@@ -115,17 +118,17 @@ def fp8_quantize_sequence(k_cache, v_cache, f8: dict, b: int, n_tokens: int, n_q
 
 def decode_step_fp8(q, q_idx, k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, tail_sum, pooled, f8: dict,
                     bufs: dict, stream=None):
-    """One decode step over the FP8 cache: append the new token (bf16 cache + pooled keys),
-    quantise the blocks it closes, select, attend (closed blocks from the e4m3 codes, the own
+    """One decode step over the FP8 cache: select, append the new token (bf16 cache + pooled
+    keys), quantise the block it closes, attend (closed blocks from the e4m3 codes, the own
     block from bf16). Returns (out, lse, sel)."""
     s, mp = bufs["shape"], bufs["max_pos"]
     l_cap = k_cache.shape[2]
     nb_cap = pooled.shape[2]
+    msa_index_select(s, q_idx, 1, ctx_len, mp, pooled, nb_cap, bufs["sel"], bufs["ws_select"], stream)
     msa_pooled_keys_append(s, k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, l_cap, tail_sum, pooled,
                            nb_cap, bufs["ws_append"], stream)
     msa_fp8_close_blocks(s, ctx_len, k_cache, v_cache, l_cap, f8["k_codes"], f8["v_codes"], f8["k_scale"],
                          f8["v_scale"], f8["nb_cap"], bufs["ws_append"], stream)
-    msa_index_select(s, q_idx, 1, ctx_len, mp, pooled, nb_cap, bufs["sel"], bufs["ws_select"], stream)
     msa_sparse_attn_decode_fp8(s, q, f8["k_codes"], f8["v_codes"], f8["k_scale"], f8["v_scale"], f8["nb_cap"],
                                k_cache, v_cache, l_cap, ctx_len, mp, bufs["sel"], bufs["out"], bufs["lse"],
                                bufs["ws_attn"], stream)

@@ -297,6 +297,11 @@ msa_status_t msa_sparse_attn_prefill_backward(const msa_shape_t *shape, const vo
  *                               multiple of Bk, else incremented by it
  *   pooled    fp32 [B, G, nb_cap, d_I]: when L_b + 1 completes block j = L_b / Bk,
  *                               pooled[b,g,j] = tail_sum / Bk
+ * The kernel is launched with programmatic dependent launch: it may start during the tail of
+ * the previous kernel of this library on the stream (the step's msa_index_select, which reads
+ * only the pooled keys of blocks below L_b / Bk) and completes only after that kernel, so a
+ * decode step may run selection, append, attention in that order; the attention needs the
+ * appended key and value.
  */
 msa_status_t msa_pooled_keys_append(const msa_shape_t *shape, const void *k_idx_new,
                                     const void *k_new, const void *v_new, const int32_t *ctx_len,
