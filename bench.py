@@ -72,8 +72,8 @@ CAPTURES = {
                 "small kernels not captured), scaled by the main-branch call's byte model",
         "profile": "profiles/attn_kvmajor_kernel_prefill8k.md, profiles/combine_kernel_prefill8k.md"},
     "topk_rows": {
-        "bytes": 536922112 + 7836928, "rows": 131072,
-        "sources": ["topk.cu"], "sha16": "a5bb54c67fd9d582",
+        "bytes": 536937472 + 7052800, "rows": 131072,
+        "sources": ["topk.cu"], "sha16": "dafaf2384b8ae8c3",
         "note": "DRAM bytes of topk_rows_kernel at 131,072 x 1,024 (ncu --set full, one launch), scaled by rows",
         "profile": "profiles/topk_rows_kernel_131072x1024.md"},
 }
