@@ -91,7 +91,8 @@ def test_recorded_captures_are_close_to_their_models():
         assert 0.9 <= c["attn_prefill"]["bytes"] / c["attn_prefill"]["model_bytes"] < 1.2
     if "topk_rows" in c:
         rows = c["topk_rows"]["rows"]
-        assert 1.0 <= c["topk_rows"]["bytes"] / (rows * 1024 * 4 + rows * 15 * 4) < 1.02
+        # reads equal the scores; some of the ids' writes can still be dirty in L2 when the kernel ends
+        assert 0.99 <= c["topk_rows"]["bytes"] / (rows * 1024 * 4 + rows * 15 * 4) < 1.02
 
 
 def test_attention_byte_model_is_part_of_the_call_model():
