@@ -8,7 +8,8 @@ import torch
 import oracle
 import synth
 from block_sparse_gqa_branch_b200 import (Shape, msa_get_device_status, msa_index_select,
-                                          msa_pool_index_keys, msa_pooled_keys_append, pipeline)
+                                          msa_pool_index_keys, msa_pooled_keys_append, msa_sparse_attn_decode,
+                                          pipeline)
 from tests.gpu_util import check_selection, dev_bf16, f32, host_bits
 from tests.msa_check import assert_close_attention
 
@@ -222,3 +223,51 @@ def test_decode_select_long_context_merge(cuda_ok, case):
         assert (sel == ref[0]).all(), (case, sel, ref[0])
     if case == "many_survivors":
         assert list(sel) == list(range(128, 142)) + [256, c]
+
+
+@pytest.mark.parametrize("order", ["append-select-attend", "select-append-attend"])
+def test_decode_step_order_gives_the_same_results(cuda_ok, order):
+    """The append may run before or after the step's selection (the selection scores only blocks
+    below the new token's own, and the append runs under programmatic dependent launch in the
+    shadow of the kernel before it): both orders, eager and replayed from a graph, give outputs
+    bit-identical to the pipeline's step, and a block that the step closes is pooled."""
+    w = synth.Workload(name="t", kind="decode", B=3, Hq=16, G=2, ctx=(2047, 3000, 383), seed=4242)
+    l_cap = 3200
+    ref = build_decode_state(w, l_cap)
+    o_ref, l_ref, s_ref = run_step(w, ref)
+    for graph in (False, True):
+        st = build_decode_state(w, l_cap)
+        s, mp = Shape.make(w.B, w.Hq, w.G), max(w.ctx)
+        bufs = pipeline.decode_buffers(w.B, w.Hq, w.G, mp, "cuda")
+
+        def step():
+            app = lambda: msa_pooled_keys_append(s, st["k_idx_new"], st["k_new"], st["v_new"], st["ctx"],  # noqa: E731
+                                                 st["k_cache"], st["v_cache"], l_cap, st["tail"], st["pooled"],
+                                                 st["nb_cap"], bufs["ws_append"])
+            sel = lambda: msa_index_select(s, st["q_idx"], 1, st["ctx"], mp, st["pooled"], st["nb_cap"],  # noqa: E731
+                                           bufs["sel"], bufs["ws_select"])
+            for f in ((app, sel) if order == "append-select-attend" else (sel, app)):
+                f()
+            msa_sparse_attn_decode(s, st["q"], st["k_cache"], st["v_cache"], l_cap, st["ctx"], mp, bufs["sel"],
+                                   bufs["out"], bufs["lse"], bufs["ws_attn"])
+
+        if graph:
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step()
+            g.replay()
+        else:
+            step()
+        torch.cuda.synchronize()
+        for key in ("ws_append", "ws_select", "ws_attn"):
+            stt, info = msa_get_device_status(bufs[key])
+            assert stt == 0, (key, stt, info)
+        assert np.array_equal(bufs["sel"].cpu().numpy(), s_ref)
+        assert np.array_equal(f32(host_bits(bufs["out"])), o_ref)
+        assert np.array_equal(bufs["lse"].cpu().numpy(), l_ref)
+        # sequence 0 (2,047 cached tokens) closes block 15 with this step
+        assert torch.equal(st["pooled"][0, :, 15], ref["pooled"][0, :, 15])
+        assert not torch.isnan(st["pooled"][0, :, 15]).any()
+        if graph:
+            del g
