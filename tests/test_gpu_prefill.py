@@ -95,3 +95,22 @@ def test_prefill_batch_of_two(cuda_ok):
             check_selection(r["sel"][b, :, g], o["sel"][b, :, g], o["kth"][b, :, g], x["q_idx"][b, :, g],
                             o["pooled"][b, g], np.arange(2400), label="prefill batch 2 N=2400")
     assert_close_attention(r["out"], o["out"], "batch 2")
+
+
+@pytest.mark.parametrize("B,N,Hq,G", [(2, 2100, 16, 8), (1, 16384 + 700, 8, 8)])
+def test_prefill_many_groups_and_two_ranges(cuda_ok, B, N, Hq, G):
+    """Eight groups over two sequences, and a sequence whose queries span two 16K-token ranges of
+    the inverted index (the second one ragged). Same bar as the other prefill cases, and the
+    outputs equal a second call bit for bit."""
+    w = synth.Workload(name="t", kind="prefill", B=B, N=N, Hq=Hq, G=G, seed=N + B)
+    x = synth.prefill_inputs_np(w)
+    r = run_prefill(w, x)
+    r2 = run_prefill(w, x)
+    assert np.array_equal(r["out"], r2["out"]) and np.array_equal(r["lse"], r2["lse"])
+    o = oracle.prefill(x, Hq, G, sel=r["sel"])
+    for b in range(B):
+        for g in range(G):
+            check_selection(r["sel"][b, :, g], o["sel"][b, :, g], o["kth"][b, :, g], x["q_idx"][b, :, g],
+                            o["pooled"][b, g], np.arange(N), label=f"prefill B={B} N={N} G={G}")
+    assert_close_attention(r["out"], o["out"], f"prefill B={B} N={N} G={G}")
+    np.testing.assert_allclose(r["lse"], o["lse"], rtol=0, atol=2e-3)
