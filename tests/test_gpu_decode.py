@@ -229,8 +229,10 @@ def test_decode_select_long_context_merge(cuda_ok, case):
 def test_decode_step_order_gives_the_same_results(cuda_ok, order):
     """The append may run before or after the step's selection (the selection scores only blocks
     below the new token's own, and the append runs under programmatic dependent launch in the
-    shadow of the kernel before it): both orders, eager and replayed from a graph, give outputs
-    bit-identical to the pipeline's step, and a block that the step closes is pooled."""
+    shadow of the kernel before it): both orders, eager and replayed from a graph, give the
+    pipeline's selection exactly and its output and lse up to the order of the fp32 merge of a
+    group split over CTAs (whichever CTA arrives last merges), and a block that the step closes
+    is pooled."""
     w = synth.Workload(name="t", kind="decode", B=3, Hq=16, G=2, ctx=(2047, 3000, 383), seed=4242)
     l_cap = 3200
     ref = build_decode_state(w, l_cap)
@@ -264,8 +266,9 @@ def test_decode_step_order_gives_the_same_results(cuda_ok, order):
             stt, info = msa_get_device_status(bufs[key])
             assert stt == 0, (key, stt, info)
         assert np.array_equal(bufs["sel"].cpu().numpy(), s_ref)
-        assert np.array_equal(f32(host_bits(bufs["out"])), o_ref)
-        assert np.array_equal(bufs["lse"].cpu().numpy(), l_ref)
+        o = f32(host_bits(bufs["out"]))
+        assert (np.abs(o - o_ref) <= np.abs(o_ref) * 2.0 ** -7 + 1e-6).all()    # one bf16 step at most
+        np.testing.assert_allclose(bufs["lse"].cpu().numpy(), l_ref, rtol=1e-6, atol=1e-6)
         # sequence 0 (2,047 cached tokens) closes block 15 with this step
         assert torch.equal(st["pooled"][0, :, 15], ref["pooled"][0, :, 15])
         assert not torch.isnan(st["pooled"][0, :, 15]).any()
