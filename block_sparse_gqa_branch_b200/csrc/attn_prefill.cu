@@ -127,17 +127,27 @@ __global__ void __launch_bounds__(1024) csr_scan_kernel(int* __restrict__ counts
         c0 = int(a / kBlock);
         c1 = int((z - 1) / kBlock) + 1;
     };
+    // the thread's counts are read kScanBatch at a time, the loads of a batch issued together
+    constexpr int kScanBatch = 8;
     long long se = 0, si = 0;
-    for (int64_t bin = lo; bin < hi; ++bin) {
-        const int j = int(bin % nbs);
-        if (j < nb) {
-            const int cnt = counts[bin];
-            se += cnt;
-            if (cnt > 0) si += (cnt + items_per_max - 1) / items_per_max;
-        } else {
-            int c0, c1;
-            diag_blocks(int((bin / nbs) % nR), c0, c1);
-            si += max(0, c1 - c0);
+    for (int64_t bin0 = lo; bin0 < hi; bin0 += kScanBatch) {
+        int cs[kScanBatch];
+#pragma unroll
+        for (int i = 0; i < kScanBatch; ++i) cs[i] = bin0 + i < hi ? counts[bin0 + i] : 0;
+#pragma unroll
+        for (int i = 0; i < kScanBatch; ++i) {
+            const int64_t bin = bin0 + i;
+            if (bin >= hi) break;
+            const int j = int(bin % nbs);
+            if (j < nb) {
+                const int cnt = cs[i];
+                se += cnt;
+                if (cnt > 0) si += (cnt + items_per_max - 1) / items_per_max;
+            } else {
+                int c0, c1;
+                diag_blocks(int((bin / nbs) % nR), c0, c1);
+                si += max(0, c1 - c0);
+            }
         }
     }
     s_e[threadIdx.x] = se;
@@ -152,27 +162,35 @@ __global__ void __launch_bounds__(1024) csr_scan_kernel(int* __restrict__ counts
         __syncthreads();
     }
     long long eoff = s_e[threadIdx.x] - se, ioff = s_i[threadIdx.x] - si;
-    for (int64_t bin = lo; bin < hi; ++bin) {
-        const int j = int(bin % nbs);
-        const int64_t seg = bin / nbs;
-        const int R = int(seg % nR);
-        const int bg = int(seg / nR);
-        if (j < nb) {
-            const int cnt = counts[bin];
-            offsets[bin] = int(eoff);
-            counts[bin] = 0;
-            for (int k0 = 0; k0 < cnt; k0 += items_per_max)
-                items[ioff++] = make_int4(bg, j, int(eoff + k0), min(items_per_max, cnt - k0));
-            eoff += cnt;
-        } else {
-            // diagonal items: the range's queries inside block c, as (first query index, count)
-            int c0, c1;
-            diag_blocks(R, c0, c1);
-            const int64_t qa = int64_t(R) * kRange, qz = imin64(N, int64_t(R + 1) * kRange);
-            for (int c = c0; c < c1; ++c) {
-                const int64_t f = int64_t(c) * kBlock - P > qa ? int64_t(c) * kBlock - P : qa;
-                const int64_t e = imin64(qz, int64_t(c + 1) * kBlock - P);
-                items[ioff++] = make_int4(bg, c | kDiagFlag, int(f), int(e - f));
+    for (int64_t bin0 = lo; bin0 < hi; bin0 += kScanBatch) {
+        int cs[kScanBatch];
+#pragma unroll
+        for (int i = 0; i < kScanBatch; ++i) cs[i] = bin0 + i < hi ? counts[bin0 + i] : 0;
+#pragma unroll
+        for (int i = 0; i < kScanBatch; ++i) {
+            const int64_t bin = bin0 + i;
+            if (bin >= hi) break;
+            const int j = int(bin % nbs);
+            const int64_t seg = bin / nbs;
+            const int R = int(seg % nR);
+            const int bg = int(seg / nR);
+            if (j < nb) {
+                const int cnt = cs[i];
+                offsets[bin] = int(eoff);
+                counts[bin] = 0;
+                for (int k0 = 0; k0 < cnt; k0 += items_per_max)
+                    items[ioff++] = make_int4(bg, j, int(eoff + k0), min(items_per_max, cnt - k0));
+                eoff += cnt;
+            } else {
+                // diagonal items: the range's queries inside block c, as (first query index, count)
+                int c0, c1;
+                diag_blocks(R, c0, c1);
+                const int64_t qa = int64_t(R) * kRange, qz = imin64(N, int64_t(R + 1) * kRange);
+                for (int c = c0; c < c1; ++c) {
+                    const int64_t f = int64_t(c) * kBlock - P > qa ? int64_t(c) * kBlock - P : qa;
+                    const int64_t e = imin64(qz, int64_t(c + 1) * kBlock - P);
+                    items[ioff++] = make_int4(bg, c | kDiagFlag, int(f), int(e - f));
+                }
             }
         }
     }
