@@ -29,6 +29,8 @@ NAN_BF16 = 0x7FC0
     (3100, 16, 2, [700, 1100, 1, 60, 1239]),
     (4000, 64, 8, [2500, 1500]),
     (2300, 8, 1, [128, 2047, 125]),
+    # the last chunk scores up to 78 candidates: two 64-candidate chunks of split pooled keys
+    (10050, 16, 2, [8100, 1950]),
 ])
 def test_chunked_prefill_matches_oracle(cuda_ok, N, Hq, G, chunks):
     assert sum(chunks) == N
