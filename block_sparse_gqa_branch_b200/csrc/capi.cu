@@ -184,6 +184,22 @@ msa_status_t make_tmap_qidx(CUtensorMap* m, const void* base, int G, uint64_t ro
     }
     return MSA_OK;
 }
+msa_status_t make_tmap_split(CUtensorMap* m, const void* base, uint64_t nbp, uint64_t nbg3) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return MSA_ERR_CUDA;
+    cuuint64_t dims[3] = {uint64_t(kIndexDim), nbp, nbg3};
+    cuuint64_t strides[2] = {uint64_t(kIndexDim) * 2, nbp * kIndexDim * 2};
+    cuuint32_t box[3] = {64, 32, 3};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error = int(r);
+        return MSA_ERR_CUDA;
+    }
+    return MSA_OK;
+}
 msa_status_t make_tmap_q_rows(CUtensorMap* m, const void* base, uint64_t rows) {
     auto fn = encode_fn();
     if (fn == nullptr) return MSA_ERR_CUDA;

@@ -48,6 +48,9 @@ msa_status_t make_tmap_qidx(CUtensorMap* m, const void* base, int G, uint64_t ro
 // Rows of 128 bf16 viewed as (64 columns, row, d half): box {64, 8, 2} lands 8 rows with both
 // halves as [half][8 rows][128 B] (128B swizzle)
 msa_status_t make_tmap_q_rows(CUtensorMap* m, const void* base, uint64_t rows);
+// Split pooled keys [nbg3][nbp][64] bf16 as a 3-D tensor {64, nbp, nbg3}; box {64, 32, 3}: 32
+// candidates of the three terms of one (sequence, group) as [term][32 rows][128 B] (128B swizzle)
+msa_status_t make_tmap_split(CUtensorMap* m, const void* base, uint64_t nbp, uint64_t nbg3);
 
 // byte offsets, inside a prefill workspace, of the inverted index's item count, items and entries
 struct IndexOffsets { size_t nitems, items, list; };

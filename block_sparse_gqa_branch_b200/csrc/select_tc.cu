@@ -8,19 +8,22 @@
 //
 // A pre-pass splits every pooled key (fp32) exactly into three bf16 terms (hi = bf16(x),
 // mid = bf16(x - hi), lo = bf16(x - hi - mid): 24 significant bits) once, into the workspace.
-// Then one CTA of 128 threads per (128-token query block c, group g, sequence b), heaviest
-// blocks first. The tile's index queries Q_I (128 x 64 bf16) arrive by TMA. The fully-past
-// candidates j < c go 64 per chunk: the threads copy the chunk's three terms into three K-major
-// shared-memory operands (the loads of chunk k + 1 are in flight while chunk k is ranked); one
-// thread issues the 12 tcgen05.mma (3 terms x 4 k-steps of 16) that accumulate
-// S = Q_I x Kbar^T (128 x 64, fp32) into tensor memory. Scores are fp32-accurate (a single bf16 term would move selections
-// beyond the near-tie rule). Two S buffers let chunk k + 1's MMAs run while chunk k is ranked;
-// 64-candidate chunks keep the CTA at 65 KB of shared memory, three CTAs per SM.
-// Thread i owns query row i (tensor-memory lane i): it reads its row's 64 scores with
-// tcgen05.ld, marks without branches the candidates that beat its current 15th best, and
-// inserts only those, in id order, into its running best 15 -- compares only, so equal scores
-// keep the lower block id. The 1/sqrt(d_I) factor is an exact power of two and cannot change
-// the order, so it is not applied.
+// Then one CTA per (128-token query block c, group g, sequence b), heaviest blocks first: four
+// ranking warps (thread i owns query row i, tensor-memory lane i) and one producer warp. The
+// producer brings the tile's index queries Q_I (128 x 64 bf16) and, 32 fully-past candidates
+// j < c per item, the three split terms by TMA into a 3-stage ring, and issues the item's 12
+// tcgen05.mma (3 terms x 4 k-steps of 16) that accumulate S = Q_I x Kbar^T (128 x 32, fp32)
+// into one of two tensor-memory buffers. Scores are fp32-accurate (a single bf16 term would
+// move selections beyond the near-tie rule).
+// The ranking runs in two passes over the candidates, exp-free and compare-only:
+//  * pass A keeps only the 15 largest score VALUES per query: the first 32 through a sorting
+//    network, then the candidates that beat the current 15th value, two per round, through a
+//    branch-free min/max merge (no block ids to carry, no dependent chain);
+//  * pass B recomputes the same scores (the same MMAs on the same operands: bit-identical) and
+//    emits, in id order, every block above the 15th value and then the first blocks equal to
+//    it until 15 are taken -- exactly "score descending, then lower block id", already sorted.
+// The 1/sqrt(d_I) factor is an exact power of two and cannot change the order, so it is not
+// applied.
 #include <atomic>
 
 #include "msa_common.cuh"
@@ -28,13 +31,17 @@
 namespace msa {
 
 constexpr int kTcRows = 128;       // queries per tile (MMA M)
-constexpr int kTcCand = 64;        // candidates per chunk (MMA N)
-constexpr int kTcKeep = kTopK - 1;
+constexpr int kTcCand = 32;        // candidates per item (MMA N)
+constexpr int kTcStages = 3;       // operand stages in flight
+constexpr int kTcThreads = 160;    // 4 ranking warps (one query row per thread) + 1 producer warp
+constexpr int kStashStride = 36;   // floats per ranking thread's stash row (16-byte rows, conflict-free stores)
+constexpr uint32_t kTcStageBytes = 3 * kTcCand * 128;
 
 struct __align__(1024) SelTcSmem {
-    uint8_t q[kTcRows * 128];               // Q_I tile [128 rows][64 bf16], 128B swizzle
-    uint8_t kb[2][3][kTcCand * 128];        // split pooled keys [buf][hi, mid, lo][64 cand][64 bf16], 128B swizzle
-    uint64_t q_full, mma_done[2];
+    uint8_t q[kTcRows * 128];                   // Q_I tile [128 rows][64 bf16], 128B swizzle
+    uint8_t kb[kTcStages][3][kTcCand * 128];    // split pooled keys [stage][hi, mid, lo][32 cand][64 bf16], 128B swizzle
+    float stash[kTcRows * kStashStride];        // each ranking thread's scores of the current item
+    uint64_t q_full, kfull[kTcStages], kempty[kTcStages], sfull[2], sempty[2];
     uint32_t tmem_base;
 };
 
@@ -73,50 +80,75 @@ __global__ void __launch_bounds__(256) split_pooled_kernel(const float* __restri
                                pack_bf16x2(ls[6], ls[7]));
 }
 
-// 64 contiguous bytes at each of three addresses (the three terms of one candidate's half
-// row), issued back to back
-__device__ __forceinline__ void ld_nc_64Bx3(const uint4* p0, const uint4* p1, const uint4* p2, uint4 (&v)[3][4]) {
-    asm volatile(
-        "ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%48];\n\tld.global.nc.v4.u32 {%4, %5, %6, %7}, [%48+16];\n\t"
-        "ld.global.nc.v4.u32 {%8, %9, %10, %11}, [%48+32];\n\tld.global.nc.v4.u32 {%12, %13, %14, %15}, [%48+48];\n\t"
-        "ld.global.nc.v4.u32 {%16, %17, %18, %19}, [%49];\n\tld.global.nc.v4.u32 {%20, %21, %22, %23}, [%49+16];\n\t"
-        "ld.global.nc.v4.u32 {%24, %25, %26, %27}, [%49+32];\n\tld.global.nc.v4.u32 {%28, %29, %30, %31}, [%49+48];\n\t"
-        "ld.global.nc.v4.u32 {%32, %33, %34, %35}, [%50];\n\tld.global.nc.v4.u32 {%36, %37, %38, %39}, [%50+16];\n\t"
-        "ld.global.nc.v4.u32 {%40, %41, %42, %43}, [%50+32];\n\tld.global.nc.v4.u32 {%44, %45, %46, %47}, [%50+48];"
-        : "=r"(v[0][0].x), "=r"(v[0][0].y), "=r"(v[0][0].z), "=r"(v[0][0].w), "=r"(v[0][1].x), "=r"(v[0][1].y),
-          "=r"(v[0][1].z), "=r"(v[0][1].w), "=r"(v[0][2].x), "=r"(v[0][2].y), "=r"(v[0][2].z), "=r"(v[0][2].w),
-          "=r"(v[0][3].x), "=r"(v[0][3].y), "=r"(v[0][3].z), "=r"(v[0][3].w), "=r"(v[1][0].x), "=r"(v[1][0].y),
-          "=r"(v[1][0].z), "=r"(v[1][0].w), "=r"(v[1][1].x), "=r"(v[1][1].y), "=r"(v[1][1].z), "=r"(v[1][1].w),
-          "=r"(v[1][2].x), "=r"(v[1][2].y), "=r"(v[1][2].z), "=r"(v[1][2].w), "=r"(v[1][3].x), "=r"(v[1][3].y),
-          "=r"(v[1][3].z), "=r"(v[1][3].w), "=r"(v[2][0].x), "=r"(v[2][0].y), "=r"(v[2][0].z), "=r"(v[2][0].w),
-          "=r"(v[2][1].x), "=r"(v[2][1].y), "=r"(v[2][1].z), "=r"(v[2][1].w), "=r"(v[2][2].x), "=r"(v[2][2].y),
-          "=r"(v[2][2].z), "=r"(v[2][2].w), "=r"(v[2][3].x), "=r"(v[2][3].y), "=r"(v[2][3].z), "=r"(v[2][3].w)
-        : "l"(p0), "l"(p1), "l"(p2));
+// compare-exchange: a takes the larger value, b the smaller
+__device__ __forceinline__ void cx_desc(float& a, float& b) {
+    const float hi = fmaxf(a, b);
+    b = fminf(a, b);
+    a = hi;
 }
 
-__device__ __forceinline__ void sort16_ids(int (&x)[16]) {
+// bitonic sorting network on 16 values, descending
+__device__ __forceinline__ void sort16_desc(float (&a)[16]) {
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
+    for (int k = 2; k <= 16; k <<= 1)
 #pragma unroll
-        for (int i = (r & 1); i + 1 < 16; i += 2) {
-            const int a = min(x[i], x[i + 1]), bb = max(x[i], x[i + 1]);
-            x[i] = a; x[i + 1] = bb;
-        }
-    }
+        for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int p = i ^ j;
+                if (p > i) {
+                    if ((i & k) == 0) cx_desc(a[i], a[p]);
+                    else cx_desc(a[p], a[i]);
+                }
+            }
+}
+
+// best = the 15 largest of v[0..31] (no NaN), descending: both halves sorted, the larger of
+// a[i] and b[15 - i] (the top 16, as a bitonic sequence), then a bitonic merge
+__device__ __forceinline__ void top15_of_32(const float (&v)[32], float (&best)[kTopK - 1]) {
+    float a[16], b[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) { a[i] = v[i]; b[i] = v[16 + i]; }
+    sort16_desc(a);
+    sort16_desc(b);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] = fmaxf(a[i], b[15 - i]);
+#pragma unroll
+    for (int j = 8; j > 0; j >>= 1)
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if ((i ^ j) > i) cx_desc(a[i], a[i ^ j]);
+#pragma unroll
+    for (int i = 0; i < kTopK - 1; ++i) best[i] = a[i];
+}
+
+// Merges two values x1, x2 (no NaN; -inf for none) into the descending list b of 15: the
+// r-th largest of the union of a sorted list and a sorted pair x >= y is
+// max(b[r], min(b[r-1], x), min(b[r-2], y)) with b[-1] = b[-2] = +inf. Branch-free, and every
+// entry is independent of the others.
+__device__ __forceinline__ void merge2(float (&b)[kTopK - 1], float x1, float x2) {
+    const float x = fmaxf(x1, x2), y = fminf(x1, x2);
+    float nb[kTopK - 1];
+    nb[0] = fmaxf(b[0], x);
+    nb[1] = fmax3(b[1], fminf(b[0], x), y);
+#pragma unroll
+    for (int r = 2; r < kTopK - 1; ++r) nb[r] = fmax3(b[r], fminf(b[r - 1], x), fminf(b[r - 2], y));
+#pragma unroll
+    for (int r = 0; r < kTopK - 1; ++r) b[r] = nb[r];
 }
 
 // Queries are the N tokens at positions P .. P + N - 1 (P = 0 for a whole prefill); query row i
 // of q_idx and sel is position P + i.
-__global__ void __launch_bounds__(128) select_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
-                                                                int64_t N, int64_t P, int G,
-                                                                const uint16_t* __restrict__ split, int64_t nbp,
-                                                                int32_t* __restrict__ sel, WsHeader* hdr) {
+__global__ void __launch_bounds__(kTcThreads, 3) select_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                                         const __grid_constant__ CUtensorMap tmS,
+                                                                         int64_t N, int64_t P, int G,
+                                                                         int32_t* __restrict__ sel, WsHeader* hdr) {
     extern __shared__ uint8_t smem_raw[];
     SelTcSmem& sm = *reinterpret_cast<SelTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int c = int((P + N - 1) / kBlock) - int(blockIdx.x), g = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int64_t t = int64_t(c) * kBlock + tid;            // this thread's query position
-    const bool live = t >= P && t < P + N;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t t = int64_t(c) * kBlock + tid;            // a ranking thread's query position
+    const bool live = warp < 4 && t >= P && t < P + N;
     int32_t* out = sel + ((size_t(b) * N + (live ? t - P : 0)) * G + g) * kTopK;
     if (c + 1 <= kTopK) {                                    // every block 0..c is taken
         if (live) {
@@ -130,10 +162,15 @@ __global__ void __launch_bounds__(128) select_prefill_tc_kernel(const __grid_con
     }
     if (tid == 0) {
         mbar_init(&sm.q_full, 1);
-        mbar_init(&sm.mma_done[0], 1);
-        mbar_init(&sm.mma_done[1], 1);
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(&sm.kfull[s], 1);
+            mbar_init(&sm.kempty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.sfull[i], 1);
+            mbar_init(&sm.sempty[i], 4);
+        }
         fence_barrier_init();
-        tma_prefetch_desc(&tmQ);
     }
     if (warp == 0) {
         tmem_alloc(&sm.tmem_base, 2 * kTcCand);
@@ -143,127 +180,157 @@ __global__ void __launch_bounds__(128) select_prefill_tc_kernel(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    if (tid == 0) {
-        // rows 128 c - P .. + 127 of this sequence's queries (rows outside the queries are read
-        // as zeros or as a neighbour's rows and never written)
-        mbar_arrive_expect_tx(&sm.q_full, kTcRows * 128);
-        tma_load_3d(sm.q, &tmQ, 0, g, int(int64_t(b) * N + int64_t(c) * kBlock - P), &sm.q_full);
-    }
-    const int nchunks = (c + kTcCand - 1) / kTcCand;
-    const uint16_t* sbase = split + size_t(b * G + g) * 3 * nbp * kIndexDim;
-    const uint32_t idesc = idesc_bf16_f32(kTcRows, kTcCand, 0, 0);   // both operands K-major
-
-    // threads 2 i and 2 i + 1 copy candidate j0 + i of a chunk, 32 dims (64 bytes) of each of the
-    // three terms: loaded into registers one chunk ahead, stored into the swizzled operands
-    uint4 pre[3][4];
-    auto load_chunk = [&](int k) {
-        const int r = tid >> 1, j = k * kTcCand + r;             // j < nbp: nbp is a multiple of 64
-        const uint4* p = reinterpret_cast<const uint4*>(sbase + size_t(j) * kIndexDim) + 4 * (tid & 1);
-        const size_t term = size_t(nbp) * kIndexDim / 8;
-        ld_nc_64Bx3(p, p + term, p + 2 * term, pre);
-    };
-    auto store_chunk = [&](int k) {
-        const int r = tid >> 1;
-        uint8_t* dst = sm.kb[k & 1][0];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            const uint32_t off = sw128(uint32_t(r), uint32_t(4 * (tid & 1) + c4));
-#pragma unroll
-            for (int t = 0; t < 3; ++t) *reinterpret_cast<uint4*>(dst + t * kTcCand * 128 + off) = pre[t][c4];
-        }
-        fence_proxy_async();                                 // visible to the tensor cores
-    };
-    // one thread: S[buf] = sum over the three terms of Q_I x term^T
-    auto issue = [&](int k) {
-        const int buf = k & 1;
-        const uint32_t qb = smem_u32(sm.q), kbase = smem_u32(sm.kb[buf][0]);
-#pragma unroll
-        for (int part = 0; part < 3; ++part)
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc_mma_ss(tmem + buf * kTcCand, sdesc_sw128(qb + ks * 32, 16, 1024),
-                          sdesc_sw128(kbase + part * kTcCand * 128 + ks * 32, 16, 1024), idesc,
-                          (part | ks) != 0);
-        tc_commit(&sm.mma_done[buf]);
-    };
-
-    float best[kTcKeep];
-    int bid[kTcKeep];
-#pragma unroll
-    for (int i = 0; i < kTcKeep; ++i) { best[i] = -INFINITY; bid[i] = 0x7fffffff; }
-    // Every wait is bounded. A wait that gives up makes its warp stop ranking; the whole CTA then
-    // leaves the loop at the next barrier, and thread 0 waits (bounded) for the MMAs it issued
-    // before the tensor memory is freed.
+    const int n = (c + kTcCand - 1) / kTcCand;               // items per pass
+    const int items = 2 * n;                                  // pass A (values), pass B (block ids)
     bool ok = true;
-    int issued = 0, waited = 0;                              // chunks whose MMAs were issued / waited for
-    load_chunk(0);
-    store_chunk(0);
-    if (nchunks > 1) load_chunk(1);
-    __syncthreads();
-    if (tid == 0) {
-        ok = mbar_wait(&sm.q_full, 0, hdr, KID_SELECT_PREFILL);
-        if (ok) {
-            tc_fence_after();
-            issue(0);
-            issued = 1;
-        }
-    }
-    ok = __syncthreads_and(ok);
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
-    for (int k = 0; ok && k < nchunks; ++k) {
-        __syncthreads();                                     // chunk k - 1's stashed scores all read
-        if (k + 1 < nchunks) {
-            store_chunk(k + 1);                              // its buffer's MMAs (chunk k - 1) are done
-            if (k + 2 < nchunks) load_chunk(k + 2);          // in flight while chunk k is ranked
-        }
-        tc_fence_before();
-        if (!__syncthreads_and(ok)) { ok = false; break; }   // stored; chunk k - 1's scores all read
-        tc_fence_after();
-        if (tid == 0 && k + 1 < nchunks) { issue(k + 1); issued = k + 2; }
-        ok = __all_sync(0xffffffffu, mbar_wait(&sm.mma_done[k & 1], (k >> 1) & 1, hdr, KID_SELECT_PREFILL));
-        if (!ok) continue;                                   // the loop ends at the next barrier
-        waited = k + 1;
-        tc_fence_after();
-        const int j0 = k * kTcCand;
-        // the chunk's operand buffer is free once its MMAs are done: it stashes each thread's
-        // 32 scores of a pass (row stride 33 floats: conflict-free), so that an insertion reads
-        // its score with one shared-memory load
-        float* stash = reinterpret_cast<float*>(sm.kb[k & 1][0]) + tid * 33;
-#pragma unroll 1
-        for (int q32 = 0; q32 < kTcCand / 32; ++q32) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_off + (k & 1) * kTcCand + q32 * 32, v);
-            tmem_wait_ld();
-            // mark the candidates that beat the current 15th score (no branches), then insert
-            // only those, in id order: the warp runs as many rounds as its busiest lane
-            unsigned msk = 0u;
-            const float thr = best[kTcKeep - 1];
+    int ids[kTopK - 1];                                       // a ranking thread's emitted blocks
+    int cnt = 0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                msk |= (j0 + q32 * 32 + i < c && __uint_as_float(v[i]) > thr) ? (1u << i) : 0u;
-            if (__any_sync(0xffffffffu, msk != 0u)) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) stash[i] = __uint_as_float(v[i]);
+    for (int i = 0; i < kTopK - 1; ++i) ids[i] = -1;
+
+    if (warp == 4) {
+        // producer: TMA of the queries and of each item's 32 candidates (three split terms), and
+        // the 12 MMAs of an item once its operands are in and its score buffer has been read
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmS);
+            const int zb = (b * G + g) * 3;
+            mbar_arrive_expect_tx(&sm.q_full, kTcRows * 128);
+            tma_load_3d(sm.q, &tmQ, 0, g, int(int64_t(b) * N + int64_t(c) * kBlock - P), &sm.q_full);
+            int loaded = 0, landed = 0, mmas = 0;             // items loaded / waited for / multiplied
+            for (; loaded < items && loaded < kTcStages; ++loaded) {
+                mbar_arrive_expect_tx(&sm.kfull[loaded], kTcStageBytes);
+                tma_load_3d(sm.kb[loaded][0], &tmS, 0, kTcCand * (loaded % n), zb, &sm.kfull[loaded]);
             }
-            while (msk != 0u) {
-                const int i = __ffs(msk) - 1;
-                msk &= msk - 1u;
-                const float sc = stash[i];
-                if (sc > best[kTcKeep - 1]) {
-                    best[kTcKeep - 1] = sc; bid[kTcKeep - 1] = j0 + q32 * 32 + i;
+            ok = mbar_wait(&sm.q_full, 0, hdr, KID_SELECT_PREFILL);
+            const uint32_t idesc = idesc_bf16_f32(kTcRows, kTcCand, 0, 0);   // both operands K-major
+            const uint32_t qb = smem_u32(sm.q);
+            for (int it = 0; ok && it < items; ++it) {
+                const int s = it % kTcStages;
+                ok = mbar_wait(&sm.kfull[s], (it / kTcStages) & 1, hdr, KID_SELECT_PREFILL);
+                if (!ok) break;
+                landed = it + 1;
+                if (it >= 2) ok = mbar_wait(&sm.sempty[it & 1], ((it >> 1) - 1) & 1, hdr, KID_SELECT_PREFILL);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t kbase = smem_u32(sm.kb[s][0]);
 #pragma unroll
-                    for (int r = kTcKeep - 1; r > 0; --r) {
-                        if (best[r] > best[r - 1]) {
-                            float tv = best[r]; best[r] = best[r - 1]; best[r - 1] = tv;
-                            int ti = bid[r]; bid[r] = bid[r - 1]; bid[r - 1] = ti;
-                        }
+                for (int part = 0; part < 3; ++part)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        tc_mma_ss(tmem + (it & 1) * kTcCand, sdesc_sw128(qb + ks * 32, 16, 1024),
+                                  sdesc_sw128(kbase + part * kTcCand * 128 + ks * 32, 16, 1024), idesc,
+                                  (part | ks) != 0);
+                tc_commit(&sm.sfull[it & 1]);
+                tc_commit(&sm.kempty[s]);
+                mmas = it + 1;
+                // item it - 1's stage is free once its MMAs are done: load item it - 1 + stages
+                if (it >= 1 && loaded < items) {
+                    const int sp = (it - 1) % kTcStages;
+                    ok = mbar_wait(&sm.kempty[sp], ((it - 1) / kTcStages) & 1, hdr, KID_SELECT_PREFILL);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&sm.kfull[sp], kTcStageBytes);
+                    tma_load_3d(sm.kb[sp][0], &tmS, 0, kTcCand * (loaded % n), zb, &sm.kfull[sp]);
+                    ++loaded;
+                }
+            }
+            // nothing may still write this CTA's shared or tensor memory when it exits: wait
+            // (bounded) for the last MMAs and for every copy not yet waited for
+            if (mmas > 0) mbar_wait(&sm.kempty[(mmas - 1) % kTcStages], ((mmas - 1) / kTcStages) & 1, hdr,
+                                    KID_SELECT_PREFILL);
+            for (int it = landed; it < loaded; ++it)
+                mbar_wait(&sm.kfull[it % kTcStages], (it / kTcStages) & 1, hdr, KID_SELECT_PREFILL);
+        }
+        __syncwarp();
+    } else {
+        // ranking thread: query row tid (tensor-memory lane tid). Pass A keeps the 15 largest
+        // score values (compare-only min/max networks); pass B recomputes the same scores and
+        // emits, in id order, every block above the 15th value and the first blocks equal to it.
+        const uint32_t lane_off = uint32_t(warp * 32) << 16;
+        float* stash = sm.stash + tid * kStashStride;
+        float best[kTopK - 1];
+        float thr = -INFINITY;
+        int eq = 0, need_eq = 0;
+#pragma unroll
+        for (int i = 0; i < kTopK - 1; ++i) best[i] = -INFINITY;
+        for (int it = 0; it < items; ++it) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.sfull[it & 1], (it >> 1) & 1, hdr, KID_SELECT_PREFILL));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + (it & 1) * kTcCand, v);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.sempty[it & 1]);
+            const bool pass_a = it < n;
+            const int j0 = (pass_a ? it : it - n) * kTcCand;
+            const unsigned valid = c - j0 >= 32 ? 0xffffffffu : (1u << (c - j0)) - 1u;
+            if (it == 0) {                                    // the first 32 candidates: a network
+                float f[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float x = __uint_as_float(v[i]);
+                    f[i] = ((valid >> i) & 1u) && x == x ? x : -INFINITY;
+                }
+                top15_of_32(f, best);
+                continue;
+            }
+            if (it == n) {                                    // pass B starts: the 15th value decides
+                thr = best[kTopK - 2];
+                int gt = 0;
+#pragma unroll
+                for (int i = 0; i < kTopK - 1; ++i) gt += best[i] > thr ? 1 : 0;
+                need_eq = kTopK - 1 - gt;
+            }
+            unsigned msk = 0u;
+            if (pass_a) {
+                const float th = best[kTopK - 2];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) msk |= __uint_as_float(v[i]) > th ? (1u << i) : 0u;
+            } else {
+                if (!__any_sync(0xffffffffu, cnt < kTopK - 1)) continue;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) msk |= __uint_as_float(v[i]) >= thr ? (1u << i) : 0u;
+                if (cnt >= kTopK - 1) msk = 0u;
+            }
+            msk &= valid;
+            if (msk != 0u) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4*>(stash + i) = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                                                        __uint_as_float(v[i + 2]),
+                                                                        __uint_as_float(v[i + 3]));
+            }
+            if (pass_a) {
+                // two candidates per round; a round merges what beat the 15th value when the item
+                // was read (a value that no longer does leaves the list unchanged)
+                while (msk != 0u) {
+                    const int i1 = __ffs(msk) - 1;
+                    msk &= msk - 1u;
+                    const float x1 = stash[i1];
+                    const int i2 = msk != 0u ? __ffs(msk) - 1 : i1;
+                    const float x2 = msk != 0u ? stash[i2] : -INFINITY;
+                    msk &= msk - 1u;
+                    merge2(best, x1, x2);
+                }
+            } else {
+                while (msk != 0u) {
+                    const int i = __ffs(msk) - 1;
+                    msk &= msk - 1u;
+                    const float x = stash[i];
+                    const bool above = x > thr;
+                    if (above || eq < need_eq) {
+                        eq += above ? 0 : 1;
+#pragma unroll
+                        for (int r = 0; r < kTopK - 2; ++r) ids[r] = ids[r + 1];
+                        ids[kTopK - 2] = j0 + i;
+                        if (++cnt == kTopK - 1) msk = 0u;
                     }
                 }
             }
         }
     }
-    if (tid == 0)                                            // MMAs issued but not waited for (failure path)
-        for (int kk = waited; kk < issued; ++kk) mbar_wait(&sm.mma_done[kk & 1], (kk >> 1) & 1, hdr, KID_SELECT_PREFILL);
     tc_fence_before();
     ok = __syncthreads_and(ok);
     if (warp == 0) {
@@ -271,23 +338,36 @@ __global__ void __launch_bounds__(128) select_prefill_tc_kernel(const __grid_con
         tmem_dealloc(tmem, 2 * kTcCand);
     }
     if (!ok || !live) return;
-    int ids[16];
+    // ids[15 - cnt ..] hold the emitted blocks in ascending order (all 15 unless scores were NaN),
+    // then the query's own block c (the largest id), then -1 padding
+    int o16[kTopK];
+    if (cnt == kTopK - 1) {
 #pragma unroll
-    for (int i = 0; i < kTcKeep; ++i) ids[i] = bid[i];
-    ids[15] = c;
-    sort16_ids(ids);
+        for (int i = 0; i < kTopK - 1; ++i) o16[i] = ids[i];
+        o16[kTopK - 1] = c;
+    } else {
+#pragma unroll
+        for (int r = 0; r < kTopK; ++r) {
+            int x = -1;
+#pragma unroll
+            for (int i = 0; i < kTopK - 1; ++i) x = (i == kTopK - 1 - cnt + r) ? ids[i] : x;
+            o16[r] = r < cnt ? x : (r == cnt ? c : -1);
+        }
+    }
     int4* o = reinterpret_cast<int4*>(out);
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) o[q4] = make_int4(ids[4 * q4], ids[4 * q4 + 1], ids[4 * q4 + 2], ids[4 * q4 + 3]);
+    for (int q4 = 0; q4 < 4; ++q4) o[q4] = make_int4(o16[4 * q4], o16[4 * q4 + 1], o16[4 * q4 + 2], o16[4 * q4 + 3]);
 }
 
 // Blocks of split pooled keys the selection for queries up to position n_end - 1 keeps in its
 // workspace (the fully-past candidates of the last query, rounded up to whole 64-candidate
 // chunks), and the workspace bytes that need.
 int64_t select_split_blocks(int64_t n_end) {
+    constexpr int64_t kRound = 64;                           // a multiple of the item size
+    static_assert(kRound % kTcCand == 0, "whole items");
     const int64_t ncand = n_end > 0 ? (n_end - 1) / kBlock : 0;
-    const int64_t chunks = (ncand + kTcCand - 1) / kTcCand;
-    return (chunks > 0 ? chunks : 1) * kTcCand;
+    const int64_t chunks = (ncand + kRound - 1) / kRound;
+    return (chunks > 0 ? chunks : 1) * kRound;
 }
 size_t select_split_offset() { return (sizeof(WsHeader) + 255) / 256 * 256; }
 size_t select_prefill_ws_bytes(int B, int G, int64_t n_end) {
@@ -296,11 +376,12 @@ size_t select_prefill_ws_bytes(int B, int G, int64_t n_end) {
 
 msa_status_t launch_select_prefill_tc(const void* q_idx, int B, int G, int64_t N, int64_t P, const float* pooled,
                                       int64_t nb_cap, int32_t* sel, void* ws, cudaStream_t st) {
-    CUtensorMap tmQ;
-    msa_status_t e = make_tmap_qidx(&tmQ, q_idx, G, uint64_t(B) * N);
-    if (e != MSA_OK) return e;
     const int64_t ncand = (P + N - 1) / kBlock, nbp = select_split_blocks(P + N);
     uint16_t* split = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + select_split_offset());
+    CUtensorMap tmQ, tmS;
+    msa_status_t e = make_tmap_qidx(&tmQ, q_idx, G, uint64_t(B) * N);
+    if (e == MSA_OK) e = make_tmap_split(&tmS, split, uint64_t(nbp), uint64_t(B) * G * 3);
+    if (e != MSA_OK) return e;
     {
         const int64_t threads = nbp * 8;
         const KernelTimer kt(KID_SPLIT, st);
@@ -318,7 +399,7 @@ msa_status_t launch_select_prefill_tc(const void* q_idx, int B, int G, int64_t N
     }
     dim3 grid(static_cast<unsigned>(nqb), static_cast<unsigned>(G), static_cast<unsigned>(B));
     const KernelTimer kt(KID_SELECT_PREFILL, st);
-    select_prefill_tc_kernel<<<grid, 128, smem, st>>>(tmQ, N, P, G, split, nbp, sel, static_cast<WsHeader*>(ws));
+    select_prefill_tc_kernel<<<grid, kTcThreads, smem, st>>>(tmQ, tmS, N, P, G, sel, static_cast<WsHeader*>(ws));
     return MSA_OK;
 }
 
