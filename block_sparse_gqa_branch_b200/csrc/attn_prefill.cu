@@ -113,121 +113,125 @@ __global__ void __launch_bounds__(256) csr_count_kernel(const int32_t* __restric
 // One CTA of 1024 threads. Bins are ordered (b, g, R, j) with j = nb the diagonal bin of the
 // range. Writes entry offsets, resets the counts (they become fill cursors), and emits the
 // work items in bin order: {b*G+g, j (| kDiagFlag), first entry (or first token), count}.
+// The bins go 1,024 at a time, thread i taking bin 1024 k + i, so every load and store of a
+// round is coalesced; a block-wide scan of (entries, items) per round plus the running totals
+// gives each bin its offsets, and the next round's counts are loaded during the current one.
+// Entry and item totals fit in int: the host bounds B N G (k - 1) below 2^31.
+__device__ __forceinline__ void warp_scan2(int& x, int& y, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int ax = __shfl_up_sync(0xffffffffu, x, off), ay = __shfl_up_sync(0xffffffffu, y, off);
+        if (lane >= off) { x += ax; y += ay; }
+    }
+}
+
 __global__ void __launch_bounds__(1024) csr_scan_kernel(int* __restrict__ counts, int* __restrict__ offsets,
                                                         int4* __restrict__ items, int* __restrict__ n_items,
                                                         int64_t nbins, int nb, int nR, int64_t N, int64_t P, int tpt) {
-    __shared__ long long s_e[1024], s_i[1024];
+    __shared__ int w_e[2][32], w_i[2][32];          // per-warp totals, one set per round parity
     const int nbs = nb + 1;
-    const int64_t per = (nbins + 1023) / 1024;
-    const int64_t lo = imin64(nbins, int64_t(threadIdx.x) * per), hi = imin64(nbins, lo + per);
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int items_per_max = kMaxTilesPerItem * tpt;
-    // query blocks [c0, c1) that hold positions of range R (queries R kRange .. (R + 1) kRange - 1)
-    auto diag_blocks = [&](int R, int& c0, int& c1) {
-        const int64_t a = P + int64_t(R) * kRange, z = P + imin64(N, int64_t(R + 1) * kRange);
-        c0 = int(a / kBlock);
-        c1 = int((z - 1) / kBlock) + 1;
-    };
-    // the thread's counts are read kScanBatch at a time, the loads of a batch issued together
-    constexpr int kScanBatch = 8;
-    long long se = 0, si = 0;
-    for (int64_t bin0 = lo; bin0 < hi; bin0 += kScanBatch) {
-        int cs[kScanBatch];
-#pragma unroll
-        for (int i = 0; i < kScanBatch; ++i) cs[i] = bin0 + i < hi ? counts[bin0 + i] : 0;
-#pragma unroll
-        for (int i = 0; i < kScanBatch; ++i) {
-            const int64_t bin = bin0 + i;
-            if (bin >= hi) break;
-            const int j = int(bin % nbs);
-            if (j < nb) {
-                const int cnt = cs[i];
-                se += cnt;
-                if (cnt > 0) si += (cnt + items_per_max - 1) / items_per_max;
-            } else {
-                int c0, c1;
-                diag_blocks(int((bin / nbs) % nR), c0, c1);
-                si += max(0, c1 - c0);
+    int carry_e = 0, carry_i = 0;                    // entries and items of the earlier rounds
+    int64_t bin = threadIdx.x;
+    int cnt_next = bin < nbins ? counts[bin] : 0;
+    for (int round = 0; int64_t(round) * 1024 < nbins; ++round, bin += 1024) {
+        const int cnt = cnt_next;
+        cnt_next = bin + 1024 < nbins ? counts[bin + 1024] : 0;
+        const bool live = bin < nbins;
+        const int j = int(bin % nbs);
+        const int64_t seg = bin / nbs;
+        const int R = int(seg % nR), bg = int(seg / nR);
+        // diagonal bin: query blocks [c0, c1) that hold positions of range R
+        const int64_t qa = int64_t(R) * kRange, qz = imin64(N, int64_t(R + 1) * kRange);
+        const int c0 = int((P + qa) / kBlock), c1 = int((P + qz - 1) / kBlock) + 1;
+        int ve = 0, vi = 0;
+        if (live) {
+            if (j < nb) { ve = cnt; vi = (cnt + items_per_max - 1) / items_per_max; }
+            else vi = max(0, c1 - c0);
+        }
+        int se = ve, si = vi;
+        warp_scan2(se, si, lane);
+        const int buf = round & 1;
+        if (lane == 31) { w_e[buf][wid] = se; w_i[buf][wid] = si; }
+        __syncthreads();
+        if (wid == 0) {
+            int te = w_e[buf][lane], ti = w_i[buf][lane];
+            warp_scan2(te, ti, lane);
+            w_e[buf][lane] = te;
+            w_i[buf][lane] = ti;
+        }
+        __syncthreads();
+        const int eoff = carry_e + (wid > 0 ? w_e[buf][wid - 1] : 0) + se - ve;
+        int ioff = carry_i + (wid > 0 ? w_i[buf][wid - 1] : 0) + si - vi;
+        carry_e += w_e[buf][31];
+        carry_i += w_i[buf][31];
+        if (!live) continue;
+        if (j < nb) {
+            offsets[bin] = eoff;
+            counts[bin] = 0;
+            for (int k0 = 0; k0 < cnt; k0 += items_per_max)
+                items[ioff++] = make_int4(bg, j, eoff + k0, min(items_per_max, cnt - k0));
+        } else {
+            // diagonal items: the range's queries inside block c, as (first query index, count)
+            for (int c = c0; c < c1; ++c) {
+                const int64_t f = int64_t(c) * kBlock - P > qa ? int64_t(c) * kBlock - P : qa;
+                const int64_t e = imin64(qz, int64_t(c + 1) * kBlock - P);
+                items[ioff++] = make_int4(bg, c | kDiagFlag, int(f), int(e - f));
             }
         }
     }
-    s_e[threadIdx.x] = se;
-    s_i[threadIdx.x] = si;
-    __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {             // inclusive Hillis-Steele scan
-        long long ae = 0, ai = 0;
-        if (threadIdx.x >= off) { ae = s_e[threadIdx.x - off]; ai = s_i[threadIdx.x - off]; }
-        __syncthreads();
-        s_e[threadIdx.x] += ae;
-        s_i[threadIdx.x] += ai;
-        __syncthreads();
-    }
-    long long eoff = s_e[threadIdx.x] - se, ioff = s_i[threadIdx.x] - si;
-    for (int64_t bin0 = lo; bin0 < hi; bin0 += kScanBatch) {
-        int cs[kScanBatch];
-#pragma unroll
-        for (int i = 0; i < kScanBatch; ++i) cs[i] = bin0 + i < hi ? counts[bin0 + i] : 0;
-#pragma unroll
-        for (int i = 0; i < kScanBatch; ++i) {
-            const int64_t bin = bin0 + i;
-            if (bin >= hi) break;
-            const int j = int(bin % nbs);
-            const int64_t seg = bin / nbs;
-            const int R = int(seg % nR);
-            const int bg = int(seg / nR);
-            if (j < nb) {
-                const int cnt = cs[i];
-                offsets[bin] = int(eoff);
-                counts[bin] = 0;
-                for (int k0 = 0; k0 < cnt; k0 += items_per_max)
-                    items[ioff++] = make_int4(bg, j, int(eoff + k0), min(items_per_max, cnt - k0));
-                eoff += cnt;
-            } else {
-                // diagonal items: the range's queries inside block c, as (first query index, count)
-                int c0, c1;
-                diag_blocks(R, c0, c1);
-                const int64_t qa = int64_t(R) * kRange, qz = imin64(N, int64_t(R + 1) * kRange);
-                for (int c = c0; c < c1; ++c) {
-                    const int64_t f = int64_t(c) * kBlock - P > qa ? int64_t(c) * kBlock - P : qa;
-                    const int64_t e = imin64(qz, int64_t(c + 1) * kBlock - P);
-                    items[ioff++] = make_int4(bg, c | kDiagFlag, int(f), int(e - f));
-                }
-            }
-        }
-    }
-    if (threadIdx.x == 1023) {
-        n_items[0] = int(ioff);
+    if (threadIdx.x == 0) {
+        n_items[0] = carry_i;
         n_items[1] = 0;                                   // work-item counter of the tensor-core kernel
     }
 }
 
 // ------------------------------------------------------------------ CSR: fill
-// one thread per (b, t, g): appends (t, slot) to the list of every fully-past selected block
-__global__ void __launch_bounds__(256) csr_fill_kernel(const int32_t* __restrict__ sel, int64_t N, int64_t P, int G,
-                                                       int nb, int nR, const int* __restrict__ offsets,
-                                                       int* __restrict__ cursors, int* __restrict__ list,
-                                                       int64_t total) {
-    const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (idx >= total) return;
-    const int g = int(idx % G);
-    const int64_t t = (idx / G) % N;                  // query index (position P + t)
-    const int b = int(idx / (int64_t(G) * N));
-    const int c = int((P + t) / kBlock);
-    const int R = int(t / kRange);
-    const int4* row = reinterpret_cast<const int4*>(sel + size_t(idx) * kTopK);
-    const size_t seg = (size_t(b * G + g) * nR + R) * (nb + 1);
+// grid (ceil(N / 1024), G, B), 1024 threads (one query each), dynamic smem nb ints. Every
+// fully-past selected block of the chunk's queries gets the entry (t, slot) in its list. The
+// chunk lies in one range (kRange is a multiple of kCountChunk), so it reserves one run of
+// each block's list with one global atomic: the queries number their entries per block in
+// shared memory, the counts reserve the runs, and each entry goes to its run's base plus its
+// number.
+__global__ void __launch_bounds__(1024) csr_fill_kernel(const int32_t* __restrict__ sel, int64_t N, int64_t P, int G,
+                                                        int nb, int nR, const int* __restrict__ offsets,
+                                                        int* __restrict__ cursors, int* __restrict__ list) {
+    extern __shared__ int runs[];                 // per block: entries of the chunk, then the run's base
+    const int g = blockIdx.y, b = blockIdx.z;
+    const int64_t t = int64_t(blockIdx.x) * kCountChunk + threadIdx.x;
+    const int R = int((int64_t(blockIdx.x) * kCountChunk) / kRange);
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) runs[i] = 0;
+    int ids[kTopK];
+    if (t < N) {
+        const int4* row = reinterpret_cast<const int4*>(sel + ((size_t(b) * N + t) * G + g) * kTopK);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int4 v = row[q];
-        const int ids[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int id = ids[e];
-            if (id >= 0 && id < c) {
-                const int pos = offsets[seg + id] + atomicAdd(cursors + seg + id, 1);
-                list[pos] = int(t) * kSlots + (4 * q + e);
-            }
+        for (int q = 0; q < 4; ++q) {
+            const int4 v = row[q];
+            ids[4 * q] = v.x; ids[4 * q + 1] = v.y; ids[4 * q + 2] = v.z; ids[4 * q + 3] = v.w;
         }
+    } else {
+#pragma unroll
+        for (int e = 0; e < kTopK; ++e) ids[e] = -1;
     }
+    const int c = int((P + t) / kBlock);
+    __syncthreads();
+    int num[kTopK];
+#pragma unroll
+    for (int e = 0; e < kTopK; ++e) {
+        const int id = ids[e];
+        num[e] = (id >= 0 && id < c) ? atomicAdd(&runs[id], 1) : -1;
+    }
+    __syncthreads();
+    const size_t seg = (size_t(b * G + g) * nR + R) * (nb + 1);
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        const int n = runs[i];
+        if (n > 0) runs[i] = offsets[seg + i] + atomicAdd(cursors + seg + i, n);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < kTopK; ++e)
+        if (num[e] >= 0) list[runs[ids[e]] + num[e]] = int(t) * kSlots + e;
 }
 
 // ------------------------------------------------------------------ the tensor-core kernel
@@ -829,10 +833,13 @@ void launch_inverted_index(const int32_t* sel, int64_t N, int64_t P, int B, int 
         csr_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, items, nitems, int64_t(L.nbins), L.nb, L.nR, N, P, L.tpt);
     }
     {
-        const int64_t total = int64_t(B) * N * G;
+        dim3 grid(static_cast<unsigned>((N + kCountChunk - 1) / kCountChunk), static_cast<unsigned>(G),
+                  static_cast<unsigned>(B));
+        const size_t smem = size_t(L.nb) * sizeof(int);
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(csr_fill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         const KernelTimer kt(KID_CSR, st);
-        csr_fill_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(sel, N, P, G, L.nb, L.nR, offsets,
-                                                                                   counts, list, total);
+        csr_fill_kernel<<<grid, kCountChunk, smem, st>>>(sel, N, P, G, L.nb, L.nR, offsets, counts, list);
     }
 }
 
