@@ -19,7 +19,7 @@ __all__ = [
     "MSAError", "Shape", "load", "lib_path",
     "msa_abi_version", "msa_status_string", "msa_workspace_size",
     "msa_pool_index_keys", "msa_index_select", "msa_sparse_attn_prefill",
-    "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_get_device_status",
+    "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_decode_step", "msa_get_device_status",
     "msa_index_select_decode_noalloc", "msa_selftest_wait_timeout", "msa_kernel_launches",
     "msa_topk_rows", "msa_fp8_quantize_blocks", "msa_fp8_close_blocks", "msa_sparse_attn_decode_fp8",
     "msa_pool_index_keys_chunk", "msa_index_select_chunk", "msa_sparse_attn_prefill_chunk",
@@ -44,7 +44,7 @@ EXPORTED_SYMBOLS = [
     "msa_abi_version", "msa_status_string", "msa_last_cuda_error", "msa_kernel_launches",
     "msa_workspace_size",
     "msa_pool_index_keys", "msa_index_select", "msa_sparse_attn_prefill",
-    "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_get_device_status",
+    "msa_pooled_keys_append", "msa_sparse_attn_decode", "msa_decode_step", "msa_get_device_status",
     "msa_index_select_decode_noalloc", "msa_selftest_wait_timeout", "msa_topk_rows",
     "msa_fp8_quantize_blocks", "msa_fp8_close_blocks", "msa_sparse_attn_decode_fp8",
     "msa_pool_index_keys_chunk", "msa_index_select_chunk", "msa_sparse_attn_prefill_chunk",
@@ -112,6 +112,7 @@ def load():
             "msa_sparse_attn_prefill": [SP, P, P, P, I64, P, P, P, P, SZ, P],
             "msa_pooled_keys_append": [SP, P, P, P, P, P, P, I64, P, P, I64, P, SZ, P],
             "msa_sparse_attn_decode": [SP, P, P, P, I64, P, I64, P, P, P, P, SZ, P],
+            "msa_decode_step": [SP, P, P, P, P, P, P, P, P, I64, P, P, I64, I64, P, P, P, P, SZ, P, SZ, P, SZ, P],
             "msa_get_device_status": [P, P, P],
             "msa_index_select_decode_noalloc": [SP, P, P, I64, P, I64, P, P],
             "msa_selftest_wait_timeout": [P, SZ, P],
@@ -231,6 +232,17 @@ def msa_sparse_attn_decode(shape: Shape, q, k_cache, v_cache, l_cap: int, q_pos,
                                          l_cap, _ptr(q_pos), max_pos, _ptr(sel), _ptr(out), _ptr(lse),
                                          _ptr(workspace), _nbytes(workspace), _stream(stream)),
            "msa_sparse_attn_decode")
+
+
+def msa_decode_step(shape: Shape, q, q_idx, k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, l_cap: int,
+                    tail_sum, pooled, nb_cap: int, max_pos: int, sel, out, lse, ws_select, ws_append, ws_attn,
+                    stream=None):
+    _check(load().msa_decode_step(ctypes.byref(shape), _ptr(q), _ptr(q_idx), _ptr(k_idx_new), _ptr(k_new),
+                                  _ptr(v_new), _ptr(ctx_len), _ptr(k_cache), _ptr(v_cache), l_cap, _ptr(tail_sum),
+                                  _ptr(pooled), nb_cap, max_pos, _ptr(sel), _ptr(out), _ptr(lse),
+                                  _ptr(ws_select), _nbytes(ws_select), _ptr(ws_append), _nbytes(ws_append),
+                                  _ptr(ws_attn), _nbytes(ws_attn), _stream(stream)),
+           "msa_decode_step")
 
 
 def msa_get_device_status(workspace, stream=None):

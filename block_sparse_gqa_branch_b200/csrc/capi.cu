@@ -258,6 +258,46 @@ size_t ws_size(const msa_shape_t* s, int32_t op, int64_t n) {
     }
 }
 
+// Argument checks shared by the decode entry points and msa_decode_step (shape already checked).
+msa_status_t check_select_decode(const msa_shape_t* shape, int64_t max_pos, int64_t nb_cap, const void* workspace,
+                                 size_t workspace_bytes) {
+    MSA_REQ(max_pos <= kMaxPos, MSA_ERR_UNSUPPORTED);
+    MSA_REQ(nb_cap >= max_pos / kBlock, MSA_ERR_INVALID_ARGUMENT);
+    const size_t need = ws_size(shape, MSA_OP_INDEX_SELECT_DECODE, max_pos);
+    MSA_REQ(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need, MSA_ERR_WORKSPACE);
+    return MSA_OK;
+}
+
+msa_status_t check_append(const void* k_idx_new, const void* k_new, const void* v_new, const int32_t* ctx_len,
+                          const void* k_cache, const void* v_cache, int64_t l_cap, const float* tail_sum,
+                          const float* pooled, int64_t nb_cap, const void* workspace, size_t workspace_bytes) {
+    MSA_REQ(k_idx_new && aligned16(k_idx_new) && ctx_len && tail_sum && aligned16(tail_sum) && pooled &&
+                aligned16(pooled),
+            MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ((k_new == nullptr) == (v_new == nullptr), MSA_ERR_INVALID_ARGUMENT);
+    if (k_new != nullptr)
+        MSA_REQ(aligned16(k_new) && aligned16(v_new) && k_cache && v_cache && aligned16(k_cache) &&
+                    aligned16(v_cache) && l_cap >= 1,
+                MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(nb_cap >= 1, MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(workspace != nullptr && workspace_bytes >= header_only(), MSA_ERR_WORKSPACE);
+    return MSA_OK;
+}
+
+msa_status_t check_attn_decode(const msa_shape_t* shape, const void* q, const void* k_cache, const void* v_cache,
+                               int64_t l_cap, const int32_t* q_pos, int64_t max_pos, const int32_t* sel,
+                               const void* out, const float* lse, const void* workspace, size_t workspace_bytes) {
+    MSA_REQ(q && k_cache && v_cache && q_pos && sel && out && aligned16(q) && aligned16(k_cache) &&
+                aligned16(v_cache) && aligned16(sel) && aligned16(out) &&
+                (lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u) == 0),
+            MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(l_cap >= 1 && max_pos >= 0 && max_pos < l_cap, MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(int64_t(shape->batch) * shape->n_kv_groups * l_cap + kBlock < (int64_t(1) << 31), MSA_ERR_UNSUPPORTED);
+    const size_t need = ws_size(shape, MSA_OP_ATTN_DECODE, max_pos);
+    MSA_REQ(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need, MSA_ERR_WORKSPACE);
+    return MSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -340,10 +380,7 @@ msa_status_t msa_index_select(const msa_shape_t* shape, const void* q_idx, int64
         MSA_TRY(launch_select_prefill_tc(q_idx, B, G, n_queries, 0, pooled, nb_cap, sel, workspace, st));
     } else {                                       // decode: one query per sequence at q_pos[b]
         MSA_REQ(n_queries == 1, MSA_ERR_INVALID_ARGUMENT);
-        MSA_REQ(max_pos <= kMaxPos, MSA_ERR_UNSUPPORTED);
-        MSA_REQ(nb_cap >= max_pos / kBlock, MSA_ERR_INVALID_ARGUMENT);
-        const size_t need = ws_size(shape, MSA_OP_INDEX_SELECT_DECODE, max_pos);
-        MSA_REQ(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need, MSA_ERR_WORKSPACE);
+        MSA_TRY(check_select_decode(shape, max_pos, nb_cap, workspace, workspace_bytes));
         launch_select_decode(q_idx, q_pos, max_pos, B, G, pooled, nb_cap, sel, workspace, st);
     }
     return cuda_status();
@@ -468,16 +505,8 @@ msa_status_t msa_pooled_keys_append(const msa_shape_t* shape, const void* k_idx_
                                     size_t workspace_bytes, msa_stream_t stream) {
     MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
-    MSA_REQ(k_idx_new && aligned16(k_idx_new) && ctx_len && tail_sum && aligned16(tail_sum) && pooled &&
-                aligned16(pooled),
-            MSA_ERR_INVALID_ARGUMENT);
-    MSA_REQ((k_new == nullptr) == (v_new == nullptr), MSA_ERR_INVALID_ARGUMENT);
-    if (k_new != nullptr)
-        MSA_REQ(aligned16(k_new) && aligned16(v_new) && k_cache && v_cache && aligned16(k_cache) &&
-                    aligned16(v_cache) && l_cap >= 1,
-                MSA_ERR_INVALID_ARGUMENT);
-    MSA_REQ(nb_cap >= 1, MSA_ERR_INVALID_ARGUMENT);
-    MSA_REQ(workspace != nullptr && workspace_bytes >= header_only(), MSA_ERR_WORKSPACE);
+    MSA_TRY(check_append(k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, l_cap, tail_sum, pooled, nb_cap,
+                         workspace, workspace_bytes));
     launch_append(k_idx_new, k_new, v_new, ctx_len, shape->batch, shape->n_kv_groups, k_cache, v_cache,
                   k_new ? l_cap : int64_t(1) << 62, tail_sum, pooled, nb_cap, workspace,
                   reinterpret_cast<cudaStream_t>(stream));
@@ -490,18 +519,39 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const void* q, con
                                     size_t workspace_bytes, msa_stream_t stream) {
     MSA_CALL_RANGE();
     MSA_TRY(check_shape(shape));
-    MSA_REQ(q && k_cache && v_cache && q_pos && sel && out && aligned16(q) && aligned16(k_cache) &&
-                aligned16(v_cache) && aligned16(sel) && aligned16(out) &&
-                (lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u) == 0),
-            MSA_ERR_INVALID_ARGUMENT);
-    MSA_REQ(l_cap >= 1 && max_pos >= 0 && max_pos < l_cap, MSA_ERR_INVALID_ARGUMENT);
+    MSA_TRY(check_attn_decode(shape, q, k_cache, v_cache, l_cap, q_pos, max_pos, sel, out, lse, workspace,
+                              workspace_bytes));
     const int B = shape->batch, G = shape->n_kv_groups;
-    MSA_REQ(int64_t(B) * G * l_cap + kBlock < (int64_t(1) << 31), MSA_ERR_UNSUPPORTED);
-    const size_t need = ws_size(shape, MSA_OP_ATTN_DECODE, max_pos);
-    MSA_REQ(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need, MSA_ERR_WORKSPACE);
     MSA_TRY(launch_attn_decode(k_cache, v_cache, q, l_cap, q_pos, max_pos, sel, B, G, shape->n_q_heads / G, out, lse,
                                workspace, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr, nullptr,
                                0));
+    return cuda_status();
+}
+
+msa_status_t msa_decode_step(const msa_shape_t* shape, const void* q, const void* q_idx, const void* k_idx_new,
+                             const void* k_new, const void* v_new, const int32_t* ctx_len, void* k_cache,
+                             void* v_cache, int64_t l_cap, float* tail_sum, float* pooled, int64_t nb_cap,
+                             int64_t max_pos, int32_t* sel, void* out, float* lse, void* ws_select,
+                             size_t ws_select_bytes, void* ws_append, size_t ws_append_bytes, void* ws_attn,
+                             size_t ws_attn_bytes, msa_stream_t stream) {
+    MSA_CALL_RANGE();
+    MSA_TRY(check_shape(shape));
+    // every argument of the three steps is checked before the first launch
+    MSA_REQ(q_idx != nullptr && aligned16(q_idx) && sel != nullptr && aligned16(sel) && aligned16(pooled),
+            MSA_ERR_INVALID_ARGUMENT);
+    MSA_REQ(k_new != nullptr && max_pos >= 0 && nb_cap >= 0, MSA_ERR_INVALID_ARGUMENT);
+    MSA_TRY(check_select_decode(shape, max_pos, nb_cap, ws_select, ws_select_bytes));
+    MSA_TRY(check_append(k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, l_cap, tail_sum, pooled, nb_cap,
+                         ws_append, ws_append_bytes));
+    MSA_TRY(check_attn_decode(shape, q, k_cache, v_cache, l_cap, ctx_len, max_pos, sel, out, lse, ws_attn,
+                              ws_attn_bytes));
+    const int B = shape->batch, G = shape->n_kv_groups, Hg = shape->n_q_heads / G;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    launch_select_decode(q_idx, ctx_len, max_pos, B, G, pooled, nb_cap, sel, ws_select, st);
+    launch_append(k_idx_new, k_new, v_new, ctx_len, B, G, k_cache, v_cache, l_cap, tail_sum, pooled, nb_cap, ws_append,
+                  st);
+    MSA_TRY(launch_attn_decode(k_cache, v_cache, q, l_cap, ctx_len, max_pos, sel, B, G, Hg, out, lse, ws_attn, st,
+                               nullptr, nullptr, nullptr, nullptr, 0));
     return cuda_status();
 }
 

@@ -10,9 +10,9 @@ import torch
 
 from . import (BLOCK, INDEX_DIM, TOPK, OP_ATTN_DECODE, OP_ATTN_PREFILL, OP_ATTN_PREFILL_BACKWARD,
                OP_INDEX_SELECT_DECODE, msa_sparse_attn_prefill_backward,
-               OP_INDEX_SELECT_PREFILL, Shape, msa_fp8_close_blocks, msa_fp8_quantize_blocks,
+               OP_INDEX_SELECT_PREFILL, Shape, msa_decode_step, msa_fp8_close_blocks, msa_fp8_quantize_blocks,
                msa_index_select, msa_index_select_chunk, msa_pool_index_keys, msa_pool_index_keys_chunk,
-               msa_pooled_keys_append, msa_prefill_chunk_workspace_size, msa_sparse_attn_decode,
+               msa_pooled_keys_append, msa_prefill_chunk_workspace_size,
                msa_sparse_attn_decode_fp8, msa_sparse_attn_prefill, msa_sparse_attn_prefill_chunk,
                msa_workspace_size)
 
@@ -81,18 +81,15 @@ def decode_step(q, q_idx, k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, ta
     """One decode step: select, append the new token (KV + pooled keys), attend.
     ctx_len [B] int32 on the device = tokens cached before the step (the new token's position).
     Caches: k_cache/v_cache [B,G,l_cap,128] bf16, pooled [B,G,nb_cap,64] fp32, tail_sum [B,G,64].
-    The selection comes first: it scores only blocks below the new token's own, which the append
-    does not change, so the append runs in its shadow (programmatic dependent launch) and the
-    attention, which needs both, waits for the append's completion (after the selection's).
+    One msa_decode_step call: the selection comes first (it scores only blocks below the new
+    token's own, which the append does not change), so the append runs in its shadow
+    (programmatic dependent launch), and the attention, which needs both, waits for the
+    append's completion (after the selection's).
     Returns (out [B,Hq,128], lse [B,Hq], sel [B,G,16])."""
     s, mp = bufs["shape"], bufs["max_pos"]
-    l_cap = k_cache.shape[2]
-    nb_cap = pooled.shape[2]
-    msa_index_select(s, q_idx, 1, ctx_len, mp, pooled, nb_cap, bufs["sel"], bufs["ws_select"], stream)
-    msa_pooled_keys_append(s, k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, l_cap, tail_sum, pooled,
-                           nb_cap, bufs["ws_append"], stream)
-    msa_sparse_attn_decode(s, q, k_cache, v_cache, l_cap, ctx_len, mp, bufs["sel"], bufs["out"], bufs["lse"],
-                           bufs["ws_attn"], stream)
+    msa_decode_step(s, q, q_idx, k_idx_new, k_new, v_new, ctx_len, k_cache, v_cache, k_cache.shape[2], tail_sum,
+                    pooled, pooled.shape[2], mp, bufs["sel"], bufs["out"], bufs["lse"], bufs["ws_select"],
+                    bufs["ws_append"], bufs["ws_attn"], stream)
     return bufs["out"], bufs["lse"], bufs["sel"]
 
 

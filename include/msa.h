@@ -327,6 +327,23 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t *shape, const void *q, con
                                     msa_stream_t stream);
 
 /*
+ * A whole decode step in one call: msa_index_select (decode, q_pos = ctx_len), then
+ * msa_pooled_keys_append, then msa_sparse_attn_decode, on the stream in that order, with the
+ * same arguments, kernels and results as those three calls (sources as theirs). The three
+ * workspaces are theirs: msa_workspace_size(MSA_OP_INDEX_SELECT_DECODE, max_pos), at least 256
+ * bytes, and msa_workspace_size(MSA_OP_ATTN_DECODE, max_pos); each records its own kernels'
+ * device errors (msa_get_device_status). k_new and v_new are required. Every argument of the
+ * three steps is checked before the first launch, so a rejected call changes nothing.
+ */
+msa_status_t msa_decode_step(const msa_shape_t *shape, const void *q, const void *q_idx,
+                             const void *k_idx_new, const void *k_new, const void *v_new,
+                             const int32_t *ctx_len, void *k_cache, void *v_cache, int64_t l_cap,
+                             float *tail_sum, float *pooled, int64_t nb_cap, int64_t max_pos,
+                             int32_t *sel, void *out, float *lse, void *ws_select,
+                             size_t ws_select_bytes, void *ws_append, size_t ws_append_bytes,
+                             void *ws_attn, size_t ws_attn_bytes, msa_stream_t stream);
+
+/*
  * FP8 (e4m3) key-value cache of the decode step. Source: KuCoin flash "MiniMax launches MSA
  * sparse attention method and MiniMax-M3 model", "ME AI News" paragraph (the SM100 attention
  * kernel also takes FP8 inputs); the pages give no format, so this library's reading is:

@@ -110,6 +110,41 @@ def test_validation_errors_before_launch(L):
     assert L.msa_pooled_keys_append(bs, FAKE, None, None, FAKE, None, None, 0, FAKE, FAKE, 1, FAKE, 16, None) == 3
 
 
+def test_decode_step_validates_all_three_steps_before_launch(L):
+    s = _shape(batch=2, n_q_heads=16, n_kv_groups=2)
+    bs = ctypes.byref(s)
+    max_pos, l_cap, nb_cap = 4095, 4096, 32     # every call below fails validation: nothing launches
+    ws_sel = msa.msa_workspace_size(s, msa.OP_INDEX_SELECT_DECODE, max_pos)
+    ws_att = msa.msa_workspace_size(s, msa.OP_ATTN_DECODE, max_pos)
+    ok = [bs, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE2, FAKE, FAKE, l_cap, FAKE, FAKE, nb_cap, max_pos,
+          FAKE2, FAKE, None, FAKE, ws_sel, FAKE, 256, FAKE, ws_att, None]
+
+    def call(**kw):
+        args = list(ok)
+        names = ["shape", "q", "q_idx", "k_idx_new", "k_new", "v_new", "ctx_len", "k_cache", "v_cache", "l_cap",
+                 "tail_sum", "pooled", "nb_cap", "max_pos", "sel", "out", "lse", "ws_select", "ws_select_bytes",
+                 "ws_append", "ws_append_bytes", "ws_attn", "ws_attn_bytes", "stream"]
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return L.msa_decode_step(*args)
+
+    assert call(shape=None) == 1
+    assert call(k_new=None, v_new=None) == 1               # the step always appends K and V
+    assert call(v_new=None) == 1
+    assert call(q_idx=FAKE + 2) == 1                       # misaligned
+    assert call(sel=None) == 1
+    assert call(q=None) == 1
+    assert call(ctx_len=None) == 1
+    assert call(max_pos=l_cap) == 1                        # positions beyond the cache
+    assert call(nb_cap=max_pos // 128 - 1) == 1             # too small for the last position
+    assert call(max_pos=1 << 26, l_cap=1 << 27, nb_cap=1 << 20) == 2
+    assert call(ws_select_bytes=ws_sel - 16) == 3
+    assert call(ws_append=None) == 3
+    assert call(ws_append_bytes=16) == 3
+    assert call(ws_attn_bytes=ws_att - 256) == 3
+    assert call(ws_attn=FAKE + 8) == 3                     # misaligned
+
+
 def test_binding_rejects_host_tensors(L):
     import torch
     with pytest.raises(ValueError):

@@ -274,3 +274,53 @@ def test_decode_step_order_gives_the_same_results(cuda_ok, order):
         assert not torch.isnan(st["pooled"][0, :, 15]).any()
         if graph:
             del g
+
+
+def test_decode_step_entry_matches_separate_calls(cuda_ok):
+    """msa_decode_step (80 groups: one attention CTA per (sequence, group)) gives the selection,
+    output and lse of the three separate calls bit for bit, eager and replayed from a graph, call
+    after call, writes the same cache rows, and leaves no device error."""
+    w = synth.Workload(name="t", kind="decode", B=10, Hq=64, G=8,
+                       ctx=(2047, 3000, 383, 4095, 128, 2500, 1000, 3333, 127, 3900), seed=777)
+    l_cap = 4224
+    s, mp = Shape.make(w.B, w.Hq, w.G), max(w.ctx)
+    ref = build_decode_state(w, l_cap)
+    rb = pipeline.decode_buffers(w.B, w.Hq, w.G, mp, "cuda")
+    msa_index_select(s, ref["q_idx"], 1, ref["ctx"], mp, ref["pooled"], ref["nb_cap"], rb["sel"], rb["ws_select"])
+    msa_pooled_keys_append(s, ref["k_idx_new"], ref["k_new"], ref["v_new"], ref["ctx"], ref["k_cache"],
+                           ref["v_cache"], l_cap, ref["tail"], ref["pooled"], ref["nb_cap"], rb["ws_append"])
+    msa_sparse_attn_decode(s, ref["q"], ref["k_cache"], ref["v_cache"], l_cap, ref["ctx"], mp, rb["sel"], rb["out"],
+                           rb["lse"], rb["ws_attn"])
+    torch.cuda.synchronize()
+    s_ref, o_ref, l_ref = rb["sel"].clone(), rb["out"].clone(), rb["lse"].clone()
+
+    st = build_decode_state(w, l_cap)
+    bufs = pipeline.decode_buffers(w.B, w.Hq, w.G, mp, "cuda")
+
+    def step():
+        pipeline.decode_step(st["q"], st["q_idx"], st["k_idx_new"], st["k_new"], st["v_new"], st["ctx"],
+                             st["k_cache"], st["v_cache"], st["tail"], st["pooled"], bufs)
+
+    def check(what):
+        torch.cuda.synchronize()
+        for key in ("ws_append", "ws_select", "ws_attn"):
+            stt, info = msa_get_device_status(bufs[key])
+            assert stt == 0, (what, key, stt, info)
+        assert torch.equal(bufs["sel"], s_ref), what
+        assert torch.equal(bufs["out"].view(torch.int16), o_ref.view(torch.int16)), what
+        assert torch.equal(bufs["lse"], l_ref), what
+        bufs["out"].zero_()
+        bufs["sel"].fill_(-7)
+
+    for i in range(3):
+        step()
+        check(f"eager call {i}")
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for i in range(3):
+        g.replay()
+        check(f"graph replay {i}")
+    del g
+    for key in ("k_cache", "v_cache"):          # bits: rows past the context hold NaNs
+        assert torch.equal(st[key].view(torch.int16), ref[key].view(torch.int16)), key
